@@ -1,0 +1,88 @@
+"""Planted mistakes in the oracle must fail its pins.
+
+Each case copies kvq_oracle.c, applies one plausible mistake (a wrong constant, a
+dropped term, a wrong sign, a transposed operand, a wrong index), compiles the copy on
+the CPU and runs the pin tests against it. A mutation no pin catches would mean the
+pins do not constrain that part of the oracle.
+"""
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "kvq_oracle.c")
+
+MUTATIONS = [
+    ("per-tensor qmax 128", "scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : 127.0f);",
+     "scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : 128.0f);"),
+    ("per-token qmax 128", "tok_scale = amax / 127.0f;", "tok_scale = amax / 128.0f;"),
+    ("per-channel qmax 255", "scale[h * D + d] = amax / 127.0f;", "scale[h * D + d] = amax / 255.0f;"),
+    ("round half away", "  float y = x / s;\n  float r = rintf(y);", "  float y = x / s;\n  float r = roundf(y);"),
+    ("clamp -128", "if (r < (float)-qmax) r = (float)-qmax;", "if (r < (float)(-qmax - 1)) r = (float)(-qmax - 1);"),
+    ("fp8 scale 240", "448.0f : 127.0f", "240.0f : 127.0f"),
+    ("e4m3 bias", "v = ldexpf((float)(8 + m), e - 10);", "v = ldexpf((float)(8 + m), e - 9);"),
+    ("e4m3 no saturation", "if (a > 448.0f) return (uint8_t)(sign | 0x7E);", "if (a > 480.0f) return (uint8_t)(sign | 0x7F);"),
+    ("asym zp sign", "float z = rintf(-lo / sc);", "float z = rintf(lo / sc);"),
+    ("asym 256 levels", "float sc = (hi - lo) / 255.0f;", "float sc = (hi - lo) / 256.0f;"),
+    ("asym page form", "float r = rintf(x / s) + (float)zp;", "float r = rintf(x / s);"),
+    ("kivi dequant sign", "  return a + mn;", "  return a - mn;"),
+    ("kivi no min shift", "float diff = x[(size_t)i * stride] - lo;", "float diff = x[(size_t)i * stride];"),
+    ("kivi key axis transposed",
+     "oq_kivi_group(xk + (size_t)gi * g * D + d, g, D, kb, codes, &s, &mn);",
+     "oq_kivi_group(xk + (size_t)gi * g * D + (size_t)d * g % (g * D), g, 1, kb, codes, &s, &mn);"),
+    ("kivi flush rule", "const int r_new = ((total - 1) % R) + 1;", "const int r_new = total % R;"),
+    ("kivi pack order", "const int byte = d / per, sh = (d % per) * bits;",
+     "const int byte = d / per, sh = (per - 1 - d % per) * bits;"),
+    ("paged slot", "(size_t)(t % c->page_size);\n}", "(size_t)((t + 1) % c->page_size);\n}"),
+    ("calibration skips last head", "      for (int h = 0; h < H; ++h)\n        for (int t = 0; t < block_len(k, b); ++t)\n          for (int d = 0; d < D; ++d) {\n            float a = fabsf",
+     "      for (int h = 0; h < H - 1; ++h)\n        for (int t = 0; t < block_len(k, b); ++t)\n          for (int d = 0; d < D; ++d) {\n            float a = fabsf"),
+    ("attention drops scale", "s[t] = acc * (double)scale;", "s[t] = acc;"),
+    ("attention no max shift", "const double p = exp(s[t] - m);", "const double p = exp(s[t]);"),
+    ("attention lse", "*lse = m + log(l);", "*lse = log(l);"),
+    ("gqa mapping", "const int hq = hk * G + j;", "const int hq = j * c->Hkv + hk;"),
+    ("bytes formula", "return 2.0 * bytes_per_elem *", "return bytes_per_elem *"),
+]
+
+
+def _pin_tests():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if params:
+            argname, values = params[0].args
+            for v in values:
+                out.append((f"{name}[{v}]", lambda fn=fn, a=argname, v=v: fn(**{a: v})))
+        else:
+            out.append((name, fn))
+    return out
+
+
+@pytest.mark.parametrize("label,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_pins_catch_mutation(label, old, new, tmp_path):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique or missing: {label}"
+    mut = tmp_path / "kvq_oracle.c"
+    mut.write_text(src.replace(old, new))
+    (tmp_path / "kvq_oracle.h").write_text(open(SRC[:-2] + ".h").read())
+    so = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), str(mut), "-lm"])
+    saved = oracle._lib
+    oracle._lib = oracle.load(str(so))
+    caught = []
+    try:
+        for name, fn in _pin_tests():
+            try:
+                fn()
+            except (AssertionError, ValueError):
+                caught.append(name)
+                break
+    finally:
+        oracle._lib = saved
+    assert caught, f"no pin failed for planted mistake: {label}"

@@ -1,0 +1,499 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a worked example the
+pages print, a closed form, an invariant, an independent library routine, or brute force.
+"""
+import decimal
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import OracleCache
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+F32 = np.float32
+
+
+def _read_golden(name):
+    sections, cur = {}, None
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line in ("tokens", "codes"):
+                cur = sections.setdefault(line, [])
+                continue
+            cur.append(line.split())
+    return sections
+
+
+def _rne(fr: Fraction) -> int:
+    """Round a rational half to even."""
+    fl = math.floor(fr)
+    rem = fr - fl
+    if rem > Fraction(1, 2):
+        return fl + 1
+    if rem < Fraction(1, 2):
+        return fl
+    return fl if fl % 2 == 0 else fl + 1
+
+
+def _sym_exact(xs, absmax):
+    s = Fraction(absmax) / 127
+    return [max(-127, min(127, _rne(Fraction(x) / s))) for x in xs]
+
+
+# --------------------------------------------------------------- worked examples
+def test_key_worked_example_per_channel():
+    g = _read_golden("key_per_channel_example.txt")
+    X = np.array([[float(v) for v in row[1:]] for row in g["tokens"]], np.float32)  # [3 tok, 4 ch]
+    c = OracleCache(1, 1, 1, 4, oracle.INT8_SYM_PER_CHANNEL, oracle.INT8_SYM_PER_CHANNEL, cap=8)
+    x = X[None, None]  # [B=1, H=1, T=3, D=4]
+    c.append(x, x, bf16=False, calibrate=True)
+    codes = c["k_codes"][0, 0, :3].view(np.int8)
+    for row in g["codes"]:
+        ch, num, want = int(row[0]) - 1, row[1], [int(v) for v in row[2:]]
+        col = [str(r[1 + ch]) for r in g["tokens"]]
+        assert _sym_exact(col, max(Fraction(v) for v in col)) == want  # fixture is exact math
+        assert list(codes[:, ch]) == want
+        # the per-channel scale is max|column| / 127; channel 3 prints s = 9.0/127
+        assert c["k_scale"][0, ch] == F32(float(num)) / F32(127)
+    assert c["k_scale"][0, 2] == F32(9.0) / F32(127)
+    # each column has its own scale: channel 3's outliers do not touch channels 1, 2, 4
+    assert len(set(c["k_scale"][0].tolist())) == 3
+
+
+def test_value_worked_example_per_token():
+    g = _read_golden("value_per_token_example.txt")
+    X = np.array([[float(v) for v in row[1:]] for row in g["tokens"]], np.float32)
+    c = OracleCache(1, 1, 1, 4, oracle.INT8_SYM_PER_TOKEN, oracle.INT8_SYM_PER_TOKEN, cap=8)
+    c.append(X[None, None], X[None, None], bf16=False)
+    codes = c["v_codes"][0, 0, :3].view(np.int8)
+    for row in g["codes"]:
+        t, num, want = int(row[0]) - 1, row[1], [int(v) for v in row[2:]]
+        tok = g["tokens"][t][1:]
+        assert _sym_exact(tok, max(Fraction(v) for v in tok)) == want
+        assert list(codes[t]) == want
+        assert c["v_scale"][0, 0, t] == F32(float(num)) / F32(127)
+
+
+# --------------------------------------------------------------- byte arithmetic
+def test_memory_table_and_formula():
+    table = []
+    with open(os.path.join(GOLDEN, "memory_table.txt")) as fh:
+        for line in fh:
+            if line.strip() and not line.startswith("#"):
+                table.append(line.split())
+    per_tok = {}
+    for name, bpe, kb, gb, req in table:
+        b = oracle.kv_bytes_per_token(80, 8, 128, float(bpe))
+        per_tok[name] = b
+        assert b / 1024 == float(kb)                       # 320 / 160 / 80 KiB
+        assert abs(b * 4096 / 2**30 - float(gb)) < 0.0051  # 1.25 / 0.63 / 0.31 GiB
+        exact = int(45 * 2**30 // (b * 4096))
+        assert abs(exact - int(req)) <= 1                  # 36/72/144 vs printed 36/71/145
+    assert per_tok["BF16"] == 327680.0 == 2 * 2 * 80 * 8 * 128
+    assert per_tok["FP8"] == 163840.0 and per_tok["INT4"] == 81920.0
+    assert per_tok["BF16"] * 4096 == 1.25 * 2**30
+
+
+# --------------------------------------------------------------- E4M3 codec
+def test_e4m3_decode_matches_torch():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    for c in codes:
+        got = oracle.e4m3_decode(int(c))
+        if np.isnan(ref[c]):
+            assert np.isnan(got)
+        else:
+            assert got == ref[c] and np.signbit(got) == np.signbit(ref[c])
+
+
+def test_e4m3_roundtrip_all_codes():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue  # NaN
+        assert oracle.e4m3_encode(oracle.e4m3_decode(c)) == c
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(7)
+    x = np.concatenate([
+        rng.uniform(-448, 448, 20000), rng.normal(0, 1, 20000), rng.normal(0, 0.01, 20000),
+        np.ldexp(rng.uniform(-1, 1, 5000), -8),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(v) for v in x], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_ties_saturation_and_zero():
+    assert oracle.e4m3_encode(1.0 + 1 / 16) == oracle.e4m3_encode(1.0)        # tie -> even (m=0)
+    assert oracle.e4m3_decode(oracle.e4m3_encode(1.0 + 3 / 16)) == 1.25         # tie -> even (m=2)
+    assert oracle.e4m3_encode(2.0**-10) == 0x00                                 # subnormal tie -> 0
+    assert oracle.e4m3_decode(oracle.e4m3_encode(3 * 2.0**-10)) == 2.0**-8      # -> even code 2
+    for big in (448.0, 449.0, 464.0, 500.0, 1e30, float("inf")):
+        assert oracle.e4m3_encode(big) == 0x7E
+        assert oracle.e4m3_encode(-big) == 0xFE
+    assert oracle.e4m3_decode(0x7E) == 448.0
+    assert oracle.e4m3_encode(-0.0) == 0x80 and oracle.e4m3_encode(0.0) == 0x00
+
+
+def test_e4m3_nearest_by_brute_force():
+    finite = [(c, oracle.e4m3_decode(c)) for c in range(128) if c != 0x7F]
+    rng = np.random.default_rng(3)
+    for x in rng.uniform(0, 448, 3000).astype(np.float32):
+        code = oracle.e4m3_encode(float(x))
+        best = min(abs(v - float(x)) for _, v in finite)
+        assert abs(oracle.e4m3_decode(code) - float(x)) == best
+
+
+# --------------------------------------------------------------- symmetric INT8
+def test_sym_round_half_even_tie():
+    s = 0.125
+    assert oracle.sym_code(62.5 * s, s) == 62   # half-away would give 63
+    assert oracle.sym_code(63.5 * s, s) == 64
+    assert oracle.sym_code(-62.5 * s, s) == -62
+    assert oracle.sym_code(5.0, 0.0) == 0       # zero range
+    assert oracle.sym_code(1000.0, 1.0) == 127 and oracle.sym_code(-1000.0, 1.0) == -127
+
+
+def test_sym_exact_roundtrip_and_half_step_bound():
+    for s in (2.0**-7, 0.25, 1.0, 8.0):
+        for k in range(-127, 128):
+            assert oracle.sym_code(k * s, s) == k
+    rng = np.random.default_rng(11)
+    x = rng.normal(0, 3, 4000).astype(np.float32)
+    s = F32(np.abs(x).max()) / F32(127)
+    for v in x:
+        q = oracle.sym_code(float(v), float(s))
+        xh = F32(q) * s
+        assert abs(float(xh) - float(v)) <= float(s) / 2 * (1 + 2**-22)
+
+
+def test_per_tensor_scale_covers_all_rows_and_heads():
+    B, H, T, D = 2, 3, 5, 8
+    rng = np.random.default_rng(1)
+    x = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    x[1, 2, 4, 7] = -50.0  # the largest magnitude sits in the last row / head / token / channel
+    c = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.INT8_SYM_PER_TENSOR, cap=16)
+    c.append(x, x, bf16=False, calibrate=True)
+    assert c["k_scale"][0] == F32(50.0) / F32(127)
+    assert c["k_codes"][1, 2, 4, 7].view(np.int8) == -127
+    # a second, non-calibrating append keeps the scale and saturates out-of-range values
+    y = np.full((B, H, 1, D), 100.0, np.float32)
+    c.append(y, y, bf16=False)
+    assert c["k_scale"][0] == F32(50.0) / F32(127)
+    assert np.all(c["k_codes"][:, :, T].view(np.int8) == 127)
+
+
+def test_fp8_per_tensor_scale_and_codes():
+    rng = np.random.default_rng(2)
+    x = rng.normal(0, 2, (1, 2, 6, 16)).astype(np.float32)
+    c = OracleCache(1, 2, 2, 16, oracle.FP8_E4M3_PER_TENSOR, oracle.FP8_E4M3_PER_TENSOR, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    s = F32(np.abs(x).max()) / F32(448)
+    assert c["k_scale"][0] == s
+    deq = c.dequantize(0, 8)[:, :, :6]
+    # E4M3 relative step is 2^-3: nearest-value error <= 2^-4 relative (normal range)
+    err = np.abs(deq - x)
+    bound = np.maximum(np.abs(x) * 2.0**-4, float(s) * 2.0**-10) * (1 + 2**-20)
+    assert np.all(err <= bound)
+    assert np.abs(deq).max() == np.abs(x).max()  # the absmax element maps to 448 exactly
+
+
+# --------------------------------------------------------------- asymmetric uint8
+def test_asym_affine_roundtrip_and_bounds():
+    s_pow2 = 2.0**-4
+    mn, mx = -100 * s_pow2, 155 * s_pow2
+    s, zp = oracle.asym_params(mn, mx)
+    assert s == F32(mx - mn) / F32(255) and zp == 100
+    for k in range(256):
+        x = (k - zp) * float(s)
+        q = oracle.asym_code(x, s, zp)
+        assert q == k and (q - zp) * s == F32(x)
+    rng = np.random.default_rng(5)
+    x = rng.normal(0.3, 2.0, 3000).astype(np.float32)
+    s, zp = oracle.asym_params(float(x.min()), float(x.max()))
+    for v in x:
+        q = oracle.asym_code(float(v), s, zp)
+        err = abs(float(F32(q - zp) * F32(s)) - float(v))
+        assert err <= float(s) * (1 + 2**-20)  # <= s/2 inside, <= s at a clamped edge
+
+
+def test_asym_range_without_zero_is_widened():
+    # The page's literal form (zp clamped to 0, codes from (x - min)/s, dequant
+    # (q - zp) * s) decodes the range [1, 2] onto [0, 1]; the affine reading keeps it.
+    s, zp = oracle.asym_params(1.0, 2.0)
+    assert zp == 0 and s == F32(2.0) / F32(255)
+    for v in (1.0, 1.5, 2.0):
+        q = oracle.asym_code(v, s, zp)
+        assert abs(float(F32(q) * F32(s)) - v) <= float(s) / 2 * (1 + 2**-20)
+
+
+def test_per_channel_asym_calibration_axis():
+    # One (scale, zp) per (kv_head, channel), reduced over batch rows and tokens.
+    B, H, T, D = 3, 2, 4, 8
+    rng = np.random.default_rng(9)
+    x = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    c = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    for h in range(H):
+        for d in range(D):
+            col = x[:, h, :, d]
+            s, zp = oracle.asym_params(float(col.min()), float(col.max()))
+            assert c["v_scale"][h, d] == s and c["v_zp"][h, d] == zp
+
+
+# --------------------------------------------------------------- KIVI
+@pytest.mark.parametrize("bits", [4, 2])
+def test_kivi_group_extremes_and_nearest_level(bits):
+    qmax = 2**bits - 1
+    rng = np.random.default_rng(bits)
+    for _ in range(200):
+        x = rng.normal(0, 1, 32).astype(np.float32)
+        codes, s, mn = oracle.kivi_group(x, bits)
+        assert mn == x.min() and s == F32(F32(x.max()) - F32(x.min())) / F32(qmax)
+        assert codes[np.argmin(x)] == 0 and codes[np.argmax(x)] == qmax
+        for xi, qi in zip(x, codes):
+            levels = [oracle.kivi_value(k, s, mn) for k in range(qmax + 1)]
+            dists = [abs(float(L) - float(xi)) for L in levels]
+            # the chosen level is a nearest one (brute force over all 2^bits codes)
+            assert dists[qi] <= min(dists) + float(s) * 2**-20
+            assert dists[qi] <= float(s) / 2 * (1 + 2**-22) + abs(float(mn)) * 2**-23
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_kivi_exact_grid_and_zero_range(bits):
+    qmax = 2**bits - 1
+    s, mn = 2.0**-3, -1.5
+    ks = np.arange(32) % (qmax + 1)
+    ks[0], ks[1] = 0, qmax
+    x = (mn + ks * s).astype(np.float32)
+    codes, s_o, mn_o = oracle.kivi_group(x, bits)
+    assert s_o == s and mn_o == mn and list(codes) == list(ks)
+    for k in range(qmax + 1):
+        assert oracle.kivi_value(k, s_o, mn_o) == F32(mn + k * s)
+    z = np.full(32, 0.75, np.float32)
+    codes, s_o, mn_o = oracle.kivi_group(z, bits)
+    assert s_o == 0 and mn_o == F32(0.75) and not codes.any()
+    neg0 = np.array([-0.0] * 32, np.float32)
+    _, s_o, mn_o = oracle.kivi_group(neg0, bits)
+    assert not np.signbit(mn_o) and not np.signbit(s_o)
+
+
+def _kivi_cache(B, H, D, cap, bits, group=32, rcap=128):
+    sch = oracle.KIVI_INT4 if bits == 4 else oracle.KIVI_INT2
+    return OracleCache(B, H, H, D, sch, sch, cap=cap, group=group, rcap=rcap)
+
+
+def _bf16(a):
+    return (np.ascontiguousarray(a, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def test_kivi_residual_page_example():
+    # "Quantized KV: [tokens 1-64 in INT4] + [tokens 65-128 in INT4] + ...
+    #  Residual: [tokens 193-200 in BF16]" with groups of 64 tokens.
+    rng = np.random.default_rng(4)
+    x = _bf16(rng.normal(0, 1, (1, 1, 200, 128)))
+    c = _kivi_cache(1, 1, 128, 256, 4, group=64, rcap=64)
+    c.append(x, x, bf16=True)
+    assert (c.length, c.residual) == (192, 8)
+    assert np.array_equal(c["k_res"][0, 0, :8], x[0, 0, 192:200])
+
+
+@pytest.mark.parametrize("n", [1, 127, 128, 129, 256, 257, 300])
+def test_kivi_bulk_equals_streaming(n):
+    rng = np.random.default_rng(n)
+    k = _bf16(rng.normal(0, 1, (2, 2, n, 64)))
+    v = _bf16(rng.normal(0, 1, (2, 2, n, 64)))
+    a = _kivi_cache(2, 2, 64, 512, 2)
+    a.append(k, v, bf16=True)
+    b = _kivi_cache(2, 2, 64, 512, 2)
+    for t in range(n):
+        b.append(k[:, :, t:t + 1], v[:, :, t:t + 1], bf16=True)
+    assert a.length == b.length == 128 * ((n - 1) // 128)
+    assert a.residual == b.residual == n - a.length
+    for name in ("k_codes", "v_codes", "k_scale", "k_zero", "v_scale", "v_zero"):
+        assert np.array_equal(a[name], b[name]), name
+    for name in ("k_res", "v_res"):  # only the first `residual` slots are state
+        assert np.array_equal(a[name][:, :, :a.residual], b[name][:, :, :b.residual]), name
+
+
+def test_kivi_axes_key_per_channel_value_per_token():
+    # Keys: one (scale, min) per channel per 32-token group; values: one per token per
+    # 32-channel group. A key outlier channel must not change other channels' scales;
+    # a large value token must not change other tokens' scales.
+    rng = np.random.default_rng(8)
+    k = rng.normal(0, 1, (1, 1, 129, 64)).astype(np.float32)
+    v = rng.normal(0, 1, (1, 1, 129, 64)).astype(np.float32)
+    k2, v2 = k.copy(), v.copy()
+    k2[0, 0, :, 5] *= 100.0
+    v2[0, 0, 17, :] *= 100.0
+    outs = []
+    for kk, vv in ((k, v), (k2, v2)):
+        c = _kivi_cache(1, 1, 64, 256, 4)
+        c.append(_bf16(kk), _bf16(vv), bf16=True)
+        outs.append(c)
+    a, b = outs
+    diff_k = (a["k_scale"] != b["k_scale"])[:, :, :4]  # [1,1,groups,D]; 128 tokens flushed
+    assert diff_k[0, 0, :, 5].all() and not np.delete(diff_k[0, 0], 5, axis=1).any()
+    diff_v = a["v_scale"] != b["v_scale"]          # [1,1,T,D/32]
+    assert diff_v[0, 0, 17].all() and not np.delete(diff_v[0, 0], 17, axis=0).any()
+    # the scale of channel d in group gi is (max - min)/15 of that column slice
+    xk = _bf16(k).astype(np.uint32) << 16
+    col = xk.view(np.float32)[0, 0, 32:64, 9]
+    assert a["k_scale"][0, 0, 1, 9] == F32(F32(col.max()) - F32(col.min())) / F32(15)
+
+
+def test_kivi_packing_low_index_low_bits():
+    x = np.zeros((1, 1, 129, 64), np.float32)
+    ramp = np.arange(32) % 4
+    x[0, 0, 0, :32] = ramp           # value token 0, channel group 0: codes 0,1,2,3,0,1,...
+    c = _kivi_cache(1, 1, 64, 256, 2)
+    c.append(_bf16(x), _bf16(x), bf16=True)
+    row = c["v_codes"][0, 0, 0]
+    assert row[0] == (0 | 1 << 2 | 2 << 4 | 3 << 6)
+
+
+# --------------------------------------------------------------- attention (fp64)
+def _attn(q, k, v, scale):
+    return oracle.attention_row(np.asarray(q, np.float32), np.asarray(k, np.float32),
+                                np.asarray(v, np.float32), scale)
+
+
+def test_attention_closed_forms():
+    rng = np.random.default_rng(0)
+    D = 16
+    q = rng.normal(0, 1, D).astype(np.float32)
+    k = rng.normal(0, 1, (5, D)).astype(np.float32)
+    v = rng.normal(0, 1, (5, D)).astype(np.float32)
+    out, lse = _attn(q, k[:1], v[:1], 0.3)
+    assert np.array_equal(out, v[0].astype(np.float64))      # T = 1 -> that value row
+    out, _ = _attn(np.zeros(D), k, v, 0.3)
+    assert np.allclose(out, v.astype(np.float64).mean(0), rtol=0, atol=1e-15)  # q = 0 -> mean
+    kk = np.repeat(k[:1], 5, 0)
+    out, lse = _attn(q, kk, v, 0.3)
+    assert np.allclose(out, v.astype(np.float64).mean(0), rtol=0, atol=1e-15)  # equal keys
+    s0 = float(np.dot(q.astype(np.float64), kk[0].astype(np.float64))) * np.float64(F32(0.3))
+    assert abs(lse - (s0 + math.log(5))) < 1e-12
+    # one score larger by >= 800 -> exactly that value row (exp(-800) underflows)
+    k3 = np.zeros((4, D), np.float32)
+    q3 = np.zeros(D, np.float32)
+    q3[0] = 1.0
+    k3[2, 0] = 1000.0
+    out, _ = _attn(q3, k3, v[:4], 1.0)
+    assert np.array_equal(out, v[2].astype(np.float64))
+
+
+def test_attention_shift_invariance_and_empty():
+    rng = np.random.default_rng(1)
+    D = 8
+    q = np.zeros(D, np.float32)
+    q[0] = 2.0
+    k = (np.round(rng.normal(0, 1, (6, D)) * 1024) / 1024).astype(np.float32)  # k + 3 is exact
+    v = rng.normal(0, 1, (6, D)).astype(np.float32)
+    a, la = _attn(q, k, v, 0.5)
+    k2 = k.copy()
+    k2[:, 0] += 3.0  # adds 2 * 3 * 0.5 = 3 to every score exactly
+    b, lb = _attn(q, k2, v, 0.5)
+    assert np.allclose(a, b, rtol=0, atol=1e-13) and abs((lb - la) - 3.0) < 1e-12
+    out, lse = _attn(q, np.zeros((0, D)), np.zeros((0, D)), 0.5)
+    assert not out.any() and lse == -math.inf
+
+
+def test_attention_against_high_precision_brute_force():
+    decimal.getcontext().prec = 50
+    rng = np.random.default_rng(2)
+    for T in (1, 3, 17, 64):
+        D = 8
+        q = rng.normal(0, 1, D).astype(np.float32)
+        k = (rng.normal(0, 3, (T, D))).astype(np.float32)
+        v = rng.normal(0, 1, (T, D)).astype(np.float32)
+        scale = F32(1 / math.sqrt(D))
+        out, lse = _attn(q, k, v, float(scale))
+        Dd = decimal.Decimal
+        s = [sum(Dd(float(q[d])) * Dd(float(k[t, d])) for d in range(D)) * Dd(float(scale)) for t in range(T)]
+        m = max(s)
+        p = [(x - m).exp() for x in s]
+        l = sum(p)
+        ref = [float(sum(p[t] * Dd(float(v[t, d])) for t in range(T)) / l) for d in range(D)]
+        assert np.allclose(out, ref, rtol=1e-13, atol=1e-13)
+        assert abs(lse - float(m + l.ln())) < 1e-12
+
+
+def test_attention_split_merge_equals_whole():
+    # LSE merge of any split of the token axis equals attention over all tokens.
+    rng = np.random.default_rng(3)
+    D, T = 16, 40
+    q = rng.normal(0, 1, D).astype(np.float32)
+    k = rng.normal(0, 2, (T, D)).astype(np.float32)
+    v = rng.normal(0, 1, (T, D)).astype(np.float32)
+    whole, lw = _attn(q, k, v, 0.25)
+    for cuts in ([13], [1, 2, 39], [10, 20, 30]):
+        bounds = [0, *cuts, T]
+        parts = [_attn(q, k[a:b], v[a:b], 0.25) for a, b in zip(bounds, bounds[1:])]
+        M = max(l for _, l in parts)
+        w = [math.exp(l - M) for _, l in parts]
+        merged = sum(wi * o for wi, (o, _) in zip(w, parts)) / sum(w)
+        assert np.allclose(merged, whole, rtol=1e-13, atol=1e-13)
+        assert abs(M + math.log(sum(w)) - lw) < 1e-12
+
+
+# --------------------------------------------------------------- cache plumbing
+def test_paged_gather_matches_dense():
+    rng = np.random.default_rng(6)
+    B, H, D, ps = 3, 2, 16, 4
+    lens = np.array([5, 9, 1], np.int32)
+    maxp = 4
+    perm = rng.permutation(12).astype(np.int32)
+    table = perm.reshape(B, maxp)
+    n = int(lens.max())
+    k = rng.normal(0, 1, (B, H, n, D)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, n, D)).astype(np.float32)
+    pg = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL,
+                     paged=True, page_size=ps, max_pages=maxp, num_pages=12, page_table=table)
+    pg.append(k, v, bf16=False, calibrate=True, new_lens=lens)
+    assert list(pg["seq_lens"]) == list(lens)
+    for b in range(B):
+        dn = OracleCache(1, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, cap=16)
+        dn["k_scale"][:] = pg["k_scale"]
+        dn["v_scale"][:] = pg["v_scale"]
+        dn["v_zp"][:] = pg["v_zp"]
+        dn.append(k[b:b + 1, :, :lens[b]], v[b:b + 1, :, :lens[b]], bf16=False)
+        for t in range(lens[b]):
+            page, slot = table[b, t // ps], t % ps
+            assert np.array_equal(pg["k_codes"][page, :, slot], dn["k_codes"][0, :, t])
+            assert np.array_equal(pg["v_codes"][page, :, slot], dn["v_codes"][0, :, t])
+        a = pg.dequantize(1, 12)[b, :, :lens[b]]
+        assert np.array_equal(a, dn.dequantize(1, 12)[0, :, :lens[b]])
+
+
+def test_gqa_head_mapping_and_decode():
+    # Query head h reads kv head h // G: with G = 2, heads 0,1 -> kv 0 and 2,3 -> kv 1.
+    rng = np.random.default_rng(12)
+    B, Hq, H, D, T = 1, 4, 2, 8, 6
+    k = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    c = OracleCache(B, Hq, H, D, oracle.INT8_SYM_PER_TOKEN, oracle.INT8_SYM_PER_TOKEN, cap=8)
+    c.append(k, v, bf16=False)
+    q = rng.normal(0, 1, (B, Hq, D)).astype(np.float32)
+    out, lse = c.decode(q, bf16=False, scale=0.35)
+    K, V = c.dequantize(0, T), c.dequantize(1, T)
+    for h in range(Hq):
+        ref, lr = _attn(q[0, h], K[0, h // 2], V[0, h // 2], 0.35)
+        assert np.array_equal(out[0, h], ref) and lse[0, h] == lr
+
+
+def test_capacity_errors():
+    c = OracleCache(1, 1, 1, 8, oracle.INT8_SYM_PER_TOKEN, oracle.INT8_SYM_PER_TOKEN, cap=4)
+    x = np.zeros((1, 1, 5, 8), np.float32)
+    with pytest.raises(ValueError):
+        c.append(x, x, bf16=False)
