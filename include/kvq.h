@@ -1,0 +1,195 @@
+/*
+ * libkvq: KV-cache quantize-on-append and decode attention over the quantized cache,
+ * for NVIDIA B200 (sm_100a). C ABI; every pointer named "device" is CUDA device memory
+ * owned by the caller. The library allocates nothing.
+ *
+ * Problem statement ("How KV cache quantization reduces GPU memory", n4n.ai, Step 1):
+ * the cache holds K and V per layer, each [batch, num_heads, seq_len, head_dim]; here
+ * num_heads are the KV heads and one descriptor describes one layer.
+ *
+ * Conventions for every entry point:
+ *  - Asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default).
+ *  - Argument errors return synchronously, before any launch, and change nothing.
+ *  - A launch failure returns KVQ_ERR_CUDA.
+ *  - Faults the device detects (a page id outside the pool, a length outside the page
+ *    table, a wait that ran out of time) set bits in the device status word
+ *    (desc->dev_status[0]); the kernel skips the affected work and never traps. Read the
+ *    word with kvq_get_device_status.
+ *  - Codes, scales and zero points are bit-exact functions of the inputs (IEEE fp32
+ *    division, round-half-to-even); attention outputs are fp32.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_ABI_VERSION 1
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, bad enum value */
+  KVQ_ERR_UNSUPPORTED = 2,   /* valid but not implemented (scheme pair, dtype, head_dim) */
+  KVQ_ERR_CAPACITY = 3,      /* the append does not fit the dense capacity */
+  KVQ_ERR_WORKSPACE = 4,     /* workspace null or smaller than the query says */
+  KVQ_ERR_CUDA = 5           /* a CUDA call or launch failed */
+} kvq_status;
+
+/* Quantization schemes, chosen separately for K and for V.
+ *  FP8_E4M3_PER_TENSOR  OCP E4M3 codes of x/s, s = absmax/448 over the calibrating append
+ *                       ("KV Cache Quantization", infra.bea.ai, §4; llms.blog §1).
+ *  INT8_SYM_PER_TENSOR  clamp(rne(x/s), -127, 127), s = absmax/127 over the calibrating
+ *                       append (n4n.ai Step 2-3; llms.blog §2).
+ *  INT8_SYM_PER_TOKEN   same, one s per (batch, kv_head, token) row (llms.blog §2).
+ *  INT8_SYM_PER_CHANNEL same, one s per (kv_head, channel) (infra.bea.ai §3 Key example).
+ *  UINT8_ASYM_PER_CHANNEL  clamp(rne(x/s) + zp, 0, 255), s = (max(mx,0) - min(mn,0))/255,
+ *                       zp = clamp(rne(-min(mn,0)/s), 0, 255) per (kv_head, channel)
+ *                       (n4n.ai Step 2 "per-channel asymmetric INT8").
+ *  KIVI_INT4 / KIVI_INT2  KIVI (infra.bea.ai §3, llms.blog §3): keys per channel over
+ *                       groups of 32 tokens, values per token over groups of 32 channels,
+ *                       s = (max - min)/(2^bits - 1), q = clamp(rne((x - min)/s)), fp32
+ *                       scale and minimum, codes packed along head_dim (lower channel in
+ *                       lower bits), recent tokens in a bf16 residual of 128 tokens.
+ * A zero range gives s = 0 and code 0. */
+typedef enum kvq_scheme {
+  KVQ_FP8_E4M3_PER_TENSOR = 0,
+  KVQ_INT8_SYM_PER_TENSOR = 1,
+  KVQ_INT8_SYM_PER_TOKEN = 2,
+  KVQ_INT8_SYM_PER_CHANNEL = 3,
+  KVQ_UINT8_ASYM_PER_CHANNEL = 4,
+  KVQ_KIVI_INT4 = 5,
+  KVQ_KIVI_INT2 = 6
+} kvq_scheme;
+
+typedef enum kvq_dtype { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
+typedef enum kvq_layout { KVQ_DENSE = 0, KVQ_PAGED = 1 } kvq_layout;
+
+/* kvq_quantize_append flags */
+#define KVQ_APPEND_CALIBRATE 0x1u  /* recompute per-tensor / per-channel scales from this block */
+
+/* device status word bits (dev_status[0]); dev_status[1] counts saturated codes */
+#define KVQ_DEV_BAD_PAGE 0x1u
+#define KVQ_DEV_BAD_LENGTH 0x2u
+#define KVQ_DEV_TIMEOUT 0x4u
+
+/*
+ * One layer's cache. Shapes (all device memory, contiguous, caller-owned):
+ *   row_bytes(scheme) = head_dim (8-bit), head_dim/2 (KIVI_INT4), head_dim/4 (KIVI_INT2)
+ *   dense codes  [batch, kv_heads, capacity, row_bytes]
+ *   paged codes  [num_pages, kv_heads, page_size, row_bytes]
+ *   per-tensor scale            float [1]
+ *   per-token scale             float [batch, kv_heads, capacity]  (paged: [num_pages, kv_heads, page_size])
+ *   per-channel scale           float [kv_heads, head_dim]; uint8 zero point (k_zp/v_zp) same shape
+ *   KIVI key scale and minimum  float [batch, kv_heads, capacity/32, head_dim] (k_scale, k_zero)
+ *   KIVI value scale and minimum float [batch, kv_heads, capacity, head_dim/32] (v_scale, v_zero)
+ *   KIVI residual               bf16  [batch, kv_heads, residual_cap, head_dim] (k_res, v_res)
+ *   paged page_table            int32 [batch, max_pages_per_seq]; seq_lens int32 [batch]
+ *   dev_status                  uint32 [2]
+ * Unused pointers may be NULL.
+ */
+typedef struct kvq_cache_desc {
+  int32_t batch, num_q_heads, num_kv_heads, head_dim;  /* head_dim must be 128 */
+  int32_t k_scheme, v_scheme;                          /* kvq_scheme */
+  int32_t layout;                                      /* kvq_layout */
+  int32_t capacity;          /* dense: tokens per (batch, kv_head); multiple of 128 */
+  int32_t page_size;         /* paged: 16, 32 or 64 tokens */
+  int32_t max_pages_per_seq, num_pages;
+  int32_t group_size;        /* KIVI: 32 */
+  int32_t residual_cap;      /* KIVI: 128 */
+  int32_t num_quantized;     /* dense: quantized tokens per row (library-maintained) */
+  int32_t num_residual;      /* KIVI: tokens in the bf16 residual (library-maintained) */
+  void* k_codes;
+  void* v_codes;
+  float* k_scale;
+  float* k_zero;
+  float* v_scale;
+  float* v_zero;
+  uint8_t* k_zp;
+  uint8_t* v_zp;
+  uint16_t* k_res;
+  uint16_t* v_res;
+  int32_t* page_table;
+  int32_t* seq_lens;
+  uint32_t* dev_status;
+} kvq_cache_desc;
+
+typedef struct kvq_footprint {
+  uint64_t code_bytes;       /* K and V codes at capacity */
+  uint64_t meta_bytes;       /* scales, minima and zero points */
+  uint64_t residual_bytes;   /* KIVI bf16 residual */
+  uint64_t total_bytes;
+  double bytes_per_token;    /* codes + per-token share of metadata + residual, per kv_head row pair */
+} kvq_footprint;
+
+int kvq_abi_version(void);
+const char* kvq_status_string(kvq_status s);
+
+/* Check a descriptor's fields (shapes, enums, pointer presence). No device access. */
+kvq_status kvq_validate(const kvq_cache_desc* desc);
+
+/* Bytes the cache arrays take (n4n.ai Step 6 "peak memory"; llms.blog memory-per-token). */
+kvq_status kvq_cache_bytes(const kvq_cache_desc* desc, kvq_footprint* out);
+
+/* Workspace kvq_quantize_append needs for `flags` (0 unless KVQ_APPEND_CALIBRATE). */
+size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t flags);
+
+/*
+ * Quantize n_new tokens per sequence and append them ("QuantizedKVCache.append",
+ * n4n.ai Step 3; KIVI residual policy, infra.bea.ai §3 "Residual Cache for Streaming").
+ *   k_new, v_new  device [batch, kv_heads, n_new, head_dim], in_dtype (KIVI: bf16 only)
+ *   new_lens      paged only, device int32 [batch] or NULL: per-sequence counts <= n_new
+ *   flags         KVQ_APPEND_CALIBRATE: per-tensor / per-channel scales from this block
+ *                 (otherwise the scales already in the descriptor are used; values beyond
+ *                 them saturate and are counted in dev_status[1])
+ * Dense: tokens go to positions num_quantized.. of every row; the library updates
+ * num_quantized / num_residual in *desc when the call is accepted. KIVI: tokens enter the
+ * residual; when a token arrives at a full residual, its 128 tokens are quantized.
+ * Paged: token i of sequence b goes to position seq_lens[b] + i, page
+ * page_table[b][pos / page_size], slot pos % page_size; seq_lens is advanced on the device.
+ * The caller assigns page_table entries before the call.
+ */
+kvq_status kvq_quantize_append(kvq_cache_desc* desc, const void* k_new, const void* v_new,
+                               int32_t in_dtype, int32_t n_new, const int32_t* new_lens,
+                               uint32_t flags, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * Dequantize K (which = 0) or V (which = 1) into device fp32 out [batch, kv_heads,
+ * out_tokens, head_dim] ("QuantizedKVCache.dequantize / get", n4n.ai Step 3). Token
+ * order: quantized tokens, then the KIVI residual. Rows at or past a sequence's length
+ * are written as zero. out_tokens must be >= every sequence's length.
+ */
+kvq_status kvq_dequantize(const kvq_cache_desc* desc, int32_t which, float* out,
+                          int32_t out_tokens, void* stream);
+
+/* Workspace kvq_decode_attention needs (split partials and the paged plan). */
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc);
+
+/*
+ * Decode attention of one query token per sequence over the quantized cache, reading the
+ * codes directly (llms.blog, section "Serving Economics and Latency Trade-Offs": decode is bound by
+ * memory bandwidth; guide.dupenodi.dev "KV cache quantization": the savings only count
+ * when the attention kernel consumes the low-precision cache itself).
+ *   q         device [batch, num_q_heads, head_dim], q_dtype (bf16 or fp32)
+ *   out       device fp32 [batch, num_q_heads, head_dim]
+ *   lse       device fp32 [batch, num_q_heads] or NULL: natural-log sum of exp of scores
+ * Query head h reads kv head h / (num_q_heads / num_kv_heads). Scores are
+ * softmax_scale * q.k over all tokens of the sequence (no mask). A sequence with no
+ * tokens gives zeros and lse = -inf.
+ */
+kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* q, int32_t q_dtype,
+                                float softmax_scale, float* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/* Copy dev_status[0..1] to host out[2] (synchronises `stream`); clear != 0 zeroes them. */
+kvq_status kvq_get_device_status(const kvq_cache_desc* desc, uint32_t* out, int32_t clear,
+                                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -41,8 +41,8 @@ uint16_t oq_f32_to_bf16(float f) {
   return (uint16_t)(u >> 16);
 }
 
-/* OCP 8-bit floating point, E4M3 ("FP8 E4M3: 1 sign bit, 4 exponent bits, 3 mantissa
- * bits", P3 §1): exponent bias 7, no infinities, S.1111.111 is NaN, largest finite
+/* OCP 8-bit floating point E4M3 (P3 §1 names it: sign, 4 exponent and 3 mantissa
+ * bits): exponent bias 7, no infinities, S.1111.111 is NaN, largest finite
  * value 1.75 * 2^8 = 448, subnormals M/8 * 2^-6. */
 float oq_e4m3_decode(uint8_t code) {
   int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
@@ -79,8 +79,8 @@ uint8_t oq_e4m3_encode(float x) {
   return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | ((int)m - 8)));
 }
 
-/* Symmetric code: clamp(rne(x / s), -qmax, qmax) (P4 Step 3 `(x / scale).round()`,
- * clamp range from P3 §2 "maps values to [-127, 127]"). */
+/* Symmetric code: clamp(rne(x / s), -qmax, qmax) (P4 Step 3 divides by the scale and
+ * rounds; P3 §2 gives the symmetric INT8 range as -127..127). */
 int oq_sym_code(float x, float s, int qmax) {
   if (s == 0.0f) return 0;
   float y = x / s;
@@ -225,7 +225,8 @@ static float block_at(const block* k, int b, int h, int t, int d) {
 }
 
 /* Fixed scales of the per-tensor and per-channel schemes, from the tokens of the
- * calibrating append (runtime statistics, P1 §2 "Must use runtime statistics").
+ * calibrating append: the cache is built online, so its scales come from runtime
+ * statistics of the data (P1 §2, weights-vs-KV comparison table).
  * Per-tensor: one scale over every batch row, head, token and channel (P4 Step 3
  * `x.abs().max() / 127`). Per-channel: one per (kv_head, channel) over batch and
  * tokens (P4 Step 3 reduces V over batch and sequence per channel). */
@@ -565,8 +566,8 @@ void oq_decode_pairs(const oq_cache* c, const void* q, int q_bf16, float scale,
                 out + (size_t)i * G * c->D, lse ? lse + (size_t)i * G : NULL);
 }
 
-/* P3: "Memory per Token = 2 x 2 x n_layers x n_kv_heads x d_head bytes" for 2-byte
- * elements; generalised to any element width. */
+/* P3 introduction: per-token KV bytes are K and V (2) times the element width times
+ * layers, KV heads and head dimension; the page states it for 2-byte elements. */
 double oq_kv_bytes_per_token(int n_layers, int n_kv_heads, int d_head, double bytes_per_elem) {
   return 2.0 * bytes_per_elem * (double)n_layers * (double)n_kv_heads * (double)d_head;
 }

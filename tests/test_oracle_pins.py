@@ -299,8 +299,8 @@ def _bf16(a):
 
 
 def test_kivi_residual_page_example():
-    # "Quantized KV: [tokens 1-64 in INT4] + [tokens 65-128 in INT4] + ...
-    #  Residual: [tokens 193-200 in BF16]" with groups of 64 tokens.
+    # The page's streaming example: with groups of 64 tokens, 200 tokens leave tokens
+    # 1..192 quantized (three groups) and tokens 193..200 in the bf16 residual.
     rng = np.random.default_rng(4)
     x = _bf16(rng.normal(0, 1, (1, 1, 200, 128)))
     c = _kivi_cache(1, 1, 128, 256, 4, group=64, rcap=64)
