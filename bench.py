@@ -1,0 +1,587 @@
+"""Benchmark: decode-attention KV GB/s (% of B200 HBM peak) and tokens/s per KV dtype.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the hot path over one batch: quantize-append of one new token per
+sequence, then split-KV decode attention (+ log-sum-exp merge) over the whole cache. The
+default workload is the Llama-3-8B-shaped FP8 E4M3 layer (batch 32, 32/8 heads, context
+4096). Inputs are seeded synthetic tensors resident in HBM; the step is captured once in a
+CUDA graph and replayed; L2 is flushed (256 MiB write) before every timed step and the
+flush is outside the step's CUDA-event interval. `value` is the step's algorithmic bytes
+(codes + scales + residual + Q + out for decode, new K/V in + codes out for the append)
+divided by the step time, summed over all ranks (weak scaling: one full workload per GPU).
+`--impl reference` times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "decode-attn KV GB/s (% of B200 HBM peak) and tokens/s, per KV dtype"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+DTYPE_NAME = {synth.FP8_E4M3_PER_TENSOR: "fp8_e4m3", synth.INT8_SYM_PER_TENSOR: "int8",
+              synth.INT8_SYM_PER_TOKEN: "int8", synth.INT8_SYM_PER_CHANNEL: "int8",
+              synth.UINT8_ASYM_PER_CHANNEL: "uint8", synth.KIVI_INT4: "int4", synth.KIVI_INT2: "int2"}
+CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
+              synth.UINT8_ASYM_PER_CHANNEL)
+KERNEL_SOURCES = ["decode_attention_quantize_b200/csrc/kvq_decode.cu",
+                  "decode_attention_quantize_b200/csrc/kvq_device.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="fp8_8b", choices=list(synth.workloads()))
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+def row_bytes(scheme):
+    return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2}.get(scheme, 8) // 8
+
+
+def meta_bytes_per_token(scheme, Hkv):
+    """Per-token-row metadata bytes that decode must read (K or V side)."""
+    if scheme == synth.INT8_SYM_PER_TOKEN:
+        return 4.0
+    if scheme in (synth.KIVI_INT4, synth.KIVI_INT2):
+        return 8.0 * 128 / 32  # fp32 (scale, min) per 32 elements
+    return 0.0
+
+
+def fixed_meta_bytes(scheme, Hkv):
+    if scheme in (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
+        return 4
+    if scheme == synth.INT8_SYM_PER_CHANNEL:
+        return Hkv * 128 * 4
+    if scheme == synth.UINT8_ASYM_PER_CHANNEL:
+        return Hkv * 128 * 5
+    return 0
+
+
+def decode_bytes(w, lens_q, len_res=0):
+    """Algorithmic bytes of one decode call: codes + metadata + residual + Q + out."""
+    rows = int(np.sum(lens_q)) * w.Hkv
+    b = rows * (row_bytes(w.k_scheme) + row_bytes(w.v_scheme))
+    b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv) + meta_bytes_per_token(w.v_scheme, w.Hkv))
+    b += fixed_meta_bytes(w.k_scheme, w.Hkv) + fixed_meta_bytes(w.v_scheme, w.Hkv)
+    b += w.B * w.Hkv * len_res * 128 * 2 * 2
+    b += w.B * w.Hq * 128 * (2 if w.bf16 else 4)  # Q
+    b += w.B * w.Hq * 128 * 4                       # out (fp32)
+    return float(b)
+
+
+def append_bytes(w, n=1):
+    """One token per sequence: read bf16/fp32 K and V, write codes (+ per-token scales)."""
+    rows = w.B * w.Hkv * n
+    elem = 2 if w.bf16 else 4
+    b = rows * 128 * elem * 2
+    if w.kivi:
+        b += rows * 128 * 2 * 2  # bf16 residual write
+    else:
+        b += rows * (row_bytes(w.k_scheme) + row_bytes(w.v_scheme))
+        b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv) + meta_bytes_per_token(w.v_scheme, w.Hkv))
+    return float(b)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            v = float(json.load(fh)["hbm_gbs"])
+            return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(workload):
+    """DRAM bytes per decode launch from the committed ncu capture, if the kernel source is
+    unchanged since the capture; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    h = hashlib.sha256()
+    for src in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, src), "rb").read())
+    if rec.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    return rec.get("dram_bytes_per_launch_full")
+
+
+# ---------------------------------------------------------------- clocks (NVML, read-only)
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8): "hw_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20): "sw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40): "hw_thermal_slowdown",
+            getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4): "sw_power_cap",
+            getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80): "hw_power_brake_slowdown",
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in names.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml" if self.nv else "unavailable"}
+
+
+# ---------------------------------------------------------------- GPU workload
+class GpuWorkload:
+    """Builds one layer's cache for a workload and exposes a graph-captured decode step."""
+
+    def __init__(self, w, rank, device):
+        import torch
+        from decode_attention_quantize_b200 import kvq
+        self.torch, self.kvq, self.w, self.dev = torch, kvq, w, device
+        self.seed_w = synth.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+        W = self.seed_w
+        if W.paged:
+            self._build_paged(W)
+        else:
+            self._build_dense(W)
+        torch.cuda.synchronize()
+
+    def _dev(self, a, bf16):
+        t = self.torch.from_numpy(np.ascontiguousarray(a)).to(self.dev)
+        return t.view(self.torch.bfloat16) if bf16 else t
+
+    def _build_dense(self, W):
+        kvq = self.kvq
+        total = W.prefill_tokens()
+        self.append_token = W.name != "tiny_int8"  # the tiny configuration decodes without appending
+        pre = total - 1 if self.append_token else total
+        cap = (total + 127) // 128 * 128
+        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap)
+        self.cache = kvq.QuantizedKVCache(spec, device=self.dev)
+        calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
+        chunk = max(1, (1 << 27) // (W.Hkv * 128 * W.B))  # generate ~256 MB of bf16 at a time
+        first = True
+        for t0 in range(0, pre, chunk if not calib else pre):
+            t1 = min(pre, t0 + (chunk if not calib else pre))
+            k = synth.keys(W, 0, W.B, 0, W.Hkv, t0, t1)
+            v = synth.values(W, 0, W.B, 0, W.Hkv, t0, t1)
+            self.cache.append(self._dev(k, W.bf16), self._dev(v, W.bf16), calibrate=calib and first)
+            first = False
+        self.torch.cuda.synchronize()
+        self.pre = pre
+        d = self.cache.desc
+        self.saved = (d.num_quantized, d.num_residual)
+        self.k_new = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, pre, pre + 1), W.bf16)
+        self.v_new = self._dev(synth.values(W, 0, W.B, 0, W.Hkv, pre, pre + 1), W.bf16)
+        self.len_q_decode = d.num_quantized if not W.kivi else None
+        self._common(W)
+
+    def _build_paged(self, W):
+        kvq, torch = self.kvq, self.torch
+        lens = W.prefill_lengths()
+        extra = 4096
+        need = [(int(L) + extra + W.page_size - 1) // W.page_size for L in lens]
+        max_pages = max(need)
+        num_pages = int(sum(need))
+        perm = synth.permutation(W.seed, num_pages)
+        table = np.full((W.B, max_pages), -1, np.int32)
+        off = 0
+        for b, n in enumerate(need):
+            table[b, :n] = perm[off:off + n]
+            off += n
+        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, paged=True, page_size=W.page_size,
+                             max_pages=max_pages, num_pages=num_pages)
+        self.cache = kvq.QuantizedKVCache(spec, device=self.dev, page_table=torch.from_numpy(table))
+        n_max = int(lens.max())
+        K = torch.zeros((W.B, W.Hkv, n_max, 128), dtype=torch.bfloat16, device=self.dev)
+        V = torch.zeros_like(K)
+        for b in range(W.B):
+            L = int(lens[b])
+            K[b, :, :L] = self._dev(synth.keys(W, b, b + 1, 0, W.Hkv, 0, L)[0], True)
+            V[b, :, :L] = self._dev(synth.values(W, b, b + 1, 0, W.Hkv, 0, L)[0], True)
+        self.cache.append(K, V, new_lens=torch.from_numpy(lens).to(self.dev), calibrate=True)
+        del K, V
+        torch.cuda.synchronize()
+        self.lens = lens
+        self.append_token = True
+        self.extra = extra
+        # step tokens: generated per step index from the same generator (positions L_b + s)
+        self.k_steps, self.v_steps = [], []
+        self._common(W)
+
+    def _common(self, W):
+        torch, kvq = self.torch, self.kvq
+        self.q_host = [synth.queries(W, s, 0, W.B) for s in range(2)]
+        self.q = self._dev(self.q_host[0], W.bf16)
+        self.out = torch.empty((W.B, W.Hq, 128), dtype=torch.float32, device=self.dev)
+        self.ws = torch.empty(kvq.kvq_decode_workspace_bytes(self.cache.desc), dtype=torch.uint8, device=self.dev)
+        self.scale = 1.0 / math.sqrt(128.0)
+
+    def paged_token(self, step):
+        W = self.seed_w
+        k = np.stack([synth.keys(W, b, b + 1, 0, W.Hkv, int(self.lens[b]) + step, int(self.lens[b]) + step + 1)[0]
+                      for b in range(W.B)])
+        v = np.stack([synth.values(W, b, b + 1, 0, W.Hkv, int(self.lens[b]) + step, int(self.lens[b]) + step + 1)[0]
+                      for b in range(W.B)])
+        return self._dev(k, True), self._dev(v, True)
+
+    # one step (eager): append + decode
+    def step(self, stream=None, k_new=None, v_new=None, q=None):
+        d = self.cache.desc
+        if self.append_token:
+            if not self.w.paged:
+                d.num_quantized, d.num_residual = self.saved
+            self.cache.append(self.k_new if k_new is None else k_new, self.v_new if v_new is None else v_new,
+                              stream=stream)
+        self.cache.decode(self.q if q is None else q, self.scale, out=self.out, workspace=self.ws, stream=stream)
+
+    def decode_lens(self, appended):
+        """(per-sequence quantized tokens, residual tokens) seen by a decode. Dense: every step
+        sees the state after its own append (recorded after the first step). Paged: the cache
+        holds the prefill plus `appended` streamed tokens."""
+        W = self.seed_w
+        if W.paged:
+            return self.lens + appended, 0
+        nq, nr = self.after
+        return np.full(W.B, nq), (nr if W.kivi else 0)
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from decode_attention_quantize_b200 import kvq
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.workloads()[args.workload]
+    G = GpuWorkload(w, rank, dev)
+    W = G.seed_w
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # capture one step in a CUDA graph (dense: positions are reset each step, so the graph
+    # replays an identical step; paged: lengths live on the device and advance per replay)
+    graph = None
+    launches_per_replay = 0
+    if not W.paged:
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            G.step(stream)  # materialise lazy state before capture
+        torch.cuda.synchronize()
+        G.after = (G.cache.desc.num_quantized, G.cache.desc.num_residual)
+        graph = torch.cuda.CUDAGraph()
+        c0 = kvq.kvq_launch_count()
+        with torch.cuda.graph(graph, stream=stream):
+            G.step(stream)
+        launches_per_replay = kvq.kvq_launch_count() - c0  # kernels in the captured step
+        torch.cuda.synchronize()
+
+    def run_step(i):
+        if graph is not None:
+            graph.replay()
+        else:
+            k, v = G.paged_token(i)
+            with torch.cuda.stream(stream):
+                G.step(stream, k_new=k, v_new=v)
+
+    # paged: pre-generate the step tokens (host generation is outside timing)
+    if W.paged:
+        total_steps = args.warmup + args.steps
+        if total_steps + 200 > G.extra:
+            raise SystemExit("too many steps for the page pool")
+        toks = [G.paged_token(i) for i in range(total_steps)]
+
+        def run_step(i):  # noqa: F811
+            with torch.cuda.stream(stream):
+                G.step(stream, k_new=toks[i][0], v_new=toks[i][1])
+
+    for i in range(args.warmup):
+        flush.zero_()
+        run_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches0 = kvq.kvq_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(args.steps):
+            with torch.cuda.stream(stream):
+                flush.zero_()
+                ev[i][0].record(stream)
+                if graph is not None:
+                    graph.replay()
+                else:
+                    run_step(args.warmup + i)
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    launches = kvq.kvq_launch_count() - launches0
+    if graph is not None:
+        launches = args.steps * launches_per_replay
+    # decode-only timing (the dominant kernel's call: split-KV kernel + merge), eager
+    dec_ms = []
+    for i in range(min(args.steps, 400)):
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            dec_ev[i][0].record(stream)
+            G.cache.decode(G.q, G.scale, out=G.out, workspace=G.ws, stream=stream)
+            dec_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev[:min(args.steps, 400)]]
+
+    t_step = sum(step_ms) / len(step_ms) / 1e3  # seconds (mean)
+    t_dec = sum(dec_ms) / len(dec_ms) / 1e3
+    lens_q, len_res = G.decode_lens(args.warmup + args.steps // 2 + 1)
+    dbytes = decode_bytes(W, lens_q, len_res)
+    lens_d, res_d = G.decode_lens(args.warmup + args.steps)  # state seen by the decode-only timing
+    dbytes_dec = decode_bytes(W, lens_d, res_d)
+    abytes = append_bytes(W) if G.append_token else 0.0
+    total_time = torch.tensor([sum(step_ms) / 1e3], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(total_time, op=dist.ReduceOp.MAX)
+    t_max = float(total_time.item()) / args.steps
+
+    # end to end through the public API: host inputs (pinned) -> device -> step -> host out
+    e2e = run_e2e(G, W, stream, flush, n=min(200, args.steps), step0=args.warmup + args.steps)
+    status = G.cache.status()
+    return dict(t_step=t_step, t_max=t_max, t_dec=t_dec, dbytes=dbytes, dbytes_dec=dbytes_dec, abytes=abytes,
+                launches=launches,
+                clocks=sampler.summary(), e2e=e2e, status=status, W=W, G=G)
+
+
+def run_e2e(G, W, stream, flush, n, step0):
+    """Same step through the public API with host buffers: pinned host K/V token and Q copied
+    in, append + decode, output copied back; all inside the event interval."""
+    import torch
+    torch_dt = torch.bfloat16 if W.bf16 else torch.float32
+    q_h = torch.from_numpy(np.ascontiguousarray(G.q_host[1])).view(torch_dt).pin_memory()
+    if W.paged:
+        toks = [G.paged_token(step0 + i) for i in range(n)]
+        k_h = [t[0].cpu().pin_memory() for t in toks]
+        v_h = [t[1].cpu().pin_memory() for t in toks]
+    else:
+        k_h = [G.k_new.detach().cpu().pin_memory()] * n
+        v_h = [G.v_new.detach().cpu().pin_memory()] * n
+    out_h = torch.empty(G.out.shape, dtype=torch.float32).pin_memory()
+    q_d = torch.empty_like(G.q)
+    kd = torch.empty_like(k_h[0], device=G.dev)
+    vd = torch.empty_like(v_h[0], device=G.dev)
+    h2d = q_h.numel() * q_h.element_size()
+    if G.append_token:
+        h2d += 2 * k_h[0].numel() * k_h[0].element_size()
+    d2h = out_h.numel() * 4
+    evs = []
+    for i in range(n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            flush.zero_()
+            a.record(stream)
+            q_d.copy_(q_h, non_blocking=True)
+            if G.append_token:
+                kd.copy_(k_h[i], non_blocking=True)
+                vd.copy_(v_h[i], non_blocking=True)
+            G.step(stream, k_new=kd, v_new=vd, q=q_d)
+            out_h.copy_(G.out, non_blocking=True)
+            b.record(stream)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / n
+    return dict(t=ms / 1e3, h2d=h2d, d2h=d2h)
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+class OracleUnit:
+    """One (sequence, kv_head) unit of the workload held by the CPU oracle: its prefill is
+    quantized once (untimed); a step is the same as on the GPU: one token appended at the
+    step position, then fp64 decode attention of the unit's query heads over its tokens."""
+
+    def __init__(self, w, b, h):
+        from oracle import OracleCache
+        self.w, self.b, self.h = w, b, h
+        L = int(w.prefill_lengths()[b])
+        self.append = w.name != "tiny_int8"
+        pre = L - 1 if self.append else L
+        K = synth.keys(w, b, b + 1, h, h + 1, 0, pre + 1)
+        V = synth.values(w, b, b + 1, h, h + 1, 0, pre + 1)
+        cap = (pre + 1 + 127) // 128 * 128
+        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap)
+        calib = w.k_scheme in CALIBRATED or w.v_scheme in CALIBRATED
+        self.oc.append(K[:, :, :pre], V[:, :, :pre], w.bf16, calibrate=calib)
+        self.saved = (self.oc.c.len, self.oc.c.res)
+        self.k1, self.v1 = K[:, :, pre:pre + 1].copy(), V[:, :, pre:pre + 1].copy()
+        qw = synth.Workload(**{**w.__dict__, "B": 1, "Hkv": 1, "Hq": w.G, "seed": w.seed + 17 * (b * w.Hkv + h)})
+        self.q = synth.queries(qw, 0, 0, 1)
+        self.unit_w = synth.Workload(**{**w.__dict__, "B": 1, "Hkv": 1, "Hq": w.G})
+
+    def step(self):
+        """Returns (algorithmic bytes, seconds) of one oracle step."""
+        self.oc.c.len, self.oc.c.res = self.saved
+        t0 = time.perf_counter()
+        if self.append:
+            self.oc.append(self.k1, self.v1, self.w.bf16)
+        self.oc.decode(self.q, self.w.bf16, 1.0 / math.sqrt(128.0))
+        dt = time.perf_counter() - t0
+        nr = self.oc.residual if self.w.kivi else 0
+        b = decode_bytes(self.unit_w, np.array([self.oc.length]), nr)
+        if self.append:
+            b += append_bytes(self.unit_w)
+        return b, dt
+
+
+def oracle_time(w, seconds, max_units=8):
+    """Time oracle steps over up to max_units distinct units until `seconds` of timed work."""
+    units, tb, tt, steps = [], 0.0, 0.0, 0
+    while tt < seconds:
+        if len(units) < max_units:
+            i = len(units)
+            units.append(OracleUnit(w, i % w.B, (i // w.B) % w.Hkv))
+        u = units[steps % len(units)]
+        b, t = u.step()
+        tb, tt, steps = tb + b, tt + t, steps + 1
+    ctx = units[0].oc.length + (units[0].oc.residual if w.kivi else 0)
+    desc = (f"{steps} oracle steps over {len(units)} (sequence, kv_head) units; each: "
+            f"{'append 1 token + ' if units[0].append else ''}fp64 decode of {w.G} query heads over "
+            f"{ctx} tokens (single-threaded C)")
+    return tb, tt, steps, desc
+
+
+def emit(obj):
+    print(json.dumps(obj), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.workloads()[args.workload]
+    dtype = DTYPE_NAME[w.k_scheme] + ("/" + DTYPE_NAME[w.v_scheme] if w.v_scheme != w.k_scheme else "")
+    config = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
+              "k_scheme": w.k_scheme, "v_scheme": w.v_scheme,
+              "context": (f"uniform {w.len_lo}..{w.len_hi}" if w.paged else w.prefill_tokens()),
+              "layout": "paged/16" if w.paged else "dense",
+              "step": ("decode only" if w.name == "tiny_int8" else "append 1 token per sequence + decode"),
+              "l2": "flushed (256 MiB write) before every timed step, outside the event interval",
+              "parallelism": f"replicas x{args.gpus}"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        unit = OracleUnit(w, 0, 0)
+        for _ in range(args.warmup):
+            unit.step()
+        tb = tt = 0.0
+        for _ in range(args.steps):
+            b, t = unit.step()
+            tb, tt = tb + b, tt + t
+        val = tb / tt / 1e9
+        ctx = unit.oc.length + (unit.oc.residual if w.kivi else 0)
+        sample = (f"each step: one (sequence 0, kv_head 0) unit of the workload step - "
+                  f"{'append 1 token + ' if unit.append else ''}fp64 decode of {w.G} query heads over {ctx} "
+                  f"tokens (single-threaded C oracle)")
+        emit({"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": tt / args.steps * 1e3,
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+              "data": "synthetic (seeded generators)", "config": config,
+              "cpu_baseline": {"value": val, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+              "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        return
+
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    r = run_gpu(args, rank, world, local_rank)
+    W = r["W"]
+    step_bytes = r["dbytes"] + r["abytes"]
+    value = world * step_bytes / r["t_max"] / 1e9
+    tokens_per_s = world * W.B / r["t_max"]
+    peak, peak_kind = measured_peak()
+    achieved = r["dbytes_dec"] / r["t_dec"] / 1e9
+    roofline = {"bound": "hbm", "kernel": "decode attention call (split-KV kernel + LSE merge)",
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": r["dbytes_dec"], "launch_ms": r["t_dec"] * 1e3,
+                "traffic": kernel_traffic(W.name)}
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": r["t_max"] * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": dtype,
+           "data": "synthetic (seeded counter-based generators; no dataset)", "config": config,
+           "tokens_per_s": tokens_per_s, "pct_of_hbm_peak": 100.0 * (value / world) / peak,
+           "roofline": roofline, "clocks": r["clocks"], "gpu_launches": r["launches"],
+           "device_status": list(r["status"])}
+    if r["e2e"]:
+        e = r["e2e"]
+        out["e2e"] = {"value": world * step_bytes / e["t"] / 1e9, "unit": UNIT,
+                      "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
+    else:
+        out["e2e"] = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        b, t, n, desc = oracle_time(W, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": b / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        emit(out)
+
+
+if __name__ == "__main__":
+    main()

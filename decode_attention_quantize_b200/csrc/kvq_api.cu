@@ -1,0 +1,340 @@
+// C-ABI entry points of libkvq: argument validation (host only, before any launch),
+// workspace queries, footprint arithmetic and kernel launches.
+#include <atomic>
+#include <cstring>
+
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+using namespace kvq;
+
+namespace kvq {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace kvq
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_KIVI_INT2; }
+
+bool needs_scale(int s) { return true; }
+bool needs_zp(int s) { return s == KVQ_UINT8_ASYM_PER_CHANNEL; }
+
+// Per-side metadata element counts (floats) for the layouts in kvq.h.
+uint64_t scale_elems(const kvq_cache_desc* d, int side) {
+  const int s = side ? d->v_scheme : d->k_scheme;
+  const uint64_t B = d->batch, H = d->num_kv_heads, D = d->head_dim;
+  const bool paged = d->layout == KVQ_PAGED;
+  switch (s) {
+    case KVQ_FP8_E4M3_PER_TENSOR:
+    case KVQ_INT8_SYM_PER_TENSOR: return 1;
+    case KVQ_INT8_SYM_PER_TOKEN:
+      return paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity;
+    case KVQ_INT8_SYM_PER_CHANNEL:
+    case KVQ_UINT8_ASYM_PER_CHANNEL: return H * D;
+    default:
+      return side == 0 ? B * H * (uint64_t)(d->capacity / 32) * D : B * H * (uint64_t)d->capacity * (D / 32);
+  }
+}
+
+kvq_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return KVQ_OK;
+  if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_ERR_CUDA;
+}
+
+int seq_capacity(const kvq_cache_desc* d) {
+  return d->layout == KVQ_PAGED ? d->max_pages_per_seq * d->page_size : d->capacity;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_abi_version(void) { return KVQ_ABI_VERSION; }
+
+uint64_t kvq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+kvq_status kvq_validate(const kvq_cache_desc* d) {
+  if (!d) return KVQ_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->num_kv_heads < 1 || d->num_q_heads < d->num_kv_heads ||
+      d->num_q_heads % d->num_kv_heads != 0 || d->batch > 65535 || d->num_kv_heads > 1024)
+    return KVQ_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return d->head_dim > 0 ? KVQ_ERR_UNSUPPORTED : KVQ_ERR_INVALID_ARG;
+  if (!valid_scheme(d->k_scheme) || !valid_scheme(d->v_scheme)) return KVQ_ERR_INVALID_ARG;
+  if (d->layout != KVQ_DENSE && d->layout != KVQ_PAGED) return KVQ_ERR_INVALID_ARG;
+  const bool kivi_k = is_kivi(d->k_scheme), kivi_v = is_kivi(d->v_scheme);
+  if (kivi_k || kivi_v) {
+    if (d->k_scheme != d->v_scheme) return KVQ_ERR_UNSUPPORTED;
+    if (d->layout == KVQ_PAGED) return KVQ_ERR_UNSUPPORTED;
+    if (d->group_size != 32 || d->residual_cap != 128) return KVQ_ERR_UNSUPPORTED;
+    if (!d->k_zero || !d->v_zero || !d->k_res || !d->v_res) return KVQ_ERR_INVALID_ARG;
+    if (!aligned16(d->k_zero) || !aligned16(d->v_zero) || !aligned16(d->k_res) || !aligned16(d->v_res))
+      return KVQ_ERR_INVALID_ARG;
+    if (d->num_residual < 0 || d->num_residual > d->residual_cap) return KVQ_ERR_INVALID_ARG;
+  }
+  if (d->layout == KVQ_DENSE) {
+    if (d->capacity < 128 || d->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;
+    if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)d->capacity >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (d->num_quantized < 0 || d->num_quantized > d->capacity) return KVQ_ERR_INVALID_ARG;
+    if ((kivi_k) && d->num_quantized % 128 != 0) return KVQ_ERR_INVALID_ARG;
+  } else {
+    if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64) return KVQ_ERR_UNSUPPORTED;
+    if (d->max_pages_per_seq < 1 || d->num_pages < 1) return KVQ_ERR_INVALID_ARG;
+    if ((uint64_t)d->num_pages * d->num_kv_heads * (uint64_t)d->page_size >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (!d->page_table || !d->seq_lens) return KVQ_ERR_INVALID_ARG;
+  }
+  if (!d->k_codes || !d->v_codes || !d->k_scale || !d->v_scale || !d->dev_status) return KVQ_ERR_INVALID_ARG;
+  if (!aligned16(d->k_codes) || !aligned16(d->v_codes) || !aligned16(d->k_scale) || !aligned16(d->v_scale))
+    return KVQ_ERR_INVALID_ARG;
+  if ((needs_zp(d->k_scheme) && !d->k_zp) || (needs_zp(d->v_scheme) && !d->v_zp)) return KVQ_ERR_INVALID_ARG;
+  (void)needs_scale;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_bytes(const kvq_cache_desc* d, kvq_footprint* out) {
+  const kvq_status st = kvq_validate(d);
+  if (st != KVQ_OK) return st;
+  if (!out) return KVQ_ERR_INVALID_ARG;
+  const bool paged = d->layout == KVQ_PAGED;
+  const uint64_t rows = paged ? (uint64_t)d->num_pages * d->num_kv_heads * d->page_size
+                              : (uint64_t)d->batch * d->num_kv_heads * d->capacity;
+  kvq_footprint f;
+  std::memset(&f, 0, sizeof(f));
+  f.code_bytes = rows * (uint64_t)(row_bytes(d->k_scheme) + row_bytes(d->v_scheme));
+  uint64_t meta = 0;
+  double per_token_meta = 0.0;
+  for (int side = 0; side < 2; ++side) {
+    const int s = side ? d->v_scheme : d->k_scheme;
+    const uint64_t n = scale_elems(d, side);
+    uint64_t bytes = n * 4;
+    if (is_kivi(s)) bytes *= 2;                       // scale + minimum
+    if (needs_zp(s)) bytes += (uint64_t)d->num_kv_heads * d->head_dim;  // uint8 zero points
+    meta += bytes;
+    if (s == KVQ_INT8_SYM_PER_TOKEN) per_token_meta += 4.0;
+    if (is_kivi(s)) per_token_meta += 8.0 * d->head_dim / 32.0;  // (scale, min) per 32 tokens or channels
+  }
+  f.meta_bytes = meta;
+  f.residual_bytes = is_kivi(d->k_scheme)
+                         ? 2ull * d->batch * d->num_kv_heads * (uint64_t)d->residual_cap * d->head_dim * 2
+                         : 0;
+  f.total_bytes = f.code_bytes + f.meta_bytes + f.residual_bytes;
+  f.bytes_per_token = (double)(row_bytes(d->k_scheme) + row_bytes(d->v_scheme)) + per_token_meta;
+  *out = f;
+  return KVQ_OK;
+}
+
+size_t kvq_append_workspace_bytes(const kvq_cache_desc* d, uint32_t flags) {
+  if (!d || !(flags & KVQ_APPEND_CALIBRATE)) return 0;
+  return round_up((2 + 4 * (size_t)d->num_kv_heads * kHeadDim) * sizeof(uint32_t));
+}
+
+kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void* v_new, int32_t in_dtype,
+                               int32_t n_new, const int32_t* new_lens, uint32_t flags, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  kvq_status st = kvq_validate(d);
+  if (st != KVQ_OK) return st;
+  if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (n_new < 0 || (flags & ~KVQ_APPEND_CALIBRATE)) return KVQ_ERR_INVALID_ARG;
+  if (n_new == 0) return KVQ_OK;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+  const bool paged = d->layout == KVQ_PAGED;
+  if (new_lens && !paged) return KVQ_ERR_INVALID_ARG;
+  const bool kivi = is_kivi(d->k_scheme);
+  if (kivi && in_dtype != KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
+  if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)n_new >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+  if (paged && n_new > seq_capacity(d)) return KVQ_ERR_CAPACITY;
+  const bool calibrate = (flags & KVQ_APPEND_CALIBRATE) != 0 && !kivi;
+  if (calibrate) {
+    if (!workspace || workspace_bytes < kvq_append_workspace_bytes(d, flags) || !aligned16(workspace))
+      return KVQ_ERR_WORKSPACE;
+  }
+  int r_old = 0, flushed = 0, r_new = 0;
+  if (!paged) {
+    if (kivi) {
+      r_old = d->num_residual;
+      const int total = r_old + n_new;
+      r_new = (total - 1) % d->residual_cap + 1;
+      flushed = total - r_new;
+      if ((int64_t)d->num_quantized + flushed > d->capacity) return KVQ_ERR_CAPACITY;
+    } else if ((int64_t)d->num_quantized + n_new > d->capacity) {
+      return KVQ_ERR_CAPACITY;
+    }
+  }
+  AppendParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = d->batch;
+  p.H = d->num_kv_heads;
+  p.n_new = n_new;
+  p.k_scheme = d->k_scheme;
+  p.v_scheme = d->v_scheme;
+  p.in_bf16 = in_dtype == KVQ_BF16;
+  p.paged = paged;
+  p.cap = d->capacity;
+  p.page_size = d->page_size;
+  p.max_pages = d->max_pages_per_seq;
+  p.num_pages = d->num_pages;
+  p.pos0 = d->num_quantized;
+  p.rcap = d->residual_cap;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.new_lens = new_lens;
+  p.k_codes = d->k_codes;
+  p.v_codes = d->v_codes;
+  p.k_scale = d->k_scale;
+  p.k_zero = d->k_zero;
+  p.v_scale = d->v_scale;
+  p.v_zero = d->v_zero;
+  p.k_zp = d->k_zp;
+  p.v_zp = d->v_zp;
+  p.k_res = d->k_res;
+  p.v_res = d->v_res;
+  p.page_table = d->page_table;
+  p.seq_lens = d->seq_lens;
+  p.status = d->dev_status;
+  const cudaError_t e = launch_append(p, static_cast<uint32_t*>(workspace), calibrate, r_old, flushed, r_new,
+                                      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return from_cuda(e);
+  if (!paged) {
+    if (kivi) {
+      d->num_quantized += flushed;
+      d->num_residual = r_new;
+    } else {
+      d->num_quantized += n_new;
+    }
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_dequantize(const kvq_cache_desc* d, int32_t which, float* out, int32_t out_tokens, void* stream) {
+  kvq_status st = kvq_validate(d);
+  if (st != KVQ_OK) return st;
+  if ((which != 0 && which != 1) || !out || out_tokens < 0 || !aligned16(out)) return KVQ_ERR_INVALID_ARG;
+  const bool paged = d->layout == KVQ_PAGED;
+  if (!paged) {
+    const int len = d->num_quantized + (is_kivi(d->k_scheme) ? d->num_residual : 0);
+    if (out_tokens < len) return KVQ_ERR_INVALID_ARG;
+  }
+  DequantParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = d->batch;
+  p.H = d->num_kv_heads;
+  p.T_out = out_tokens;
+  p.which = which;
+  p.scheme = which ? d->v_scheme : d->k_scheme;
+  p.paged = paged;
+  p.cap = d->capacity;
+  p.page_size = d->page_size;
+  p.max_pages = d->max_pages_per_seq;
+  p.num_pages = d->num_pages;
+  p.len_q = d->num_quantized;
+  p.len_res = d->num_residual;
+  p.rcap = d->residual_cap;
+  p.codes = static_cast<const uint8_t*>(which ? d->v_codes : d->k_codes);
+  p.scale = which ? d->v_scale : d->k_scale;
+  p.zero = which ? d->v_zero : d->k_zero;
+  p.zp = which ? d->v_zp : d->k_zp;
+  p.res = which ? d->v_res : d->k_res;
+  p.page_table = d->page_table;
+  p.seq_lens = d->seq_lens;
+  p.status = d->dev_status;
+  p.out = out;
+  return from_cuda(launch_dequantize(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* d) {
+  if (!d || d->num_kv_heads < 1 || d->batch < 1 || d->num_q_heads < d->num_kv_heads) return 0;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  const size_t pairs = (size_t)d->batch * d->num_kv_heads * ((G + 7) / 8);
+  const size_t slots = pairs + kMaxCtas;
+  return round_up(slots * 8 * kHeadDim * sizeof(float)) + round_up(slots * 8 * 2 * sizeof(float)) +
+         round_up((2 * (size_t)d->batch + 2) * sizeof(int32_t));
+}
+
+kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t q_dtype, float softmax_scale,
+                                float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  kvq_status st = kvq_validate(d);
+  if (st != KVQ_OK) return st;
+  if (!q || !out || (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16)) return KVQ_ERR_INVALID_ARG;
+  if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.0f) return KVQ_ERR_INVALID_ARG;
+  const size_t need = kvq_decode_workspace_bytes(d);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KVQ_ERR_WORKSPACE;
+  const bool paged = d->layout == KVQ_PAGED;
+  if (!decode_supported(d->k_scheme, d->v_scheme, paged)) return KVQ_ERR_UNSUPPORTED;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = d->batch;
+  p.Hq = d->num_q_heads;
+  p.Hkv = d->num_kv_heads;
+  p.G = G;
+  p.HG = (G + 7) / 8;
+  p.k_scheme = d->k_scheme;
+  p.v_scheme = d->v_scheme;
+  p.paged = paged;
+  p.cap = d->capacity;
+  p.page_size = d->page_size;
+  p.max_pages = d->max_pages_per_seq;
+  p.num_pages = d->num_pages;
+  p.len_q = d->num_quantized;
+  p.len_res = is_kivi(d->k_scheme) ? d->num_residual : 0;
+  p.rcap = d->residual_cap;
+  p.k_codes = static_cast<const uint8_t*>(d->k_codes);
+  p.v_codes = static_cast<const uint8_t*>(d->v_codes);
+  p.k_scale = d->k_scale;
+  p.k_zero = d->k_zero;
+  p.v_scale = d->v_scale;
+  p.v_zero = d->v_zero;
+  p.k_zp = d->k_zp;
+  p.v_zp = d->v_zp;
+  p.k_res = d->k_res;
+  p.v_res = d->v_res;
+  p.page_table = d->page_table;
+  p.seq_lens = d->seq_lens;
+  p.status = d->dev_status;
+  p.q = q;
+  p.q_bf16 = q_dtype == KVQ_BF16;
+  p.softmax_scale = softmax_scale;
+  p.out = out;
+  p.lse = lse;
+  p.n_pairs = d->batch * d->num_kv_heads * p.HG;
+  const size_t slots = (size_t)p.n_pairs + kMaxCtas;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.part_o = reinterpret_cast<float*>(ws);
+  ws += round_up(slots * 8 * kHeadDim * sizeof(float));
+  p.part_ml = reinterpret_cast<float*>(ws);
+  ws += round_up(slots * 8 * 2 * sizeof(float));
+  p.plan = reinterpret_cast<int32_t*>(ws);
+  return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_get_device_status(const kvq_cache_desc* d, uint32_t* out, int32_t clear, void* stream) {
+  if (!d || !d->dev_status || !out) return KVQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(out, d->dev_status, 2 * sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && clear) {
+    e = cudaMemsetAsync(d->dev_status, 0, 2 * sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  return from_cuda(e);
+}
+
+}  // extern "C"

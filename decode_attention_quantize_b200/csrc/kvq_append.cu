@@ -1,0 +1,547 @@
+// Quantize-on-append, calibration and dequantize kernels (sm_100a).
+//
+// Every code, scale and zero point is computed with one correctly rounded fp32 operation
+// per step (IEEE division, round-half-to-even), so results are bit-identical to a plain
+// sequential statement of the schemes:
+//  - symmetric INT8: s = absmax/127, q = clamp(rne(x/s), -127, 127)
+//    ("KV Cache Quantization in Production LLM Serving", llms.blog, §2);
+//  - FP8 E4M3: s = absmax/448, q = e4m3_rn_satfinite(x/s) (infra.bea.ai §4, llms.blog §1);
+//  - asymmetric uint8 per channel: affine form over a range widened to contain 0
+//    ("How KV cache quantization reduces GPU memory", n4n.ai, Steps 2-3);
+//  - KIVI: keys per channel over 32-token groups, values per token over 32-channel
+//    groups, min-max with 2^bits - 1 steps, bf16 residual of 128 tokens
+//    (infra.bea.ai §3; llms.blog §3).
+#include <cuda_fp8.h>
+
+#include "kvq_device.cuh"
+#include "kvq_internal.h"
+
+namespace kvq {
+
+// ------------------------------------------------------------------ element helpers
+template <bool kBf16>
+__device__ __forceinline__ void load8(const void* base, size_t elem, float (&x)[8]) {
+  if constexpr (kBf16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = bf16_bits_to_float(w[i] & 0xFFFFu);
+      x[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+    const float4 a = p[0], b = p[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ int sym_code(float x, float s, int qmax, int& sat) {
+  if (s == 0.0f) return 0;
+  float r = rintf(__fdiv_rn(x, s));
+  if (r > (float)qmax) { r = (float)qmax; ++sat; }
+  if (r < (float)-qmax) { r = (float)-qmax; ++sat; }
+  return (int)r;
+}
+
+__device__ __forceinline__ int asym_code(float x, float s, int zp, int& sat) {
+  if (s == 0.0f) return 0;
+  float r = __fadd_rn(rintf(__fdiv_rn(x, s)), (float)zp);
+  if (r < 0.0f) { r = 0.0f; ++sat; }
+  if (r > 255.0f) { r = 255.0f; ++sat; }
+  return (int)r;
+}
+
+__device__ __forceinline__ int fp8_code(float x, float s, int& sat) {
+  if (s == 0.0f) return 0;
+  const float y = __fdiv_rn(x, s);
+  if (fabsf(y) > 448.0f) ++sat;
+  return (int)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Row of token `pos` of (b, h): dense [B,H,cap]; paged via the page table. Returns false
+// (and flags the status word) when the page slot is outside the table or the pool.
+__device__ __forceinline__ bool cache_row(const AppendParams& p, int b, int h, int pos, size_t& row) {
+  if (!p.paged) {
+    row = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)pos;
+    return true;
+  }
+  const int pi = pos / p.page_size;
+  if (pos < 0 || pi >= p.max_pages) {
+    flag(p.status, KVQ_DEV_BAD_LENGTH);
+    return false;
+  }
+  const int page = p.page_table[(size_t)b * p.max_pages + pi];
+  if (page < 0 || page >= p.num_pages) {
+    flag(p.status, KVQ_DEV_BAD_PAGE);
+    return false;
+  }
+  row = ((size_t)page * p.H + h) * (size_t)p.page_size + (size_t)(pos % p.page_size);
+  return true;
+}
+
+__device__ __forceinline__ int new_count(const AppendParams& p, int b) {
+  if (!p.new_lens) return p.n_new;
+  int n = p.new_lens[b];
+  return n < 0 ? 0 : (n > p.n_new ? p.n_new : n);
+}
+
+// ------------------------------------------------------------------ calibration
+// Workspace keys (uint32): [0] K absmax, [1] V absmax, then per side two arrays of H*D
+// (absmax or order-key min, and order-key max).
+__global__ void calib_init_kernel(uint32_t* keys, int hd) {
+  const int n = 2 + 4 * hd;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    uint32_t v = 0u;
+    if (i >= 2) {
+      const int j = (i - 2) % (2 * hd);
+      v = j < hd ? 0xFFFFFFFFu : 0u;  // first array: min keys start high; absmax uses max
+    }
+    keys[i] = v;
+  }
+}
+
+// One block per (token chunk, b*H + h, side). 256 threads: 16 row lanes x 16 lanes of
+// 8 channels. Reduces absmax (per-tensor), absmax per channel, or min/max per channel.
+template <bool kBf16>
+__global__ void __launch_bounds__(256) calib_reduce_kernel(AppendParams p, uint32_t* keys) {
+  constexpr int kChunk = 256;
+  const int side = blockIdx.z;
+  const int scheme = side ? p.v_scheme : p.k_scheme;
+  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR;
+  const bool per_channel = scheme == KVQ_INT8_SYM_PER_CHANNEL || scheme == KVQ_UINT8_ASYM_PER_CHANNEL;
+  if (!per_tensor && !per_channel) return;
+  const bool asym = scheme == KVQ_UINT8_ASYM_PER_CHANNEL;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  const int n_b = new_count(p, b);
+  const int t_begin = blockIdx.x * kChunk;
+  if (t_begin >= n_b) return;
+  const int t_end = min(n_b, t_begin + kChunk);
+  const void* x = side ? p.v_new : p.k_new;
+  const int lane8 = threadIdx.x & 15, rl = threadIdx.x >> 4;
+  float lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    lo[i] = INFINITY;
+    hi[i] = asym ? -INFINITY : 0.0f;
+  }
+  for (int t = t_begin + rl; t < t_end; t += 16) {
+    float v[8];
+    load8<kBf16>(x, (((size_t)b * p.H + h) * (size_t)p.n_new + t) * kHeadDim + lane8 * 8, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (asym) {
+        lo[i] = fminf(lo[i], v[i]);
+        hi[i] = fmaxf(hi[i], v[i]);
+      } else {
+        hi[i] = fmaxf(hi[i], fabsf(v[i]));
+      }
+    }
+  }
+  __shared__ float s_lo[16][kHeadDim], s_hi[16][kHeadDim];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s_lo[rl][lane8 * 8 + i] = lo[i];
+    s_hi[rl][lane8 * 8 + i] = hi[i];
+  }
+  __syncthreads();
+  const int hd = p.H * kHeadDim;
+  uint32_t* base = keys + 2 + side * 2 * hd;
+  if (threadIdx.x < kHeadDim) {
+    const int d = threadIdx.x;
+    float a = s_lo[0][d], m = s_hi[0][d];
+    for (int r = 1; r < 16; ++r) {
+      a = fminf(a, s_lo[r][d]);
+      m = fmaxf(m, s_hi[r][d]);
+    }
+    if (per_channel) {
+      if (asym) {
+        atomicMin(base + h * kHeadDim + d, order_key(a));
+        atomicMax(base + hd + h * kHeadDim + d, order_key(m));
+      } else {
+        atomicMax(base + hd + h * kHeadDim + d, __float_as_uint(m));  // m >= +0
+      }
+    } else {
+      s_hi[0][d] = m;
+    }
+  }
+  if (per_tensor) {
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float m = 0.0f;
+      for (int d = threadIdx.x; d < kHeadDim; d += 32) m = fmaxf(m, s_hi[0][d]);
+      m = warp_max(m);
+      if (threadIdx.x == 0) atomicMax(keys + side, __float_as_uint(m));
+    }
+  }
+}
+
+// Turn the reduced statistics into scales (and zero points): one block.
+__global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
+  const int hd = p.H * kHeadDim;
+  for (int side = 0; side < 2; ++side) {
+    const int scheme = side ? p.v_scheme : p.k_scheme;
+    float* scale = side ? p.v_scale : p.k_scale;
+    uint8_t* zp = side ? p.v_zp : p.k_zp;
+    const uint32_t* base = keys + 2 + side * 2 * hd;
+    if (scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR) {
+      if (threadIdx.x == 0) {
+        const float amax = __uint_as_float(keys[side]);
+        scale[0] = __fdiv_rn(amax, scheme == KVQ_FP8_E4M3_PER_TENSOR ? 448.0f : 127.0f);
+      }
+    } else if (scheme == KVQ_INT8_SYM_PER_CHANNEL) {
+      for (int i = threadIdx.x; i < hd; i += blockDim.x)
+        scale[i] = __fdiv_rn(__uint_as_float(base[hd + i]), 127.0f);
+    } else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
+      for (int i = threadIdx.x; i < hd; i += blockDim.x) {
+        const float mn = key_to_float(base[i]), mx = key_to_float(base[hd + i]);
+        const float lo = mn < 0.0f ? mn : 0.0f;
+        const float hi = mx > 0.0f ? mx : 0.0f;
+        const float s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
+        int z = 0;
+        if (s != 0.0f) {
+          float zf = rintf(__fdiv_rn(-lo, s));
+          zf = fminf(fmaxf(zf, 0.0f), 255.0f);
+          z = (int)zf;
+        }
+        scale[i] = s;
+        zp[i] = (uint8_t)z;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ 8-bit quantize-store
+// Rows (b, h, i) of the new block; 16 threads per row, 8 channels each; blockIdx.y = side.
+template <bool kBf16>
+__global__ void __launch_bounds__(256) quantize_rows_kernel(AppendParams p) {
+  const int side = blockIdx.y;
+  const int scheme = side ? p.v_scheme : p.k_scheme;
+  const long long rows = (long long)p.B * p.H * p.n_new;
+  const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+  const int lane8 = threadIdx.x & 15;
+  const unsigned half_mask = (threadIdx.x & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+  int sat = 0;
+  bool active = r < rows;
+  int b = 0, h = 0, i = 0;
+  if (active) {
+    i = (int)(r % p.n_new);
+    h = (int)((r / p.n_new) % p.H);
+    b = (int)(r / ((long long)p.n_new * p.H));
+    active = i < new_count(p, b);
+  }
+  float x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (active) load8<kBf16>(side ? p.v_new : p.k_new, (size_t)r * kHeadDim + lane8 * 8, x);
+  float* scale = side ? p.v_scale : p.k_scale;
+  // per-token scale: absmax over the 16 lanes of this row (all 32 lanes take part)
+  float tok_s = 0.0f;
+  if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    tok_s = __fdiv_rn(m, 127.0f);
+  }
+  (void)half_mask;
+  if (!active) return;
+  const int pos = (p.paged ? p.seq_lens[b] : p.pos0) + i;
+  size_t row;
+  if (!cache_row(p, b, h, pos, row)) return;
+  uint8_t* codes = static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8;
+  const uint8_t* zp = side ? p.v_zp : p.k_zp;
+  uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int d = lane8 * 8 + k;
+    int q = 0;
+    switch (scheme) {
+      case KVQ_FP8_E4M3_PER_TENSOR: q = fp8_code(x[k], scale[0], sat); break;
+      case KVQ_INT8_SYM_PER_TENSOR: q = sym_code(x[k], scale[0], 127, sat); break;
+      case KVQ_INT8_SYM_PER_TOKEN: q = sym_code(x[k], tok_s, 127, sat); break;
+      case KVQ_INT8_SYM_PER_CHANNEL: q = sym_code(x[k], scale[h * kHeadDim + d], 127, sat); break;
+      case KVQ_UINT8_ASYM_PER_CHANNEL:
+        q = asym_code(x[k], scale[h * kHeadDim + d], zp[h * kHeadDim + d], sat);
+        break;
+    }
+    packed[k >> 2] |= (uint32_t)(q & 0xFF) << (8 * (k & 3));
+  }
+  *reinterpret_cast<uint2*>(codes) = make_uint2(packed[0], packed[1]);
+  if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
+  if (sat && p.status) atomicAdd(p.status + 1, (uint32_t)sat);
+}
+
+__global__ void seq_lens_advance_kernel(AppendParams p) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < p.B) p.seq_lens[b] += new_count(p, b);
+}
+
+// ------------------------------------------------------------------ KIVI
+// One block per (R-token chunk, b*H + h): quantize R consecutive tokens of the combined
+// stream (old residual tokens, then the new block) into the cache at pos0 + chunk*R.
+template <int kBits>
+__global__ void __launch_bounds__(256) kivi_flush_kernel(AppendParams p, int r_old) {
+  constexpr int R = 128, G = 32, kQmax = (1 << kBits) - 1, kPer = 8 / kBits;
+  constexpr int kRowBytes = kHeadDim * kBits / 8;
+  extern __shared__ __align__(16) uint8_t smem[];
+  uint16_t* xk = reinterpret_cast<uint16_t*>(smem);           // [R][D] bf16
+  uint16_t* xv = xk + R * kHeadDim;                            // [R][D] bf16
+  uint8_t* kcodes = reinterpret_cast<uint8_t*>(xv + R * kHeadDim);  // [R][row bytes]
+  const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  const int pos0 = p.pos0 + chunk * R;
+  // gather the combined stream: 16-byte pieces, 16 per token row
+  for (int e = threadIdx.x; e < R * 16; e += blockDim.x) {
+    const int tok = e >> 4, piece = e & 15;
+    const int s = chunk * R + tok;  // index in the combined stream
+    const uint16_t *srck, *srcv;
+    if (s < r_old) {
+      const size_t o = (((size_t)b * p.H + h) * p.rcap + s) * kHeadDim;
+      srck = p.k_res + o;
+      srcv = p.v_res + o;
+    } else {
+      const size_t o = (((size_t)b * p.H + h) * (size_t)p.n_new + (s - r_old)) * kHeadDim;
+      srck = static_cast<const uint16_t*>(p.k_new) + o;
+      srcv = static_cast<const uint16_t*>(p.v_new) + o;
+    }
+    reinterpret_cast<uint4*>(xk + tok * kHeadDim)[piece] = reinterpret_cast<const uint4*>(srck)[piece];
+    reinterpret_cast<uint4*>(xv + tok * kHeadDim)[piece] = reinterpret_cast<const uint4*>(srcv)[piece];
+  }
+  __syncthreads();
+  // keys: task = (group gi, kPer adjacent channels)
+  constexpr int kKTasks = (R / G) * (kHeadDim / kPer);
+  for (int task = threadIdx.x; task < kKTasks; task += blockDim.x) {
+    const int gi = task / (kHeadDim / kPer), c0 = (task % (kHeadDim / kPer)) * kPer;
+    uint8_t bytes[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) bytes[j] = 0;
+    const size_t meta = (((size_t)b * p.H + h) * (size_t)(p.cap / G) + (size_t)(pos0 / G + gi)) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int d = c0 + k;
+      float lo = bf16_bits_to_float(xk[(gi * G) * kHeadDim + d]), hi = lo;
+      for (int j = 1; j < G; ++j) {
+        const float v = bf16_bits_to_float(xk[(gi * G + j) * kHeadDim + d]);
+        lo = fminf(lo, v);
+        hi = fmaxf(hi, v);
+      }
+      if (lo == 0.0f) lo = 0.0f;
+      if (hi == 0.0f) hi = 0.0f;
+      const float s = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+      p.k_scale[meta + d] = s;
+      p.k_zero[meta + d] = lo;
+      for (int j = 0; j < G; ++j) {
+        int q = 0;
+        if (s != 0.0f) {
+          const float v = bf16_bits_to_float(xk[(gi * G + j) * kHeadDim + d]);
+          float r = rintf(__fdiv_rn(__fsub_rn(v, lo), s));
+          r = fminf(fmaxf(r, 0.0f), (float)kQmax);
+          q = (int)r;
+        }
+        bytes[j] |= (uint8_t)(q << (k * kBits));
+      }
+    }
+    for (int j = 0; j < G; ++j) kcodes[(gi * G + j) * kRowBytes + c0 / kPer] = bytes[j];
+  }
+  // values: task = (token, channel group)
+  for (int task = threadIdx.x; task < R * (kHeadDim / G); task += blockDim.x) {
+    const int tok = task / (kHeadDim / G), j = task % (kHeadDim / G);
+    const uint16_t* row = xv + tok * kHeadDim + j * G;
+    float lo = bf16_bits_to_float(row[0]), hi = lo;
+    for (int i = 1; i < G; ++i) {
+      const float v = bf16_bits_to_float(row[i]);
+      lo = fminf(lo, v);
+      hi = fmaxf(hi, v);
+    }
+    if (lo == 0.0f) lo = 0.0f;
+    if (hi == 0.0f) hi = 0.0f;
+    const float s = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+    uint32_t words[G * kBits / 32];
+#pragma unroll
+    for (int w = 0; w < G * kBits / 32; ++w) words[w] = 0u;
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      int q = 0;
+      if (s != 0.0f) {
+        float r = rintf(__fdiv_rn(__fsub_rn(bf16_bits_to_float(row[i]), lo), s));
+        r = fminf(fmaxf(r, 0.0f), (float)kQmax);
+        q = (int)r;
+      }
+      words[(i * kBits) / 32] |= (uint32_t)q << ((i * kBits) % 32);
+    }
+    const size_t crow = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)(pos0 + tok);
+    uint8_t* dst = static_cast<uint8_t*>(p.v_codes) + crow * kRowBytes + j * (G * kBits / 8);
+    if constexpr (kBits == 4) {
+      *reinterpret_cast<uint4*>(dst) = make_uint4(words[0], words[1], words[2], words[3]);
+    } else {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
+    }
+    p.v_scale[crow * (kHeadDim / G) + j] = s;
+    p.v_zero[crow * (kHeadDim / G) + j] = lo;
+  }
+  __syncthreads();
+  // key codes: R rows x kRowBytes, contiguous in the cache
+  uint8_t* kdst = static_cast<uint8_t*>(p.k_codes) + (((size_t)b * p.H + h) * (size_t)p.cap + pos0) * kRowBytes;
+  for (int e = threadIdx.x; e < R * kRowBytes / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(kdst)[e] = reinterpret_cast<const uint4*>(kcodes)[e];
+}
+
+// Copy `count` new tokens (input rows src0..) into residual slots dst0.. for every (b, h).
+__global__ void kivi_residual_kernel(AppendParams p, int src0, int dst0, int count) {
+  const long long total = (long long)p.B * p.H * count * 16;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int piece = (int)(e & 15);
+    const long long rr = e >> 4;
+    const int i = (int)(rr % count);
+    const long long bh = rr / count;
+    const size_t src = ((size_t)bh * p.n_new + src0 + i) * kHeadDim;
+    const size_t dst = ((size_t)bh * p.rcap + dst0 + i) * kHeadDim;
+    reinterpret_cast<uint4*>(p.k_res + dst)[piece] =
+        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.k_new) + src)[piece];
+    reinterpret_cast<uint4*>(p.v_res + dst)[piece] =
+        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.v_new) + src)[piece];
+  }
+}
+
+// ------------------------------------------------------------------ dequantize
+// out [B, H, T_out, D]; one thread per 8 channels of one row.
+__global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
+  const long long rows = (long long)p.B * p.H * p.T_out;
+  const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
+  if (r >= rows) return;
+  const int lane8 = threadIdx.x & 15;
+  const int t = (int)(r % p.T_out);
+  const int h = (int)((r / p.T_out) % p.H);
+  const int b = (int)(r / ((long long)p.T_out * p.H));
+  float y[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const int scheme = p.scheme;
+  const int len = p.paged ? p.seq_lens[b] : p.len_q + (is_kivi(scheme) ? p.len_res : 0);
+  if (t < len) {
+    if (is_kivi(scheme) && t >= p.len_q) {
+      const uint16_t* res = p.res + (((size_t)b * p.H + h) * p.rcap + (t - p.len_q)) * kHeadDim + lane8 * 8;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) y[k] = bf16_bits_to_float(res[k]);
+    } else {
+      size_t row;
+      bool ok = true;
+      if (!p.paged) {
+        row = ((size_t)b * p.H + h) * (size_t)p.cap + t;
+      } else {
+        const int pi = t / p.page_size;
+        const int page = pi < p.max_pages ? p.page_table[(size_t)b * p.max_pages + pi] : -1;
+        ok = page >= 0 && page < p.num_pages;
+        if (!ok) flag(p.status, KVQ_DEV_BAD_PAGE);
+        row = ((size_t)page * p.H + h) * (size_t)p.page_size + (t % p.page_size);
+      }
+      if (ok) {
+        const int bits = code_bits(scheme);
+        const uint8_t* codes = p.codes + row * (size_t)row_bytes(scheme);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int d = lane8 * 8 + k;
+          int q;
+          if (bits == 8) {
+            q = codes[d];
+          } else {
+            const int per = 8 / bits;
+            q = (codes[d / per] >> ((d % per) * bits)) & ((1 << bits) - 1);
+          }
+          float v = 0.0f;
+          switch (scheme) {
+            case KVQ_FP8_E4M3_PER_TENSOR: {
+              const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q, __NV_E4M3);
+              v = __fmul_rn(__half2float(__half(hr)), p.scale[0]);
+              break;
+            }
+            case KVQ_INT8_SYM_PER_TENSOR: v = __fmul_rn((float)(int8_t)q, p.scale[0]); break;
+            case KVQ_INT8_SYM_PER_TOKEN: v = __fmul_rn((float)(int8_t)q, p.scale[row]); break;
+            case KVQ_INT8_SYM_PER_CHANNEL: v = __fmul_rn((float)(int8_t)q, p.scale[h * kHeadDim + d]); break;
+            case KVQ_UINT8_ASYM_PER_CHANNEL:
+              v = __fmul_rn((float)(q - (int)p.zp[h * kHeadDim + d]), p.scale[h * kHeadDim + d]);
+              break;
+            default: {  // KIVI
+              size_t m;
+              if (p.which == 0)
+                m = (((size_t)b * p.H + h) * (size_t)(p.cap / 32) + (size_t)(t / 32)) * kHeadDim + d;
+              else
+                m = row * (kHeadDim / 32) + d / 32;
+              v = __fadd_rn(__fmul_rn((float)q, p.scale[m]), p.zero[m]);
+            }
+          }
+          y[k] = v;
+        }
+      }
+    }
+  }
+  float4* o = reinterpret_cast<float4*>(p.out + (size_t)r * kHeadDim + lane8 * 8);
+  o[0] = make_float4(y[0], y[1], y[2], y[3]);
+  o[1] = make_float4(y[4], y[5], y[6], y[7]);
+}
+
+// ------------------------------------------------------------------ launchers
+cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
+                          int flushed, int r_new, cudaStream_t st) {
+  const bool kivi = is_kivi(p.k_scheme);
+  if (kivi) {
+    if (flushed > 0) {
+      const int bits = code_bits(p.k_scheme);
+      const size_t smem = 2 * 128 * kHeadDim * 2 + 128 * (kHeadDim * bits / 8);
+      dim3 grid(flushed / 128, p.B * p.H);
+      if (bits == 4) {
+        cudaFuncSetAttribute(kivi_flush_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kivi_flush_kernel<4><<<grid, 256, smem, st>>>(p, r_old);
+        count_launches(1);
+      } else {
+        cudaFuncSetAttribute(kivi_flush_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kivi_flush_kernel<2><<<grid, 256, smem, st>>>(p, r_old);
+        count_launches(1);
+      }
+    }
+    // residual update: only new tokens ever move into it
+    const int count = flushed > 0 ? r_new : p.n_new;
+    const int src0 = flushed > 0 ? p.n_new - r_new : 0;
+    const int dst0 = flushed > 0 ? 0 : r_old;
+    if (count > 0) {
+      const long long pieces = (long long)p.B * p.H * count * 16;
+      const long long want = (pieces + 255) / 256;
+      const int blocks = (int)(want < 65535 ? want : 65535);
+      kivi_residual_kernel<<<blocks, 256, 0, st>>>(p, src0, dst0, count);
+      count_launches(1);
+    }
+    return cudaGetLastError();
+  }
+  if (calibrate) {
+    const int hd = p.H * kHeadDim;
+    calib_init_kernel<<<(2 + 4 * hd + 255) / 256, 256, 0, st>>>(calib_keys, hd);
+    dim3 grid((p.n_new + 255) / 256, p.B * p.H, 2);
+    if (p.in_bf16)
+      calib_reduce_kernel<true><<<grid, 256, 0, st>>>(p, calib_keys);
+    else
+      calib_reduce_kernel<false><<<grid, 256, 0, st>>>(p, calib_keys);
+    calib_finalize_kernel<<<1, 256, 0, st>>>(p, calib_keys);
+    count_launches(3);
+  }
+  const long long rows = (long long)p.B * p.H * p.n_new;
+  dim3 grid((unsigned)((rows + 15) / 16), 2);
+  if (p.in_bf16)
+    quantize_rows_kernel<true><<<grid, 256, 0, st>>>(p);
+  else
+    quantize_rows_kernel<false><<<grid, 256, 0, st>>>(p);
+  count_launches(1);
+  if (p.paged) {
+    seq_lens_advance_kernel<<<(p.B + 255) / 256, 256, 0, st>>>(p);
+    count_launches(1);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const DequantParams& p, cudaStream_t st) {
+  const long long rows = (long long)p.B * p.H * p.T_out;
+  if (rows == 0) return cudaSuccess;
+  dequantize_kernel<<<(unsigned)((rows + 15) / 16), 256, 0, st>>>(p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace kvq

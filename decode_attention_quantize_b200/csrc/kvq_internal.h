@@ -1,0 +1,96 @@
+// Kernel parameter blocks and launchers shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+struct AppendParams {
+  int B, H, n_new;
+  int k_scheme, v_scheme;
+  int in_bf16;
+  int paged, cap, page_size, max_pages, num_pages;
+  int pos0;  // dense: first position written (quantized tokens so far)
+  int rcap;
+  const void* k_new;
+  const void* v_new;
+  const int32_t* new_lens;
+  void* k_codes;
+  void* v_codes;
+  float* k_scale;
+  float* k_zero;
+  float* v_scale;
+  float* v_zero;
+  uint8_t* k_zp;
+  uint8_t* v_zp;
+  uint16_t* k_res;
+  uint16_t* v_res;
+  const int32_t* page_table;
+  int32_t* seq_lens;
+  uint32_t* status;
+};
+
+struct DequantParams {
+  int B, H, T_out, which, scheme;
+  int paged, cap, page_size, max_pages, num_pages;
+  int len_q, len_res, rcap;
+  const uint8_t* codes;
+  const float* scale;
+  const float* zero;
+  const uint8_t* zp;
+  const uint16_t* res;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  uint32_t* status;
+  float* out;
+};
+
+struct DecodeParams {
+  int B, Hq, Hkv, G, HG;        // G = Hq / Hkv, HG = ceil(G / 8) head groups of 8
+  int k_scheme, v_scheme;
+  int paged, cap, page_size, max_pages, num_pages;
+  int len_q, len_res, rcap;     // dense lengths (uniform over the batch)
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const float* k_scale;
+  const float* k_zero;
+  const float* v_scale;
+  const float* v_zero;
+  const uint8_t* k_zp;
+  const uint8_t* v_zp;
+  const uint16_t* k_res;
+  const uint16_t* v_res;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  uint32_t* status;
+  const void* q;
+  int q_bf16;
+  float softmax_scale;
+  float* out;
+  float* lse;
+  // workspace
+  float* part_o;                // [slots, 8, 128]
+  float* part_ml;               // [slots, 8, 2]
+  int32_t* plan;                // paged: [B + 1] tile prefix over sequences
+  int ncta;
+  int n_pairs;
+  int ts;                       // tokens per quantized tile of the chosen kernel
+  int nq, nr;                   // dense: quantized / residual tiles per pair
+};
+
+constexpr int kMaxCtas = 1024;
+
+// Count of kernel launches issued by the library (reported by kvq_launch_count).
+void count_launches(int n);  // decode grid bound used to size the workspace
+
+cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
+                          int flushed, int r_new, cudaStream_t st);
+cudaError_t launch_dequantize(const DequantParams& p, cudaStream_t st);
+// Returns cudaErrorNotSupported when the (k_scheme, v_scheme, layout) pair has no kernel.
+cudaError_t launch_decode(DecodeParams p, cudaStream_t st);
+bool decode_supported(int k_scheme, int v_scheme, int paged);
+
+}  // namespace kvq

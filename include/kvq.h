@@ -30,6 +30,12 @@ extern "C" {
 
 #define KVQ_ABI_VERSION 1
 
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
 typedef enum kvq_status {
   KVQ_OK = 0,
   KVQ_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, bad enum value */
@@ -125,17 +131,17 @@ typedef struct kvq_footprint {
   double bytes_per_token;    /* codes + per-token share of metadata + residual, per kv_head row pair */
 } kvq_footprint;
 
-int kvq_abi_version(void);
-const char* kvq_status_string(kvq_status s);
+KVQ_API int kvq_abi_version(void);
+KVQ_API const char* kvq_status_string(kvq_status s);
 
 /* Check a descriptor's fields (shapes, enums, pointer presence). No device access. */
-kvq_status kvq_validate(const kvq_cache_desc* desc);
+KVQ_API kvq_status kvq_validate(const kvq_cache_desc* desc);
 
 /* Bytes the cache arrays take (n4n.ai Step 6 "peak memory"; llms.blog memory-per-token). */
-kvq_status kvq_cache_bytes(const kvq_cache_desc* desc, kvq_footprint* out);
+KVQ_API kvq_status kvq_cache_bytes(const kvq_cache_desc* desc, kvq_footprint* out);
 
 /* Workspace kvq_quantize_append needs for `flags` (0 unless KVQ_APPEND_CALIBRATE). */
-size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t flags);
+KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t flags);
 
 /*
  * Quantize n_new tokens per sequence and append them ("QuantizedKVCache.append",
@@ -152,7 +158,7 @@ size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t flags);
  * page_table[b][pos / page_size], slot pos % page_size; seq_lens is advanced on the device.
  * The caller assigns page_table entries before the call.
  */
-kvq_status kvq_quantize_append(kvq_cache_desc* desc, const void* k_new, const void* v_new,
+KVQ_API kvq_status kvq_quantize_append(kvq_cache_desc* desc, const void* k_new, const void* v_new,
                                int32_t in_dtype, int32_t n_new, const int32_t* new_lens,
                                uint32_t flags, void* workspace, size_t workspace_bytes,
                                void* stream);
@@ -163,11 +169,11 @@ kvq_status kvq_quantize_append(kvq_cache_desc* desc, const void* k_new, const vo
  * order: quantized tokens, then the KIVI residual. Rows at or past a sequence's length
  * are written as zero. out_tokens must be >= every sequence's length.
  */
-kvq_status kvq_dequantize(const kvq_cache_desc* desc, int32_t which, float* out,
+KVQ_API kvq_status kvq_dequantize(const kvq_cache_desc* desc, int32_t which, float* out,
                           int32_t out_tokens, void* stream);
 
 /* Workspace kvq_decode_attention needs (split partials and the paged plan). */
-size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc);
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc);
 
 /*
  * Decode attention of one query token per sequence over the quantized cache, reading the
@@ -181,12 +187,15 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc);
  * softmax_scale * q.k over all tokens of the sequence (no mask). A sequence with no
  * tokens gives zeros and lse = -inf.
  */
-kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* q, int32_t q_dtype,
+KVQ_API kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* q, int32_t q_dtype,
                                 float softmax_scale, float* out, float* lse, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Number of kernels this process has launched through the library (all entry points). */
+KVQ_API uint64_t kvq_launch_count(void);
+
 /* Copy dev_status[0..1] to host out[2] (synchronises `stream`); clear != 0 zeroes them. */
-kvq_status kvq_get_device_status(const kvq_cache_desc* desc, uint32_t* out, int32_t clear,
+KVQ_API kvq_status kvq_get_device_status(const kvq_cache_desc* desc, uint32_t* out, int32_t clear,
                                  void* stream);
 
 #ifdef __cplusplus

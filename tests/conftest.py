@@ -26,3 +26,20 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    try:
+        from tests import harness
+    except Exception:
+        return
+    if harness.ERRORS:
+        worst = max(e for _, e in harness.ERRORS)
+        terminalreporter.write_line(
+            f"attention parity: {len(harness.ERRORS)} comparisons, worst max|err|/max|ref| = {worst:.3e} "
+            f"(bound {harness.ATTN_RTOL})")
+        out = os.environ.get("KVQ_PARITY_REPORT")
+        if out:
+            import json
+            with open(out, "w") as fh:
+                json.dump(harness.ERRORS, fh, indent=0)

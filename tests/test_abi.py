@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every symbol its header declares, and rejects bad
+arguments on the host before touching a device (no compute calls here)."""
+import ctypes
+import re
+import os
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]*?\b(kvq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = _declared()
+    for must in ("kvq_quantize_append", "kvq_dequantize", "kvq_decode_attention"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    from decode_attention_quantize_b200 import kvq
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert sorted(kvq.EXPORTS) == _declared()
+    assert lib.kvq_abi_version() == 1
+
+
+def _desc(**kw):
+    from decode_attention_quantize_b200.kvq import KvqDesc
+    d = KvqDesc()
+    d.batch, d.num_q_heads, d.num_kv_heads, d.head_dim = 2, 8, 2, 128
+    d.k_scheme = d.v_scheme = 0
+    d.layout, d.capacity = 0, 256
+    d.group_size, d.residual_cap = 32, 128
+    fake = 0x10000  # never dereferenced: validation is host-only
+    for f in ("k_codes", "v_codes", "k_scale", "v_scale", "dev_status"):
+        setattr(d, f, fake)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_validation_is_host_side():
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    ok = _desc()
+    assert L.kvq_validate(ctypes.byref(ok)) == kvq.KVQ_OK
+    cases = [
+        (dict(head_dim=64), kvq.KVQ_ERR_UNSUPPORTED),
+        (dict(num_q_heads=7), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(capacity=200), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(k_scheme=9), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(k_scheme=5, v_scheme=6), kvq.KVQ_ERR_UNSUPPORTED),
+        (dict(k_codes=None), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(k_codes=0x10004), kvq.KVQ_ERR_INVALID_ARG),   # not 16-byte aligned
+        (dict(layout=1, page_size=16, max_pages_per_seq=4, num_pages=8), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(layout=1, page_size=24, max_pages_per_seq=4, num_pages=8, page_table=0x10000, seq_lens=0x10000),
+         kvq.KVQ_ERR_UNSUPPORTED),
+        (dict(v_scheme=4), kvq.KVQ_ERR_INVALID_ARG),          # asym needs a zero-point array
+        (dict(k_scheme=5, v_scheme=5), kvq.KVQ_ERR_INVALID_ARG),  # KIVI needs minima and residual
+    ]
+    for kw, want in cases:
+        d = _desc(**kw)
+        assert L.kvq_validate(ctypes.byref(d)) == want, kw
+
+
+def test_append_and_decode_reject_before_launch():
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    d = _desc(num_quantized=250)
+    buf = 0x20000
+    # capacity: 250 + 8 > 256
+    st = L.kvq_quantize_append(ctypes.byref(d), buf, buf, kvq.KVQ_BF16, 8, None, 0, None, 0, None)
+    assert st == kvq.KVQ_ERR_CAPACITY and d.num_quantized == 250
+    # calibration without workspace
+    d2 = _desc()
+    st = L.kvq_quantize_append(ctypes.byref(d2), buf, buf, kvq.KVQ_BF16, 8, None, kvq.KVQ_APPEND_CALIBRATE,
+                               None, 0, None)
+    assert st == kvq.KVQ_ERR_WORKSPACE and d2.num_quantized == 0
+    # KIVI takes bf16 only
+    d3 = _desc(k_scheme=5, v_scheme=5, k_zero=buf, v_zero=buf, k_res=buf, v_res=buf)
+    st = L.kvq_quantize_append(ctypes.byref(d3), buf, buf, kvq.KVQ_F32, 8, None, 0, None, 0, None)
+    assert st == kvq.KVQ_ERR_UNSUPPORTED
+    # per-sequence counts are for the paged layout only
+    st = L.kvq_quantize_append(ctypes.byref(d2), buf, buf, kvq.KVQ_BF16, 8, buf, 0, None, 0, None)
+    assert st == kvq.KVQ_ERR_INVALID_ARG
+    # decode: workspace too small, bad dtype, bad scale
+    need = L.kvq_decode_workspace_bytes(ctypes.byref(d2))
+    assert need > 0
+    assert L.kvq_decode_attention(ctypes.byref(d2), buf, 1, ctypes.c_float(0.088), buf, None, buf, need - 1,
+                                  None) == kvq.KVQ_ERR_WORKSPACE
+    assert L.kvq_decode_attention(ctypes.byref(d2), buf, 7, ctypes.c_float(0.088), buf, None, buf, need,
+                                  None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attention(ctypes.byref(d2), buf, 1, ctypes.c_float(-1.0), buf, None, buf, need,
+                                  None) == kvq.KVQ_ERR_INVALID_ARG
+    # dequantize needs room for every token
+    d4 = _desc(num_quantized=100)
+    assert L.kvq_dequantize(ctypes.byref(d4), 0, buf, 99, None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_status_string(kvq.KVQ_ERR_CAPACITY) == b"cache capacity exceeded"
+
+
+def test_footprint_matches_the_pages_per_token_bytes():
+    # 70B shape, one layer: 8 KV heads x 128 channels. BF16 would take 2 * 2 * 8 * 128 bytes per
+    # token per layer; FP8 codes take half of that and INT4 a quarter (memory table, infra.bea.ai).
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    d = _desc(batch=1, num_q_heads=64, num_kv_heads=8, capacity=4096)
+    f = kvq.KvqFootprint()
+    assert L.kvq_cache_bytes(ctypes.byref(d), ctypes.byref(f)) == kvq.KVQ_OK
+    assert f.code_bytes == 4096 * 2 * 8 * 128 and f.bytes_per_token == 2 * 128
+    assert f.code_bytes * 80 / 4096 == 163840  # FP8 row of the memory table: 160 KiB per token
+    buf = 0x30000
+    d5 = _desc(batch=1, num_q_heads=64, num_kv_heads=8, capacity=4096, k_scheme=5, v_scheme=5, k_zero=buf,
+               v_zero=buf, k_res=buf, v_res=buf)
+    assert L.kvq_cache_bytes(ctypes.byref(d5), ctypes.byref(f)) == kvq.KVQ_OK
+    assert f.code_bytes * 80 / 4096 == 81920  # INT4 codes: 80 KiB per token for 80 layers
+    assert f.bytes_per_token == 2 * 64 + 2 * 8 * 4  # codes + fp32 (scale, min) per 32 elements

@@ -1,0 +1,165 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Codes, scales, zero points and residual tokens must match bit for bit; decode attention
+must satisfy max|err| <= 2e-4 * max|ref| against the fp64 oracle on the same cache.
+Sizes span several tiles with ragged tails; every scheme pair, both layouts, GQA group
+sizes 1, 4, 8 and 16, streaming appends and the KIVI flush boundary are covered.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+S = synth
+
+
+# ------------------------------------------------------------------ dense, 8-bit schemes
+@pytest.mark.parametrize("ks,vs", [
+    (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR),
+    (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TENSOR),
+    (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN),
+    (S.INT8_SYM_PER_CHANNEL, S.INT8_SYM_PER_CHANNEL),
+    (S.UINT8_ASYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL),
+    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
+    (S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL),
+])
+def test_dense_8bit_schemes(ks, vs):
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=ks, vs=vs, prefill=300, steps=2)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_gqa_group_sizes(G):
+    H.dense_case(B=2, Hq=2 * G, Hkv=2, ks=S.FP8_E4M3_PER_TENSOR, vs=S.FP8_E4M3_PER_TENSOR, prefill=200, steps=1)
+
+
+def test_fp32_inputs_and_queries():
+    # fp32 K/V/Q (the tiny configuration's input type); Q needs the hi/lo split
+    H.dense_case(B=1, Hq=4, Hkv=1, ks=S.INT8_SYM_PER_TOKEN, vs=S.INT8_SYM_PER_TOKEN, prefill=257, steps=2,
+                 bf16=False, rope=0.0)
+    H.dense_case(B=2, Hq=8, Hkv=2, ks=S.FP8_E4M3_PER_TENSOR, vs=S.FP8_E4M3_PER_TENSOR, prefill=130, steps=1,
+                 bf16=True, q_bf16=False)
+
+
+def test_tiny_int8_configuration_full_size():
+    w = synth.workloads()["tiny_int8"]
+    _, _, err = H.dense_case(B=w.B, Hq=w.Hq, Hkv=w.Hkv, ks=w.k_scheme, vs=w.v_scheme, prefill=w.context,
+                             steps=0, bf16=False, seed=w.seed, outlier=w.outlier_scale, rope=w.rope_theta)
+    assert err <= H.ATTN_RTOL
+
+
+def test_single_token_and_chunked_prefill():
+    H.dense_case(B=1, Hq=8, Hkv=1, ks=S.FP8_E4M3_PER_TENSOR, vs=S.FP8_E4M3_PER_TENSOR, prefill=1, steps=3)
+    H.dense_case(B=2, Hq=8, Hkv=2, ks=S.INT8_SYM_PER_TOKEN, vs=S.INT8_SYM_PER_TOKEN, prefill=333, steps=1,
+                 chunks=[17, 200])
+
+
+def test_outliers_x100_int8_per_channel():
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=S.INT8_SYM_PER_CHANNEL, vs=S.UINT8_ASYM_PER_CHANNEL, prefill=190, steps=1,
+                 outlier=100.0)
+
+
+# ------------------------------------------------------------------ KIVI
+@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2])
+@pytest.mark.parametrize("prefill", [44, 128, 129, 300, 384, 385])
+def test_kivi_prefill_and_stream(scheme, prefill):
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=scheme, vs=scheme, prefill=prefill, steps=2, cap=640)
+
+
+@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2])
+def test_kivi_flush_on_stream_boundary(scheme):
+    # 127 + 1 fills the residual; the next token flushes 128 tokens into 4 key groups
+    H.dense_case(B=1, Hq=8, Hkv=1, ks=scheme, vs=scheme, prefill=127, steps=3, cap=256)
+    H.dense_case(B=2, Hq=8, Hkv=2, ks=scheme, vs=scheme, prefill=256, steps=2, cap=512, outlier=100.0)
+
+
+def test_kivi_chunked_appends_match_bulk():
+    H.dense_case(B=1, Hq=16, Hkv=2, ks=S.KIVI_INT4, vs=S.KIVI_INT4, prefill=400, steps=1, cap=512,
+                 chunks=[5, 100, 260])
+
+
+# ------------------------------------------------------------------ paged
+@pytest.mark.parametrize("ks,vs,ps", [
+    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL, 16),
+    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL, 32),
+    (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR, 16),
+    (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN, 64),
+    (S.INT8_SYM_PER_CHANNEL, S.INT8_SYM_PER_CHANNEL, 16),
+])
+def test_paged(ks, vs, ps):
+    B, Hq, Hkv = 4, 16, 4
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, ks, vs, lens=[37, 100, 5, 64], page_size=ps,
+                                                    steps=3)
+    oc.append(K, V, True, calibrate=calib, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=calib)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc, "prefill")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), True, "paged decode 0")
+    for s in range(3):
+        kk = np.stack([synth.keys(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(B)])
+        vv = np.stack([synth.values(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(B)])
+        oc.append(kk, vv, True)
+        gc.append(H.dev(kk, True), H.dev(vv, True))
+        torch.cuda.synchronize()
+        H.compare_paged(oc, gc, f"step {s}")
+        H.decode_both(oc, gc, synth.queries(w, s + 1, 0, B), True, f"paged decode {s + 1}")
+    assert gc.status()[0] == 0
+
+
+def test_paged_empty_sequence_and_variable_lengths():
+    B, Hq, Hkv = 3, 8, 2
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL,
+                                                    lens=[0, 250, 1], steps=0)
+    oc.append(K, V, True, calibrate=True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc)
+    q = synth.queries(w, 0, 0, B)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    out, _ = gc.decode(H.dev(q, True), float(H.SCALE), lse=lse)
+    ref, ref_lse = oc.decode(q, True, float(H.SCALE))
+    torch.cuda.synchronize()
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))  # empty sequence
+    H.attn_check(out, ref, lse, ref_lse, "variable lengths")
+    assert np.abs(ref[1]).max() > 0
+
+
+def test_bad_page_id_is_flagged_not_dereferenced():
+    B, Hq, Hkv = 2, 8, 2
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL,
+                                                    lens=[40, 40], steps=0, bad_page=(1, 1))
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
+    out, _ = gc.decode(H.dev(synth.queries(w, 0, 0, B), True), float(H.SCALE))
+    torch.cuda.synchronize()
+    st = gc.status(clear=True)
+    assert st[0] & H.kvq().KVQ_DEV_BAD_PAGE
+    assert torch.isfinite(out).all()
+    assert gc.status()[0] == 0
+
+
+def test_saturation_is_counted():
+    # fixed per-tensor scale from a small prefill; a later token 50x larger saturates
+    B, Hq, Hkv = 1, 8, 1
+    gc = H.kvq().QuantizedKVCache(H.kvq().CacheSpec(B, Hq, Hkv, S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TENSOR,
+                                                    capacity=128))
+    x = torch.randn(B, Hkv, 4, 128, device="cuda", dtype=torch.float32)
+    gc.append(x, x, calibrate=True)
+    big = x[:, :, :1] * 50
+    gc.append(big.contiguous(), big.contiguous())
+    torch.cuda.synchronize()
+    assert gc.status()[1] > 0
+
+
+# ------------------------------------------------------------------ dequantize
+@pytest.mark.parametrize("ks,vs", [(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.KIVI_INT2, S.KIVI_INT2),
+                                   (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL)])
+def test_dequantize_matches_oracle(ks, vs):
+    oc, gc, _ = H.dense_case(B=2, Hq=8, Hkv=2, ks=ks, vs=vs, prefill=200, steps=1, cap=384)
+    T = oc.tokens()
+    for which in (0, 1):
+        got = gc.dequantize(which, T + 3).cpu().numpy()
+        ref = oc.dequantize(which, T + 3)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), f"dequantize side {which}"
