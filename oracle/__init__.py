@@ -89,6 +89,8 @@ def load(path: str):
     L.oq_kivi_value.restype = f32
     L.oq_append.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp, i32]
     L.oq_append.restype = i32
+    L.oq_calibrate.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp]
+    L.oq_calibrate.restype = i32
     L.oq_tokens.argtypes = [ctypes.POINTER(_Cache), i32]
     L.oq_tokens.restype = i32
     L.oq_dequantize.argtypes = [ctypes.POINTER(_Cache), i32, vp, i32]
@@ -229,6 +231,15 @@ class OracleCache:
                              _ptr(nl), int(bool(calibrate)))
         if rc != 0:
             raise ValueError("oracle append rejected the call (capacity or arguments)")
+
+    def calibrate(self, k, v, bf16: bool, new_lens=None):
+        """Scales of the calibrating append for block k, v (nothing is quantized)."""
+        k = np.ascontiguousarray(k)
+        v = np.ascontiguousarray(v)
+        nl = None if new_lens is None else np.ascontiguousarray(new_lens, np.int32)
+        if lib().oq_calibrate(ctypes.byref(self.c), k.ctypes.data, v.ctypes.data, int(bf16), k.shape[2],
+                              _ptr(nl)) != 0:
+            raise ValueError("oracle calibrate rejected the call")
 
     def dequantize(self, which: int, T_out: int) -> np.ndarray:
         out = np.zeros((self.B, self.Hkv, T_out, self.D), np.float32)

@@ -436,6 +436,16 @@ int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, in
   return 0;
 }
 
+int oq_calibrate(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
+                 const int32_t* new_lens) {
+  block kb = {k_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
+  block vb = {v_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
+  if (is_kivi(c->k_scheme) || is_kivi(c->v_scheme)) return -1;
+  calibrate(c, &kb, c->k_scheme, c->k_scale, c->k_zp);
+  calibrate(c, &vb, c->v_scheme, c->v_scale, c->v_zp);
+  return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* dequantize                                                                */
 /* ------------------------------------------------------------------------- */

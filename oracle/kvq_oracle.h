@@ -77,6 +77,11 @@ typedef struct {
 int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
               const int32_t* new_lens, int calibrate);
 
+/* Only the calibration of oq_append: recompute the per-tensor / per-channel scales of the
+ * cache from the block (same arguments), quantize nothing. */
+int oq_calibrate(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
+                 const int32_t* new_lens);
+
 /* Tokens visible to decode for sequence b. */
 int oq_tokens(const oq_cache* c, int b);
 

@@ -497,3 +497,20 @@ def test_capacity_errors():
     x = np.zeros((1, 1, 5, 8), np.float32)
     with pytest.raises(ValueError):
         c.append(x, x, bf16=False)
+
+
+def test_calibrate_only_equals_calibrating_append():
+    rng = np.random.default_rng(13)
+    B, H, T, D = 3, 2, 9, 16
+    k = rng.normal(0, 2, (B, H, T, D)).astype(np.float32)
+    v = rng.normal(0.5, 1, (B, H, T, D)).astype(np.float32)
+    lens = np.array([9, 4, 0], np.int32)
+    table = np.arange(3 * 4, dtype=np.int32).reshape(3, 4)
+    mk = lambda: OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, paged=True,
+                             page_size=4, max_pages=4, num_pages=12, page_table=table)
+    a, b = mk(), mk()
+    a.append(k, v, bf16=False, calibrate=True, new_lens=lens)
+    b.calibrate(k, v, bf16=False, new_lens=lens)
+    for name in ("k_scale", "v_scale", "v_zp"):
+        assert np.array_equal(a[name], b[name]), name
+    assert not b["k_codes"].any() and not b["seq_lens"].any()
