@@ -183,6 +183,28 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml" if self.nv else "unavailable"}
 
 
+# ---------------------------------------------------------------- multi-rank plumbing
+def rank_workload(w, rank):
+    """Weak scaling: rank r runs the whole per-GPU workload on its own seeded batch."""
+    return synth.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def max_over_ranks(seconds, world, device=None):
+    """Slowest rank's timed interval (the job's time); a no-op for one process."""
+    if world <= 1:
+        return float(seconds)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(seconds)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(step_bytes, steps, t_max_total, world):
+    """Whole-job GB/s: every rank processed `steps` steps of `step_bytes` in t_max_total."""
+    return world * step_bytes * steps / t_max_total / 1e9
+
+
 # ---------------------------------------------------------------- GPU workload
 class GpuWorkload:
     """Builds one layer's cache for a workload and exposes a graph-captured decode step."""
@@ -191,7 +213,7 @@ class GpuWorkload:
         import torch
         from decode_attention_quantize_b200 import kvq
         self.torch, self.kvq, self.w, self.dev = torch, kvq, w, device
-        self.seed_w = synth.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+        self.seed_w = rank_workload(w, rank)
         W = self.seed_w
         if W.paged:
             self._build_paged(W)
@@ -391,10 +413,7 @@ def run_gpu(args, rank, world, local_rank):
     lens_d, res_d = G.decode_lens(args.warmup + args.steps)  # state seen by the decode-only timing
     dbytes_dec = decode_bytes(W, lens_d, res_d)
     abytes = append_bytes(W) if G.append_token else 0.0
-    total_time = torch.tensor([sum(step_ms) / 1e3], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(total_time, op=dist.ReduceOp.MAX)
-    t_max = float(total_time.item()) / args.steps
+    t_max = max_over_ranks(sum(step_ms) / 1e3, world, device=dev) / args.steps
 
     # end to end through the public API: host inputs (pinned) -> device -> step -> host out
     e2e = run_e2e(G, W, stream, flush, n=min(200, args.steps), step0=args.warmup + args.steps)
@@ -549,7 +568,7 @@ def main():
     r = run_gpu(args, rank, world, local_rank)
     W = r["W"]
     step_bytes = r["dbytes"] + r["abytes"]
-    value = world * step_bytes / r["t_max"] / 1e9
+    value = job_value(step_bytes, args.steps, r["t_max"] * args.steps, world)
     tokens_per_s = world * W.B / r["t_max"]
     peak, peak_kind = measured_peak()
     achieved = r["dbytes_dec"] / r["t_dec"] / 1e9
