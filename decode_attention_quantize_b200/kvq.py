@@ -35,7 +35,9 @@ EXPORTS = [
     "kvq_abi_version", "kvq_status_string", "kvq_validate", "kvq_cache_bytes",
     "kvq_append_workspace_bytes", "kvq_quantize_append", "kvq_dequantize",
     "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_get_device_status", "kvq_launch_count",
+    "kvq_decode_attention_noalloc",
 ]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class KvqDesc(ctypes.Structure):
@@ -82,6 +84,8 @@ def _load():
     L.kvq_decode_attention.argtypes = [P, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.kvq_get_device_status.argtypes = [P, vp, i32, vp]
     L.kvq_launch_count.restype = ctypes.c_uint64
+    L.kvq_decode_attention_noalloc.argtypes = [P, vp, i32, ctypes.c_float, vp, vp, vp]
+    L.kvq_decode_attention_noalloc.restype = ctypes.c_int
     for name in ("kvq_validate", "kvq_cache_bytes", "kvq_quantize_append", "kvq_dequantize",
                  "kvq_decode_attention", "kvq_get_device_status"):
         getattr(L, name).restype = ctypes.c_int
@@ -168,6 +172,18 @@ def kvq_decode_attention(desc: KvqDesc, q, softmax_scale: float, out=None, lse=N
                                     _ptr(out), _ptr(lse), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
            "kvq_decode_attention")
+    return out, lse
+
+
+def kvq_decode_attention_noalloc(desc: KvqDesc, q, softmax_scale: float, out=None, lse=None, stream=None):
+    """kvq_decode_attention without a workspace: for callers that cannot allocate device
+    memory (the library's static scratch array holds the partials; see include/kvq.h)."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    _check(lib.kvq_decode_attention_noalloc(ctypes.byref(desc), _ptr(q), _dtype_code(q), float(softmax_scale),
+                                            _ptr(out), _ptr(lse), _stream(stream)),
+           "kvq_decode_attention_noalloc")
     return out, lse
 
 

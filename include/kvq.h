@@ -194,6 +194,27 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* 
 /* Number of kernels this process has launched through the library (all entry points). */
 KVQ_API uint64_t kvq_launch_count(void);
 
+/*
+ * Decode attention that allocates nothing and takes no workspace. The paper has no
+ * counterpart; this exists for callers that cannot call cudaMalloc: an inference-engine
+ * plugin handed only its input and output buffers, code running while a CUDA graph is
+ * being captured (a new allocation is not allowed there), or a serving loop that forbids
+ * allocation after start-up so it never synchronises the device or fragments its pool.
+ *
+ * The split partials live in a static device array of KVQ_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads the library holds until the process exits. A cache whose
+ * kvq_decode_workspace_bytes exceeds that size is rejected with KVQ_ERR_WORKSPACE
+ * before any launch. The first call on a device looks up the array's device address
+ * (with that device current), so make the first call on each device before any stream
+ * capture. Every call shares the one array: calls that overlap on the GPU (different
+ * streams, or devices sharing a context) race, so serialise them. The array keeps the
+ * previous call's contents; nothing in it needs to start at zero. Arguments and results
+ * are those of kvq_decode_attention.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+KVQ_API kvq_status kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, int32_t q_dtype,
+                                                float softmax_scale, float* out, float* lse, void* stream);
+
 /* Copy dev_status[0..1] to host out[2] (synchronises `stream`); clear != 0 zeroes them. */
 KVQ_API kvq_status kvq_get_device_status(const kvq_cache_desc* desc, uint32_t* out, int32_t clear,
                                  void* stream);
