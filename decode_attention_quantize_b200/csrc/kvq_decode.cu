@@ -77,7 +77,8 @@ struct Cfg {
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
-  static constexpr int kStages = kKivi ? 3 : 4;
+  static constexpr int kStages = kKivi ? 3 : 3;
+  static constexpr int kMinBlocks = kKivi ? 2 : 3;  // resident CTAs per SM the registers are sized for
   static constexpr int kOffDesc = kStages * kStageBytes;
   static constexpr int kOffBar = kOffDesc + kStages * 64;
   static constexpr int kOffRedO = kOffBar + 2 * kStages * 8 + 64;
@@ -112,35 +113,66 @@ __device__ __forceinline__ Sched make_sched(const DecodeParams& p) {
   return s;
 }
 
-__device__ __forceinline__ TileDesc locate(const DecodeParams& p, const Sched& s, int t, int tb, int te) {
-  TileDesc d;
-  int j, npt;
-  if (p.paged) {
-    int lo = 0, hi = p.B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.plan[mid] <= t) lo = mid; else hi = mid - 1;
+// Walks a CTA's contiguous range of the flattened tile list without per-tile divisions.
+struct TileIter {
+  int t, tb, te;
+  int b, hh, j, npt;  // sequence, (kv head, head group) index in the sequence, tile in pair, tiles per pair
+  int L;              // paged: sequence length
+
+  __device__ __forceinline__ void init(const DecodeParams& p, const Sched& s, int tb_, int te_) {
+    t = tb = tb_;
+    te = te_;
+    L = 0;
+    if (p.paged) {
+      int lo = 0, hi = p.B - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.plan[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      b = lo;
+      npt = (p.plan[lo + 1] - p.plan[lo]) / s.per_seq;
+      const int local = t - p.plan[lo];
+      hh = local / npt;
+      j = local % npt;
+      L = p.plan[p.B + 1 + lo];
+    } else {
+      npt = p.nq + p.nr;
+      const int pair = t / npt;
+      j = t % npt;
+      b = pair / s.per_seq;
+      hh = pair % s.per_seq;
     }
-    d.b = lo;
-    npt = (p.plan[lo + 1] - p.plan[lo]) / s.per_seq;
-    const int local = t - p.plan[lo];
-    const int hh = local / npt;
-    j = local % npt;
-    d.pair = lo * s.per_seq + hh;
-    d.hk = hh / p.HG;
-    d.hg = hh % p.HG;
-    d.kind = 0;
-    d.t0 = j * p.ts;
-    d.n = min(p.ts, p.plan[p.B + 1 + lo] - d.t0);
-  } else {
-    npt = p.nq + p.nr;
-    d.pair = t / npt;
-    j = t % npt;
-    d.b = d.pair / s.per_seq;
-    const int hh = d.pair % s.per_seq;
-    d.hk = hh / p.HG;
-    d.hg = hh % p.HG;
-    if (j < p.nq) {
+  }
+
+  __device__ __forceinline__ void next(const DecodeParams& p, const Sched& s) {
+    ++t;
+    if (++j < npt) return;
+    j = 0;
+    if (++hh < s.per_seq) return;
+    hh = 0;
+    ++b;
+    if (p.paged && t < te) {
+      while ((npt = (p.plan[b + 1] - p.plan[b]) / s.per_seq) == 0) ++b;  // skip empty sequences
+      L = p.plan[p.B + 1 + b];
+    }
+  }
+
+  __device__ __forceinline__ TileDesc desc(const DecodeParams& p, const Sched& s) const {
+    TileDesc d;
+    d.b = b;
+    d.pair = b * s.per_seq + hh;
+    if (p.HG == 1) {
+      d.hk = hh;
+      d.hg = 0;
+    } else {
+      d.hk = hh / p.HG;
+      d.hg = hh - d.hk * p.HG;
+    }
+    if (p.paged) {
+      d.kind = 0;
+      d.t0 = j * p.ts;
+      d.n = min(p.ts, L - d.t0);
+    } else if (j < p.nq) {
       d.kind = 0;
       d.t0 = j * p.ts;
       d.n = min(p.ts, p.len_q - d.t0);
@@ -149,12 +181,12 @@ __device__ __forceinline__ TileDesc locate(const DecodeParams& p, const Sched& s
       d.t0 = (j - p.nq) * kRT;
       d.n = min(kRT, p.len_res - d.t0);
     }
+    d.first = (t == tb) || (j == 0);
+    d.last = (t == te - 1) || (j == npt - 1);
+    d.valid = 0xFFFFFFFFu;
+    return d;
   }
-  d.first = (t == tb) || (j == 0);
-  d.last = (t == te - 1) || (j == npt - 1);
-  d.valid = 0xFFFFFFFFu;
-  return d;
-}
+};
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -180,16 +212,22 @@ template <class C>
 __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                          uint8_t* stages, TileDesc* descs, uint32_t full0, uint32_t empty0,
                          const Sched& s, int tb, int te) {
-  for (int t = tb, it = 0; t < te; ++t, ++it) {
-    const int st = it % C::kStages;
-    if (it >= C::kStages && !mbar_wait(empty0 + 8 * st, ((it / C::kStages) - 1) & 1, p.status)) return;
-    TileDesc d = locate(p, s, t, tb, te);
-    const uint32_t sb = smem_addr(stages + st * C::kStageBytes);
-    const uint32_t bar = full0 + 8 * st;
+  TileIter ti;
+  ti.init(p, s, tb, te);
+  for (int it = 0, st = 0, phase = 0; ti.t < te; ti.next(p, s), ++it) {
+    if (it >= C::kStages && !mbar_wait(empty0 + 8 * st, phase ^ 1, p.status)) return;
+    TileDesc d = ti.desc(p, s);
+    const int cur = st;
+    if (++st == C::kStages) {
+      st = 0;
+      phase ^= 1;
+    }
+    const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
+    const uint32_t bar = full0 + 8 * cur;
     const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
     if (d.kind == 1) {  // KIVI residual: bf16 rows, whole 32-token slab (inside rcap)
       const size_t r0 = (pair_row * p.rcap + d.t0) * kHeadDim;
-      descs[st] = d;
+      descs[cur] = d;
       mbar_arrive_expect_tx(bar, 2 * kRT * kHeadDim * 2);
       bulk_g2s(sb, p.k_res + r0, kRT * kHeadDim * 2, bar);
       bulk_g2s(sb + kRT * kHeadDim * 2, p.v_res + r0, kRT * kHeadDim * 2, bar);
@@ -199,7 +237,7 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       // whole tile: capacity is a multiple of 128 tokens, so the tile lies inside the row
       const size_t row0 = pair_row * p.cap + d.t0;
       const uint32_t bytes = C::kTS * (C::kKRow + C::kVRow) + C::kKMeta + C::kVMeta;
-      descs[st] = d;
+      descs[cur] = d;
       mbar_arrive_expect_tx(bar, bytes);
       tma_2d(sb + C::kOffK, tk, 0, (int)row0, bar);
       tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar);
@@ -236,7 +274,7 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
         }
       }
       d.valid = valid;
-      descs[st] = d;
+      descs[cur] = d;
       uint32_t per_page = ps * (C::kKRow + C::kVRow);
       if constexpr (C::kKFold == FOLD_TOKEN) per_page += ps * 4;
       if constexpr (C::kVFold == FOLD_TOKEN) per_page += ps * 4;
@@ -272,15 +310,19 @@ __device__ __forceinline__ int dmap_v(int g, int mt, int rh) {
   return 16 * g + 2 * mt + rh;
 }
 
-// 16-bit piece (two 8-bit codes) -> f16x2 of the code values.
+// Bytes 0,1 (lo) and 2,3 (hi) of a word of 8-bit codes -> two f16x2 of the code values.
 template <int FMT>
-__device__ __forceinline__ uint32_t cvt8x2(uint32_t piece16, uint32_t zp_bias) {
+__device__ __forceinline__ void cvt8x4(uint32_t w, uint32_t zlo, uint32_t zhi, uint32_t& lo, uint32_t& hi) {
   if constexpr (FMT == FMT_E4M3) {
-    return e4m3x2_to_f16x2(piece16);
-  } else if constexpr (FMT == FMT_S8) {  // piece already XORed with 0x80: biased by 128
-    return hsub2_u(prmt(piece16, 0x64646464u, 0x5150u), 0x64806480u);  // - 1152
+    asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+  } else if constexpr (FMT == FMT_S8) {  // word already XORed with 0x80808080: codes biased by 128
+    lo = hsub2_u(prmt(w, 0x64646464u, 0x5150u), 0x64806480u);  // (1024 + 128 + q) - 1152
+    hi = hsub2_u(prmt(w, 0x64646464u, 0x5352u), 0x64806480u);
   } else {  // FMT_U8: subtract 1024 + zero point
-    return hsub2_u(prmt(piece16, 0x64646464u, 0x5150u), zp_bias);
+    lo = hsub2_u(prmt(w, 0x64646464u, 0x5150u), zlo);
+    hi = hsub2_u(prmt(w, 0x64646464u, 0x5352u), zhi);
   }
 }
 
@@ -311,10 +353,14 @@ __device__ __forceinline__ T lds(const uint8_t* p) {
   return *reinterpret_cast<const T*>(p);
 }
 
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
+  return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+
 // ------------------------------------------------------------------ consumer state
 template <class C>
 struct Consumer {
-  int w, lane, g, c;
+  int w, g, c;
   float o[8][4];
   float m[2], l[2];
   int ev;            // O accumulator holds (true value) * 2^ev
@@ -325,6 +371,7 @@ struct Consumer {
   float kmul;        // score multiplier (log2 domain)
   float bias[2];     // KIVI group bias (raw units), heads 2c, 2c+1
   int qmode;         // 0: fragments for codes built, 1: for bf16 residual rows
+  uint32_t zpk[8][2], zpv[8][2];  // uint8 asymmetric: f16x2 (1024 + zero point)
 };
 
 // Build Q' fragments (head g, this thread's channels) from q_s, optionally multiplied by
@@ -356,9 +403,357 @@ __device__ __forceinline__ int build_q(const float* q_s, const float* fold, int 
   return eq;
 }
 
+// ------------------------------------------------------------------ one tile, one warp
+// kMasked: the warp's tokens are not all valid (ragged tail or missing pages).
+template <class C, bool kMasked>
+__device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p, const uint8_t* base,
+                                          const TileDesc& d, uint32_t valid, bool residual, int tok_base,
+                                          float sc_log2, const float* q_s) {
+  const int g = S.g, c = S.c, w = S.w;
+  // validity of a token of this warp's range (tile-relative index)
+  auto tok_ok = [&](int tok) -> bool {
+    if constexpr (!kMasked) return true;
+    bool ok = tok < d.n;
+    if constexpr (C::kPaged) ok = ok && ((valid >> (tok / p.page_size)) & 1u);
+    return ok;
+  };
+
+  // (1) query fragments that change per tile (KIVI key groups, residual rows)
+  if constexpr (C::kKivi) {
+    if (!residual) {
+      const float* ksm = reinterpret_cast<const float*>(base + C::kOffKM) + w * kHeadDim;
+      const float* kzm = reinterpret_cast<const float*>(base + C::kOffKM + C::kKMeta / 2) + w * kHeadDim;
+      const int eq = build_q<C::kKFmt>(q_s, ksm, g, c, S.qh, S.ql);
+      float bs = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int dd = 32 * c + i;
+        bs = fmaf(q_s[g * 132 + dd + (dd >> 5)], kzm[dd], bs);
+      }
+      bs += __shfl_xor_sync(0xffffffffu, bs, 1);
+      bs += __shfl_xor_sync(0xffffffffu, bs, 2);
+      S.bias[0] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c));
+      S.bias[1] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c + 1));
+      S.kmul = pow2i(-eq);
+      S.qsplit = true;
+      S.qmode = 0;
+    } else if (S.qmode != 1) {
+      const int eq = build_q<FMT_S8>(q_s, nullptr, g, c, S.qh, S.ql);
+      S.kmul = sc_log2 * pow2i(-eq);
+      S.qsplit = !p.q_bf16;
+      S.qmode = 1;
+    }
+  }
+
+  // (2) S^T = K . Q'^T for kNSub blocks of 16 tokens; two accumulators halve the MMA chain
+  float acc[C::kNSub][4];
+#pragma unroll
+  for (int sb = 0; sb < C::kNSub; ++sb) {
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const int r0 = tok_base + sb * 16 + g, r1 = r0 + 8;
+    auto mma2 = [&](int ks, uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, bool split) {
+      float(&acc_k)[4] = (ks & 1) ? a1 : a0;
+      mma_16816(acc_k, x0, x1, x2, x3, S.qh[ks][0], S.qh[ks][1]);
+      if (split) mma_16816(acc_k, x0, x1, x2, x3, S.ql[ks][0], S.ql[ks][1]);
+    };
+    if (residual) {
+      const uint8_t* kr = base;  // bf16 rows of 256 bytes
+      uint32_t w0[16], w1[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 x = lds<uint4>(kr + r0 * 256 + c * 64 + i * 16);
+        const uint4 y = lds<uint4>(kr + r1 * 256 + c * 64 + i * 16);
+        w0[4 * i] = x.x; w0[4 * i + 1] = x.y; w0[4 * i + 2] = x.z; w0[4 * i + 3] = x.w;
+        w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
+      }
+      const bool split = S.qsplit;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma2(ks, bf16x2_to_f16x2(w0[2 * ks]), bf16x2_to_f16x2(w1[2 * ks]), bf16x2_to_f16x2(w0[2 * ks + 1]),
+             bf16x2_to_f16x2(w1[2 * ks + 1]), split);
+    } else if constexpr (C::kKFmt == FMT_U4) {
+      const uint4 x = lds<uint4>(base + C::kOffK + swz<64>(r0, c));
+      const uint4 y = lds<uint4>(base + C::kOffK + swz<64>(r1, c));
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int i = ks >> 1, k0 = 2 * (ks & 1);
+        const uint32_t u = word_of(x, i), v = word_of(y, i);
+        mma2(ks, u4_pair(u, k0), u4_pair(v, k0), u4_pair(u, k0 + 1), u4_pair(v, k0 + 1), true);
+      }
+    } else if constexpr (C::kKFmt == FMT_U2) {
+      const uint2 x = lds<uint2>(base + C::kOffK + swz<32>(r0, c >> 1) + 8 * (c & 1));
+      const uint2 y = lds<uint2>(base + C::kOffK + swz<32>(r1, c >> 1) + 8 * (c & 1));
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int i = ks >> 2, k0 = 2 * (ks & 3);
+        const uint32_t u = i ? x.y : x.x, v = i ? y.y : y.x;
+        mma2(ks, u2_pair(u, k0), u2_pair(v, k0), u2_pair(u, k0 + 1), u2_pair(v, k0 + 1), true);
+      }
+    } else {
+      // 8-bit codes, 128-byte rows: chunks 2c and 2c+1 of rows g and g+8 (swizzled)
+      const uint4 x0 = lds<uint4>(base + C::kOffK + swz<128>(r0, 2 * c));
+      const uint4 x1 = lds<uint4>(base + C::kOffK + swz<128>(r0, 2 * c + 1));
+      const uint4 y0 = lds<uint4>(base + C::kOffK + swz<128>(r1, 2 * c));
+      const uint4 y1 = lds<uint4>(base + C::kOffK + swz<128>(r1, 2 * c + 1));
+      const bool split = S.qsplit;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        uint32_t u = word_of(ks < 4 ? x0 : x1, ks & 3), v = word_of(ks < 4 ? y0 : y1, ks & 3);
+        if constexpr (C::kKFmt == FMT_S8) {
+          u ^= 0x80808080u;
+          v ^= 0x80808080u;
+        }
+        uint32_t u_lo, u_hi, v_lo, v_hi;
+        cvt8x4<C::kKFmt>(u, S.zpk[ks][0], S.zpk[ks][1], u_lo, u_hi);
+        cvt8x4<C::kKFmt>(v, S.zpk[ks][0], S.zpk[ks][1], v_lo, v_hi);
+        mma2(ks, u_lo, v_lo, u_hi, v_hi, split);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[sb][k] = a0[k] + a1[k];
+  }
+
+  // (3) scores (log2 domain) with masking
+  float sco[C::kNSub][4];
+#pragma unroll
+  for (int sb = 0; sb < C::kNSub; ++sb)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int tok = tok_base + sb * 16 + g + 8 * r;
+      const bool ok = tok_ok(tok);
+      float mul = S.kmul;
+      if constexpr (C::kKFold == FOLD_TOKEN) mul *= reinterpret_cast<const float*>(base + C::kOffKM)[tok];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float sv;
+        if (C::kKivi && !residual)
+          sv = fmaf(acc[sb][2 * r + j], S.kmul, S.bias[j]) * sc_log2;
+        else
+          sv = acc[sb][2 * r + j] * mul;
+        sco[sb][2 * r + j] = ok ? sv : kNegInf;
+      }
+    }
+
+  // (4) online softmax over this warp's tokens
+  float alpha[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float mx = kNegInf;
+#pragma unroll
+    for (int sb = 0; sb < C::kNSub; ++sb) mx = fmaxf(mx, fmaxf(sco[sb][j], sco[sb][2 + j]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float mnew = fmaxf(S.m[j], mx);
+    const float ms = mnew == kNegInf ? 0.0f : mnew;
+    alpha[j] = fast_exp2(S.m[j] - ms);
+    float ls = 0.0f;
+#pragma unroll
+    for (int sb = 0; sb < C::kNSub; ++sb) {
+      sco[sb][j] = fast_exp2(sco[sb][j] - ms);
+      sco[sb][2 + j] = fast_exp2(sco[sb][2 + j] - ms);
+      ls += sco[sb][j] + sco[sb][2 + j];
+    }
+    S.l[j] = S.l[j] * alpha[j] + ls;
+    S.m[j] = mnew;
+  }
+
+  // (5) probabilities to the B-operand layout: head g, tokens 2c, 2c+1, 2c+8, 2c+9
+  float pt[C::kNSub][4];
+  const int srcA = 4 * (2 * c) + (g >> 1), srcB = srcA + 4;
+  const bool odd = g & 1;
+#pragma unroll
+  for (int sb = 0; sb < C::kNSub; ++sb) {
+    const float a0 = __shfl_sync(0xffffffffu, sco[sb][0], srcA);
+    const float a1 = __shfl_sync(0xffffffffu, sco[sb][1], srcA);
+    const float a2 = __shfl_sync(0xffffffffu, sco[sb][2], srcA);
+    const float a3 = __shfl_sync(0xffffffffu, sco[sb][3], srcA);
+    const float b0 = __shfl_sync(0xffffffffu, sco[sb][0], srcB);
+    const float b1 = __shfl_sync(0xffffffffu, sco[sb][1], srcB);
+    const float b2 = __shfl_sync(0xffffffffu, sco[sb][2], srcB);
+    const float b3 = __shfl_sync(0xffffffffu, sco[sb][3], srcB);
+    pt[sb][0] = odd ? a1 : a0;
+    pt[sb][1] = odd ? b1 : b0;
+    pt[sb][2] = odd ? a3 : a2;
+    pt[sb][3] = odd ? b3 : b2;
+  }
+
+  // (6) value-side fold and accumulator exponent
+  constexpr bool kVPerToken = C::kVFold == FOLD_TOKEN || C::kKivi;
+  float vs[C::kNSub][4][4];  // [sb][token][group] folded value scale (token fold: group 0)
+  int evn = 15;
+  if (kVPerToken && !residual) {
+    float smax = 0.0f;
+#pragma unroll
+    for (int sb = 0; sb < C::kNSub; ++sb)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int tok = tok_base + sb * 16 + 2 * c + (k & 1) + 8 * (k >> 1);
+        const bool ok = tok_ok(tok);
+        if constexpr (C::kKivi) {
+          const float4 s4 = lds<float4>(base + C::kOffVM + tok * 16);
+          vs[sb][k][0] = ok ? s4.x : 0.0f;
+          vs[sb][k][1] = ok ? s4.y : 0.0f;
+          vs[sb][k][2] = ok ? s4.z : 0.0f;
+          vs[sb][k][3] = ok ? s4.w : 0.0f;
+          smax = fmaxf(smax, fmaxf(fmaxf(vs[sb][k][0], vs[sb][k][1]), fmaxf(vs[sb][k][2], vs[sb][k][3])));
+        } else {
+          const float s1 = reinterpret_cast<const float*>(base + C::kOffVM)[tok];
+          vs[sb][k][0] = ok ? s1 : 0.0f;
+          smax = fmaxf(smax, vs[sb][k][0]);
+        }
+      }
+    smax = warp_max(smax);
+    evn = smax > 0.0f ? range_shift(smax) : (S.ev_set ? S.ev : 15);
+  }
+  // rescale the accumulator only when some head's max moved or the exponent changed
+  const bool moved = (alpha[0] != 1.0f) || (alpha[1] != 1.0f) || (S.ev_set && evn != S.ev);
+  if (__any_sync(0xffffffffu, moved)) {
+    float f0 = alpha[0], f1 = alpha[1];
+    if (S.ev_set) {
+      const float r = fast_exp2((float)(evn - S.ev));
+      f0 *= r;
+      f1 *= r;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      S.o[mt][0] *= f0;
+      S.o[mt][1] *= f1;
+      S.o[mt][2] *= f0;
+      S.o[mt][3] *= f1;
+    }
+  }
+  S.ev = evn;
+  S.ev_set = true;
+  const float pscale = pow2i(evn);
+
+  // (7) O^T += V^T . P'^T
+  if constexpr (C::kKivi) {
+    // alpha for head g rescales the min-term accumulator
+    const float ag0 = __shfl_sync(0xffffffffu, alpha[0], g >> 1);
+    const float ag1 = __shfl_sync(0xffffffffu, alpha[1], g >> 1);
+    const float ag = odd ? ag1 : ag0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) S.zacc[j] *= ag;
+  }
+#pragma unroll
+  for (int sb = 0; sb < C::kNSub; ++sb) {
+    const int tb0 = tok_base + sb * 16;
+    const int tk[4] = {tb0 + 2 * c, tb0 + 2 * c + 1, tb0 + 2 * c + 8, tb0 + 2 * c + 9};
+    bool ok[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ok[k] = tok_ok(tk[k]);
+    if constexpr (!C::kKivi) {
+      float pv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pv[k] = (C::kVFold == FOLD_TOKEN ? pt[sb][k] * vs[sb][k][0] : pt[sb][k]) * pscale;
+      uint32_t bh0, bl0, bh1, bl1;
+      split_f16x2(pv[0], pv[1], bh0, bl0);
+      split_f16x2(pv[2], pv[3], bh1, bl1);
+      uint4 W[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        W[k] = lds<uint4>(base + C::kOffV + swz<128>(tk[k], g));
+        if (kMasked && !ok[k]) W[k] = make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (C::kVFmt == FMT_S8) {
+          W[k].x ^= 0x80808080u; W[k].y ^= 0x80808080u; W[k].z ^= 0x80808080u; W[k].w ^= 0x80808080u;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t x0 = word_of(W[0], q), x1 = word_of(W[1], q);
+        const uint32_t x2 = word_of(W[2], q), x3 = word_of(W[3], q);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int mt = 2 * q + half;
+          // (token 2c, token 2c+1) bytes at channels d (lo) and d+1 (hi) of this m-tile
+          const uint32_t ta = prmt(x0, x1, half ? 0x7362u : 0x5140u);
+          const uint32_t tb2 = prmt(x2, x3, half ? 0x7362u : 0x5140u);
+          uint32_t a0, a1, a2, a3;
+          cvt8x4<C::kVFmt>(ta, S.zpv[mt][0], S.zpv[mt][1], a0, a1);
+          cvt8x4<C::kVFmt>(tb2, S.zpv[mt][0], S.zpv[mt][1], a2, a3);
+          mma_16816(S.o[mt], a0, a1, a2, a3, bh0, bh1);
+          mma_16816(S.o[mt], a0, a1, a2, a3, bl0, bl1);
+        }
+      }
+    } else {
+      // KIVI: one B operand per 32-channel group; zero-point term on CUDA cores
+      uint32_t bh[4][2], bl[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float pv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pv[k] = residual ? pt[sb][k] * pscale : pt[sb][k] * vs[sb][k][j] * pscale;
+        split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
+        split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
+      }
+      if (!residual) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (!ok[k]) continue;
+          const float4 z4 = lds<float4>(base + C::kOffVM + C::kVMeta / 2 + tk[k] * 16);
+          S.zacc[0] = fmaf(pt[sb][k], z4.x, S.zacc[0]);
+          S.zacc[1] = fmaf(pt[sb][k], z4.y, S.zacc[1]);
+          S.zacc[2] = fmaf(pt[sb][k], z4.z, S.zacc[2]);
+          S.zacc[3] = fmaf(pt[sb][k], z4.w, S.zacc[3]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t pr[2][4];  // [token pair][channel e]: f16x2 (token even, token odd)
+        if (residual) {
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            const uint8_t* vr = base + kRT * kHeadDim * 2;
+            uint2 u0 = lds<uint2>(vr + tk[2 * pp] * 256 + (32 * j + 4 * g) * 2);
+            uint2 u1 = lds<uint2>(vr + tk[2 * pp + 1] * 256 + (32 * j + 4 * g) * 2);
+            if (!ok[2 * pp]) u0 = make_uint2(0u, 0u);
+            if (!ok[2 * pp + 1]) u1 = make_uint2(0u, 0u);
+            pr[pp][0] = float2_to_f16x2(bf16_bits_to_float(u0.x & 0xFFFFu), bf16_bits_to_float(u1.x & 0xFFFFu));
+            pr[pp][1] = float2_to_f16x2(bf16_bits_to_float(u0.x >> 16), bf16_bits_to_float(u1.x >> 16));
+            pr[pp][2] = float2_to_f16x2(bf16_bits_to_float(u0.y & 0xFFFFu), bf16_bits_to_float(u1.y & 0xFFFFu));
+            pr[pp][3] = float2_to_f16x2(bf16_bits_to_float(u0.y >> 16), bf16_bits_to_float(u1.y >> 16));
+          }
+        } else if constexpr (C::kVFmt == FMT_U4) {
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            uint32_t u0 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp], j) + 2 * g);
+            uint32_t u1 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp + 1], j) + 2 * g);
+            if (kMasked && !ok[2 * pp]) u0 = 0u;
+            if (kMasked && !ok[2 * pp + 1]) u1 = 0u;
+            const uint32_t wv = prmt(u0, u1, 0x5410u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[pp][e] = u4_pair(wv, e);
+          }
+        } else {
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            uint32_t u0 = lds<uint8_t>(base + C::kOffV + swz<32>(tk[2 * pp], j >> 1) + 8 * (j & 1) + g);
+            uint32_t u1 = lds<uint8_t>(base + C::kOffV + swz<32>(tk[2 * pp + 1], j >> 1) + 8 * (j & 1) + g);
+            if (kMasked && !ok[2 * pp]) u0 = 0u;
+            if (kMasked && !ok[2 * pp + 1]) u1 = 0u;
+            const uint32_t wv = prmt(u0, u1, 0x5410u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[pp][e] = u2_pair(wv, e);
+          }
+        }
+        // channel e = 2 * (mt & 1) + rh within the group: mt = 2j + (e >> 1)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int mt = 2 * j + half;
+          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bh[j][0],
+                    bh[j][1]);
+          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bl[j][0],
+                    bl[j][1]);
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int KS, int VS, bool PAGED>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
   using C = Cfg<KS, VS, PAGED>;
@@ -388,7 +783,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   // ---------------------------------------------------------------- consumers
   Consumer<C> S;
   S.w = warp;
-  S.lane = lane;
   S.g = lane >> 2;
   S.c = lane & 3;
   const int g = S.g, c = S.c, w = S.w;
@@ -399,12 +793,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   float* q_s = reinterpret_cast<float*>(smem + C::kOffQ);
   const float sc_log2 = p.softmax_scale * kLog2e;
   bool dead = false;
-  uint32_t zpk[8][2], zpv[8][2];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) S.zpk[ks][0] = S.zpk[ks][1] = S.zpv[ks][0] = S.zpv[ks][1] = 0u;
 
-  for (int t = tb, it = 0; t < te; ++t, ++it) {
-    const int st = it % C::kStages;
-    const TileDesc d = locate(p, sc, t, tb, te);
-    if (!dead && !mbar_wait(full0 + 8 * st, (it / C::kStages) & 1, p.status)) dead = true;
+  TileIter ti;
+  ti.init(p, sc, tb, te);
+  for (int st = 0, phase = 0; ti.t < te; ti.next(p, sc)) {
+    const TileDesc d = ti.desc(p, sc);
+    if (!dead && !mbar_wait(full0 + 8 * st, phase, p.status)) dead = true;
     const uint8_t* base = smem + st * C::kStageBytes;
     const uint32_t valid = C::kPaged ? descs[st].valid : 0xFFFFFFFFu;
 
@@ -451,7 +847,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               const int d0 = dmap_k<C::kKFmt>(c, ks, h, 0);
               const float z0 = 1024.0f + p.k_zp[d.hk * kHeadDim + d0];
               const float z1 = 1024.0f + p.k_zp[d.hk * kHeadDim + d0 + 1];
-              zpk[ks][h] = float2_to_f16x2(z0, z1);
+              S.zpk[ks][h] = float2_to_f16x2(z0, z1);
             }
         }
       }
@@ -461,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int rh = 0; rh < 2; ++rh) {
             const float z = 1024.0f + p.v_zp[d.hk * kHeadDim + dmap_v<false>(g, mt, rh)];
-            zpv[mt][rh] = float2_to_f16x2(z, z);
+            S.zpv[mt][rh] = float2_to_f16x2(z, z);
           }
       }
     }
@@ -471,362 +867,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int tok_base = residual ? 0 : w * C::kTPW;
     const bool busy = !dead && (residual ? (w == 0) : true) && (d.n - tok_base > 0);
     if (busy) {
-      // (1) query fragments for this tile
-      if constexpr (C::kKivi) {
-        if (!residual) {
-          const float* ksm = reinterpret_cast<const float*>(base + C::kOffKM) + w * kHeadDim;
-          const float* kzm = reinterpret_cast<const float*>(base + C::kOffKM + C::kKMeta / 2) + w * kHeadDim;
-          const int eq = build_q<C::kKFmt>(q_s, ksm, g, c, S.qh, S.ql);
-          float bs = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int dd = 32 * c + i;
-            bs = fmaf(q_s[g * 132 + dd + (dd >> 5)], kzm[dd], bs);
-          }
-          bs += __shfl_xor_sync(0xffffffffu, bs, 1);
-          bs += __shfl_xor_sync(0xffffffffu, bs, 2);
-          S.bias[0] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c));
-          S.bias[1] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c + 1));
-          S.kmul = pow2i(-eq);
-          S.qsplit = true;
-          S.qmode = 0;
-        } else if (S.qmode != 1) {
-          const int eq = build_q<FMT_S8>(q_s, nullptr, g, c, S.qh, S.ql);
-          S.kmul = sc_log2 * pow2i(-eq);
-          S.qsplit = !p.q_bf16;
-          S.qmode = 1;
-        }
-      }
-
-      // (2) S^T = K . Q'^T for kNSub blocks of 16 tokens
-      float acc[C::kNSub][4];
-#pragma unroll
-      for (int sb = 0; sb < C::kNSub; ++sb) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[sb][k] = 0.0f;
-        const int r0 = tok_base + sb * 16 + g, r1 = r0 + 8;
-        if (residual) {
-          const uint8_t* kr = base;  // bf16 rows of 256 bytes
-          uint32_t w0[16], w1[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 a = lds<uint4>(kr + r0 * 256 + c * 64 + i * 16);
-            const uint4 b = lds<uint4>(kr + r1 * 256 + c * 64 + i * 16);
-            w0[4 * i] = a.x; w0[4 * i + 1] = a.y; w0[4 * i + 2] = a.z; w0[4 * i + 3] = a.w;
-            w1[4 * i] = b.x; w1[4 * i + 1] = b.y; w1[4 * i + 2] = b.z; w1[4 * i + 3] = b.w;
-          }
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t a0 = bf16x2_to_f16x2(w0[2 * ks]), a1 = bf16x2_to_f16x2(w1[2 * ks]);
-            const uint32_t a2 = bf16x2_to_f16x2(w0[2 * ks + 1]), a3 = bf16x2_to_f16x2(w1[2 * ks + 1]);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.qh[ks][0], S.qh[ks][1]);
-            if (S.qsplit) mma_16816(acc[sb], a0, a1, a2, a3, S.ql[ks][0], S.ql[ks][1]);
-          }
-        } else if constexpr (C::kKFmt == FMT_U4) {
-          const uint4 a = lds<uint4>(base + C::kOffK + swz<64>(r0, c));
-          const uint4 b = lds<uint4>(base + C::kOffK + swz<64>(r1, c));
-          const uint32_t w0[4] = {a.x, a.y, a.z, a.w}, w1[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const int i = ks >> 1, k0 = 2 * (ks & 1);
-            const uint32_t a0 = u4_pair(w0[i], k0), a1 = u4_pair(w1[i], k0);
-            const uint32_t a2 = u4_pair(w0[i], k0 + 1), a3 = u4_pair(w1[i], k0 + 1);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.qh[ks][0], S.qh[ks][1]);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.ql[ks][0], S.ql[ks][1]);
-          }
-        } else if constexpr (C::kKFmt == FMT_U2) {
-          const uint2 a = lds<uint2>(base + C::kOffK + swz<32>(r0, c >> 1) + 8 * (c & 1));
-          const uint2 b = lds<uint2>(base + C::kOffK + swz<32>(r1, c >> 1) + 8 * (c & 1));
-          const uint32_t w0[2] = {a.x, a.y}, w1[2] = {b.x, b.y};
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const int i = ks >> 2, k0 = 2 * (ks & 3);
-            const uint32_t a0 = u2_pair(w0[i], k0), a1 = u2_pair(w1[i], k0);
-            const uint32_t a2 = u2_pair(w0[i], k0 + 1), a3 = u2_pair(w1[i], k0 + 1);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.qh[ks][0], S.qh[ks][1]);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.ql[ks][0], S.ql[ks][1]);
-          }
-        } else {
-          // 8-bit codes, 128-byte rows: chunks 2c, 2c+1 (order swapped on odd rows so the
-          // eight lanes of a load phase touch distinct banks)
-          const int sw0 = g & 1;
-          const uint4 a0v = lds<uint4>(base + C::kOffK + swz<128>(r0, 2 * c + sw0));
-          const uint4 a1v = lds<uint4>(base + C::kOffK + swz<128>(r0, 2 * c + (sw0 ^ 1)));
-          const uint4 b0v = lds<uint4>(base + C::kOffK + swz<128>(r1, 2 * c + sw0));
-          const uint4 b1v = lds<uint4>(base + C::kOffK + swz<128>(r1, 2 * c + (sw0 ^ 1)));
-          const uint4 a_lo = sw0 ? a1v : a0v, a_hi = sw0 ? a0v : a1v;
-          const uint4 b_lo = sw0 ? b1v : b0v, b_hi = sw0 ? b0v : b1v;
-          uint32_t w0[8] = {a_lo.x, a_lo.y, a_lo.z, a_lo.w, a_hi.x, a_hi.y, a_hi.z, a_hi.w};
-          uint32_t w1[8] = {b_lo.x, b_lo.y, b_lo.z, b_lo.w, b_hi.x, b_hi.y, b_hi.z, b_hi.w};
-          if constexpr (C::kKFmt == FMT_S8) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              w0[i] ^= 0x80808080u;
-              w1[i] ^= 0x80808080u;
-            }
-          }
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t z0 = C::kKFmt == FMT_U8 ? zpk[ks][0] : 0u;
-            const uint32_t z1 = C::kKFmt == FMT_U8 ? zpk[ks][1] : 0u;
-            const uint32_t a0 = cvt8x2<C::kKFmt>(w0[ks] & 0xFFFFu, z0);
-            const uint32_t a1 = cvt8x2<C::kKFmt>(w1[ks] & 0xFFFFu, z0);
-            const uint32_t a2 = cvt8x2<C::kKFmt>(w0[ks] >> 16, z1);
-            const uint32_t a3 = cvt8x2<C::kKFmt>(w1[ks] >> 16, z1);
-            mma_16816(acc[sb], a0, a1, a2, a3, S.qh[ks][0], S.qh[ks][1]);
-            if (S.qsplit) mma_16816(acc[sb], a0, a1, a2, a3, S.ql[ks][0], S.ql[ks][1]);
-          }
-        }
-      }
-
-      // (3) scores (log2 domain) with masking
-      float sco[C::kNSub][4];
-#pragma unroll
-      for (int sb = 0; sb < C::kNSub; ++sb)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int tok = tok_base + sb * 16 + g + 8 * r;
-          bool ok = tok < d.n;
-          if constexpr (C::kPaged) ok = ok && ((valid >> (tok / p.page_size)) & 1u);
-          float mul = S.kmul;
-          if constexpr (C::kKFold == FOLD_TOKEN) mul *= reinterpret_cast<const float*>(base + C::kOffKM)[tok];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            float s;
-            if (C::kKivi && !residual)
-              s = fmaf(acc[sb][2 * r + j], S.kmul, S.bias[j]) * sc_log2;
-            else
-              s = acc[sb][2 * r + j] * mul;
-            sco[sb][2 * r + j] = ok ? s : kNegInf;
-          }
-        }
-
-      // (4) online softmax over this warp's tokens
-      float alpha[2];
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float mx = kNegInf;
-#pragma unroll
-        for (int sb = 0; sb < C::kNSub; ++sb) mx = fmaxf(mx, fmaxf(sco[sb][j], sco[sb][2 + j]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float mnew = fmaxf(S.m[j], mx);
-        const float ms = mnew == kNegInf ? 0.0f : mnew;
-        alpha[j] = fast_exp2(S.m[j] - ms);
-        float ls = 0.0f;
-#pragma unroll
-        for (int sb = 0; sb < C::kNSub; ++sb) {
-          sco[sb][j] = fast_exp2(sco[sb][j] - ms);
-          sco[sb][2 + j] = fast_exp2(sco[sb][2 + j] - ms);
-          ls += sco[sb][j] + sco[sb][2 + j];
-        }
-        S.l[j] = S.l[j] * alpha[j] + ls;
-        S.m[j] = mnew;
-      }
-
-      // (5) probabilities to the B-operand layout: head g, tokens 2c, 2c+1, 2c+8, 2c+9
-      float pt[C::kNSub][4];
-      const int srcA = 4 * (2 * c) + (g >> 1), srcB = srcA + 4;
-#pragma unroll
-      for (int sb = 0; sb < C::kNSub; ++sb) {
-        const float a0 = __shfl_sync(0xffffffffu, sco[sb][0], srcA);
-        const float a1 = __shfl_sync(0xffffffffu, sco[sb][1], srcA);
-        const float a2 = __shfl_sync(0xffffffffu, sco[sb][2], srcA);
-        const float a3 = __shfl_sync(0xffffffffu, sco[sb][3], srcA);
-        const float b0 = __shfl_sync(0xffffffffu, sco[sb][0], srcB);
-        const float b1 = __shfl_sync(0xffffffffu, sco[sb][1], srcB);
-        const float b2 = __shfl_sync(0xffffffffu, sco[sb][2], srcB);
-        const float b3 = __shfl_sync(0xffffffffu, sco[sb][3], srcB);
-        const bool odd = g & 1;
-        pt[sb][0] = odd ? a1 : a0;
-        pt[sb][1] = odd ? b1 : b0;
-        pt[sb][2] = odd ? a3 : a2;
-        pt[sb][3] = odd ? b3 : b2;
-      }
-
-      // (6) value-side fold and accumulator exponent
-      constexpr bool kVPerToken = C::kVFold == FOLD_TOKEN || C::kKivi;
-      float vs[C::kNSub][4][4];  // [sb][token][group] folded scale (token fold: group 0)
-      int evn = 15;
-      if (kVPerToken && !residual) {
-        float smax = 0.0f;
-#pragma unroll
-        for (int sb = 0; sb < C::kNSub; ++sb)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int tok = tok_base + sb * 16 + 2 * c + (k & 1) + 8 * (k >> 1);
-            bool ok = tok < d.n;
-            if constexpr (C::kPaged) ok = ok && ((valid >> (tok / p.page_size)) & 1u);
-            if constexpr (C::kKivi) {
-              const float4 s4 = lds<float4>(base + C::kOffVM + tok * 16);
-              vs[sb][k][0] = ok ? s4.x : 0.0f;
-              vs[sb][k][1] = ok ? s4.y : 0.0f;
-              vs[sb][k][2] = ok ? s4.z : 0.0f;
-              vs[sb][k][3] = ok ? s4.w : 0.0f;
-              smax = fmaxf(smax, fmaxf(fmaxf(vs[sb][k][0], vs[sb][k][1]), fmaxf(vs[sb][k][2], vs[sb][k][3])));
-            } else {
-              const float s1 = reinterpret_cast<const float*>(base + C::kOffVM)[tok];
-              vs[sb][k][0] = ok ? s1 : 0.0f;
-              smax = fmaxf(smax, vs[sb][k][0]);
-            }
-          }
-        smax = warp_max(smax);
-        evn = smax > 0.0f ? range_shift(smax) : (S.ev_set ? S.ev : 15);
-      }
-      float f0 = alpha[0], f1 = alpha[1];
-      if (S.ev_set) {
-        const float r = fast_exp2((float)(evn - S.ev));
-        f0 *= r;
-        f1 *= r;
-      }
-      S.ev = evn;
-      S.ev_set = true;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        S.o[mt][0] *= f0;
-        S.o[mt][1] *= f1;
-        S.o[mt][2] *= f0;
-        S.o[mt][3] *= f1;
-      }
-      const float pscale = pow2i(evn);
-
-      // (7) O^T += V^T . P'^T
-      if constexpr (C::kKivi) {
-        // alpha for head g rescales the min-term accumulator
-        const float ag0 = __shfl_sync(0xffffffffu, alpha[0], g >> 1);
-        const float ag1 = __shfl_sync(0xffffffffu, alpha[1], g >> 1);
-        const float ag = (g & 1) ? ag1 : ag0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) S.zacc[j] *= ag;
-      }
-#pragma unroll
-      for (int sb = 0; sb < C::kNSub; ++sb) {
-        const int tb0 = tok_base + sb * 16;
-        const int tk[4] = {tb0 + 2 * c, tb0 + 2 * c + 1, tb0 + 2 * c + 8, tb0 + 2 * c + 9};
-        bool ok[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          ok[k] = tk[k] < d.n;
-          if constexpr (C::kPaged) ok[k] = ok[k] && ((valid >> (tk[k] / p.page_size)) & 1u);
-        }
-        if constexpr (!C::kKivi) {
-          float pv[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            pv[k] = (C::kVFold == FOLD_TOKEN ? pt[sb][k] * vs[sb][k][0] : pt[sb][k]) * pscale;
-          uint32_t bh0, bl0, bh1, bl1;
-          split_f16x2(pv[0], pv[1], bh0, bl0);
-          split_f16x2(pv[2], pv[3], bh1, bl1);
-          const int vrow = 16 * g;  // chunk g of each 128-byte row
-          uint4 W[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            W[k] = lds<uint4>(base + C::kOffV + swz<128>(tk[k], g));
-            if (!ok[k]) W[k] = make_uint4(0u, 0u, 0u, 0u);
-            if constexpr (C::kVFmt == FMT_S8) {
-              W[k].x ^= 0x80808080u; W[k].y ^= 0x80808080u; W[k].z ^= 0x80808080u; W[k].w ^= 0x80808080u;
-            }
-          }
-          (void)vrow;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t x0 = q == 0 ? W[0].x : q == 1 ? W[0].y : q == 2 ? W[0].z : W[0].w;
-            const uint32_t x1 = q == 0 ? W[1].x : q == 1 ? W[1].y : q == 2 ? W[1].z : W[1].w;
-            const uint32_t x2 = q == 0 ? W[2].x : q == 1 ? W[2].y : q == 2 ? W[2].z : W[2].w;
-            const uint32_t x3 = q == 0 ? W[3].x : q == 1 ? W[3].y : q == 2 ? W[3].z : W[3].w;
-            const uint32_t t01a = prmt(x0, x1, 0x5140u), t01b = prmt(x0, x1, 0x7362u);
-            const uint32_t t23a = prmt(x2, x3, 0x5140u), t23b = prmt(x2, x3, 0x7362u);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int mt = 2 * q + half;
-              const uint32_t ta = half ? t01b : t01a, tb2 = half ? t23b : t23a;
-              const uint32_t zr0 = C::kVFmt == FMT_U8 ? zpv[mt][0] : 0u;
-              const uint32_t zr1 = C::kVFmt == FMT_U8 ? zpv[mt][1] : 0u;
-              const uint32_t a0 = cvt8x2<C::kVFmt>(ta & 0xFFFFu, zr0);
-              const uint32_t a1 = cvt8x2<C::kVFmt>(ta >> 16, zr1);
-              const uint32_t a2 = cvt8x2<C::kVFmt>(tb2 & 0xFFFFu, zr0);
-              const uint32_t a3 = cvt8x2<C::kVFmt>(tb2 >> 16, zr1);
-              mma_16816(S.o[mt], a0, a1, a2, a3, bh0, bh1);
-              mma_16816(S.o[mt], a0, a1, a2, a3, bl0, bl1);
-            }
-          }
-        } else {
-          // KIVI: one B operand per 32-channel group; zero-point term on CUDA cores
-          uint32_t bh[4][2], bl[4][2];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float pv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) pv[k] = residual ? pt[sb][k] * pscale : pt[sb][k] * vs[sb][k][j] * pscale;
-            split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
-            split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
-          }
-          if (!residual) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              if (!ok[k]) continue;
-              const float4 z4 = lds<float4>(base + C::kOffVM + C::kVMeta / 2 + tk[k] * 16);
-              S.zacc[0] = fmaf(pt[sb][k], z4.x, S.zacc[0]);
-              S.zacc[1] = fmaf(pt[sb][k], z4.y, S.zacc[1]);
-              S.zacc[2] = fmaf(pt[sb][k], z4.z, S.zacc[2]);
-              S.zacc[3] = fmaf(pt[sb][k], z4.w, S.zacc[3]);
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t pr[2][4];  // [token pair][channel e]: f16x2 (token even, token odd)
-            if (residual) {
-#pragma unroll
-              for (int pp = 0; pp < 2; ++pp) {
-                const uint8_t* vr = base + kRT * kHeadDim * 2;
-                uint2 u0 = lds<uint2>(vr + tk[2 * pp] * 256 + (32 * j + 4 * g) * 2);
-                uint2 u1 = lds<uint2>(vr + tk[2 * pp + 1] * 256 + (32 * j + 4 * g) * 2);
-                if (!ok[2 * pp]) u0 = make_uint2(0u, 0u);
-                if (!ok[2 * pp + 1]) u1 = make_uint2(0u, 0u);
-                pr[pp][0] = float2_to_f16x2(bf16_bits_to_float(u0.x & 0xFFFFu), bf16_bits_to_float(u1.x & 0xFFFFu));
-                pr[pp][1] = float2_to_f16x2(bf16_bits_to_float(u0.x >> 16), bf16_bits_to_float(u1.x >> 16));
-                pr[pp][2] = float2_to_f16x2(bf16_bits_to_float(u0.y & 0xFFFFu), bf16_bits_to_float(u1.y & 0xFFFFu));
-                pr[pp][3] = float2_to_f16x2(bf16_bits_to_float(u0.y >> 16), bf16_bits_to_float(u1.y >> 16));
-              }
-            } else if constexpr (C::kVFmt == FMT_U4) {
-#pragma unroll
-              for (int pp = 0; pp < 2; ++pp) {
-                uint32_t u0 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp], j) + 2 * g);
-                uint32_t u1 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp + 1], j) + 2 * g);
-                if (!ok[2 * pp]) u0 = 0u;
-                if (!ok[2 * pp + 1]) u1 = 0u;
-                const uint32_t wv = prmt(u0, u1, 0x5410u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pr[pp][e] = u4_pair(wv, e);
-              }
-            } else {
-#pragma unroll
-              for (int pp = 0; pp < 2; ++pp) {
-                uint32_t u0 = lds<uint8_t>(base + C::kOffV + swz<32>(tk[2 * pp], j >> 1) + 8 * (j & 1) + g);
-                uint32_t u1 = lds<uint8_t>(base + C::kOffV + swz<32>(tk[2 * pp + 1], j >> 1) + 8 * (j & 1) + g);
-                if (!ok[2 * pp]) u0 = 0u;
-                if (!ok[2 * pp + 1]) u1 = 0u;
-                const uint32_t wv = prmt(u0, u1, 0x5410u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pr[pp][e] = u2_pair(wv, e);
-              }
-            }
-            // channel e = 2 * (mt & 1) + rh within the group: mt = 2j + (e >> 1)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int mt = 2 * j + half;
-              const uint32_t a0 = pr[0][2 * half], a1 = pr[0][2 * half + 1];
-              const uint32_t a2 = pr[1][2 * half], a3 = pr[1][2 * half + 1];
-              mma_16816(S.o[mt], a0, a1, a2, a3, bh[j][0], bh[j][1]);
-              mma_16816(S.o[mt], a0, a1, a2, a3, bl[j][0], bl[j][1]);
-            }
-          }
-        }
-      }
+      const bool full = d.n - tok_base >= C::kTPW && (!C::kPaged || valid == 0xFFFFFFFFu ||
+                                                       ((valid >> (tok_base / p.page_size)) &
+                                                        ((1u << (C::kTPW + p.page_size - 1) / p.page_size) - 1u)) ==
+                                                           ((1u << (C::kTPW + p.page_size - 1) / p.page_size) - 1u));
+      if (full)
+        warp_tile<C, false>(S, p, base, d, valid, residual, tok_base, sc_log2, q_s);
+      else
+        warp_tile<C, true>(S, p, base, d, valid, residual, tok_base, sc_log2, q_s);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * st);
+    if (++st == C::kStages) {
+      st = 0;
+      phase ^= 1;
+    }
 
     // ------------------------------------------------ pair end: merge the warps
     if (d.last) {
@@ -894,10 +949,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ------------------------------------------------------------------ merge
+// One block per (pair, query head of the pair's group); 128 threads = channels. The (m, l)
+// of every covering CTA are staged in shared memory first, so the output costs two
+// dependent global round trips however many CTAs covered the pair.
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
-  const int pair = blockIdx.x, dd = threadIdx.x;
+  __shared__ float s_m[128], s_w[128];
+  __shared__ float s_M, s_L;
+  const int pair = blockIdx.x, j = blockIdx.y, dd = threadIdx.x;
   const int per_seq = p.Hkv * p.HG;
   const int b = pair / per_seq, hh = pair % per_seq, hk = hh / p.HG, hg = hh % p.HG;
+  const int hl = hg * 8 + j;
+  if (hl >= p.G) return;
+  const int hq = hk * p.G + hl;
   int off, n, N;
   if (p.paged) {
     N = p.plan[p.B];
@@ -908,31 +971,47 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
     N = p.n_pairs * n;
     off = pair * n;
   }
-  const int W = (N + p.ncta - 1) / p.ncta;
-  for (int j = 0; j < 8; ++j) {
-    const int hl = hg * 8 + j;
-    if (hl >= p.G) break;
-    const int hq = hk * p.G + hl;
-    float ov = 0.0f, lse = kNegInf;
-    if (n > 0) {
-      const int c0 = off / W, c1 = (off + n - 1) / W;
-      float M = kNegInf;
-      for (int cta = c0; cta <= c1; ++cta) M = fmaxf(M, p.part_ml[((size_t)(pair + cta) * 8 + j) * 2]);
-      if (M != kNegInf) {
-        float L = 0.0f, acc = 0.0f;
-        for (int cta = c0; cta <= c1; ++cta) {
-          const size_t sl = (size_t)(pair + cta) * 8 + j;
-          const float a = exp2f(p.part_ml[sl * 2] - M);
-          L = fmaf(a, p.part_ml[sl * 2 + 1], L);
-          acc = fmaf(a, p.part_o[sl * kHeadDim + dd], acc);
-        }
-        ov = acc / L;
-        lse = (M + log2f(L)) * 0.69314718055994531f;
+  float ov = 0.0f, lse = kNegInf;
+  if (n > 0) {
+    const int W = (N + p.ncta - 1) / p.ncta;
+    const int c0 = off / W, c1 = (off + n - 1) / W;
+    float acc = 0.0f, M = kNegInf, L = 0.0f;
+    // chunks of up to 128 covering CTAs (almost always one chunk)
+    for (int base = c0; base <= c1; base += 128) {
+      const int cnt = min(128, c1 - base + 1);
+      if (dd < cnt) {
+        const size_t sl = (size_t)(pair + base + dd) * 8 + j;
+        s_m[dd] = p.part_ml[sl * 2];
+        s_w[dd] = p.part_ml[sl * 2 + 1];
       }
+      __syncthreads();
+      if (dd == 0) {
+        float mc = M;
+        for (int i = 0; i < cnt; ++i) mc = fmaxf(mc, s_m[i]);
+        float Lc = (M == kNegInf || mc == kNegInf) ? 0.0f : L * exp2f(M - mc);
+        for (int i = 0; i < cnt; ++i) {
+          const float a = mc == kNegInf ? 0.0f : exp2f(s_m[i] - mc);
+          Lc = fmaf(a, s_w[i], Lc);
+          s_w[i] = a;
+        }
+        s_M = mc;
+        s_L = Lc;
+      }
+      __syncthreads();
+      const float mc = s_M;
+      acc = (M == kNegInf || mc == kNegInf) ? 0.0f : acc * exp2f(M - mc);
+      for (int i = 0; i < cnt; ++i) acc = fmaf(s_w[i], p.part_o[((size_t)(pair + base + i) * 8 + j) * kHeadDim + dd], acc);
+      M = mc;
+      L = s_L;
+      __syncthreads();
     }
-    p.out[((size_t)b * p.Hq + hq) * kHeadDim + dd] = ov;
-    if (dd == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
+    if (M != kNegInf && L > 0.0f) {
+      ov = acc / L;
+      lse = (M + log2f(L)) * 0.69314718055994531f;
+    }
   }
+  p.out[((size_t)b * p.Hq + hq) * kHeadDim + dd] = ov;
+  if (dd == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
 }
 
 // ------------------------------------------------------------------ paged plan
@@ -1099,7 +1178,7 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
     return cudaErrorInvalidValue;
   if (p.paged) plan_kernel<<<1, 1024, 0, st>>>(p);
   var->kernel<<<ncta, kThreads, var->smem, st>>>(p, tk, tv);
-  merge_kernel<<<p.n_pairs, 128, 0, st>>>(p);
+  merge_kernel<<<dim3(p.n_pairs, 8), 128, 0, st>>>(p);
   count_launches(p.paged ? 3 : 2);
   return cudaGetLastError();
 }
