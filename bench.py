@@ -6,7 +6,7 @@ A step is one pass of the hot path over one batch: quantize-append of one new to
 sequence, then split-KV decode attention (+ log-sum-exp merge) over the whole cache. The
 default workload is the Llama-3-8B-shaped FP8 E4M3 layer (batch 32, 32/8 heads, context
 4096). Inputs are seeded synthetic tensors resident in HBM; the step is captured once in a
-CUDA graph and replayed; L2 is flushed (256 MiB write) before every timed step and the
+CUDA graph and replayed; L2 is flushed (256 MiB written, then 256 MiB read) before every timed step; the
 flush is outside the step's CUDA-event interval. `value` is the step's algorithmic bytes
 (codes + scales + residual + Q + out for decode, new K/V in + codes out for the append)
 divided by the step time, summed over all ranks (weak scaling: one full workload per GPU).
@@ -183,6 +183,23 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml" if self.nv else "unavailable"}
 
 
+class L2Flush:
+    """Evicts the 126 MB L2 between timed steps: writes a 256 MiB buffer, then reads another
+    256 MiB buffer so the write-backs of the first happen before the timed interval and the
+    timed step starts with clean lines that hold none of its inputs."""
+
+    def __init__(self, dev):
+        import torch
+        self.a = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.b = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        self.out = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.a.zero_()
+        torch.amax(self.b, dim=0, out=self.out)
+
+
 # ---------------------------------------------------------------- multi-rank plumbing
 def rank_workload(w, rank):
     """Weak scaling: rank r runs the whole per-GPU workload on its own seeded batch."""
@@ -233,23 +250,64 @@ class GpuWorkload:
         cap = (total + 127) // 128 * 128
         spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev)
-        calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
-        chunk = max(1, (1 << 27) // (W.Hkv * 128 * W.B))  # generate ~256 MB of bf16 at a time
-        first = True
-        for t0 in range(0, pre, chunk if not calib else pre):
-            t1 = min(pre, t0 + (chunk if not calib else pre))
-            k = synth.keys(W, 0, W.B, 0, W.Hkv, t0, t1)
-            v = synth.values(W, 0, W.B, 0, W.Hkv, t0, t1)
-            self.cache.append(self._dev(k, W.bf16), self._dev(v, W.bf16), calibrate=calib and first)
-            first = False
+        self.calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
+        self.pre_k = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, 0, pre), W.bf16)
+        self.pre_v = self._dev(synth.values(W, 0, W.B, 0, W.Hkv, 0, pre), W.bf16)
+        self.pre_lens = None
+        self.cache.append(self.pre_k, self.pre_v, calibrate=self.calib)
         self.torch.cuda.synchronize()
         self.pre = pre
+        self.prefill_rows = W.B * W.Hkv * pre
         d = self.cache.desc
         self.saved = (d.num_quantized, d.num_residual)
         self.k_new = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, pre, pre + 1), W.bf16)
         self.v_new = self._dev(synth.values(W, 0, W.B, 0, W.Hkv, pre, pre + 1), W.bf16)
-        self.len_q_decode = d.num_quantized if not W.kivi else None
         self._common(W)
+
+    def reset_to_empty(self):
+        """Forget every token (dense: host lengths; paged: device lengths) so the prefill can be
+        appended again onto the same positions."""
+        d = self.cache.desc
+        if self.w.paged:
+            self.cache["seq_lens"].zero_()
+        else:
+            d.num_quantized, d.num_residual = 0, 0
+
+    def prefill_bytes(self):
+        """Algorithmic bytes of the prefill append: the block is read once (twice when it
+        calibrates a per-tensor / per-channel scale) and codes, metadata and residual written."""
+        W = self.seed_w
+        rows = self.prefill_rows
+        elem = 2 if W.bf16 else 4
+        b = rows * 128 * elem * 2 * (2 if self.calib else 1)
+        if W.kivi:
+            nq = (self.cache.desc.num_quantized if not W.paged else 0)
+            qrows = W.B * W.Hkv * nq
+            b += qrows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme)) + qrows * 2 * 8.0 * 128 / 32
+            b += W.B * W.Hkv * self.cache.desc.num_residual * 128 * 2 * 2
+        else:
+            b += rows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme))
+            b += rows * (meta_bytes_per_token(W.k_scheme, W.Hkv) + meta_bytes_per_token(W.v_scheme, W.Hkv))
+        return float(b)
+
+    def time_prefill(self, flush, stream, reps=3):
+        torch = self.torch
+        ms = []
+        saved = (self.cache.desc.num_quantized, self.cache.desc.num_residual)
+        for _ in range(reps):
+            self.reset_to_empty()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                flush()
+                a.record(stream)
+                self.cache.append(self.pre_k, self.pre_v, new_lens=self.pre_lens, calibrate=self.calib,
+                                  stream=stream)
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        if not self.w.paged:
+            self.cache.desc.num_quantized, self.cache.desc.num_residual = saved
+        return sum(ms) / len(ms) / 1e3
 
     def _build_paged(self, W):
         kvq, torch = self.kvq, self.torch
@@ -274,8 +332,11 @@ class GpuWorkload:
             L = int(lens[b])
             K[b, :, :L] = self._dev(synth.keys(W, b, b + 1, 0, W.Hkv, 0, L)[0], True)
             V[b, :, :L] = self._dev(synth.values(W, b, b + 1, 0, W.Hkv, 0, L)[0], True)
-        self.cache.append(K, V, new_lens=torch.from_numpy(lens).to(self.dev), calibrate=True)
-        del K, V
+        self.pre_k, self.pre_v = K, V
+        self.pre_lens = torch.from_numpy(lens).to(self.dev)
+        self.calib = True
+        self.prefill_rows = int(lens.sum()) * W.Hkv
+        self.cache.append(K, V, new_lens=self.pre_lens, calibrate=True)
         torch.cuda.synchronize()
         self.lens = lens
         self.append_token = True
@@ -331,7 +392,12 @@ def run_gpu(args, rank, world, local_rank):
     G = GpuWorkload(w, rank, dev)
     W = G.seed_w
     stream = torch.cuda.Stream(device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    t_prefill = G.time_prefill(flush, stream)
+    prefill = {"ms": t_prefill * 1e3, "bytes": G.prefill_bytes(), "tokens": G.prefill_rows // W.Hkv,
+               "calibrating": bool(G.calib)}
+    G.pre_k = G.pre_v = None  # release the prefill block before timing the steps
+    torch.cuda.empty_cache()
 
     # capture one step in a CUDA graph (dense: positions are reset each step, so the graph
     # replays an identical step; paged: lengths live on the device and advance per replay)
@@ -370,7 +436,7 @@ def run_gpu(args, rank, world, local_rank):
                 G.step(stream, k_new=toks[i][0], v_new=toks[i][1])
 
     for i in range(args.warmup):
-        flush.zero_()
+        flush()
         run_step(i)
     torch.cuda.synchronize()
     if world > 1:
@@ -383,7 +449,7 @@ def run_gpu(args, rank, world, local_rank):
     with sampler:
         for i in range(args.steps):
             with torch.cuda.stream(stream):
-                flush.zero_()
+                flush()
                 ev[i][0].record(stream)
                 if graph is not None:
                     graph.replay()
@@ -399,7 +465,7 @@ def run_gpu(args, rank, world, local_rank):
     dec_ms = []
     for i in range(min(args.steps, 400)):
         with torch.cuda.stream(stream):
-            flush.zero_()
+            flush()
             dec_ev[i][0].record(stream)
             G.cache.decode(G.q, G.scale, out=G.out, workspace=G.ws, stream=stream)
             dec_ev[i][1].record(stream)
@@ -419,7 +485,7 @@ def run_gpu(args, rank, world, local_rank):
     e2e = run_e2e(G, W, stream, flush, n=min(200, args.steps), step0=args.warmup + args.steps)
     status = G.cache.status()
     return dict(t_step=t_step, t_max=t_max, t_dec=t_dec, dbytes=dbytes, dbytes_dec=dbytes_dec, abytes=abytes,
-                launches=launches,
+                launches=launches, prefill=prefill,
                 clocks=sampler.summary(), e2e=e2e, status=status, W=W, G=G)
 
 
@@ -448,7 +514,7 @@ def run_e2e(G, W, stream, flush, n, step0):
     for i in range(n):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
-            flush.zero_()
+            flush()
             a.record(stream)
             q_d.copy_(q_h, non_blocking=True)
             if G.append_token:
@@ -535,7 +601,7 @@ def main():
               "context": (f"uniform {w.len_lo}..{w.len_hi}" if w.paged else w.prefill_tokens()),
               "layout": "paged/16" if w.paged else "dense",
               "step": ("decode only" if w.name == "tiny_int8" else "append 1 token per sequence + decode"),
-              "l2": "flushed (256 MiB write) before every timed step, outside the event interval",
+              "l2": "flushed before every timed step (256 MiB write, then 256 MiB read), outside the event interval",
               "parallelism": f"replicas x{args.gpus}"}
     if args.impl == "reference":
         if rank != 0:
@@ -584,6 +650,13 @@ def main():
            "tokens_per_s": tokens_per_s, "pct_of_hbm_peak": 100.0 * (value / world) / peak,
            "roofline": roofline, "clocks": r["clocks"], "gpu_launches": r["launches"],
            "device_status": list(r["status"])}
+    pf = r["prefill"]
+    pf_gbs = pf["bytes"] / (pf["ms"] / 1e3) / 1e9
+    out["append_bulk"] = {"what": "prefill quantize-append of the whole context (calibrating when the scheme "
+                                  "has batch-wide scales), mean of 3, L2 flushed before each",
+                          "ms": pf["ms"], "algorithmic_bytes": pf["bytes"], "GBps": pf_gbs, "frac": pf_gbs / peak,
+                          "tokens_per_seq": pf["tokens"] if not W.paged else "variable",
+                          "calibrating": pf["calibrating"]}
     if r["e2e"]:
         e = r["e2e"]
         out["e2e"] = {"value": world * step_bytes / e["t"] / 1e9, "unit": UNIT,

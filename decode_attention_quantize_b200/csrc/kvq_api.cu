@@ -159,6 +159,7 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   if (new_lens && !paged) return KVQ_ERR_INVALID_ARG;
   const bool kivi = is_kivi(d->k_scheme);
   if (kivi && in_dtype != KVQ_BF16) return KVQ_ERR_UNSUPPORTED;
+  if (!append_pair_supported(d->k_scheme, d->v_scheme)) return KVQ_ERR_UNSUPPORTED;
   if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)n_new >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
   if (paged && n_new > seq_capacity(d)) return KVQ_ERR_CAPACITY;
   const bool calibrate = (flags & KVQ_APPEND_CALIBRATE) != 0 && !kivi;

@@ -37,27 +37,54 @@ __device__ __forceinline__ void load8(const void* base, size_t elem, float (&x)[
   }
 }
 
-__device__ __forceinline__ int sym_code(float x, float s, int qmax, int& sat) {
-  if (s == 0.0f) return 0;
-  float r = rintf(__fdiv_rn(x, s));
-  if (r > (float)qmax) { r = (float)qmax; ++sat; }
-  if (r < (float)-qmax) { r = (float)-qmax; ++sat; }
-  return (int)r;
+// KIVI codes without a division per element. With r = RN(1/s) (s normal and not near the
+// ends of the range), y = RN(x * r) lies within 2^-22 * |y| of RN(x / s). Rounding half to
+// even and clamping is monotone, so when no rounding boundary lies within 2^-20 * |y| of y,
+// the code of y is the code of RN(x / s); otherwise the IEEE division decides. Rounding uses
+// the 1.5 * 2^23 add-and-subtract identity (exact round-half-to-even for |v| < 2^22) so the
+// common path stays on the FP32 pipes.
+struct Recip {
+  float s, r;
+  bool fast;
+};
+
+__device__ __forceinline__ Recip recip_of(float s) {
+  Recip q;
+  q.s = s;
+  q.r = __fdiv_rn(1.0f, s);
+  q.fast = s >= 7.52316385e-37f && s <= 1.32922800e+36f;  // 2^-120 .. 2^120
+  return q;
 }
 
-__device__ __forceinline__ int asym_code(float x, float s, int zp, int& sat) {
-  if (s == 0.0f) return 0;
-  float r = __fadd_rn(rintf(__fdiv_rn(x, s)), (float)zp);
-  if (r < 0.0f) { r = 0.0f; ++sat; }
-  if (r > 255.0f) { r = 255.0f; ++sat; }
-  return (int)r;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ float rne_small(float v) { return __fsub_rn(__fadd_rn(v, kRoundMagic), kRoundMagic); }
+// an integer-valued float in [-2^22, 2^22] -> int
+__device__ __forceinline__ int int_of(float v) { return __float_as_int(__fadd_rn(v, kRoundMagic)) - kRoundMagicBits; }
+
+// The rare exact fallback, kept out of line so the common path stays compact.
+__device__ __noinline__ float slow_quot_code(float x, float s, float lo, float hi) {
+  return fminf(fmaxf(rintf(__fdiv_rn(x, s)), lo), hi);
 }
 
-__device__ __forceinline__ int fp8_code(float x, float s, int& sat) {
-  if (s == 0.0f) return 0;
-  const float y = __fdiv_rn(x, s);
-  if (fabsf(y) > 448.0f) ++sat;
-  return (int)__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E4M3);
+// clamp(rne(RN(x / s)), lo, hi) for integer lo < hi with |lo|, |hi| < 2^21
+__device__ __forceinline__ float quot_code(float x, const Recip& q, float lo, float hi) {
+  if (q.fast) {
+    const float y = fminf(fmaxf(__fmul_rn(x, q.r), lo - 1.0f), hi + 1.0f);
+    const float r = rne_small(y);
+    const float d = fabsf(__fsub_rn(y, r));                 // exact, <= 0.5
+    if (__fsub_rn(0.5f, d) > __fmul_rn(fabsf(y), 9.5367431640625e-07f))  // boundary farther than 2^-20|y|
+      return fminf(fmaxf(r, lo), hi);
+  }
+  return slow_quot_code(x, q.s, lo, hi);
+}
+
+// Two E4M3 codes, RN-even with saturation: lo -> low byte, hi -> high byte.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Row of token `pos` of (b, h): dense [B,H,cap]; paged via the page table. Returns false
@@ -213,62 +240,256 @@ __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
 }
 
 // ------------------------------------------------------------------ 8-bit quantize-store
-// Rows (b, h, i) of the new block; 16 threads per row, 8 channels each; blockIdx.y = side.
+// Bracketing reciprocals. With r = RN(1/s), lo = RN(r * (1 - 2^-20)) and hi = RN(r * (1 + 2^-20)),
+// the products RN(x * lo) and RN(x * hi) are floats on either side of x / s (for s and x * r in
+// the normal range), hence also on either side of RN(x / s). Every code map used here is monotone
+// (round half to even then clamp; E4M3 round-to-nearest-even with saturation), so when the two
+// products give the same code, that code is the code of RN(x / s). A row whose products disagree
+// anywhere, or that may saturate, is redone element by element with the IEEE division.
+struct Bracket {
+  float lo, hi;
+};
+
+// `fast` is cleared when s is outside 2^-120 .. 2^120 (zero included): such rows go exact.
+__device__ __forceinline__ Bracket bracket_of(float s, bool& fast) {
+  Bracket q;
+  const float r = __fdiv_rn(1.0f, s);
+  q.lo = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
+  q.hi = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
+  fast &= s >= 7.52316385e-37f && s <= 1.32922800e+36f;
+  return q;
+}
+
+// Eight input elements, kept as loaded until they are quantized.
 template <bool kBf16>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(AppendParams p) {
-  const int side = blockIdx.y;
-  const int scheme = side ? p.v_scheme : p.k_scheme;
-  const long long rows = (long long)p.B * p.H * p.n_new;
-  const long long r = (long long)blockIdx.x * 16 + (threadIdx.x >> 4);
-  const int lane8 = threadIdx.x & 15;
-  const unsigned half_mask = (threadIdx.x & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-  int sat = 0;
-  bool active = r < rows;
-  int b = 0, h = 0, i = 0;
-  if (active) {
-    i = (int)(r % p.n_new);
-    h = (int)((r / p.n_new) % p.H);
-    b = (int)(r / ((long long)p.n_new * p.H));
-    active = i < new_count(p, b);
+struct Raw8;
+template <>
+struct Raw8<true> {
+  uint4 v;
+  __device__ __forceinline__ void load(const void* base, size_t elem) {
+    v = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem);
   }
-  float x[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  if (active) load8<kBf16>(side ? p.v_new : p.k_new, (size_t)r * kHeadDim + lane8 * 8, x);
-  float* scale = side ? p.v_scale : p.k_scale;
-  // per-token scale: absmax over the 16 lanes of this row (all 32 lanes take part)
-  float tok_s = 0.0f;
-  if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
-    float m = 0.0f;
+  __device__ __forceinline__ void clear() { v = make_uint4(0u, 0u, 0u, 0u); }
+  __device__ __forceinline__ void unpack(float (&x)[8]) const {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    tok_s = __fdiv_rn(m, 127.0f);
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
   }
-  (void)half_mask;
-  if (!active) return;
-  const int pos = (p.paged ? p.seq_lens[b] : p.pos0) + i;
-  size_t row;
-  if (!cache_row(p, b, h, pos, row)) return;
-  uint8_t* codes = static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8;
-  const uint8_t* zp = side ? p.v_zp : p.k_zp;
-  uint32_t packed[2] = {0u, 0u};
+};
+template <>
+struct Raw8<false> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const void* base, size_t elem) {
+    const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+    a = q[0];
+    b = q[1];
+  }
+  __device__ __forceinline__ void clear() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void unpack(float (&x)[8]) const {
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+};
+
+// Low bytes of four words -> one word (byte i from word i).
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  return prmt(prmt(w0, w1, 0x0040u), prmt(w2, w3, 0x0040u), 0x5410u);
+}
+
+// Fast rows. Each returns false when the row must be redone exactly.
+__device__ __forceinline__ bool fp8_row(const float (&x)[8], const Bracket& q, uint2& out) {
+  uint32_t c[4], diff = 0u;
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float a0 = __fmul_rn(x[2 * k], q.lo), a1 = __fmul_rn(x[2 * k + 1], q.lo);
+    const float b0 = __fmul_rn(x[2 * k], q.hi), b1 = __fmul_rn(x[2 * k + 1], q.hi);
+    c[k] = e4m3x2_rn(a0, a1);
+    diff |= c[k] ^ e4m3x2_rn(b0, b1);
+    amax = fmaxf(amax, fmaxf(fabsf(b0), fabsf(b1)));  // |x * hi| >= |RN(x / s)|
+  }
+  out = make_uint2(prmt(c[0], c[1], 0x5410u), prmt(c[2], c[3], 0x5410u));
+  return diff == 0u && amax <= 448.0f;
+}
+
+// symmetric: clamp(rne(x / s), -qmax, qmax); y + 1.5 * 2^23 holds rne(y) in its low bits
+template <int kQmax>
+__device__ __forceinline__ bool sym_row(const float (&x)[8], const Bracket (&q)[8], uint2& out) {
+  uint32_t c[8], diff = 0u;
+  float amax = 0.0f;
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const int d = lane8 * 8 + k;
-    int q = 0;
-    switch (scheme) {
-      case KVQ_FP8_E4M3_PER_TENSOR: q = fp8_code(x[k], scale[0], sat); break;
-      case KVQ_INT8_SYM_PER_TENSOR: q = sym_code(x[k], scale[0], 127, sat); break;
-      case KVQ_INT8_SYM_PER_TOKEN: q = sym_code(x[k], tok_s, 127, sat); break;
-      case KVQ_INT8_SYM_PER_CHANNEL: q = sym_code(x[k], scale[h * kHeadDim + d], 127, sat); break;
-      case KVQ_UINT8_ASYM_PER_CHANNEL:
-        q = asym_code(x[k], scale[h * kHeadDim + d], zp[h * kHeadDim + d], sat);
-        break;
-    }
-    packed[k >> 2] |= (uint32_t)(q & 0xFF) << (8 * (k & 3));
+    const float a = __fmul_rn(x[k], q[k].lo), b = __fmul_rn(x[k], q[k].hi);
+    c[k] = __float_as_uint(__fadd_rn(a, kRoundMagic));
+    diff |= c[k] ^ __float_as_uint(__fadd_rn(b, kRoundMagic));
+    amax = fmaxf(amax, fabsf(b));
   }
-  *reinterpret_cast<uint2*>(codes) = make_uint2(packed[0], packed[1]);
-  if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
+  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
+  return diff == 0u && amax <= (float)kQmax;
+}
+
+// asymmetric uint8: clamp(rne(x / s) + zp, 0, 255); off = zp - bits(1.5 * 2^23)
+__device__ __forceinline__ bool asym_row(const float (&x)[8], const Bracket (&q)[8], const int (&off)[8],
+                                         uint2& out) {
+  uint32_t c[8], diff = 0u, range = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float a = __fmul_rn(x[k], q[k].lo), b = __fmul_rn(x[k], q[k].hi);
+    const uint32_t ta = __float_as_uint(__fadd_rn(a, kRoundMagic));
+    diff |= ta ^ __float_as_uint(__fadd_rn(b, kRoundMagic));
+    c[k] = ta + (uint32_t)off[k];  // the code when it lies in [0, 255]
+    range |= c[k];
+  }
+  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
+  return diff == 0u && (range & 0xFFFFFF00u) == 0u;
+}
+
+// The exact row: one IEEE division per element; counts saturated elements.
+__device__ __noinline__ uint2 exact_row(const float* x, const float* s, const uint8_t* zp, int scheme,
+                                        int* sat) {
+  uint32_t w[2] = {0u, 0u};
+  int n = 0;
+  for (int k = 0; k < 8; ++k) {
+    uint32_t code = 0u;
+    if (s[k] != 0.0f) {
+      const float z = __fdiv_rn(x[k], s[k]);
+      if (scheme == KVQ_FP8_E4M3_PER_TENSOR) {
+        n += fabsf(z) > 448.0f;
+        code = e4m3x2_rn(z, 0.0f) & 0xFFu;
+      } else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
+        float c = __fadd_rn(rintf(z), (float)zp[k]);
+        if (c < 0.0f || c > 255.0f) ++n;
+        code = (uint32_t)(int)fminf(fmaxf(c, 0.0f), 255.0f);
+      } else {
+        float c = rintf(z);
+        if (fabsf(c) > 127.0f) {
+          ++n;
+          c = c > 0.0f ? 127.0f : -127.0f;
+        }
+        code = (uint32_t)(int)c & 0xFFu;
+      }
+    }
+    w[k >> 2] |= code << (8 * (k & 3));
+  }
+  *sat += n;
+  return make_uint2(w[0], w[1]);
+}
+
+// Rows (b, h, i) of the new block; 16 threads per row, 8 channels each; blockIdx.z = side.
+// Bulk form (kR > 1): blockIdx.y = b * H + h and blockIdx.x a run of 16 * kR tokens of that
+// row, so no thread divides and every row of the block belongs to one head; each thread loads
+// its kR rows before quantizing any. Small form (kR == 1): blockIdx.x covers 16 consecutive
+// flattened rows.
+constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL; }
+
+template <bool kBf16, int kR, int KS, int VS>
+__global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)) ? 3 : 4)
+    quantize_rows_kernel(AppendParams p) {
+  const int side = blockIdx.z;
+  const int scheme = side ? VS : KS;  // compile-time per side
+  const int lane8 = threadIdx.x & 15;
+  const bool per_channel = side ? is_per_channel(VS) : is_per_channel(KS);
+  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR;
+  float* scale = side ? p.v_scale : p.k_scale;
+  const uint8_t* zp = side ? p.v_zp : p.k_zp;
+  const void* src_base = side ? p.v_new : p.k_new;
+  Raw8<kBf16> in[kR];
+  int rb[kR], rh[kR], ri[kR];
+  bool act[kR];
+  if constexpr (kR > 1) {
+    const int bh = blockIdx.y;
+    const int b = bh / p.H, h = bh - b * p.H;
+    const int n_b = new_count(p, b);
+#pragma unroll
+    for (int it = 0; it < kR; ++it) {
+      const int i = blockIdx.x * 16 * kR + 16 * it + (threadIdx.x >> 4);
+      rb[it] = b;
+      rh[it] = h;
+      ri[it] = i;
+      act[it] = i < n_b;
+      in[it].clear();
+      if (act[it]) in[it].load(src_base, ((size_t)bh * p.n_new + i) * kHeadDim + lane8 * 8);
+    }
+  } else {
+    const int r = blockIdx.x * 16 + (threadIdx.x >> 4);
+    const int rows = p.B * p.H * p.n_new;
+    const int i = r % p.n_new, bh = r / p.n_new;
+    rb[0] = bh / p.H;
+    rh[0] = bh - rb[0] * p.H;
+    ri[0] = i;
+    act[0] = r < rows && i < new_count(p, rb[0]);
+    in[0].clear();
+    if (act[0]) in[0].load(src_base, (size_t)r * kHeadDim + lane8 * 8);
+  }
+  Bracket q[8];
+  int off[8];
+  bool fixed_fast = true;  // the per-tensor or per-channel scales are all in the fast range
+  if (per_tensor) {
+    const Bracket whole = bracket_of(scale[0], fixed_fast);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) q[k] = whole;
+  }
+  int chan_head = -1;
+  int sat = 0;
+#pragma unroll
+  for (int it = 0; it < kR; ++it) {
+    float x[8];
+    in[it].unpack(x);
+    // per-token scale: absmax over the 16 lanes of this row (a half warp)
+    float tok_s = 0.0f;
+    if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
+      float m = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      tok_s = __fdiv_rn(m, 127.0f);
+    }
+    if (!act[it]) continue;
+    const int b = rb[it], h = rh[it];
+    const int pos = (p.paged ? p.seq_lens[b] : p.pos0) + ri[it];
+    size_t row;
+    if (!cache_row(p, b, h, pos, row)) continue;
+    if (per_channel && h != chan_head) {
+      fixed_fast = true;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        q[k] = bracket_of(scale[h * kHeadDim + lane8 * 8 + k], fixed_fast);
+        off[k] = (scheme == KVQ_UINT8_ASYM_PER_CHANNEL ? (int)zp[h * kHeadDim + lane8 * 8 + k] : 0) - kRoundMagicBits;
+      }
+      chan_head = h;
+    }
+    bool row_fast = fixed_fast;
+    if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
+      row_fast = true;
+      const Bracket tok = bracket_of(tok_s, row_fast);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) q[k] = tok;
+    }
+    uint2 codes;
+    bool ok;
+    if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
+      ok = fp8_row(x, q[0], codes);
+    else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
+      ok = asym_row(x, q, off, codes);
+    else
+      ok = sym_row<127>(x, q, codes);
+    if (!(ok && row_fast)) {
+      float sv[8];
+      uint8_t zv[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        sv[k] = scheme == KVQ_INT8_SYM_PER_TOKEN ? tok_s : scale[per_channel ? h * kHeadDim + lane8 * 8 + k : 0];
+        zv[k] = scheme == KVQ_UINT8_ASYM_PER_CHANNEL ? zp[h * kHeadDim + lane8 * 8 + k] : 0;
+      }
+      codes = exact_row(x, sv, zv, scheme, &sat);
+    }
+    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8) = codes;
+    if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
+  }
   if (sat && p.status) atomicAdd(p.status + 1, (uint32_t)sat);
 }
 
@@ -281,7 +502,7 @@ __global__ void seq_lens_advance_kernel(AppendParams p) {
 // One block per (R-token chunk, b*H + h): quantize R consecutive tokens of the combined
 // stream (old residual tokens, then the new block) into the cache at pos0 + chunk*R.
 template <int kBits>
-__global__ void __launch_bounds__(256) kivi_flush_kernel(AppendParams p, int r_old) {
+__global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int r_old) {
   constexpr int R = 128, G = 32, kQmax = (1 << kBits) - 1, kPer = 8 / kBits;
   constexpr int kRowBytes = kHeadDim * kBits / 8;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -308,66 +529,87 @@ __global__ void __launch_bounds__(256) kivi_flush_kernel(AppendParams p, int r_o
     reinterpret_cast<uint4*>(xv + tok * kHeadDim)[piece] = reinterpret_cast<const uint4*>(srcv)[piece];
   }
   __syncthreads();
-  // keys: task = (group gi, kPer adjacent channels)
-  constexpr int kKTasks = (R / G) * (kHeadDim / kPer);
-  for (int task = threadIdx.x; task < kKTasks; task += blockDim.x) {
-    const int gi = task / (kHeadDim / kPer), c0 = (task % (kHeadDim / kPer)) * kPer;
-    uint8_t bytes[G];
+  // keys: task = (group gi, 2 adjacent channels); the thread keeps the 32 tokens' 4-byte
+  // words (both channels as bf16) in registers and widens a channel when it needs it. The
+  // codes of token j sit in byte j % 4 of word j / 4; with 2-bit codes a byte holds 4
+  // channels and the two threads of neighbouring tasks combine their halves.
+  constexpr int kKTasks = (R / G) * (kHeadDim / 2);  // 256
+  static_assert(kKTasks == 256, "one key task per thread");
+  {
+    const int task = threadIdx.x;
+    const int gi = task / (kHeadDim / 2), c0 = (task % (kHeadDim / 2)) * 2;
+    uint32_t raw[G];
 #pragma unroll
-    for (int j = 0; j < G; ++j) bytes[j] = 0;
+    for (int j = 0; j < G; ++j) raw[j] = *reinterpret_cast<const uint32_t*>(xk + (gi * G + j) * kHeadDim + c0);
+    uint32_t bits[G / 4];
+#pragma unroll
+    for (int j = 0; j < G / 4; ++j) bits[j] = 0u;
     const size_t meta = (((size_t)b * p.H + h) * (size_t)(p.cap / G) + (size_t)(pos0 / G + gi)) * kHeadDim;
+    const int shift0 = (c0 % kPer) * kBits;  // position of channel c0 inside its byte
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int d = c0 + k;
-      float lo = bf16_bits_to_float(xk[(gi * G) * kHeadDim + d]), hi = lo;
+    for (int k = 0; k < 2; ++k) {
+      auto val = [&](int j) { return __uint_as_float(k ? (raw[j] & 0xFFFF0000u) : (raw[j] << 16)); };
+      float lo = val(0), hi = lo;
+#pragma unroll
       for (int j = 1; j < G; ++j) {
-        const float v = bf16_bits_to_float(xk[(gi * G + j) * kHeadDim + d]);
-        lo = fminf(lo, v);
-        hi = fmaxf(hi, v);
+        lo = fminf(lo, val(j));
+        hi = fmaxf(hi, val(j));
       }
       if (lo == 0.0f) lo = 0.0f;
       if (hi == 0.0f) hi = 0.0f;
-      const float s = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
-      p.k_scale[meta + d] = s;
-      p.k_zero[meta + d] = lo;
-      for (int j = 0; j < G; ++j) {
-        int q = 0;
-        if (s != 0.0f) {
-          const float v = bf16_bits_to_float(xk[(gi * G + j) * kHeadDim + d]);
-          float r = rintf(__fdiv_rn(__fsub_rn(v, lo), s));
-          r = fminf(fmaxf(r, 0.0f), (float)kQmax);
-          q = (int)r;
-        }
-        bytes[j] |= (uint8_t)(q << (k * kBits));
+      const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+      p.k_scale[meta + c0 + k] = sc;
+      p.k_zero[meta + c0 + k] = lo;
+      if (sc != 0.0f) {
+        const Recip rq = recip_of(sc);
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+          bits[j / 4] |= (uint32_t)int_of(quot_code(__fsub_rn(val(j), lo), rq, 0.0f, (float)kQmax))
+                         << (8 * (j % 4) + shift0 + k * kBits);
       }
     }
-    for (int j = 0; j < G; ++j) kcodes[(gi * G + j) * kRowBytes + c0 / kPer] = bytes[j];
+#pragma unroll
+    for (int w = 0; w < G / 4; ++w) {
+      uint32_t word = bits[w];
+      if constexpr (kBits == 2) word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      if (kBits == 4 || (c0 % kPer) == 0) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) kcodes[(gi * G + 4 * w + t) * kRowBytes + c0 / kPer] = (uint8_t)(word >> (8 * t));
+      }
+    }
   }
-  // values: task = (token, channel group)
+  // values: task = (token, channel group); 32 channels = four 16-byte shared loads
   for (int task = threadIdx.x; task < R * (kHeadDim / G); task += blockDim.x) {
     const int tok = task / (kHeadDim / G), j = task % (kHeadDim / G);
-    const uint16_t* row = xv + tok * kHeadDim + j * G;
-    float lo = bf16_bits_to_float(row[0]), hi = lo;
+    const uint4* row = reinterpret_cast<const uint4*>(xv + tok * kHeadDim + j * G);
+    uint32_t raw[G / 2];
+#pragma unroll
+    for (int q4 = 0; q4 < G / 8; ++q4) {
+      const uint4 w = row[q4];
+      raw[4 * q4] = w.x;
+      raw[4 * q4 + 1] = w.y;
+      raw[4 * q4 + 2] = w.z;
+      raw[4 * q4 + 3] = w.w;
+    }
+    auto val = [&](int i) { return __uint_as_float((i & 1) ? (raw[i >> 1] & 0xFFFF0000u) : (raw[i >> 1] << 16)); };
+    float lo = val(0), hi = lo;
+#pragma unroll
     for (int i = 1; i < G; ++i) {
-      const float v = bf16_bits_to_float(row[i]);
-      lo = fminf(lo, v);
-      hi = fmaxf(hi, v);
+      lo = fminf(lo, val(i));
+      hi = fmaxf(hi, val(i));
     }
     if (lo == 0.0f) lo = 0.0f;
     if (hi == 0.0f) hi = 0.0f;
-    const float s = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+    const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
     uint32_t words[G * kBits / 32];
 #pragma unroll
     for (int w = 0; w < G * kBits / 32; ++w) words[w] = 0u;
+    if (sc != 0.0f) {
+      const Recip rq = recip_of(sc);
 #pragma unroll
-    for (int i = 0; i < G; ++i) {
-      int q = 0;
-      if (s != 0.0f) {
-        float r = rintf(__fdiv_rn(__fsub_rn(bf16_bits_to_float(row[i]), lo), s));
-        r = fminf(fmaxf(r, 0.0f), (float)kQmax);
-        q = (int)r;
-      }
-      words[(i * kBits) / 32] |= (uint32_t)q << ((i * kBits) % 32);
+      for (int i = 0; i < G; ++i)
+        words[(i * kBits) / 32] |= (uint32_t)int_of(quot_code(__fsub_rn(val(i), lo), rq, 0.0f, (float)kQmax))
+                                   << ((i * kBits) % 32);
     }
     const size_t crow = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)(pos0 + tok);
     uint8_t* dst = static_cast<uint8_t*>(p.v_codes) + crow * kRowBytes + j * (G * kBits / 8);
@@ -376,7 +618,7 @@ __global__ void __launch_bounds__(256) kivi_flush_kernel(AppendParams p, int r_o
     } else {
       *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
     }
-    p.v_scale[crow * (kHeadDim / G) + j] = s;
+    p.v_scale[crow * (kHeadDim / G) + j] = sc;
     p.v_zero[crow * (kHeadDim / G) + j] = lo;
   }
   __syncthreads();
@@ -480,6 +722,47 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
 }
 
 // ------------------------------------------------------------------ launchers
+template <int KS, int VS>
+cudaError_t launch_quantize_rows_pair(const AppendParams& p, long long rows, cudaStream_t st) {
+  // four rows per thread once every (batch, kv head) row has enough new tokens
+  if (p.n_new >= 64 && rows >= 16LL * 4 * 148 * 8 && p.B * p.H <= 65535) {
+    dim3 grid((unsigned)((p.n_new + 64 - 1) / 64), (unsigned)(p.B * p.H), 2);
+    if (p.in_bf16)
+      quantize_rows_kernel<true, 4, KS, VS><<<grid, 256, 0, st>>>(p);
+    else
+      quantize_rows_kernel<false, 4, KS, VS><<<grid, 256, 0, st>>>(p);
+  } else {
+    dim3 grid((unsigned)((rows + 15) / 16), 1, 2);
+    if (p.in_bf16)
+      quantize_rows_kernel<true, 1, KS, VS><<<grid, 256, 0, st>>>(p);
+    else
+      quantize_rows_kernel<false, 1, KS, VS><<<grid, 256, 0, st>>>(p);
+  }
+  return cudaSuccess;
+}
+
+bool append_pair_supported(int ks, int vs) {
+  if (is_kivi(ks) || is_kivi(vs)) return ks == vs;
+  constexpr int F = KVQ_FP8_E4M3_PER_TENSOR, T = KVQ_INT8_SYM_PER_TENSOR, K = KVQ_INT8_SYM_PER_TOKEN,
+                C = KVQ_INT8_SYM_PER_CHANNEL, U = KVQ_UINT8_ASYM_PER_CHANNEL;
+  const int pairs[][2] = {{F, F}, {T, T}, {K, K}, {C, C}, {U, U}, {T, U}, {C, U}, {K, U}, {T, K}, {F, T}, {T, F}};
+  for (const auto& pr : pairs)
+    if (pr[0] == ks && pr[1] == vs) return true;
+  return false;
+}
+
+cudaError_t launch_quantize_rows(const AppendParams& p, long long rows, cudaStream_t st) {
+  constexpr int F = KVQ_FP8_E4M3_PER_TENSOR, T = KVQ_INT8_SYM_PER_TENSOR, K = KVQ_INT8_SYM_PER_TOKEN,
+                C = KVQ_INT8_SYM_PER_CHANNEL, U = KVQ_UINT8_ASYM_PER_CHANNEL;
+  const int ks = p.k_scheme, vs = p.v_scheme;
+#define KVQ_PAIR(A, B) \
+  if (ks == A && vs == B) return launch_quantize_rows_pair<A, B>(p, rows, st);
+  KVQ_PAIR(F, F) KVQ_PAIR(T, T) KVQ_PAIR(K, K) KVQ_PAIR(C, C) KVQ_PAIR(U, U)
+  KVQ_PAIR(T, U) KVQ_PAIR(C, U) KVQ_PAIR(K, U) KVQ_PAIR(T, K) KVQ_PAIR(F, T) KVQ_PAIR(T, F)
+#undef KVQ_PAIR
+  return cudaErrorNotSupported;
+}
+
 cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
                           int flushed, int r_new, cudaStream_t st) {
   const bool kivi = is_kivi(p.k_scheme);
@@ -523,11 +806,8 @@ cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool cali
     count_launches(3);
   }
   const long long rows = (long long)p.B * p.H * p.n_new;
-  dim3 grid((unsigned)((rows + 15) / 16), 2);
-  if (p.in_bf16)
-    quantize_rows_kernel<true><<<grid, 256, 0, st>>>(p);
-  else
-    quantize_rows_kernel<false><<<grid, 256, 0, st>>>(p);
+  const cudaError_t e = launch_quantize_rows(p, rows, st);
+  if (e != cudaSuccess) return e;
   count_launches(1);
   if (p.paged) {
     seq_lens_advance_kernel<<<(p.B + 255) / 256, 256, 0, st>>>(p);

@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <utility>
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -759,6 +760,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
   using C = Cfg<KS, VS, PAGED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+  grid_dependency_wait();    // the cache, the queries and the plan come from earlier kernels
+  grid_launch_dependents();  // the merge may be scheduled now; it waits for this grid to finish
   const Sched sc = make_sched(p);
   const int tb = blockIdx.x * sc.W;
   const int te = min(sc.N, tb + sc.W);
@@ -955,6 +958,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
   __shared__ float s_m[128], s_w[128];
   __shared__ float s_M, s_L;
+  grid_dependency_wait();  // the partials of the decode kernel
   const int pair = blockIdx.x, j = blockIdx.y, dd = threadIdx.x;
   const int per_seq = p.Hkv * p.HG;
   const int b = pair / per_seq, hh = pair % per_seq, hk = hh / p.HG, hg = hh % p.HG;
@@ -1019,6 +1023,7 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeParams p) {
   __shared__ int warp_sum[32];
   __shared__ int carry;
+  grid_dependency_wait();  // sequence lengths advanced by the append
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -1122,6 +1127,14 @@ const Variant* find_variant(int k, int v, int paged) {
       variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_UINT8_ASYM_PER_CHANNEL, true>(),
       variant<KVQ_INT8_SYM_PER_CHANNEL, KVQ_UINT8_ASYM_PER_CHANNEL, false>(),
       variant<KVQ_INT8_SYM_PER_CHANNEL, KVQ_UINT8_ASYM_PER_CHANNEL, true>(),
+      variant<KVQ_INT8_SYM_PER_TOKEN, KVQ_UINT8_ASYM_PER_CHANNEL, false>(),
+      variant<KVQ_INT8_SYM_PER_TOKEN, KVQ_UINT8_ASYM_PER_CHANNEL, true>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_INT8_SYM_PER_TOKEN, false>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_INT8_SYM_PER_TOKEN, true>(),
+      variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_INT8_SYM_PER_TENSOR, false>(),
+      variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_INT8_SYM_PER_TENSOR, true>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, false>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, true>(),
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
   };
@@ -1139,6 +1152,22 @@ int sm_count() {
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace
@@ -1176,9 +1205,16 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
   const int box = p.paged ? p.page_size : var->ts;
   if (!make_map(&tk, p.k_codes, kr, rows, box) || !make_map(&tv, p.v_codes, vr, rows, box))
     return cudaErrorInvalidValue;
-  if (p.paged) plan_kernel<<<1, 1024, 0, st>>>(p);
-  var->kernel<<<ncta, kThreads, var->smem, st>>>(p, tk, tv);
-  merge_kernel<<<dim3(p.n_pairs, 8), 128, 0, st>>>(p);
+  // Programmatic dependent launches: each kernel may be scheduled while its predecessor
+  // drains and waits in griddepcontrol.wait, hiding the launch gaps between the three.
+  if (p.paged) {
+    e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, p);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_pdl(var->kernel, dim3(ncta), dim3(kThreads), (size_t)var->smem, st, p, tk, tv);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(merge_kernel, dim3(p.n_pairs, 8), dim3(128), 0, st, p);
+  if (e != cudaSuccess) return e;
   count_launches(p.paged ? 3 : 2);
   return cudaGetLastError();
 }

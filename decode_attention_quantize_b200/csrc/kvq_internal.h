@@ -74,7 +74,7 @@ struct DecodeParams {
   // workspace
   float* part_o;                // [slots, 8, 128]
   float* part_ml;               // [slots, 8, 2]
-  int32_t* plan;                // paged: [B + 1] tile prefix over sequences
+  int32_t* plan;                // paged: [2B + 2] tile prefix over sequences, then lengths
   int ncta;
   int n_pairs;
   int ts;                       // tokens per quantized tile of the chosen kernel
@@ -92,5 +92,6 @@ cudaError_t launch_dequantize(const DequantParams& p, cudaStream_t st);
 // Returns cudaErrorNotSupported when the (k_scheme, v_scheme, layout) pair has no kernel.
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st);
 bool decode_supported(int k_scheme, int v_scheme, int paged);
+bool append_pair_supported(int k_scheme, int v_scheme);
 
 }  // namespace kvq

@@ -62,6 +62,41 @@ def test_outliers_x100_int8_per_channel():
                  outlier=100.0)
 
 
+# ------------------------------------------------------------------ bulk prefill (four rows per thread)
+# 4 x 2 x 9600 rows is past the size where the append switches to its bulk form; every pair
+# the library accepts goes through it, the oracle recomputing every code bit for bit.
+BULK_PAIRS = [
+    (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TENSOR),
+    (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN), (S.INT8_SYM_PER_CHANNEL, S.INT8_SYM_PER_CHANNEL),
+    (S.UINT8_ASYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL), (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
+    (S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL), (S.INT8_SYM_PER_TOKEN, S.UINT8_ASYM_PER_CHANNEL),
+    (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TOKEN), (S.FP8_E4M3_PER_TENSOR, S.INT8_SYM_PER_TENSOR),
+    (S.INT8_SYM_PER_TENSOR, S.FP8_E4M3_PER_TENSOR),
+]
+
+
+@pytest.mark.parametrize("ks,vs", BULK_PAIRS)
+def test_bulk_prefill_every_pair(ks, vs):
+    H.dense_case(B=4, Hq=8, Hkv=2, ks=ks, vs=vs, prefill=9600, steps=1, outlier=100.0)
+
+
+def test_bulk_prefill_fp32_inputs():
+    H.dense_case(B=4, Hq=8, Hkv=2, ks=S.INT8_SYM_PER_CHANNEL, vs=S.UINT8_ASYM_PER_CHANNEL, prefill=9600, steps=1,
+                 bf16=False)
+
+
+def test_bulk_prefill_paged():
+    B, Hq, Hkv = 4, 8, 2
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL,
+                                                    lens=[9600, 5000, 1, 9001], steps=0)
+    oc.append(K, V, True, calibrate=True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc, "bulk paged prefill")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), True, "bulk paged decode")
+    assert gc.status()[0] == 0
+
+
 # ------------------------------------------------------------------ KIVI
 @pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2])
 @pytest.mark.parametrize("prefill", [44, 128, 129, 300, 384, 385])
