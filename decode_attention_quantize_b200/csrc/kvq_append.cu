@@ -240,25 +240,21 @@ __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
 }
 
 // ------------------------------------------------------------------ 8-bit quantize-store
-// Bracketing reciprocals. With r = RN(1/s), lo = RN(r * (1 - 2^-20)) and hi = RN(r * (1 + 2^-20)),
-// the products RN(x * lo) and RN(x * hi) are floats on either side of x / s (for s and x * r in
-// the normal range), hence also on either side of RN(x / s). Every code map used here is monotone
-// (round half to even then clamp; E4M3 round-to-nearest-even with saturation), so when the two
-// products give the same code, that code is the code of RN(x / s). A row whose products disagree
-// anywhere, or that may saturate, is redone element by element with the IEEE division.
-struct Bracket {
-  float lo, hi;
-};
-
-// `fast` is cleared when s is outside 2^-120 .. 2^120 (zero included): such rows go exact.
-__device__ __forceinline__ Bracket bracket_of(float s, bool& fast) {
-  Bracket q;
-  const float r = __fdiv_rn(1.0f, s);
-  q.lo = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
-  q.hi = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
-  fast &= s >= 7.52316385e-37f && s <= 1.32922800e+36f;
-  return q;
+// The quotient RN(x / s) without a division per element (Markstein's fma correction, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", 1990): with y = RN(1/s),
+// q = RN(x * y) and the residual e = RN(q * s - x) (exact under fma), RN(q - e * y) is the
+// correctly rounded quotient. For bf16 x this has been checked against IEEE division for every
+// pair of bf16 and fp32 significands (the operations scale exactly with the exponents while the
+// intermediate results stay normal, which the range of s below guarantees for every x that can
+// produce a nonzero code). Writing the residual as q * s - x keeps the sign of a zero quotient.
+// fp32 inputs divide: they are not covered by that check.
+__device__ __forceinline__ float quot(float x, float s, float y, float& q) {
+  q = __fmul_rn(x, y);
+  return __fmaf_rn(-__fmaf_rn(q, s, -x), y, q);
 }
+
+// s with a normal reciprocal and room for the correction's residual: 2^-60 .. 2^60
+__device__ __forceinline__ bool quot_range(float s) { return s >= 8.67361738e-19f && s <= 1.15292150e+18f; }
 
 // Eight input elements, kept as loaded until they are quantized.
 template <bool kBf16>
@@ -299,92 +295,105 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t w0, uint32_t w1, uin
   return prmt(prmt(w0, w1, 0x0040u), prmt(w2, w3, 0x0040u), 0x5410u);
 }
 
-// Fast rows. Each returns false when the row must be redone exactly.
-__device__ __forceinline__ bool fp8_row(const float (&x)[8], const Bracket& q, uint2& out) {
-  uint32_t c[4], diff = 0u;
-  float amax = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float a0 = __fmul_rn(x[2 * k], q.lo), a1 = __fmul_rn(x[2 * k + 1], q.lo);
-    const float b0 = __fmul_rn(x[2 * k], q.hi), b1 = __fmul_rn(x[2 * k + 1], q.hi);
-    c[k] = e4m3x2_rn(a0, a1);
-    diff |= c[k] ^ e4m3x2_rn(b0, b1);
-    amax = fmaxf(amax, fmaxf(fabsf(b0), fabsf(b1)));  // |x * hi| >= |RN(x / s)|
+// Scales of one row's eight channels (one value repeated for per-tensor and per-token).
+struct Scales8 {
+  float s[8], y[8];
+  int zp[8];  // asymmetric only
+};
+
+// The code of one element from its exact quotient z (|z| < 2^22), counting saturation.
+__device__ __forceinline__ uint32_t code_of(float z, int zp, int scheme, int& sat) {
+  if (scheme == KVQ_FP8_E4M3_PER_TENSOR) {
+    sat += fabsf(z) > 448.0f;
+    return e4m3x2_rn(z, 0.0f) & 0xFFu;
   }
-  out = make_uint2(prmt(c[0], c[1], 0x5410u), prmt(c[2], c[3], 0x5410u));
-  return diff == 0u && amax <= 448.0f;
+  if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
+    const float c = __fadd_rn(rintf(z), (float)zp);
+    sat += c < 0.0f || c > 255.0f;
+    return (uint32_t)(int)fminf(fmaxf(c, 0.0f), 255.0f);
+  }
+  float c = rintf(z);
+  if (fabsf(c) > 127.0f) {
+    ++sat;
+    c = c > 0.0f ? 127.0f : -127.0f;
+  }
+  return (uint32_t)(int)c & 0xFFu;
 }
 
-// symmetric: clamp(rne(x / s), -qmax, qmax); y + 1.5 * 2^23 holds rne(y) in its low bits
-template <int kQmax>
-__device__ __forceinline__ bool sym_row(const float (&x)[8], const Bracket (&q)[8], uint2& out) {
-  uint32_t c[8], diff = 0u;
-  float amax = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float a = __fmul_rn(x[k], q[k].lo), b = __fmul_rn(x[k], q[k].hi);
-    c[k] = __float_as_uint(__fadd_rn(a, kRoundMagic));
-    diff |= c[k] ^ __float_as_uint(__fadd_rn(b, kRoundMagic));
-    amax = fmaxf(amax, fabsf(b));
-  }
-  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
-  return diff == 0u && amax <= (float)kQmax;
-}
-
-// asymmetric uint8: clamp(rne(x / s) + zp, 0, 255); off = zp - bits(1.5 * 2^23)
-__device__ __forceinline__ bool asym_row(const float (&x)[8], const Bracket (&q)[8], const int (&off)[8],
-                                         uint2& out) {
-  uint32_t c[8], diff = 0u, range = 0u;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float a = __fmul_rn(x[k], q[k].lo), b = __fmul_rn(x[k], q[k].hi);
-    const uint32_t ta = __float_as_uint(__fadd_rn(a, kRoundMagic));
-    diff |= ta ^ __float_as_uint(__fadd_rn(b, kRoundMagic));
-    c[k] = ta + (uint32_t)off[k];  // the code when it lies in [0, 255]
-    range |= c[k];
-  }
-  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
-  return diff == 0u && (range & 0xFFFFFF00u) == 0u;
-}
-
-// The exact row: one IEEE division per element; counts saturated elements.
-__device__ __noinline__ uint2 exact_row(const float* x, const float* s, const uint8_t* zp, int scheme,
-                                        int* sat) {
+// The slow form of a row: element by element, dividing where the quotient may be out of the
+// correction's range (and for fp32 inputs); counts saturation.
+template <bool kBf16>
+__device__ __forceinline__ uint2 careful_row(const float (&x)[8], const Scales8& sc, bool fast, int scheme, int& sat) {
   uint32_t w[2] = {0u, 0u};
-  int n = 0;
+#pragma unroll
   for (int k = 0; k < 8; ++k) {
     uint32_t code = 0u;
-    if (s[k] != 0.0f) {
-      const float z = __fdiv_rn(x[k], s[k]);
-      if (scheme == KVQ_FP8_E4M3_PER_TENSOR) {
-        n += fabsf(z) > 448.0f;
-        code = e4m3x2_rn(z, 0.0f) & 0xFFu;
-      } else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
-        float c = __fadd_rn(rintf(z), (float)zp[k]);
-        if (c < 0.0f || c > 255.0f) ++n;
-        code = (uint32_t)(int)fminf(fmaxf(c, 0.0f), 255.0f);
+    if (sc.s[k] != 0.0f) {
+      float q, z;
+      if (kBf16 && fast) {
+        z = quot(x[k], sc.s[k], sc.y[k], q);
+        if (!(fabsf(q) < 4194304.0f)) z = __fdiv_rn(x[k], sc.s[k]);  // huge or not finite
       } else {
-        float c = rintf(z);
-        if (fabsf(c) > 127.0f) {
-          ++n;
-          c = c > 0.0f ? 127.0f : -127.0f;
-        }
-        code = (uint32_t)(int)c & 0xFFu;
+        z = __fdiv_rn(x[k], sc.s[k]);
       }
+      code = code_of(z, sc.zp[k], scheme, sat);
     }
     w[k >> 2] |= code << (8 * (k & 3));
   }
-  *sat += n;
   return make_uint2(w[0], w[1]);
 }
+
+// Fast rows (bf16 inputs, s in range): false when a value may saturate or is out of range.
+__device__ __forceinline__ bool fp8_row(const float (&x)[8], const Scales8& sc, uint2& out) {
+  uint32_t c[4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float q0, q1;
+    const float z0 = quot(x[2 * k], sc.s[0], sc.y[0], q0), z1 = quot(x[2 * k + 1], sc.s[0], sc.y[0], q1);
+    c[k] = e4m3x2_rn(z0, z1);
+    amax = fmaxf(amax, fmaxf(fabsf(q0), fabsf(q1)));
+  }
+  out = make_uint2(prmt(c[0], c[1], 0x5410u), prmt(c[2], c[3], 0x5410u));
+  return amax < 447.9f;  // |z| < 448: nothing saturates (q is within a few ulps of z)
+}
+
+// symmetric: clamp(rne(z), -127, 127); z + 1.5 * 2^23 holds rne(z) (ties to even) in its low bits
+__device__ __forceinline__ bool sym_row(const float (&x)[8], const Scales8& sc, uint2& out) {
+  uint32_t c[8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float q;
+    const float z = quot(x[k], sc.s[k], sc.y[k], q);
+    c[k] = __float_as_uint(__fadd_rn(z, kRoundMagic));
+    amax = fmaxf(amax, fabsf(q));
+  }
+  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
+  return amax < 127.25f;  // |z| < 127.5: no clamp, no saturation
+}
+
+// asymmetric uint8: rne(z) + zp must lie in [0, 255]
+__device__ __forceinline__ bool asym_row(const float (&x)[8], const Scales8& sc, uint2& out) {
+  uint32_t c[8], range = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float q;
+    const float z = quot(x[k], sc.s[k], sc.y[k], q);
+    c[k] = __float_as_uint(__fadd_rn(z, kRoundMagic)) - (uint32_t)(kRoundMagicBits - sc.zp[k]);
+    range |= c[k];
+  }
+  out = make_uint2(pack_low_bytes(c[0], c[1], c[2], c[3]), pack_low_bytes(c[4], c[5], c[6], c[7]));
+  return (range & 0xFFFFFF00u) == 0u;  // also fails for huge or non-finite quotients
+}
+
+constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL; }
 
 // Rows (b, h, i) of the new block; 16 threads per row, 8 channels each; blockIdx.z = side.
 // Bulk form (kR > 1): blockIdx.y = b * H + h and blockIdx.x a run of 16 * kR tokens of that
 // row, so no thread divides and every row of the block belongs to one head; each thread loads
 // its kR rows before quantizing any. Small form (kR == 1): blockIdx.x covers 16 consecutive
 // flattened rows.
-constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL; }
-
 template <bool kBf16, int kR, int KS, int VS>
 __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)) ? 3 : 4)
     quantize_rows_kernel(AppendParams p) {
@@ -399,10 +408,12 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   Raw8<kBf16> in[kR];
   int rb[kR], rh[kR], ri[kR];
   bool act[kR];
+  int pos_base = 0;  // bulk form: the sequence's first new position, read once (stores may alias it)
   if constexpr (kR > 1) {
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh - b * p.H;
     const int n_b = new_count(p, b);
+    pos_base = p.paged ? p.seq_lens[b] : p.pos0;
 #pragma unroll
     for (int it = 0; it < kR; ++it) {
       const int i = blockIdx.x * 16 * kR + 16 * it + (threadIdx.x >> 4);
@@ -424,13 +435,18 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
     in[0].clear();
     if (act[0]) in[0].load(src_base, (size_t)r * kHeadDim + lane8 * 8);
   }
-  Bracket q[8];
-  int off[8];
-  bool fixed_fast = true;  // the per-tensor or per-channel scales are all in the fast range
-  if (per_tensor) {
-    const Bracket whole = bracket_of(scale[0], fixed_fast);
+  Scales8 sc;
+  bool fixed_fast = true;  // the per-tensor or per-channel scales are all in the correction's range
 #pragma unroll
-    for (int k = 0; k < 8; ++k) q[k] = whole;
+  for (int k = 0; k < 8; ++k) sc.zp[k] = 0;
+  if (per_tensor) {
+    const float s0 = scale[0], y0 = __frcp_rn(s0);
+    fixed_fast = quot_range(s0);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      sc.s[k] = s0;
+      sc.y[k] = y0;
+    }
   }
   int chan_head = -1;
   int sat = 0;
@@ -450,43 +466,42 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
     }
     if (!act[it]) continue;
     const int b = rb[it], h = rh[it];
-    const int pos = (p.paged ? p.seq_lens[b] : p.pos0) + ri[it];
+    const int pos = (kR > 1 ? pos_base : (p.paged ? p.seq_lens[b] : p.pos0)) + ri[it];
     size_t row;
     if (!cache_row(p, b, h, pos, row)) continue;
     if (per_channel && h != chan_head) {
       fixed_fast = true;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        q[k] = bracket_of(scale[h * kHeadDim + lane8 * 8 + k], fixed_fast);
-        off[k] = (scheme == KVQ_UINT8_ASYM_PER_CHANNEL ? (int)zp[h * kHeadDim + lane8 * 8 + k] : 0) - kRoundMagicBits;
+        const int c = h * kHeadDim + lane8 * 8 + k;
+        sc.s[k] = scale[c];
+        sc.y[k] = __frcp_rn(sc.s[k]);
+        fixed_fast &= quot_range(sc.s[k]);
+        if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) sc.zp[k] = zp[c];
       }
       chan_head = h;
     }
     bool row_fast = fixed_fast;
     if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
-      row_fast = true;
-      const Bracket tok = bracket_of(tok_s, row_fast);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q[k] = tok;
-    }
-    uint2 codes;
-    bool ok;
-    if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
-      ok = fp8_row(x, q[0], codes);
-    else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
-      ok = asym_row(x, q, off, codes);
-    else
-      ok = sym_row<127>(x, q, codes);
-    if (!(ok && row_fast)) {
-      float sv[8];
-      uint8_t zv[8];
+      const float y = __frcp_rn(tok_s);
+      row_fast = quot_range(tok_s);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        sv[k] = scheme == KVQ_INT8_SYM_PER_TOKEN ? tok_s : scale[per_channel ? h * kHeadDim + lane8 * 8 + k : 0];
-        zv[k] = scheme == KVQ_UINT8_ASYM_PER_CHANNEL ? zp[h * kHeadDim + lane8 * 8 + k] : 0;
+        sc.s[k] = tok_s;
+        sc.y[k] = y;
       }
-      codes = exact_row(x, sv, zv, scheme, &sat);
     }
+    uint2 codes;
+    bool ok = false;
+    if (kBf16 && row_fast) {
+      if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
+        ok = fp8_row(x, sc, codes);
+      else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
+        ok = asym_row(x, sc, codes);
+      else
+        ok = sym_row(x, sc, codes);
+    }
+    if (!ok) codes = careful_row<kBf16>(x, sc, row_fast, scheme, sat);  // saturating, out of range, fp32
     *reinterpret_cast<uint2*>(static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8) = codes;
     if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
   }
