@@ -37,49 +37,6 @@ __device__ __forceinline__ void load8(const void* base, size_t elem, float (&x)[
   }
 }
 
-// KIVI codes without a division per element. With r = RN(1/s) (s normal and not near the
-// ends of the range), y = RN(x * r) lies within 2^-22 * |y| of RN(x / s). Rounding half to
-// even and clamping is monotone, so when no rounding boundary lies within 2^-20 * |y| of y,
-// the code of y is the code of RN(x / s); otherwise the IEEE division decides. Rounding uses
-// the 1.5 * 2^23 add-and-subtract identity (exact round-half-to-even for |v| < 2^22) so the
-// common path stays on the FP32 pipes.
-struct Recip {
-  float s, r;
-  bool fast;
-};
-
-__device__ __forceinline__ Recip recip_of(float s) {
-  Recip q;
-  q.s = s;
-  q.r = __fdiv_rn(1.0f, s);
-  q.fast = s >= 7.52316385e-37f && s <= 1.32922800e+36f;  // 2^-120 .. 2^120
-  return q;
-}
-
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-constexpr int kRoundMagicBits = 0x4B400000;
-
-__device__ __forceinline__ float rne_small(float v) { return __fsub_rn(__fadd_rn(v, kRoundMagic), kRoundMagic); }
-// an integer-valued float in [-2^22, 2^22] -> int
-__device__ __forceinline__ int int_of(float v) { return __float_as_int(__fadd_rn(v, kRoundMagic)) - kRoundMagicBits; }
-
-// The rare exact fallback, kept out of line so the common path stays compact.
-__device__ __noinline__ float slow_quot_code(float x, float s, float lo, float hi) {
-  return fminf(fmaxf(rintf(__fdiv_rn(x, s)), lo), hi);
-}
-
-// clamp(rne(RN(x / s)), lo, hi) for integer lo < hi with |lo|, |hi| < 2^21
-__device__ __forceinline__ float quot_code(float x, const Recip& q, float lo, float hi) {
-  if (q.fast) {
-    const float y = fminf(fmaxf(__fmul_rn(x, q.r), lo - 1.0f), hi + 1.0f);
-    const float r = rne_small(y);
-    const float d = fabsf(__fsub_rn(y, r));                 // exact, <= 0.5
-    if (__fsub_rn(0.5f, d) > __fmul_rn(fabsf(y), 9.5367431640625e-07f))  // boundary farther than 2^-20|y|
-      return fminf(fmaxf(r, lo), hi);
-  }
-  return slow_quot_code(x, q.s, lo, hi);
-}
-
 // Two E4M3 codes, RN-even with saturation: lo -> low byte, hi -> high byte.
 __device__ __forceinline__ uint32_t e4m3x2_rn(float lo, float hi) {
   uint16_t r;
@@ -240,22 +197,6 @@ __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
 }
 
 // ------------------------------------------------------------------ 8-bit quantize-store
-// The quotient RN(x / s) without a division per element (Markstein's fma correction, "Computation
-// of elementary functions on the IBM RISC System/6000 processor", 1990): with y = RN(1/s),
-// q = RN(x * y) and the residual e = RN(q * s - x) (exact under fma), RN(q - e * y) is the
-// correctly rounded quotient. For bf16 x this has been checked against IEEE division for every
-// pair of bf16 and fp32 significands (the operations scale exactly with the exponents while the
-// intermediate results stay normal, which the range of s below guarantees for every x that can
-// produce a nonzero code). Writing the residual as q * s - x keeps the sign of a zero quotient.
-// fp32 inputs divide: they are not covered by that check.
-__device__ __forceinline__ float quot(float x, float s, float y, float& q) {
-  q = __fmul_rn(x, y);
-  return __fmaf_rn(-__fmaf_rn(q, s, -x), y, q);
-}
-
-// s with a normal reciprocal and room for the correction's residual: 2^-60 .. 2^60
-__device__ __forceinline__ bool quot_range(float s) { return s >= 8.67361738e-19f && s <= 1.15292150e+18f; }
-
 // Eight input elements, kept as loaded until they are quantized.
 template <bool kBf16>
 struct Raw8;
@@ -321,8 +262,7 @@ __device__ __forceinline__ uint32_t code_of(float z, int zp, int scheme, int& sa
 }
 
 // The slow form of a row: element by element, dividing where the quotient may be out of the
-// correction's range (and for fp32 inputs); counts saturation.
-template <bool kBf16>
+// correction's range; counts saturation.
 __device__ __forceinline__ uint2 careful_row(const float (&x)[8], const Scales8& sc, bool fast, int scheme, int& sat) {
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -330,7 +270,7 @@ __device__ __forceinline__ uint2 careful_row(const float (&x)[8], const Scales8&
     uint32_t code = 0u;
     if (sc.s[k] != 0.0f) {
       float q, z;
-      if (kBf16 && fast) {
+      if (fast) {
         z = quot(x[k], sc.s[k], sc.y[k], q);
         if (!(fabsf(q) < 4194304.0f)) z = __fdiv_rn(x[k], sc.s[k]);  // huge or not finite
       } else {
@@ -343,7 +283,7 @@ __device__ __forceinline__ uint2 careful_row(const float (&x)[8], const Scales8&
   return make_uint2(w[0], w[1]);
 }
 
-// Fast rows (bf16 inputs, s in range): false when a value may saturate or is out of range.
+// Fast rows (s in range): false when a value may saturate or is out of range.
 __device__ __forceinline__ bool fp8_row(const float (&x)[8], const Scales8& sc, uint2& out) {
   uint32_t c[4];
   float amax = 0.0f;
@@ -493,7 +433,7 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
     }
     uint2 codes;
     bool ok = false;
-    if (kBf16 && row_fast) {
+    if (row_fast) {
       if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
         ok = fp8_row(x, sc, codes);
       else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
@@ -501,7 +441,7 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
       else
         ok = sym_row(x, sc, codes);
     }
-    if (!ok) codes = careful_row<kBf16>(x, sc, row_fast, scheme, sat);  // saturating, out of range, fp32
+    if (!ok) codes = careful_row(x, sc, row_fast, scheme, sat);  // may saturate, or out of range
     *reinterpret_cast<uint2*>(static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8) = codes;
     if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
   }
@@ -514,6 +454,15 @@ __global__ void seq_lens_advance_kernel(AppendParams p) {
 }
 
 // ------------------------------------------------------------------ KIVI
+// Code of d = RN(x - min) >= 0 with step s: rne(RN(d / s)); d <= max - min keeps it <= qmax.
+template <int kQmax>
+__device__ __forceinline__ uint32_t kivi_code(float d, float s, float y, bool fast) {
+  float q;
+  const float z = fast ? quot(d, s, y, q) : __fdiv_rn(d, s);
+  const uint32_t c = __float_as_uint(__fadd_rn(z, kRoundMagic)) - (uint32_t)kRoundMagicBits;
+  return c < (uint32_t)kQmax ? c : (uint32_t)kQmax;
+}
+
 // One block per (R-token chunk, b*H + h): quantize R consecutive tokens of the combined
 // stream (old residual tokens, then the new block) into the cache at pos0 + chunk*R.
 template <int kBits>
@@ -576,11 +525,11 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
       p.k_scale[meta + c0 + k] = sc;
       p.k_zero[meta + c0 + k] = lo;
       if (sc != 0.0f) {
-        const Recip rq = recip_of(sc);
+        const float y = __frcp_rn(sc);
+        const bool fast = quot_range(sc);
 #pragma unroll
         for (int j = 0; j < G; ++j)
-          bits[j / 4] |= (uint32_t)int_of(quot_code(__fsub_rn(val(j), lo), rq, 0.0f, (float)kQmax))
-                         << (8 * (j % 4) + shift0 + k * kBits);
+          bits[j / 4] |= kivi_code<kQmax>(__fsub_rn(val(j), lo), sc, y, fast) << (8 * (j % 4) + shift0 + k * kBits);
       }
     }
 #pragma unroll
@@ -620,11 +569,11 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
 #pragma unroll
     for (int w = 0; w < G * kBits / 32; ++w) words[w] = 0u;
     if (sc != 0.0f) {
-      const Recip rq = recip_of(sc);
+      const float y = __frcp_rn(sc);
+      const bool fast = quot_range(sc);
 #pragma unroll
       for (int i = 0; i < G; ++i)
-        words[(i * kBits) / 32] |= (uint32_t)int_of(quot_code(__fsub_rn(val(i), lo), rq, 0.0f, (float)kQmax))
-                                   << ((i * kBits) % 32);
+        words[(i * kBits) / 32] |= kivi_code<kQmax>(__fsub_rn(val(i), lo), sc, y, fast) << ((i * kBits) % 32);
     }
     const size_t crow = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)(pos0 + tok);
     uint8_t* dst = static_cast<uint8_t*>(p.v_codes) + crow * kRowBytes + j * (G * kBits / 8);
@@ -739,13 +688,15 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
 // ------------------------------------------------------------------ launchers
 template <int KS, int VS>
 cudaError_t launch_quantize_rows_pair(const AppendParams& p, long long rows, cudaStream_t st) {
-  // four rows per thread once every (batch, kv head) row has enough new tokens
+  // several rows per thread once every (batch, kv head) row has enough new tokens: four of
+  // bf16, two of fp32 (the same bytes in flight per thread)
   if (p.n_new >= 64 && rows >= 16LL * 4 * 148 * 8 && p.B * p.H <= 65535) {
-    dim3 grid((unsigned)((p.n_new + 64 - 1) / 64), (unsigned)(p.B * p.H), 2);
+    const int per_block = p.in_bf16 ? 64 : 32;
+    dim3 grid((unsigned)((p.n_new + per_block - 1) / per_block), (unsigned)(p.B * p.H), 2);
     if (p.in_bf16)
       quantize_rows_kernel<true, 4, KS, VS><<<grid, 256, 0, st>>>(p);
     else
-      quantize_rows_kernel<false, 4, KS, VS><<<grid, 256, 0, st>>>(p);
+      quantize_rows_kernel<false, 2, KS, VS><<<grid, 256, 0, st>>>(p);
   } else {
     dim3 grid((unsigned)((rows + 15) / 16), 1, 2);
     if (p.in_bf16)
