@@ -358,6 +358,16 @@ __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
 
+// Column of channel dd of head `head` in the merge staging rows: an XOR within the channel's
+// aligned group of 16 (8-bit layout) or 4 (KIVI layout) so that the accumulator stores of a warp
+// (lanes spread over heads 2c and channels 16g or 4g) and the merge's channel-order reads both
+// touch 32 distinct banks.
+template <bool kKivi>
+__device__ __forceinline__ int red_col(int dd, int head) {
+  const int c = (head >> 1) & 3;
+  return dd ^ (kKivi ? c : (c | (((dd >> 5) & 3) << 2)));
+}
+
 // ------------------------------------------------------------------ consumer state
 template <class C>
 struct Consumer {
@@ -906,8 +916,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
 #pragma unroll
         for (int rh = 0; rh < 2; ++rh) {
           const int dd = dmap_v<C::kKivi>(g, mt, rh);
-          red_o[(w * 8 + 2 * c) * kHeadDim + dd] = S.o[mt][2 * rh] * oscale;
-          red_o[(w * 8 + 2 * c + 1) * kHeadDim + dd] = S.o[mt][2 * rh + 1] * oscale;
+          red_o[(w * 8 + 2 * c) * kHeadDim + red_col<C::kKivi>(dd, 2 * c)] = S.o[mt][2 * rh] * oscale;
+          red_o[(w * 8 + 2 * c + 1) * kHeadDim + red_col<C::kKivi>(dd, 2 * c + 1)] = S.o[mt][2 * rh + 1] * oscale;
         }
       if constexpr (C::kKivi) {
 #pragma unroll
@@ -934,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
 #pragma unroll
           for (int ww = 0; ww < kCW; ++ww) {
             const float a = fast_exp2(red_m[ww * 8 + j] - M);
-            float x = red_o[(ww * 8 + j) * kHeadDim + dd];
+            float x = red_o[(ww * 8 + j) * kHeadDim + red_col<C::kKivi>(dd, j)];
             if constexpr (C::kKivi) x += red_z[(ww * 8 + j) * 4 + (dd >> 5)];
             ov = fmaf(a, x, ov);
             L = fmaf(a, red_l[ww * 8 + j], L);
