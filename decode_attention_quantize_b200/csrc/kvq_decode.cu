@@ -87,7 +87,7 @@ struct Cfg {
   static constexpr int kOffRedL = kOffRedM + kCW * 8 * 4;
   static constexpr int kOffRedZ = kOffRedL + kCW * 8 * 4;
   static constexpr int kOffQ = kOffRedZ + kCW * 8 * 4 * 4;
-  static constexpr int kQStride = 132;          // q row stride (floats), conflict-free reads
+  static constexpr int kQStride = 144;          // q row stride (floats): see q_off
   static constexpr int kSmemBytes = kOffQ + 8 * kQStride * 4 + 1024;  // + alignment slack
 };
 
@@ -385,32 +385,59 @@ struct Consumer {
   uint32_t zpk[8][2], zpv[8][2];  // uint8 asymmetric: f16x2 (1024 + zero point)
 };
 
-// Build Q' fragments (head g, this thread's channels) from q_s, optionally multiplied by
-// a per-channel fold; returns the power-of-two shift applied.
+// Staged query rows: head j, channel d at j * 144 + d + 4 * (d >> 5). Each 32-channel block
+// starts on a 16-byte boundary, so a lane reads its block with eight 128-bit loads, and the
+// lanes of a quarter warp (two heads, four blocks) cover all 32 banks.
+__device__ __forceinline__ int q_off(int j, int d) { return j * 144 + d + 4 * (d >> 5); }
+
+// Build Q' fragments (head g, this thread's 32 channels 32c..32c+31) from q_s, optionally
+// multiplied by a per-channel fold; with `zmin` also returns sum_d q_d * zmin_d over those
+// channels (the KIVI key-minimum term). Returns the power-of-two shift applied to Q'.
 template <int FMT>
-__device__ __forceinline__ int build_q(const float* q_s, const float* fold, int g, int c,
-                                       uint32_t (&qh)[8][2], uint32_t (&ql)[8][2]) {
-  float v[8][2][2];
+__device__ __forceinline__ int build_q(const float* q_s, const float* fold, const float* zmin, int g, int c,
+                                       uint32_t (&qh)[8][2], uint32_t (&ql)[8][2], float* bias = nullptr) {
+  const float4* qrow = reinterpret_cast<const float4*>(q_s + q_off(g, 32 * c));
+  const float4* frow = fold ? reinterpret_cast<const float4*>(fold + 32 * c) : nullptr;
+  // pass 1: the largest |q'| of the warp sets the range shift
   float mx = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float4 q4 = qrow[i];
+    if (frow) {
+      const float4 f4 = frow[i];
+      q4.x *= f4.x; q4.y *= f4.y; q4.z *= f4.z; q4.w *= f4.w;
+    }
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w))));
+  }
+  mx = warp_max(mx);
+  const int eq = range_shift(mx);
+  const float sh = pow2i(eq);
+  // pass 2: scaled products by local channel, then the fragment split
+  float pl[32];
+  float bs = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 q4 = qrow[i];
+    float4 m4 = make_float4(sh, sh, sh, sh);
+    if (frow) {
+      const float4 f4 = frow[i];
+      m4 = make_float4(f4.x * sh, f4.y * sh, f4.z * sh, f4.w * sh);
+    }
+    if (zmin) {
+      const float4 z4 = reinterpret_cast<const float4*>(zmin + 32 * c)[i];
+      bs = fmaf(q4.x, z4.x, fmaf(q4.y, z4.y, fmaf(q4.z, z4.z, fmaf(q4.w, z4.w, bs))));
+    }
+    pl[4 * i] = q4.x * m4.x;
+    pl[4 * i + 1] = q4.y * m4.y;
+    pl[4 * i + 2] = q4.z * m4.z;
+    pl[4 * i + 3] = q4.w * m4.w;
+  }
+  if (bias) *bias = bs;
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
     for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int d = dmap_k<FMT>(c, ks, h, e);
-        float x = q_s[g * 132 + d + (d >> 5)];
-        if (fold) x *= fold[d];
-        v[ks][h][e] = x;
-        mx = fmaxf(mx, fabsf(x));
-      }
-  mx = warp_max(mx);
-  const int eq = range_shift(mx);
-  const float f = pow2i(eq);
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-    for (int h = 0; h < 2; ++h) split_f16x2(v[ks][h][0] * f, v[ks][h][1] * f, qh[ks][h], ql[ks][h]);
+      split_f16x2(pl[dmap_k<FMT>(0, ks, h, 0)], pl[dmap_k<FMT>(0, ks, h, 1)], qh[ks][h], ql[ks][h]);
   return eq;
 }
 
@@ -434,13 +461,8 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     if (!residual) {
       const float* ksm = reinterpret_cast<const float*>(base + C::kOffKM) + w * kHeadDim;
       const float* kzm = reinterpret_cast<const float*>(base + C::kOffKM + C::kKMeta / 2) + w * kHeadDim;
-      const int eq = build_q<C::kKFmt>(q_s, ksm, g, c, S.qh, S.ql);
-      float bs = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int dd = 32 * c + i;
-        bs = fmaf(q_s[g * 132 + dd + (dd >> 5)], kzm[dd], bs);
-      }
+      float bs;
+      const int eq = build_q<C::kKFmt>(q_s, ksm, kzm, g, c, S.qh, S.ql, &bs);
       bs += __shfl_xor_sync(0xffffffffu, bs, 1);
       bs += __shfl_xor_sync(0xffffffffu, bs, 2);
       S.bias[0] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c));
@@ -449,7 +471,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       S.qsplit = true;
       S.qmode = 0;
     } else if (S.qmode != 1) {
-      const int eq = build_q<FMT_S8>(q_s, nullptr, g, c, S.qh, S.ql);
+      const int eq = build_q<FMT_S8>(q_s, nullptr, nullptr, g, c, S.qh, S.ql);
       S.kmul = sc_log2 * pow2i(-eq);
       S.qsplit = !p.q_bf16;
       S.qmode = 1;
@@ -829,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
           v = p.q_bf16 ? bf16_bits_to_float(static_cast<const uint16_t*>(p.q)[qi])
                        : static_cast<const float*>(p.q)[qi];
         }
-        q_s[j * 132 + dd + (dd >> 5)] = v;
+        q_s[q_off(j, dd)] = v;
       }
       named_sync(1, kCW * 32);
 #pragma unroll
@@ -846,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
       if constexpr (!C::kKivi) {
         const float* fold = nullptr;
         if constexpr (C::kKFold == FOLD_CHANNEL) fold = p.k_scale + (size_t)d.hk * kHeadDim;
-        const int eq = build_q<C::kKFmt>(q_s, fold, g, c, S.qh, S.ql);
+        const int eq = build_q<C::kKFmt>(q_s, fold, nullptr, g, c, S.qh, S.ql);
         S.qsplit = (C::kKFold == FOLD_CHANNEL) || !p.q_bf16;
         float mul = sc_log2 * pow2i(-eq);
         if constexpr (C::kKFold == FOLD_TENSOR) mul *= p.k_scale[0];
