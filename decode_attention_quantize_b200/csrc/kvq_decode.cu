@@ -354,6 +354,15 @@ __device__ __forceinline__ T lds(const uint8_t* p) {
   return *reinterpret_cast<const T*>(p);
 }
 
+// Four 8x8 matrices of 16-bit elements, transposed: lane 8m + r supplies the shared address of
+// row r of matrix m; the thread with row group g and column group c receives, for each m,
+// elements (row 2c, column g) in its low half and (row 2c + 1, column g) in its high half.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int q) {
   return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
@@ -731,6 +740,23 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
           S.zacc[3] = fmaf(pt[sb][k], z4.w, S.zacc[3]);
         }
       }
+      // INT4 codes: one transposed matrix load per 8 tokens gives every lane its (token 2c,
+      // token 2c + 1) pair of 16-bit words (4 channels) for all four channel groups
+      uint32_t v4[2][4];
+      if constexpr (C::kVFmt == FMT_U4) {
+        if (!residual) {
+          const int lane = threadIdx.x & 31;
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp) {
+            ldsm_x4_trans(smem_addr(base + C::kOffV + swz<64>(tb0 + 8 * pp + (lane & 7), lane >> 3)), v4[pp]);
+            if constexpr (kMasked) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                v4[pp][j] &= (ok[2 * pp] ? 0x0000FFFFu : 0u) | (ok[2 * pp + 1] ? 0xFFFF0000u : 0u);
+            }
+          }
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t pr[2][4];  // [token pair][channel e]: f16x2 (token even, token odd)
@@ -749,15 +775,9 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
           }
         } else if constexpr (C::kVFmt == FMT_U4) {
 #pragma unroll
-          for (int pp = 0; pp < 2; ++pp) {
-            uint32_t u0 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp], j) + 2 * g);
-            uint32_t u1 = lds<uint16_t>(base + C::kOffV + swz<64>(tk[2 * pp + 1], j) + 2 * g);
-            if (kMasked && !ok[2 * pp]) u0 = 0u;
-            if (kMasked && !ok[2 * pp + 1]) u1 = 0u;
-            const uint32_t wv = prmt(u0, u1, 0x5410u);
+          for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) pr[pp][e] = u4_pair(wv, e);
-          }
+            for (int e = 0; e < 4; ++e) pr[pp][e] = u4_pair(v4[pp][j], e);
         } else {
 #pragma unroll
           for (int pp = 0; pp < 2; ++pp) {
