@@ -622,7 +622,13 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 
   // (6) value-side fold and accumulator exponent
   constexpr bool kVPerToken = C::kVFold == FOLD_TOKEN || C::kKivi;
-  float vs[C::kNSub][4][4];  // [sb][token][group] folded value scale (token fold: group 0)
+  // folded value scale of token tok, group j (per-token fold: group 0); 0 for masked tokens.
+  // Read from shared memory where it is used, so the 16 (KIVI: 32) values are not held live.
+  auto vscale = [&](int tok, int j) -> float {
+    if (!tok_ok(tok)) return 0.0f;
+    if constexpr (C::kKivi) return reinterpret_cast<const float*>(base + C::kOffVM)[tok * 4 + j];
+    return reinterpret_cast<const float*>(base + C::kOffVM)[tok];
+  };
   int evn = 15;
   if (kVPerToken && !residual) {
     float smax = 0.0f;
@@ -634,15 +640,11 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         const bool ok = tok_ok(tok);
         if constexpr (C::kKivi) {
           const float4 s4 = lds<float4>(base + C::kOffVM + tok * 16);
-          vs[sb][k][0] = ok ? s4.x : 0.0f;
-          vs[sb][k][1] = ok ? s4.y : 0.0f;
-          vs[sb][k][2] = ok ? s4.z : 0.0f;
-          vs[sb][k][3] = ok ? s4.w : 0.0f;
-          smax = fmaxf(smax, fmaxf(fmaxf(vs[sb][k][0], vs[sb][k][1]), fmaxf(vs[sb][k][2], vs[sb][k][3])));
+          const float m4 = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
+          smax = fmaxf(smax, ok ? m4 : 0.0f);
         } else {
           const float s1 = reinterpret_cast<const float*>(base + C::kOffVM)[tok];
-          vs[sb][k][0] = ok ? s1 : 0.0f;
-          smax = fmaxf(smax, vs[sb][k][0]);
+          smax = fmaxf(smax, ok ? s1 : 0.0f);
         }
       }
     smax = warp_max(smax);
@@ -688,7 +690,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     if constexpr (!C::kKivi) {
       float pv[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) pv[k] = (C::kVFold == FOLD_TOKEN ? pt[sb][k] * vs[sb][k][0] : pt[sb][k]) * pscale;
+      for (int k = 0; k < 4; ++k) pv[k] = (C::kVFold == FOLD_TOKEN ? pt[sb][k] * vscale(tk[k], 0) : pt[sb][k]) * pscale;
       uint32_t bh0, bl0, bh1, bl1;
       split_f16x2(pv[0], pv[1], bh0, bl0);
       split_f16x2(pv[2], pv[3], bh1, bl1);
@@ -721,11 +723,20 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     } else {
       // KIVI: one B operand per 32-channel group; zero-point term on CUDA cores
       uint32_t bh[4][2], bl[4][2];
+      float4 s4[4];  // value scales of this thread's four tokens, groups 0..3
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        s4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (!residual && ok[k]) s4[k] = lds<float4>(base + C::kOffVM + tk[k] * 16);
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float pv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) pv[k] = residual ? pt[sb][k] * pscale : pt[sb][k] * vs[sb][k][j] * pscale;
+        for (int k = 0; k < 4; ++k) {
+          const float sj = j == 0 ? s4[k].x : j == 1 ? s4[k].y : j == 2 ? s4[k].z : s4[k].w;
+          pv[k] = residual ? pt[sb][k] * pscale : pt[sb][k] * sj * pscale;
+        }
         split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
         split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
       }
