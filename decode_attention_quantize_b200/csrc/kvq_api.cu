@@ -273,7 +273,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
                                 float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
   kvq_status st = kvq_validate(d);
   if (st != KVQ_OK) return st;
-  if (!q || !out || (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16)) return KVQ_ERR_INVALID_ARG;
+  if (!q || !out || !aligned16(out) || (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16)) return KVQ_ERR_INVALID_ARG;
   if (!(softmax_scale == softmax_scale) || softmax_scale <= 0.0f) return KVQ_ERR_INVALID_ARG;
   const size_t need = kvq_decode_workspace_bytes(d);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KVQ_ERR_WORKSPACE;

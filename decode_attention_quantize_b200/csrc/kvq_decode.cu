@@ -1018,15 +1018,17 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
 // One block per (pair, query head of the pair's group); 128 threads = channels. The (m, l)
 // of every covering CTA are staged in shared memory first, so the output costs two
 // dependent global round trips however many CTAs covered the pair.
+// One warp per (pair, query head): lanes read the partials' (m, l) in parallel and combine
+// them with shuffles; each lane then accumulates a float4 of channels over the partials.
+// Grid (pairs, 2), four warps per block (heads 4 * blockIdx.y + warp).
 __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
-  __shared__ float s_m[128], s_w[128];
-  __shared__ float s_M, s_L;
   grid_dependency_wait();  // the partials of the decode kernel
-  const int pair = blockIdx.x, j = blockIdx.y, dd = threadIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, j = blockIdx.y * 4 + warp;
   const int per_seq = p.Hkv * p.HG;
   const int b = pair / per_seq, hh = pair % per_seq, hk = hh / p.HG, hg = hh % p.HG;
   const int hl = hg * 8 + j;
-  if (hl >= p.G) return;
+  if (hl >= p.G) return;  // whole warp
   const int hq = hk * p.G + hl;
   int off, n, N;
   if (p.paged) {
@@ -1038,47 +1040,47 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
     N = p.n_pairs * n;
     off = pair * n;
   }
-  float ov = 0.0f, lse = kNegInf;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float M = kNegInf, L = 0.0f;
   if (n > 0) {
     const int W = (N + p.ncta - 1) / p.ncta;
     const int c0 = off / W, c1 = (off + n - 1) / W;
-    float acc = 0.0f, M = kNegInf, L = 0.0f;
-    // chunks of up to 128 covering CTAs (almost always one chunk)
-    for (int base = c0; base <= c1; base += 128) {
-      const int cnt = min(128, c1 - base + 1);
-      if (dd < cnt) {
-        const size_t sl = (size_t)(pair + base + dd) * 8 + j;
-        s_m[dd] = p.part_ml[sl * 2];
-        s_w[dd] = p.part_ml[sl * 2 + 1];
+    for (int base = c0; base <= c1; base += 32) {
+      const int cnt = min(32, c1 - base + 1);
+      float mi = kNegInf, li = 0.0f;
+      if (lane < cnt) {
+        const size_t sl = (size_t)(pair + base + lane) * 8 + j;
+        mi = p.part_ml[sl * 2];
+        li = p.part_ml[sl * 2 + 1];
       }
-      __syncthreads();
-      if (dd == 0) {
-        float mc = M;
-        for (int i = 0; i < cnt; ++i) mc = fmaxf(mc, s_m[i]);
-        float Lc = (M == kNegInf || mc == kNegInf) ? 0.0f : L * exp2f(M - mc);
-        for (int i = 0; i < cnt; ++i) {
-          const float a = mc == kNegInf ? 0.0f : exp2f(s_m[i] - mc);
-          Lc = fmaf(a, s_w[i], Lc);
-          s_w[i] = a;
-        }
-        s_M = mc;
-        s_L = Lc;
+      const float mc = warp_max(fmaxf(M, mi));
+      const float f = (M == kNegInf || mc == kNegInf) ? 0.0f : exp2f(M - mc);
+      const float ai = (mi == kNegInf || mc == kNegInf) ? 0.0f : exp2f(mi - mc);
+      float lw = ai * li;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+      L = fmaf(L, f, lw);
+      acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+      const float4* po = reinterpret_cast<const float4*>(p.part_o) + ((size_t)(pair + base) * 8 + j) * (kHeadDim / 4) + lane;
+      for (int i = 0; i < cnt; ++i) {
+        const float a = __shfl_sync(0xffffffffu, ai, i);
+        const float4 o4 = po[(size_t)i * 8 * (kHeadDim / 4)];
+        acc.x = fmaf(a, o4.x, acc.x);
+        acc.y = fmaf(a, o4.y, acc.y);
+        acc.z = fmaf(a, o4.z, acc.z);
+        acc.w = fmaf(a, o4.w, acc.w);
       }
-      __syncthreads();
-      const float mc = s_M;
-      acc = (M == kNegInf || mc == kNegInf) ? 0.0f : acc * exp2f(M - mc);
-      for (int i = 0; i < cnt; ++i) acc = fmaf(s_w[i], p.part_o[((size_t)(pair + base + i) * 8 + j) * kHeadDim + dd], acc);
       M = mc;
-      L = s_L;
-      __syncthreads();
-    }
-    if (M != kNegInf && L > 0.0f) {
-      ov = acc / L;
-      lse = (M + log2f(L)) * 0.69314718055994531f;
     }
   }
-  p.out[((size_t)b * p.Hq + hq) * kHeadDim + dd] = ov;
-  if (dd == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
+  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lse = kNegInf;
+  if (M != kNegInf && L > 0.0f) {
+    ov = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+    lse = (M + log2f(L)) * 0.69314718055994531f;
+  }
+  reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + hq) * kHeadDim)[lane] = ov;
+  if (lane == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
 }
 
 // ------------------------------------------------------------------ paged plan
@@ -1276,7 +1278,7 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
   }
   e = launch_pdl(var->kernel, dim3(ncta), dim3(kThreads), (size_t)var->smem, st, p, tk, tv);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(merge_kernel, dim3(p.n_pairs, 8), dim3(128), 0, st, p);
+  e = launch_pdl(merge_kernel, dim3(p.n_pairs, 2), dim3(128), 0, st, p);
   if (e != cudaSuccess) return e;
   count_launches(p.paged ? 3 : 2);
   return cudaGetLastError();

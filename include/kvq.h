@@ -181,7 +181,8 @@ KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc);
  * memory bandwidth; guide.dupenodi.dev "KV cache quantization": the savings only count
  * when the attention kernel consumes the low-precision cache itself).
  *   q         device [batch, num_q_heads, head_dim], q_dtype (bf16 or fp32)
- *   out       device fp32 [batch, num_q_heads, head_dim]
+ *   out       device fp32 [batch, num_q_heads, head_dim], 16-byte aligned (else
+ *             KVQ_ERR_INVALID_ARG, returned before anything is launched)
  *   lse       device fp32 [batch, num_q_heads] or NULL: natural-log sum of exp of scores
  * Query head h reads kv head h / (num_q_heads / num_kv_heads). Scores are
  * softmax_scale * q.k over all tokens of the sequence (no mask). A sequence with no

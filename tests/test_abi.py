@@ -97,6 +97,9 @@ def test_append_and_decode_reject_before_launch():
                                   None) == kvq.KVQ_ERR_INVALID_ARG
     assert L.kvq_decode_attention(ctypes.byref(d2), buf, 1, ctypes.c_float(-1.0), buf, None, buf, need,
                                   None) == kvq.KVQ_ERR_INVALID_ARG
+    # the output is written with 16-byte stores: a misaligned pointer is refused on the host
+    assert L.kvq_decode_attention(ctypes.byref(d2), buf, 1, ctypes.c_float(0.088), buf + 4, None, buf, need,
+                                  None) == kvq.KVQ_ERR_INVALID_ARG
     # dequantize needs room for every token
     d4 = _desc(num_quantized=100)
     assert L.kvq_dequantize(ctypes.byref(d4), 0, buf, 99, None) == kvq.KVQ_ERR_INVALID_ARG
