@@ -65,7 +65,9 @@ struct Cfg {
   static constexpr int kKFmt = fmt_of(KS), kVFmt = fmt_of(VS);
   static constexpr int kKFold = fold_of(KS), kVFold = fold_of(VS);
   static constexpr bool kKivi = kKFold == FOLD_KIVI;
-  static constexpr int kTPW = kKivi ? 32 : 16;  // tokens per consumer warp per tile
+  // 32 tokens per consumer warp per tile: two independent 16-token MMA chains per warp, and
+  // the per-tile bookkeeping and softmax reductions shared by twice the tokens
+  static constexpr int kTPW = 32;
   static constexpr int kNSub = kTPW / 16;
   static constexpr int kTS = kTPW * kCW;        // tokens per quantized tile
   static constexpr int kKRow = row_bytes(KS), kVRow = row_bytes(VS);
@@ -78,8 +80,9 @@ struct Cfg {
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
-  static constexpr int kStages = kKivi ? 3 : 3;
-  static constexpr int kMinBlocks = kKivi ? 2 : 3;  // resident CTAs per SM the registers are sized for
+  // 128-token stages: three fit next to a second CTA for the 4-bit / 2-bit codes, two for 8-bit
+  static constexpr int kStages = kKivi ? 3 : 2;
+  static constexpr int kMinBlocks = 2;  // resident CTAs per SM the registers (168) are sized for
   static constexpr int kOffDesc = kStages * kStageBytes;
   static constexpr int kOffBar = kOffDesc + kStages * 64;
   static constexpr int kOffRedO = kOffBar + 2 * kStages * 8 + 64;
