@@ -80,18 +80,24 @@ struct Cfg {
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
-  // 128-token stages: three fit next to a second CTA for the 4-bit / 2-bit codes, two for 8-bit
-  static constexpr int kStages = kKivi ? 3 : 2;
+  // heads staged per pass of the per-pair warp merge: all eight for INT4 KIVI (whose register
+  // allocation suffers from the two-pass form), else four (half the staging, room for a stage)
+  static constexpr int kMergeHeads = KS == KVQ_KIVI_INT4 ? 8 : 4;
+  // 128-token stages: three when three still fit next to a second CTA on the SM
+  static constexpr int kFixedBytes =
+      2048 + kCW * kMergeHeads * kHeadDim * 4 + kCW * 8 * 4 * 2 + kCW * kMergeHeads * 4 * 4 + 8 * 144 * 4 + 1024;
+  static constexpr int kStages = (3 * kStageBytes + kFixedBytes <= 112 * 1024) ? 3 : 2;
   static constexpr int kMinBlocks = 2;  // resident CTAs per SM the registers (168) are sized for
   static constexpr int kOffDesc = kStages * kStageBytes;
   static constexpr int kOffBar = kOffDesc + kStages * 64;
   static constexpr int kOffRedO = kOffBar + 2 * kStages * 8 + 64;
-  static constexpr int kOffRedM = kOffRedO + kCW * 8 * kHeadDim * 4;
+  static constexpr int kOffRedM = kOffRedO + kCW * kMergeHeads * kHeadDim * 4;
   static constexpr int kOffRedL = kOffRedM + kCW * 8 * 4;
   static constexpr int kOffRedZ = kOffRedL + kCW * 8 * 4;
-  static constexpr int kOffQ = kOffRedZ + kCW * 8 * 4 * 4;
+  static constexpr int kOffQ = kOffRedZ + kCW * kMergeHeads * 4 * 4;
   static constexpr int kQStride = 144;          // q row stride (floats): see q_off
   static constexpr int kSmemBytes = kOffQ + 8 * kQStride * 4 + 1024;  // + alignment slack
+  static_assert(kMinBlocks * (kSmemBytes + 1024) <= 227 * 1024, "the resident CTAs must fit in shared memory");
 };
 
 struct TileDesc {
@@ -967,60 +973,69 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
         red_l[w * 8 + 2 * c + 1] = l1;
       }
       const float oscale = S.ev_set ? pow2i(-S.ev) : 0.0f;
-#pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh) {
-          const int dd = dmap_v<C::kKivi>(g, mt, rh);
-          red_o[(w * 8 + 2 * c) * kHeadDim + red_col<C::kKivi>(dd, 2 * c)] = S.o[mt][2 * rh] * oscale;
-          red_o[(w * 8 + 2 * c + 1) * kHeadDim + red_col<C::kKivi>(dd, 2 * c + 1)] = S.o[mt][2 * rh + 1] * oscale;
-        }
-      if constexpr (C::kKivi) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          float z = S.zacc[j];
-          z += __shfl_xor_sync(0xffffffffu, z, 1);
-          z += __shfl_xor_sync(0xffffffffu, z, 2);
-          if (c == 0) red_z[(w * 8 + g) * 4 + j] = z;
-        }
-      }
-      named_sync(1, kCW * 32);
       const int dd = threadIdx.x;  // channel
       const int slot = d.pair + blockIdx.x;
       float vsc = 1.0f;
       if constexpr (C::kVFold == FOLD_TENSOR) vsc = p.v_scale[0];
       if constexpr (C::kVFold == FOLD_CHANNEL) vsc = p.v_scale[(size_t)d.hk * kHeadDim + dd];
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        float M = kNegInf;
+      if constexpr (C::kKivi) {  // minimum-term sums of head g over the four lanes c
 #pragma unroll
-        for (int ww = 0; ww < kCW; ++ww) M = fmaxf(M, red_m[ww * 8 + j]);
-        float ov = 0.0f, L = 0.0f;
-        if (M != kNegInf) {
-#pragma unroll
-          for (int ww = 0; ww < kCW; ++ww) {
-            const float a = fast_exp2(red_m[ww * 8 + j] - M);
-            float x = red_o[(ww * 8 + j) * kHeadDim + red_col<C::kKivi>(dd, j)];
-            if constexpr (C::kKivi) x += red_z[(ww * 8 + j) * 4 + (dd >> 5)];
-            ov = fmaf(a, x, ov);
-            L = fmaf(a, red_l[ww * 8 + j], L);
-          }
-        }
-        p.part_o[((size_t)slot * 8 + j) * kHeadDim + dd] = ov * vsc;
-        if (dd == 0) {
-          p.part_ml[((size_t)slot * 8 + j) * 2] = M;
-          p.part_ml[((size_t)slot * 8 + j) * 2 + 1] = L;
+        for (int j = 0; j < 4; ++j) {
+          S.zacc[j] += __shfl_xor_sync(0xffffffffu, S.zacc[j], 1);
+          S.zacc[j] += __shfl_xor_sync(0xffffffffu, S.zacc[j], 2);
         }
       }
-      named_sync(1, kCW * 32);
+      // O is staged and merged kMergeHeads heads at a time (lanes hold heads 2c, 2c + 1)
+      constexpr int kMH = C::kMergeHeads;
+#pragma unroll
+      for (int half = 0; half < 8 / kMH; ++half) {
+        if ((2 * c) / kMH == half) {
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int rh = 0; rh < 2; ++rh) {
+              const int ch = dmap_v<C::kKivi>(g, mt, rh);
+              red_o[(w * kMH + 2 * c - kMH * half) * kHeadDim + red_col<C::kKivi>(ch, 2 * c)] = S.o[mt][2 * rh] * oscale;
+              red_o[(w * kMH + 2 * c + 1 - kMH * half) * kHeadDim + red_col<C::kKivi>(ch, 2 * c + 1)] =
+                  S.o[mt][2 * rh + 1] * oscale;
+            }
+        }
+        if constexpr (C::kKivi) {
+          if (c == 0 && g / kMH == half) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) red_z[(w * kMH + g - kMH * half) * 4 + j] = S.zacc[j];
+          }
+        }
+        named_sync(1, kCW * 32);
+#pragma unroll 1
+        for (int j = kMH * half; j < kMH * half + kMH; ++j) {
+          float M = kNegInf;
+#pragma unroll
+          for (int ww = 0; ww < kCW; ++ww) M = fmaxf(M, red_m[ww * 8 + j]);
+          float ov = 0.0f, L = 0.0f;
+          if (M != kNegInf) {
+#pragma unroll
+            for (int ww = 0; ww < kCW; ++ww) {
+              const float a = fast_exp2(red_m[ww * 8 + j] - M);
+              float x = red_o[(ww * kMH + j - kMH * half) * kHeadDim + red_col<C::kKivi>(dd, j)];
+              if constexpr (C::kKivi) x += red_z[(ww * kMH + j - kMH * half) * 4 + (dd >> 5)];
+              ov = fmaf(a, x, ov);
+              L = fmaf(a, red_l[ww * 8 + j], L);
+            }
+          }
+          p.part_o[((size_t)slot * 8 + j) * kHeadDim + dd] = ov * vsc;
+          if (dd == 0) {
+            p.part_ml[((size_t)slot * 8 + j) * 2] = M;
+            p.part_ml[((size_t)slot * 8 + j) * 2 + 1] = L;
+          }
+        }
+        named_sync(1, kCW * 32);
+      }
     }
   }
 }
 
 // ------------------------------------------------------------------ merge
-// One block per (pair, query head of the pair's group); 128 threads = channels. The (m, l)
-// of every covering CTA are staged in shared memory first, so the output costs two
-// dependent global round trips however many CTAs covered the pair.
 // One warp per (pair, query head): lanes read the partials' (m, l) in parallel and combine
 // them with shuffles; each lane then accumulates a float4 of channels over the partials.
 // Grid (pairs, 2), four warps per block (heads 4 * blockIdx.y + warp).
