@@ -475,24 +475,37 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
   uint8_t* kcodes = reinterpret_cast<uint8_t*>(xv + R * kHeadDim);  // [R][row bytes]
   const int chunk = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
   const int pos0 = p.pos0 + chunk * R;
-  // gather the combined stream: 16-byte pieces, 16 per token row
-  for (int e = threadIdx.x; e < R * 16; e += blockDim.x) {
-    const int tok = e >> 4, piece = e & 15;
-    const int s = chunk * R + tok;  // index in the combined stream
-    const uint16_t *srck, *srcv;
-    if (s < r_old) {
-      const size_t o = (((size_t)b * p.H + h) * p.rcap + s) * kHeadDim;
-      srck = p.k_res + o;
-      srcv = p.v_res + o;
-    } else {
-      const size_t o = (((size_t)b * p.H + h) * (size_t)p.n_new + (s - r_old)) * kHeadDim;
-      srck = static_cast<const uint16_t*>(p.k_new) + o;
-      srcv = static_cast<const uint16_t*>(p.v_new) + o;
-    }
-    reinterpret_cast<uint4*>(xk + tok * kHeadDim)[piece] = reinterpret_cast<const uint4*>(srck)[piece];
-    reinterpret_cast<uint4*>(xv + tok * kHeadDim)[piece] = reinterpret_cast<const uint4*>(srcv)[piece];
+  // gather the combined stream (old residual rows, then new rows: at most two contiguous runs
+  // of 256-byte rows per side) with the bulk copy engine; completion on one mbarrier
+  __shared__ __align__(8) uint64_t bar_storage;
+  const uint32_t bar = smem_addr(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
   }
   __syncthreads();
+  if (threadIdx.x == 0) {
+    const int s0 = chunk * R;
+    const int nres = min(max(r_old - s0, 0), R);  // rows taken from the residual
+    const size_t bhs = (size_t)b * p.H + h;
+    mbar_arrive_expect_tx(bar, 2u * R * kHeadDim * 2u);
+    if (nres > 0) {
+      const size_t o = (bhs * p.rcap + s0) * kHeadDim;
+      bulk_g2s(smem_addr(xk), p.k_res + o, (uint32_t)nres * kHeadDim * 2u, bar);
+      bulk_g2s(smem_addr(xv), p.v_res + o, (uint32_t)nres * kHeadDim * 2u, bar);
+    }
+    if (nres < R) {
+      const size_t o = (bhs * (size_t)p.n_new + (size_t)(s0 + nres - r_old)) * kHeadDim;
+      bulk_g2s(smem_addr(xk + nres * kHeadDim), static_cast<const uint16_t*>(p.k_new) + o,
+               (uint32_t)(R - nres) * kHeadDim * 2u, bar);
+      bulk_g2s(smem_addr(xv + nres * kHeadDim), static_cast<const uint16_t*>(p.v_new) + o,
+               (uint32_t)(R - nres) * kHeadDim * 2u, bar);
+    }
+  }
+  if (!mbar_wait(bar, 0, p.status)) {
+    mbar_wait(bar, 0, p.status);  // give copies still in flight a second bounded wait, then leave
+    return;
+  }
   // keys: task = (group gi, 2 adjacent channels); the thread keeps the 32 tokens' 4-byte
   // words (both channels as bf16) in registers and widens a channel when it needs it. The
   // codes of token j sit in byte j % 4 of word j / 4; with 2-bit codes a byte holds 4
