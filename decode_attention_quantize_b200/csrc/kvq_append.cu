@@ -454,6 +454,19 @@ __global__ void seq_lens_advance_kernel(AppendParams p) {
 }
 
 // ------------------------------------------------------------------ KIVI
+// Lane-wise minimum / maximum of two bf16 pairs (exact: a selection; a NaN lane yields the
+// other operand, as fminf / fmaxf do).
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Code of d = RN(x - min) >= 0 with step s: rne(RN(d / s)); d <= max - min keeps it <= qmax.
 template <int kQmax>
 __device__ __forceinline__ uint32_t kivi_code(float d, float s, float y, bool fast) {
@@ -523,15 +536,17 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
     for (int j = 0; j < G / 4; ++j) bits[j] = 0u;
     const size_t meta = (((size_t)b * p.H + h) * (size_t)(p.cap / G) + (size_t)(pos0 / G + gi)) * kHeadDim;
     const int shift0 = (c0 % kPer) * kBits;  // position of channel c0 inside its byte
+    uint32_t mn2 = raw[0], mx2 = raw[0];  // both channels at once
+#pragma unroll
+    for (int j = 1; j < G; ++j) {
+      mn2 = bmin2(mn2, raw[j]);
+      mx2 = bmax2(mx2, raw[j]);
+    }
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       auto val = [&](int j) { return __uint_as_float(k ? (raw[j] & 0xFFFF0000u) : (raw[j] << 16)); };
-      float lo = val(0), hi = lo;
-#pragma unroll
-      for (int j = 1; j < G; ++j) {
-        lo = fminf(lo, val(j));
-        hi = fmaxf(hi, val(j));
-      }
+      float lo = __uint_as_float(k ? (mn2 & 0xFFFF0000u) : (mn2 << 16));
+      float hi = __uint_as_float(k ? (mx2 & 0xFFFF0000u) : (mx2 << 16));
       if (lo == 0.0f) lo = 0.0f;
       if (hi == 0.0f) hi = 0.0f;
       const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
@@ -569,12 +584,14 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
       raw[4 * q4 + 3] = w.w;
     }
     auto val = [&](int i) { return __uint_as_float((i & 1) ? (raw[i >> 1] & 0xFFFF0000u) : (raw[i >> 1] << 16)); };
-    float lo = val(0), hi = lo;
+    uint32_t mn2 = raw[0], mx2 = raw[0];
 #pragma unroll
-    for (int i = 1; i < G; ++i) {
-      lo = fminf(lo, val(i));
-      hi = fmaxf(hi, val(i));
+    for (int i = 1; i < G / 2; ++i) {
+      mn2 = bmin2(mn2, raw[i]);
+      mx2 = bmax2(mx2, raw[i]);
     }
+    float lo = fminf(__uint_as_float(mn2 << 16), __uint_as_float(mn2 & 0xFFFF0000u));
+    float hi = fmaxf(__uint_as_float(mx2 << 16), __uint_as_float(mx2 & 0xFFFF0000u));
     if (lo == 0.0f) lo = 0.0f;
     if (hi == 0.0f) hi = 0.0f;
     const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
