@@ -529,6 +529,66 @@ def run_e2e(G, W, stream, flush, n, step0):
     return dict(t=ms / 1e3, h2d=h2d, d2h=d2h)
 
 
+# ---------------------------------------------------------------- quantization error
+def _f64(a, bf16):
+    a = np.asarray(a)
+    if bf16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def quant_error(G, W, stream, n_pairs=8):
+    """Quantization error of the step's output: the library's decode of the final cache state
+    against fp64 attention over the unquantized inputs the cache was built from, on sampled
+    (sequence, kv head) pairs; dense caches also report the per-element error of the
+    dequantized K and V of those pairs. Informational (not a parity check)."""
+    import torch
+    d = G.cache.desc
+    with torch.cuda.stream(stream):
+        G.cache.decode(G.q, G.scale, out=G.out, workspace=G.ws, stream=stream)
+    torch.cuda.synchronize()
+    out = G.out.cpu().numpy().astype(np.float64)
+    if W.paged:
+        lens = G.cache["seq_lens"].cpu().numpy().astype(np.int64)
+    else:
+        lens = np.full(W.B, d.num_quantized + (d.num_residual if W.kivi else 0), np.int64)
+    allp = [(b, h) for b in range(W.B) for h in range(W.Hkv)]
+    rng = np.random.default_rng(W.seed + 99)
+    pairs = [allp[i] for i in sorted(rng.choice(len(allp), size=min(n_pairs, len(allp)), replace=False))]
+    q = _f64(G.q_host[0], W.bf16)
+    scale = float(np.float32(G.scale))
+    diffs, refs, kd, kx, vd, vx = [], [], [], [], [], []
+    deq = None if W.paged else [G.cache.dequantize(which, int(lens[0])) for which in (0, 1)]
+    torch.cuda.synchronize()
+    for b, h in pairs:
+        L = int(lens[b])
+        K = _f64(synth.keys(W, b, b + 1, h, h + 1, 0, L)[0, 0], W.bf16)
+        V = _f64(synth.values(W, b, b + 1, h, h + 1, 0, L)[0, 0], W.bf16)
+        qs = q[b, h * W.G:(h + 1) * W.G]
+        sc = qs @ K.T * scale
+        pr = np.exp(sc - sc.max(axis=1, keepdims=True))
+        ref = (pr @ V) / pr.sum(axis=1, keepdims=True)
+        diffs.append(out[b, h * W.G:(h + 1) * W.G] - ref)
+        refs.append(ref)
+        if deq is not None:
+            kd.append(deq[0][b, h, :L].cpu().numpy().astype(np.float64) - K)
+            kx.append(K)
+            vd.append(deq[1][b, h, :L].cpu().numpy().astype(np.float64) - V)
+            vx.append(V)
+    dd, rr = np.concatenate([x.ravel() for x in diffs]), np.concatenate([x.ravel() for x in refs])
+    res = {"vs": "fp64 attention over the unquantized inputs (same tokens, same queries)",
+           "pairs": len(pairs), "max_abs": float(np.abs(dd).max()),
+           "max_abs_rel": float(np.abs(dd).max() / np.abs(rr).max()),
+           "rel_l2": float(np.linalg.norm(dd) / np.linalg.norm(rr)),
+           "clamped_elements": int(G.cache.status()[1])}
+    if deq is not None:
+        for name, dl, xl in (("k", kd, kx), ("v", vd, vx)):
+            e, x = np.concatenate([a.ravel() for a in dl]), np.concatenate([a.ravel() for a in xl])
+            res[f"{name}_dequant_rel_l2"] = float(np.linalg.norm(e) / np.linalg.norm(x))
+            res[f"{name}_dequant_max_abs"] = float(np.abs(e).max())
+    return res
+
+
 # ---------------------------------------------------------------- CPU oracle sample
 class OracleUnit:
     """One (sequence, kv_head) unit of the workload held by the CPU oracle: its prefill is
@@ -566,6 +626,39 @@ class OracleUnit:
         if self.append:
             b += append_bytes(self.unit_w)
         return b, dt
+
+
+_UNITS = {}
+
+
+def _oracle_worker(job):
+    """One process of the all-cores oracle baseline: unit `i` of the workload (built once per
+    process, untimed), stepped until `seconds` of timed work. Returns (bytes, seconds, steps)."""
+    name, i, seconds = job
+    w = synth.workloads()[name]
+    if (name, i) not in _UNITS:
+        _UNITS[(name, i)] = OracleUnit(w, i % w.B, (i // w.B) % w.Hkv)
+    u = _UNITS[(name, i)]
+    tb = tt = 0.0
+    n = 0
+    while tt < seconds:
+        b, t = u.step()
+        tb, tt, n = tb + b, tt + t, n + 1
+    return tb, tt, n
+
+
+def oracle_time_all_cores(w, seconds):
+    """The oracle over independent (sequence, kv_head) units, one process per host core (spawned:
+    the parent has already used the GPU). The processes run concurrently, so the aggregate
+    throughput is the sum of their rates over their timed work."""
+    import multiprocessing as mp
+    n = max(1, min(os.cpu_count() or 1, 64, w.B * w.Hkv))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(n) as pool:
+        res = pool.map(_oracle_worker, [(w.name, i, seconds) for i in range(n)], chunksize=1)
+    rate = sum(r[0] / r[1] for r in res)
+    steps = sum(r[2] for r in res)
+    return rate, n, f"{steps} oracle steps, {n} concurrent processes (one unit each, {seconds:.0f} s of timed work each)"
 
 
 def oracle_time(w, seconds, max_units=8):
@@ -663,10 +756,14 @@ def main():
                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]}
     else:
         out["e2e"] = None
+    if rank == 0:
+        out["quant_error"] = quant_error(r["G"], W, torch.cuda.current_stream())
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         b, t, n, desc = oracle_time(W, args.cpu_seconds)
         out["cpu_baseline"] = {"value": b / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                                "sample": desc}
+        rate, ncores, desc_all = oracle_time_all_cores(W, args.cpu_seconds / 2)
+        out["cpu_baseline"]["all_cores"] = {"value": rate / 1e9, "unit": UNIT, "cores": ncores, "sample": desc_all}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
