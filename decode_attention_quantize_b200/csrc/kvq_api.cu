@@ -11,6 +11,19 @@ using namespace kvq;
 namespace kvq {
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// One warp waits on a barrier whose phase never completes (nothing arrives), through the
+// library's bounded wait: it gives up after the wait limit and flags KVQ_DEV_TIMEOUT.
+__global__ void bounded_wait_check_kernel(uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar_storage;
+  const uint32_t bar = smem_addr(&bar_storage);
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  mbar_wait(bar, 0, status);
+}
 }  // namespace kvq
 
 namespace {
@@ -324,6 +337,13 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   ws += round_up(slots * 8 * 2 * sizeof(float));
   p.plan = reinterpret_cast<int32_t*>(ws);
   return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+kvq_status kvq_check_bounded_wait(uint32_t* dev_status, void* stream) {
+  if (!dev_status || (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0) return KVQ_ERR_INVALID_ARG;
+  bounded_wait_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(dev_status);
+  count_launches(1);
+  return from_cuda(cudaGetLastError());
 }
 
 kvq_status kvq_get_device_status(const kvq_cache_desc* d, uint32_t* out, int32_t clear, void* stream) {

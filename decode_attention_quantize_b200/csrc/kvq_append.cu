@@ -348,11 +348,13 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   Raw8<kBf16> in[kR];
   int rb[kR], rh[kR], ri[kR];
   bool act[kR];
+  int rows_at[kR];  // bulk form: cache row of each of the thread's rows (< 2^31, checked at the API)
   int pos_base = 0;  // bulk form: the sequence's first new position, read once (stores may alias it)
   if constexpr (kR > 1) {
     const int bh = blockIdx.y;
     const int b = bh / p.H, h = bh - b * p.H;
     const int n_b = new_count(p, b);
+    if (blockIdx.x * 16 * kR >= n_b) return;  // a padded block with no token of this sequence
     pos_base = p.paged ? p.seq_lens[b] : p.pos0;
 #pragma unroll
     for (int it = 0; it < kR; ++it) {
@@ -363,6 +365,14 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
       act[it] = i < n_b;
       in[it].clear();
       if (act[it]) in[it].load(src_base, ((size_t)bh * p.n_new + i) * kHeadDim + lane8 * 8);
+    }
+    // every row's cache slot (page-table reads) before any code store: the stores may alias
+    // the table, so a lookup left inside the row loop would wait for the previous row's store
+#pragma unroll
+    for (int it = 0; it < kR; ++it) {
+      size_t r64 = 0;
+      if (act[it] && !cache_row(p, b, h, pos_base + ri[it], r64)) act[it] = false;
+      rows_at[it] = (int)r64;
     }
   } else {
     const int r = blockIdx.x * 16 + (threadIdx.x >> 4);
@@ -406,9 +416,12 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
     }
     if (!act[it]) continue;
     const int b = rb[it], h = rh[it];
-    const int pos = (kR > 1 ? pos_base : (p.paged ? p.seq_lens[b] : p.pos0)) + ri[it];
     size_t row;
-    if (!cache_row(p, b, h, pos, row)) continue;
+    if constexpr (kR > 1) {
+      row = (size_t)rows_at[it];
+    } else {
+      if (!cache_row(p, b, h, (p.paged ? p.seq_lens[b] : p.pos0) + ri[it], row)) continue;
+    }
     if (per_channel && h != chan_head) {
       fixed_fast = true;
 #pragma unroll

@@ -35,7 +35,7 @@ EXPORTS = [
     "kvq_abi_version", "kvq_status_string", "kvq_validate", "kvq_cache_bytes",
     "kvq_append_workspace_bytes", "kvq_quantize_append", "kvq_dequantize",
     "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_get_device_status", "kvq_launch_count",
-    "kvq_decode_attention_noalloc",
+    "kvq_decode_attention_noalloc", "kvq_check_bounded_wait",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -86,6 +86,8 @@ def _load():
     L.kvq_launch_count.restype = ctypes.c_uint64
     L.kvq_decode_attention_noalloc.argtypes = [P, vp, i32, ctypes.c_float, vp, vp, vp]
     L.kvq_decode_attention_noalloc.restype = ctypes.c_int
+    L.kvq_check_bounded_wait.argtypes = [vp, vp]
+    L.kvq_check_bounded_wait.restype = ctypes.c_int
     for name in ("kvq_validate", "kvq_cache_bytes", "kvq_quantize_append", "kvq_dequantize",
                  "kvq_decode_attention", "kvq_get_device_status"):
         getattr(L, name).restype = ctypes.c_int
@@ -192,6 +194,12 @@ def kvq_get_device_status(desc: KvqDesc, clear=False, stream=None):
     _check(lib.kvq_get_device_status(ctypes.byref(desc), ctypes.cast(buf, ctypes.c_void_p), int(clear),
                                      _stream(stream)), "kvq_get_device_status")
     return int(buf[0]), int(buf[1])
+
+
+def kvq_check_bounded_wait(status, stream=None):
+    """Run the library's bounded-wait self-check (a wait that nothing completes); it sets
+    KVQ_DEV_TIMEOUT in status[0] after about a second. `status`: CUDA int32/uint32 tensor [2]."""
+    _check(lib.kvq_check_bounded_wait(_ptr(status), _stream(stream)), "kvq_check_bounded_wait")
 
 
 def kvq_launch_count() -> int:

@@ -192,6 +192,17 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* 
                                 float softmax_scale, float* out, float* lse, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/*
+ * Test support; the pages have no counterpart. Launches one warp that waits on a
+ * shared-memory barrier nothing ever arrives at, through the same bounded wait every kernel
+ * of the library uses for its copy barriers. After about one second the wait gives up, sets
+ * KVQ_DEV_TIMEOUT in dev_status[0] and the kernel returns, leaving the context usable. This
+ * lets a test exercise the timeout path on a GPU without hanging or faulting it.
+ *   dev_status  device uint32[2] (caller-owned; only bits are ORed in)
+ * Asynchronous on `stream`; KVQ_ERR_INVALID_ARG for a null or misaligned pointer.
+ */
+KVQ_API kvq_status kvq_check_bounded_wait(uint32_t* dev_status, void* stream);
+
 /* Number of kernels this process has launched through the library (all entry points). */
 KVQ_API uint64_t kvq_launch_count(void);
 

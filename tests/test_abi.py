@@ -100,6 +100,8 @@ def test_append_and_decode_reject_before_launch():
     # the output is written with 16-byte stores: a misaligned pointer is refused on the host
     assert L.kvq_decode_attention(ctypes.byref(d2), buf, 1, ctypes.c_float(0.088), buf + 4, None, buf, need,
                                   None) == kvq.KVQ_ERR_INVALID_ARG
+    # the bounded-wait self-check refuses a null status pointer before launching
+    assert L.kvq_check_bounded_wait(None, None) == kvq.KVQ_ERR_INVALID_ARG
     # dequantize needs room for every token
     d4 = _desc(num_quantized=100)
     assert L.kvq_dequantize(ctypes.byref(d4), 0, buf, 99, None) == kvq.KVQ_ERR_INVALID_ARG
