@@ -337,6 +337,11 @@ constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s
 template <bool kBf16, int kR, int KS, int VS>
 __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)) ? 3 : 4)
     quantize_rows_kernel(AppendParams p) {
+  // Launched as a programmatic dependent: wait for the previous kernel (its writes of the
+  // inputs, its reads of the cache) before touching memory, then let the next kernel (the
+  // decode of this step) be scheduled; it waits for this grid to finish before it reads.
+  grid_dependency_wait();
+  grid_launch_dependents();
   const int side = blockIdx.z;
   const int scheme = side ? VS : KS;  // compile-time per side
   const int lane8 = threadIdx.x & 15;
@@ -480,6 +485,53 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
   return r;
 }
 
+// Two fp32 lanes in one 64-bit register for the packed f32x2 arithmetic of sm_100 (each lane is
+// the same correctly rounded IEEE operation as its scalar form).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Two KIVI codes at once: d = RN(v - min), then the division-free quotient of `quot` in its
+// residual form r = RN(d - q * s) (the same values; zero signs do not reach integer codes),
+// then rne. v2 holds the two values; lo2, s2, ns2 (= -s), y2 (= RN(1/s)) the lanes' group terms.
+template <int kQmax>
+__device__ __forceinline__ void kivi_code2(f32x2 v2, f32x2 lo2, f32x2 s2n, f32x2 y2, uint32_t& c0, uint32_t& c1) {
+  const f32x2 d = sub2(v2, lo2);
+  const f32x2 q = mul2(d, y2);
+  const f32x2 r = fma2(q, s2n, d);
+  const f32x2 t = add2(fma2(r, y2, q), pk2(kRoundMagic, kRoundMagic));
+  float t0, t1;
+  upk2(t, t0, t1);
+  c0 = __float_as_uint(t0) - (uint32_t)kRoundMagicBits;
+  c1 = __float_as_uint(t1) - (uint32_t)kRoundMagicBits;
+  c0 = c0 < (uint32_t)kQmax ? c0 : (uint32_t)kQmax;
+  c1 = c1 < (uint32_t)kQmax ? c1 : (uint32_t)kQmax;
+}
+
 // Code of d = RN(x - min) >= 0 with step s: rne(RN(d / s)); d <= max - min keeps it <= qmax.
 template <int kQmax>
 __device__ __forceinline__ uint32_t kivi_code(float d, float s, float y, bool fast) {
@@ -555,22 +607,38 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
       mn2 = bmin2(mn2, raw[j]);
       mx2 = bmax2(mx2, raw[j]);
     }
+    float lo[2], sc[2], yr[2];
+    bool fast[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-      auto val = [&](int j) { return __uint_as_float(k ? (raw[j] & 0xFFFF0000u) : (raw[j] << 16)); };
-      float lo = __uint_as_float(k ? (mn2 & 0xFFFF0000u) : (mn2 << 16));
+      lo[k] = __uint_as_float(k ? (mn2 & 0xFFFF0000u) : (mn2 << 16));
       float hi = __uint_as_float(k ? (mx2 & 0xFFFF0000u) : (mx2 << 16));
-      if (lo == 0.0f) lo = 0.0f;
+      if (lo[k] == 0.0f) lo[k] = 0.0f;
       if (hi == 0.0f) hi = 0.0f;
-      const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
-      p.k_scale[meta + c0 + k] = sc;
-      p.k_zero[meta + c0 + k] = lo;
-      if (sc != 0.0f) {
-        const float y = __frcp_rn(sc);
-        const bool fast = quot_range(sc);
+      sc[k] = __fdiv_rn(__fsub_rn(hi, lo[k]), (float)kQmax);
+      yr[k] = __frcp_rn(sc[k]);
+      fast[k] = sc[k] != 0.0f && quot_range(sc[k]);
+      p.k_scale[meta + c0 + k] = sc[k];
+      p.k_zero[meta + c0 + k] = lo[k];
+    }
+    if (fast[0] && fast[1]) {
+      // both channels of a token in one packed operation
+      const f32x2 lo2 = pk2(lo[0], lo[1]), s2n = pk2(-sc[0], -sc[1]), y2 = pk2(yr[0], yr[1]);
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        uint32_t a, bb;
+        kivi_code2<kQmax>(pk2(__uint_as_float(raw[j] << 16), __uint_as_float(raw[j] & 0xFFFF0000u)), lo2, s2n, y2, a, bb);
+        bits[j / 4] |= (a << (8 * (j % 4) + shift0)) | (bb << (8 * (j % 4) + shift0 + kBits));
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (sc[k] == 0.0f) continue;
+        auto val = [&](int j) { return __uint_as_float(k ? (raw[j] & 0xFFFF0000u) : (raw[j] << 16)); };
 #pragma unroll
         for (int j = 0; j < G; ++j)
-          bits[j / 4] |= kivi_code<kQmax>(__fsub_rn(val(j), lo), sc, y, fast) << (8 * (j % 4) + shift0 + k * kBits);
+          bits[j / 4] |= kivi_code<kQmax>(__fsub_rn(val(j), lo[k]), sc[k], yr[k], fast[k])
+                         << (8 * (j % 4) + shift0 + k * kBits);
       }
     }
 #pragma unroll
@@ -613,10 +681,20 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
     for (int w = 0; w < G * kBits / 32; ++w) words[w] = 0u;
     if (sc != 0.0f) {
       const float y = __frcp_rn(sc);
-      const bool fast = quot_range(sc);
+      if (quot_range(sc)) {
+        // channel pairs (2i, 2i + 1) in one packed operation
+        const f32x2 lo2 = pk2(lo, lo), s2n = pk2(-sc, -sc), y2 = pk2(y, y);
 #pragma unroll
-      for (int i = 0; i < G; ++i)
-        words[(i * kBits) / 32] |= kivi_code<kQmax>(__fsub_rn(val(i), lo), sc, y, fast) << ((i * kBits) % 32);
+        for (int i = 0; i < G / 2; ++i) {
+          uint32_t a, bb;
+          kivi_code2<kQmax>(pk2(__uint_as_float(raw[i] << 16), __uint_as_float(raw[i] & 0xFFFF0000u)), lo2, s2n, y2, a, bb);
+          words[(2 * i * kBits) / 32] |= (a << ((2 * i * kBits) % 32)) | (bb << ((2 * i * kBits) % 32 + kBits));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < G; ++i)
+          words[(i * kBits) / 32] |= kivi_code<kQmax>(__fsub_rn(val(i), lo), sc, y, false) << ((i * kBits) % 32);
+      }
     }
     const size_t crow = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)(pos0 + tok);
     uint8_t* dst = static_cast<uint8_t*>(p.v_codes) + crow * kRowBytes + j * (G * kBits / 8);
@@ -736,18 +814,12 @@ cudaError_t launch_quantize_rows_pair(const AppendParams& p, long long rows, cud
   if (p.n_new >= 64 && rows >= 16LL * 4 * 148 * 8 && p.B * p.H <= 65535) {
     const int per_block = p.in_bf16 ? 64 : 32;
     dim3 grid((unsigned)((p.n_new + per_block - 1) / per_block), (unsigned)(p.B * p.H), 2);
-    if (p.in_bf16)
-      quantize_rows_kernel<true, 4, KS, VS><<<grid, 256, 0, st>>>(p);
-    else
-      quantize_rows_kernel<false, 2, KS, VS><<<grid, 256, 0, st>>>(p);
-  } else {
-    dim3 grid((unsigned)((rows + 15) / 16), 1, 2);
-    if (p.in_bf16)
-      quantize_rows_kernel<true, 1, KS, VS><<<grid, 256, 0, st>>>(p);
-    else
-      quantize_rows_kernel<false, 1, KS, VS><<<grid, 256, 0, st>>>(p);
+    if (p.in_bf16) return launch_pdl(quantize_rows_kernel<true, 4, KS, VS>, grid, dim3(256), 0, st, p);
+    return launch_pdl(quantize_rows_kernel<false, 2, KS, VS>, grid, dim3(256), 0, st, p);
   }
-  return cudaSuccess;
+  dim3 grid((unsigned)((rows + 15) / 16), 1, 2);
+  if (p.in_bf16) return launch_pdl(quantize_rows_kernel<true, 1, KS, VS>, grid, dim3(256), 0, st, p);
+  return launch_pdl(quantize_rows_kernel<false, 1, KS, VS>, grid, dim3(256), 0, st, p);
 }
 
 bool append_pair_supported(int ks, int vs) {

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <utility>
 #include <stdint.h>
 
 #include "kvq.h"
@@ -89,6 +90,25 @@ void count_launches(int n);  // decode grid bound used to size the workspace
 cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
                           int flushed, int r_new, cudaStream_t st);
 cudaError_t launch_dequantize(const DequantParams& p, cudaStream_t st);
+// Launch with programmatic dependent launch: the kernel may be scheduled while the previous
+// kernel in the stream is still running and must call griddepcontrol.wait before it touches
+// memory that kernel writes (or reads, for memory it overwrites).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Returns cudaErrorNotSupported when the (k_scheme, v_scheme, layout) pair has no kernel.
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st);
 bool decode_supported(int k_scheme, int v_scheme, int paged);
