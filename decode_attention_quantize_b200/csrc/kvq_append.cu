@@ -350,46 +350,6 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   float* scale = side ? p.v_scale : p.k_scale;
   const uint8_t* zp = side ? p.v_zp : p.k_zp;
   const void* src_base = side ? p.v_new : p.k_new;
-  Raw8<kBf16> in[kR];
-  int rb[kR], rh[kR], ri[kR];
-  bool act[kR];
-  int rows_at[kR];  // bulk form: cache row of each of the thread's rows (< 2^31, checked at the API)
-  int pos_base = 0;  // bulk form: the sequence's first new position, read once (stores may alias it)
-  if constexpr (kR > 1) {
-    const int bh = blockIdx.y;
-    const int b = bh / p.H, h = bh - b * p.H;
-    const int n_b = new_count(p, b);
-    if (blockIdx.x * 16 * kR >= n_b) return;  // a padded block with no token of this sequence
-    pos_base = p.paged ? p.seq_lens[b] : p.pos0;
-#pragma unroll
-    for (int it = 0; it < kR; ++it) {
-      const int i = blockIdx.x * 16 * kR + 16 * it + (threadIdx.x >> 4);
-      rb[it] = b;
-      rh[it] = h;
-      ri[it] = i;
-      act[it] = i < n_b;
-      in[it].clear();
-      if (act[it]) in[it].load(src_base, ((size_t)bh * p.n_new + i) * kHeadDim + lane8 * 8);
-    }
-    // every row's cache slot (page-table reads) before any code store: the stores may alias
-    // the table, so a lookup left inside the row loop would wait for the previous row's store
-#pragma unroll
-    for (int it = 0; it < kR; ++it) {
-      size_t r64 = 0;
-      if (act[it] && !cache_row(p, b, h, pos_base + ri[it], r64)) act[it] = false;
-      rows_at[it] = (int)r64;
-    }
-  } else {
-    const int r = blockIdx.x * 16 + (threadIdx.x >> 4);
-    const int rows = p.B * p.H * p.n_new;
-    const int i = r % p.n_new, bh = r / p.n_new;
-    rb[0] = bh / p.H;
-    rh[0] = bh - rb[0] * p.H;
-    ri[0] = i;
-    act[0] = r < rows && i < new_count(p, rb[0]);
-    in[0].clear();
-    if (act[0]) in[0].load(src_base, (size_t)r * kHeadDim + lane8 * 8);
-  }
   Scales8 sc;
   bool fixed_fast = true;  // the per-tensor or per-channel scales are all in the correction's range
 #pragma unroll
@@ -405,63 +365,110 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   }
   int chan_head = -1;
   int sat = 0;
-#pragma unroll
-  for (int it = 0; it < kR; ++it) {
-    float x[8];
-    in[it].unpack(x);
-    // per-token scale: absmax over the 16 lanes of this row (a half warp)
-    float tok_s = 0.0f;
-    if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
-      float m = 0.0f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      tok_s = __fdiv_rn(m, 127.0f);
-    }
-    if (!act[it]) continue;
-    const int b = rb[it], h = rh[it];
-    size_t row;
+  // Bulk form: a grid-stride walk over (chunk of 16 * kR tokens, sequence x head) items, so
+  // chunks past a sequence's new tokens (a padded paged prefill) cost only a compare, and the
+  // per-tensor scale is read once per block. Small form: one item.
+  const int nx = kR > 1 ? (p.n_new + 16 * kR - 1) / (16 * kR) : 1;
+  const int n_items = kR > 1 ? nx * p.B * p.H : 1;
+  for (int item = kR > 1 ? (int)blockIdx.x : 0; item < n_items; item += kR > 1 ? (int)gridDim.x : n_items) {
+    Raw8<kBf16> in[kR];
+    int rb[kR], rh[kR], ri[kR];
+    bool act[kR];
+    int rows_at[kR];  // bulk form: cache row of each of the thread's rows (< 2^31, checked at the API)
+    int pos_base = 0;  // bulk form: the sequence's first new position, read once (stores may alias it)
     if constexpr (kR > 1) {
-      row = (size_t)rows_at[it];
+      const int bh = item / nx, chunk = item - bh * nx;
+      const int b = bh / p.H, h = bh - b * p.H;
+      const int n_b = new_count(p, b);
+      if (chunk * 16 * kR >= n_b) continue;  // a padded chunk with no token of this sequence
+      pos_base = p.paged ? p.seq_lens[b] : p.pos0;
+#pragma unroll
+      for (int it = 0; it < kR; ++it) {
+        const int i = chunk * 16 * kR + 16 * it + (threadIdx.x >> 4);
+        rb[it] = b;
+        rh[it] = h;
+        ri[it] = i;
+        act[it] = i < n_b;
+        in[it].clear();
+        if (act[it]) in[it].load(src_base, ((size_t)bh * p.n_new + i) * kHeadDim + lane8 * 8);
+      }
+      // every row's cache slot (page-table reads) before any code store: the stores may alias
+      // the table, so a lookup left inside the row loop would wait for the previous row's store
+#pragma unroll
+      for (int it = 0; it < kR; ++it) {
+        size_t r64 = 0;
+        if (act[it] && !cache_row(p, b, h, pos_base + ri[it], r64)) act[it] = false;
+        rows_at[it] = (int)r64;
+      }
     } else {
-      if (!cache_row(p, b, h, (p.paged ? p.seq_lens[b] : p.pos0) + ri[it], row)) continue;
+      const int r = blockIdx.x * 16 + (threadIdx.x >> 4);
+      const int rows = p.B * p.H * p.n_new;
+      const int i = r % p.n_new, bh = r / p.n_new;
+      rb[0] = bh / p.H;
+      rh[0] = bh - rb[0] * p.H;
+      ri[0] = i;
+      act[0] = r < rows && i < new_count(p, rb[0]);
+      in[0].clear();
+      if (act[0]) in[0].load(src_base, (size_t)r * kHeadDim + lane8 * 8);
     }
-    if (per_channel && h != chan_head) {
-      fixed_fast = true;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int c = h * kHeadDim + lane8 * 8 + k;
-        sc.s[k] = scale[c];
-        sc.y[k] = __frcp_rn(sc.s[k]);
-        fixed_fast &= quot_range(sc.s[k]);
-        if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) sc.zp[k] = zp[c];
-      }
-      chan_head = h;
-    }
-    bool row_fast = fixed_fast;
-    if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
-      const float y = __frcp_rn(tok_s);
-      row_fast = quot_range(tok_s);
+    for (int it = 0; it < kR; ++it) {
+      float x[8];
+      in[it].unpack(x);
+      // per-token scale: absmax over the 16 lanes of this row (a half warp)
+      float tok_s = 0.0f;
+      if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
+        float m = 0.0f;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        sc.s[k] = tok_s;
-        sc.y[k] = y;
+        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        tok_s = __fdiv_rn(m, 127.0f);
       }
+      if (!act[it]) continue;
+      const int b = rb[it], h = rh[it];
+      size_t row;
+      if constexpr (kR > 1) {
+        row = (size_t)rows_at[it];
+      } else {
+        if (!cache_row(p, b, h, (p.paged ? p.seq_lens[b] : p.pos0) + ri[it], row)) continue;
+      }
+      if (per_channel && h != chan_head) {
+        fixed_fast = true;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int c = h * kHeadDim + lane8 * 8 + k;
+          sc.s[k] = scale[c];
+          sc.y[k] = __frcp_rn(sc.s[k]);
+          fixed_fast &= quot_range(sc.s[k]);
+          if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) sc.zp[k] = zp[c];
+        }
+        chan_head = h;
+      }
+      bool row_fast = fixed_fast;
+      if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
+        const float y = __frcp_rn(tok_s);
+        row_fast = quot_range(tok_s);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          sc.s[k] = tok_s;
+          sc.y[k] = y;
+        }
+      }
+      uint2 codes;
+      bool ok = false;
+      if (row_fast) {
+        if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
+          ok = fp8_row(x, sc, codes);
+        else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
+          ok = asym_row(x, sc, codes);
+        else
+          ok = sym_row(x, sc, codes);
+      }
+      if (!ok) codes = careful_row(x, sc, row_fast, scheme, sat);  // may saturate, or out of range
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8) = codes;
+      if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
     }
-    uint2 codes;
-    bool ok = false;
-    if (row_fast) {
-      if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
-        ok = fp8_row(x, sc, codes);
-      else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
-        ok = asym_row(x, sc, codes);
-      else
-        ok = sym_row(x, sc, codes);
-    }
-    if (!ok) codes = careful_row(x, sc, row_fast, scheme, sat);  // may saturate, or out of range
-    *reinterpret_cast<uint2*>(static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * kHeadDim + lane8 * 8) = codes;
-    if (scheme == KVQ_INT8_SYM_PER_TOKEN && lane8 == 0) scale[row] = tok_s;
   }
   if (sat && p.status) atomicAdd(p.status + 1, (uint32_t)sat);
 }
@@ -807,13 +814,30 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
 }
 
 // ------------------------------------------------------------------ launchers
+// Streaming multiprocessors of the current device (queried once per device).
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 template <int KS, int VS>
 cudaError_t launch_quantize_rows_pair(const AppendParams& p, long long rows, cudaStream_t st) {
   // several rows per thread once every (batch, kv head) row has enough new tokens: four of
-  // bf16, two of fp32 (the same bytes in flight per thread)
+  // bf16, two of fp32 (the same bytes in flight per thread); a grid of a few waves of the SMs
+  // walks the (chunk, sequence x head) items
   if (p.n_new >= 64 && rows >= 16LL * 4 * 148 * 8 && p.B * p.H <= 65535) {
-    const int per_block = p.in_bf16 ? 64 : 32;
-    dim3 grid((unsigned)((p.n_new + per_block - 1) / per_block), (unsigned)(p.B * p.H), 2);
+    const int per_item = p.in_bf16 ? 64 : 32;
+    const long long items = (long long)((p.n_new + per_item - 1) / per_item) * p.B * p.H;
+    const long long cap = 16LL * sm_count();
+    dim3 grid((unsigned)(items < cap ? items : cap), 1, 2);
     if (p.in_bf16) return launch_pdl(quantize_rows_kernel<true, 4, KS, VS>, grid, dim3(256), 0, st, p);
     return launch_pdl(quantize_rows_kernel<false, 2, KS, VS>, grid, dim3(256), 0, st, p);
   }
