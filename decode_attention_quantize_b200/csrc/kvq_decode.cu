@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -1194,7 +1195,10 @@ Variant variant() {
   return Variant{KS, VS, PG ? 1 : 0, decode_kernel<KS, VS, PG>, C::kSmemBytes, C::kTS};
 }
 
-const Variant* find_variant(int k, int v, int paged) {
+constexpr int kNumVariants = 24;
+constexpr int kMaxDevices = 64;
+
+const Variant* variants() {
   static const Variant table[] = {
       variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, false>(),
       variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, true>(),
@@ -1221,8 +1225,14 @@ const Variant* find_variant(int k, int v, int paged) {
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
   };
-  for (const Variant& x : table)
-    if (x.k == k && x.v == v && x.paged == paged) return &x;
+  static_assert(sizeof(table) / sizeof(table[0]) == kNumVariants, "variant count");
+  return table;
+}
+
+const Variant* find_variant(int k, int v, int paged) {
+  const Variant* table = variants();
+  for (int i = 0; i < kNumVariants; ++i)
+    if (table[i].k == k && table[i].v == v && table[i].paged == paged) return &table[i];
   return nullptr;
 }
 
@@ -1254,12 +1264,21 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
   } else {
     p.nq = p.nr = 0;
   }
-  cudaError_t e = cudaFuncSetAttribute(var->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, var->smem);
+  // shared-memory opt-in and resident CTAs per SM: set up once per (variant, device)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int occ = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var->kernel, kThreads, var->smem);
-  if (e != cudaSuccess) return e;
-  if (occ < 1) occ = 1;
+  static std::atomic<int> occ_cache[kNumVariants][kMaxDevices];
+  const int vi = (int)(var - variants());
+  int occ = dev < kMaxDevices ? occ_cache[vi][dev].load(std::memory_order_relaxed) : 0;
+  if (occ <= 0) {
+    e = cudaFuncSetAttribute(var->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, var->smem);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var->kernel, kThreads, var->smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    if (dev < kMaxDevices) occ_cache[vi][dev].store(occ, std::memory_order_relaxed);
+  }
   int ncta = sm_count() * occ;
   if (ncta > kMaxCtas) ncta = kMaxCtas;
   if (!p.paged) {
@@ -1280,7 +1299,10 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
   }
   e = launch_pdl(var->kernel, dim3(ncta), dim3(kThreads), (size_t)var->smem, st, p, tk, tv);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {
+    if (dev < kMaxDevices) occ_cache[vi][dev].store(0, std::memory_order_relaxed);  // set up again next call
+    return e;
+  }
   e = launch_pdl(merge_kernel, dim3(p.n_pairs, 2), dim3(128), 0, st, p);
   if (e != cudaSuccess) return e;
   count_launches(p.paged ? 3 : 2);

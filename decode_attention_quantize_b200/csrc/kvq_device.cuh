@@ -132,23 +132,9 @@ __device__ __forceinline__ uint32_t hfma2_u(uint32_t a, uint32_t b, uint32_t c) 
   return r;
 }
 
-// Two E4M3 codes (low byte first) -> f16x2, exact (every E4M3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  uint32_t r;
-  const uint16_t v = static_cast<uint16_t>(two_codes);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
-  return r;
-}
-
 // f16 bit pattern 0x6400 is 1024; OR-ing an integer n < 1024 into the mantissa gives
 // exactly 1024 + n.
 constexpr uint32_t kF16Magic1024x2 = 0x64006400u;
-
-// Bytes (b0, b1) at the low halves of `lo_pair` -> f16x2 (b0 + 1024, b1 + 1024); the
-// caller subtracts the bias it wants (1024 for uint8 codes, 1152 for xor-0x80 int8).
-__device__ __forceinline__ uint32_t bytes_to_biased_f16x2(uint32_t two_bytes_lo16) {
-  return prmt(two_bytes_lo16, 0x64646464u, 0x5150u) ;
-}
 
 __device__ __forceinline__ float2 f16x2_to_float2(uint32_t h) {
   __half2 v = *reinterpret_cast<__half2*>(&h);
