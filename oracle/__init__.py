@@ -34,6 +34,7 @@ INT8_SYM_PER_CHANNEL = 3
 UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
+FP8_E5M2_PER_TENSOR = 7
 
 _lib = None
 
@@ -79,6 +80,10 @@ def load(path: str):
     L.oq_e4m3_encode.restype = ctypes.c_uint8
     L.oq_e4m3_decode.argtypes = [ctypes.c_uint8]
     L.oq_e4m3_decode.restype = f32
+    L.oq_e5m2_encode.argtypes = [f32]
+    L.oq_e5m2_encode.restype = ctypes.c_uint8
+    L.oq_e5m2_decode.argtypes = [ctypes.c_uint8]
+    L.oq_e5m2_decode.restype = f32
     L.oq_sym_code.argtypes = [f32, f32, i32]
     L.oq_sym_code.restype = i32
     L.oq_asym_params.argtypes = [f32, f32, vp, vp]
@@ -113,6 +118,14 @@ def e4m3_encode(x: float) -> int:
 
 def e4m3_decode(code: int) -> float:
     return float(lib().oq_e4m3_decode(int(code)))
+
+
+def e5m2_encode(x: float) -> int:
+    return int(lib().oq_e5m2_encode(float(x)))
+
+
+def e5m2_decode(code: int) -> float:
+    return float(lib().oq_e5m2_decode(int(code)))
 
 
 def sym_code(x: float, s: float, qmax: int = 127) -> int:
@@ -182,7 +195,7 @@ class OracleCache:
             else:
                 self.arrays[side + "_codes"] = np.zeros((B, Hkv, cap, rb), np.uint8)
             scale = zero = zp = None
-            if scheme in (FP8_E4M3_PER_TENSOR, INT8_SYM_PER_TENSOR):
+            if scheme in (FP8_E4M3_PER_TENSOR, FP8_E5M2_PER_TENSOR, INT8_SYM_PER_TENSOR):
                 scale = np.zeros(1, np.float32)
             elif scheme == INT8_SYM_PER_TOKEN:
                 scale = np.zeros((num_pages, Hkv, page_size) if paged else (B, Hkv, cap), np.float32)

@@ -79,6 +79,44 @@ uint8_t oq_e4m3_encode(float x) {
   return (uint8_t)(sign | (uint8_t)(((E + 7) << 3) | ((int)m - 8)));
 }
 
+/* OCP FP8 E5M2: sign, 5 exponent bits (bias 15), 2 mantissa bits; exponent 31 holds infinity
+ * and NaN; largest finite value 1.75 * 2^15 = 57344; subnormals M/4 * 2^-14. */
+float oq_e5m2_decode(uint8_t code) {
+  const int s = code >> 7, E = (code >> 2) & 0x1F, M = code & 3;
+  float v;
+  if (E == 31)
+    v = M == 0 ? INFINITY : NAN;
+  else if (E == 0)
+    v = ldexpf((float)M, -16);
+  else
+    v = ldexpf(1.0f + (float)M / 4.0f, E - 15);
+  return s ? -v : v;
+}
+
+/* Nearest E5M2 value, ties to even mantissa; finite values above 57344 saturate to 57344
+ * (as for E4M3). The sign of zero is kept. */
+uint8_t oq_e5m2_encode(float x) {
+  const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  const float a = fabsf(x);
+  if (isnan(x)) return (uint8_t)(sign | 0x7F);
+  if (a > 57344.0f) return (uint8_t)(sign | 0x7B);
+  if (a < ldexpf(1.0f, -14)) {
+    /* subnormal grid: multiples of 2^-16; 4 * 2^-16 is the smallest normal (code 0x04) */
+    float m = rintf(ldexpf(a, 16));
+    return (uint8_t)(sign | (uint8_t)m);
+  }
+  int e2;
+  frexpf(a, &e2);            /* a in [2^(e2-1), 2^e2) */
+  int E = e2 - 1;            /* unbiased exponent, -14..15 */
+  float m = rintf(ldexpf(a, 2 - E)); /* significand * 4, in [4, 8] */
+  if (m == 8.0f) {
+    m = 4.0f;
+    E += 1;
+  }
+  if (E > 15 || (E == 15 && m > 7.0f)) return (uint8_t)(sign | 0x7B);
+  return (uint8_t)(sign | (uint8_t)(((E + 15) << 2) | ((int)m - 4)));
+}
+
 /* Symmetric code: clamp(rne(x / s), -qmax, qmax) (P4 Step 3 divides by the scale and
  * rounds; P3 §2 gives the symmetric INT8 range as -127..127). */
 int oq_sym_code(float x, float s, int qmax) {
@@ -232,7 +270,7 @@ static float block_at(const block* k, int b, int h, int t, int d) {
  * tokens (P4 Step 3 reduces V over batch and sequence per channel). */
 static void calibrate(const oq_cache* c, const block* k, int scheme, float* scale, uint8_t* zp) {
   const int B = c->B, H = c->Hkv, D = c->D;
-  if (scheme == OQ_FP8_E4M3_PER_TENSOR || scheme == OQ_INT8_SYM_PER_TENSOR) {
+  if (scheme == OQ_FP8_E4M3_PER_TENSOR || scheme == OQ_FP8_E5M2_PER_TENSOR || scheme == OQ_INT8_SYM_PER_TENSOR) {
     float amax = 0.0f;
     for (int b = 0; b < B; ++b)
       for (int h = 0; h < H; ++h)
@@ -241,7 +279,7 @@ static void calibrate(const oq_cache* c, const block* k, int scheme, float* scal
             float a = fabsf(block_at(k, b, h, t, d));
             if (a > amax) amax = a;
           }
-    scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : 127.0f);
+    scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : scheme == OQ_FP8_E5M2_PER_TENSOR ? 57344.0f : 127.0f);
   } else if (scheme == OQ_INT8_SYM_PER_CHANNEL) {
     for (int h = 0; h < H; ++h)
       for (int d = 0; d < D; ++d) {
@@ -291,6 +329,9 @@ static void quantize_token(const oq_cache* c, const block* k, int scheme, uint8_
     switch (scheme) {
       case OQ_FP8_E4M3_PER_TENSOR:
         q = scale[0] == 0.0f ? 0 : oq_e4m3_encode(x / scale[0]);
+        break;
+      case OQ_FP8_E5M2_PER_TENSOR:
+        q = scale[0] == 0.0f ? 0 : oq_e5m2_encode(x / scale[0]);
         break;
       case OQ_INT8_SYM_PER_TENSOR:
         q = oq_sym_code(x, scale[0], 127);
@@ -479,6 +520,8 @@ static float value_at(const oq_cache* c, int which, int b, int h, int t, int d) 
   switch (scheme) {
     case OQ_FP8_E4M3_PER_TENSOR:
       return oq_e4m3_decode((uint8_t)q) * scale[0];
+    case OQ_FP8_E5M2_PER_TENSOR:
+      return oq_e5m2_decode((uint8_t)q) * scale[0];
     case OQ_INT8_SYM_PER_TENSOR:
       return (float)(int8_t)q * scale[0];
     case OQ_INT8_SYM_PER_TOKEN:

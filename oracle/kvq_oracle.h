@@ -12,8 +12,9 @@
  *  [P1] "KV Cache Quantization" (infra.bea.ai guide): §1 memory table, §3 KIVI
  *       (Key per-channel, Value per-token, residual cache), §4 FP8 KV cache.
  *  [P3] "KV Cache Quantization in Production LLM Serving: Comparing FP8, INT8, INT4,
- *       KIVI, and KVQuant" (llms.blog): memory-per-token formula, §1 FP8 E4M3,
- *       §2 INT8 symmetric [-127,127], §3 KIVI.
+ *       KIVI, and KVQuant" (llms.blog): memory-per-token formula, §1 FP8 E4M3 (and
+ *       E5M2, the other OCP FP8 format the section compares it with), §2 INT8 symmetric
+ *       [-127,127], §3 KIVI.
  *  [P4] "How KV cache quantization reduces GPU memory" (n4n.ai): Step 1 tensor shape,
  *       Step 2 schemes, Step 3 QuantizedKVCache (quantize / dequantize / append).
  *
@@ -40,7 +41,8 @@ enum {
   OQ_INT8_SYM_PER_CHANNEL = 3,
   OQ_UINT8_ASYM_PER_CHANNEL = 4,
   OQ_KIVI_INT4 = 5,
-  OQ_KIVI_INT2 = 6
+  OQ_KIVI_INT2 = 6,
+  OQ_FP8_E5M2_PER_TENSOR = 7
 };
 
 /* ---- element codecs ---- */
@@ -48,6 +50,8 @@ float oq_bf16_to_f32(uint16_t h);
 uint16_t oq_f32_to_bf16(float f);
 uint8_t oq_e4m3_encode(float x);            /* round-to-nearest-even, saturate finite */
 float oq_e4m3_decode(uint8_t code);
+uint8_t oq_e5m2_encode(float x);            /* round-to-nearest-even, saturate finite */
+float oq_e5m2_decode(uint8_t code);
 int oq_sym_code(float x, float s, int qmax); /* clamp(rne(x/s), -qmax, qmax); 0 if s == 0 */
 void oq_asym_params(float mn, float mx, float* s, uint8_t* zp);
 int oq_asym_code(float x, float s, uint8_t zp);

@@ -17,13 +17,16 @@ from tests import test_oracle_pins as pins
 SRC = os.path.join(os.path.dirname(oracle.__file__), "kvq_oracle.c")
 
 MUTATIONS = [
-    ("per-tensor qmax 128", "scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : 127.0f);",
-     "scale[0] = amax / (scheme == OQ_FP8_E4M3_PER_TENSOR ? 448.0f : 128.0f);"),
+    ("per-tensor qmax 128", "scheme == OQ_FP8_E5M2_PER_TENSOR ? 57344.0f : 127.0f);",
+     "scheme == OQ_FP8_E5M2_PER_TENSOR ? 57344.0f : 128.0f);"),
     ("per-token qmax 128", "tok_scale = amax / 127.0f;", "tok_scale = amax / 128.0f;"),
     ("per-channel qmax 255", "scale[h * D + d] = amax / 127.0f;", "scale[h * D + d] = amax / 255.0f;"),
     ("round half away", "  float y = x / s;\n  float r = rintf(y);", "  float y = x / s;\n  float r = roundf(y);"),
     ("clamp -128", "if (r < (float)-qmax) r = (float)-qmax;", "if (r < (float)(-qmax - 1)) r = (float)(-qmax - 1);"),
-    ("fp8 scale 240", "448.0f : 127.0f", "240.0f : 127.0f"),
+    ("fp8 scale 240", "OQ_FP8_E4M3_PER_TENSOR ? 448.0f :", "OQ_FP8_E4M3_PER_TENSOR ? 240.0f :"),
+    ("e5m2 scale 61440", "57344.0f : 127.0f", "61440.0f : 127.0f"),
+    ("e5m2 bias", "v = ldexpf(1.0f + (float)M / 4.0f, E - 15);", "v = ldexpf(1.0f + (float)M / 4.0f, E - 14);"),
+    ("e5m2 subnormal grid", "v = ldexpf((float)M, -16);", "v = ldexpf((float)M, -15);"),
     ("e4m3 bias", "v = ldexpf((float)(8 + m), e - 10);", "v = ldexpf((float)(8 + m), e - 9);"),
     ("e4m3 no saturation", "if (a > 448.0f) return (uint8_t)(sign | 0x7E);", "if (a > 480.0f) return (uint8_t)(sign | 0x7F);"),
     ("asym zp sign", "float z = rintf(-lo / sc);", "float z = rintf(lo / sc);"),

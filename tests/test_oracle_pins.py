@@ -155,6 +155,74 @@ def test_e4m3_nearest_by_brute_force():
         assert abs(oracle.e4m3_decode(code) - float(x)) == best
 
 
+# --------------------------------------------------------------- FP8 E5M2 (a next-row format)
+def test_e5m2_decode_matches_torch():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes.copy()).view(torch.float8_e5m2).float().numpy()
+    for c in codes:
+        got = oracle.e5m2_decode(int(c))
+        if np.isnan(ref[c]):
+            assert np.isnan(got)
+        else:
+            assert got == ref[c] and np.signbit(got) == np.signbit(ref[c])
+
+
+def test_e5m2_roundtrip_all_finite_codes():
+    for c in range(256):
+        if (c >> 2) & 0x1F == 0x1F:
+            continue  # infinity and NaN
+        assert oracle.e5m2_encode(oracle.e5m2_decode(c)) == c
+
+
+def test_e5m2_encode_matches_torch_in_range():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(8)
+    x = np.concatenate([
+        rng.uniform(-57344, 57344, 20000), rng.normal(0, 1, 20000), rng.normal(0, 1e-3, 20000),
+        np.ldexp(rng.uniform(-1, 1, 5000), -15),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    got = np.array([oracle.e5m2_encode(v) for v in x], np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_e5m2_ties_saturation_and_zero():
+    assert oracle.e5m2_encode(1.125) == oracle.e5m2_encode(1.0)                 # tie -> even (m=0)
+    assert oracle.e5m2_decode(oracle.e5m2_encode(1.375)) == 1.5                 # tie -> even (m=2)
+    assert oracle.e5m2_encode(2.0**-17) == 0x00                                 # subnormal tie -> 0
+    assert oracle.e5m2_decode(oracle.e5m2_encode(3 * 2.0**-17)) == 2.0**-15     # -> even code 2
+    for big in (57344.0, 57345.0, 61440.0, 70000.0, 1e30, float("inf")):
+        assert oracle.e5m2_encode(big) == 0x7B
+        assert oracle.e5m2_encode(-big) == 0xFB
+    assert oracle.e5m2_decode(0x7B) == 57344.0
+    assert oracle.e5m2_encode(-0.0) == 0x80 and oracle.e5m2_encode(0.0) == 0x00
+
+
+def test_e5m2_nearest_by_brute_force():
+    finite = [(c, oracle.e5m2_decode(c)) for c in range(124)]
+    rng = np.random.default_rng(4)
+    for x in np.concatenate([rng.uniform(0, 57344, 1500), rng.uniform(0, 4, 1500)]).astype(np.float32):
+        code = oracle.e5m2_encode(float(x))
+        best = min(abs(v - float(x)) for _, v in finite)
+        assert abs(oracle.e5m2_decode(code) - float(x)) == best
+
+
+def test_e5m2_per_tensor_scale_and_codes():
+    rng = np.random.default_rng(5)
+    x = rng.normal(0, 2, (1, 2, 6, 16)).astype(np.float32)
+    c = OracleCache(1, 2, 2, 16, oracle.FP8_E5M2_PER_TENSOR, oracle.FP8_E5M2_PER_TENSOR, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    s = F32(np.abs(x).max()) / F32(57344)
+    assert c["k_scale"][0] == s and c["v_scale"][0] == s
+    deq = c.dequantize(1, 8)[:, :, :6]
+    # E5M2 relative step is 2^-2: nearest-value error <= 2^-3 relative (normal range)
+    err = np.abs(deq - x)
+    bound = np.maximum(np.abs(x) * 2.0**-3, float(s) * 2.0**-17) * (1 + 2**-20)
+    assert np.all(err <= bound)
+    assert np.abs(deq).max() == np.abs(x).max()  # the absmax element maps to 57344 exactly
+
+
 # --------------------------------------------------------------- symmetric INT8
 def test_sym_round_half_even_tie():
     s = 0.125
