@@ -34,10 +34,10 @@ import synth  # noqa: E402
 METRIC = "decode-attn KV GB/s (% of B200 HBM peak) and tokens/s, per KV dtype"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-DTYPE_NAME = {synth.FP8_E4M3_PER_TENSOR: "fp8_e4m3", synth.INT8_SYM_PER_TENSOR: "int8",
+DTYPE_NAME = {synth.FP8_E4M3_PER_TENSOR: "fp8_e4m3", synth.FP8_E5M2_PER_TENSOR: "fp8_e5m2", synth.INT8_SYM_PER_TENSOR: "int8",
               synth.INT8_SYM_PER_TOKEN: "int8", synth.INT8_SYM_PER_CHANNEL: "int8",
               synth.UINT8_ASYM_PER_CHANNEL: "uint8", synth.KIVI_INT4: "int4", synth.KIVI_INT2: "int2"}
-CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
+CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
               synth.UINT8_ASYM_PER_CHANNEL)
 KERNEL_SOURCES = ["decode_attention_quantize_b200/csrc/kvq_decode.cu",
                   "decode_attention_quantize_b200/csrc/kvq_device.cuh"]
@@ -70,7 +70,7 @@ def meta_bytes_per_token(scheme, Hkv):
 
 
 def fixed_meta_bytes(scheme, Hkv):
-    if scheme in (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
+    if scheme in (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
         return 4
     if scheme == synth.INT8_SYM_PER_CHANNEL:
         return Hkv * 128 * 4

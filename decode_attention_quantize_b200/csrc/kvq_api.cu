@@ -33,7 +33,7 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_KIVI_INT2; }
+bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_FP8_E5M2_PER_TENSOR; }
 
 bool needs_scale(int s) { return true; }
 bool needs_zp(int s) { return s == KVQ_UINT8_ASYM_PER_CHANNEL; }
@@ -45,6 +45,7 @@ uint64_t scale_elems(const kvq_cache_desc* d, int side) {
   const bool paged = d->layout == KVQ_PAGED;
   switch (s) {
     case KVQ_FP8_E4M3_PER_TENSOR:
+    case KVQ_FP8_E5M2_PER_TENSOR:
     case KVQ_INT8_SYM_PER_TENSOR: return 1;
     case KVQ_INT8_SYM_PER_TOKEN:
       return paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity;

@@ -6,6 +6,8 @@
 //  - symmetric INT8: s = absmax/127, q = clamp(rne(x/s), -127, 127)
 //    ("KV Cache Quantization in Production LLM Serving", llms.blog, §2);
 //  - FP8 E4M3: s = absmax/448, q = e4m3_rn_satfinite(x/s) (infra.bea.ai §4, llms.blog §1);
+//  - FP8 E5M2: s = absmax/57344, q = e5m2_rn_satfinite(x/s) (the other OCP format llms.blog §1
+//    compares);
 //  - asymmetric uint8 per channel: affine form over a range widened to contain 0
 //    ("How KV cache quantization reduces GPU memory", n4n.ai, Steps 2-3);
 //  - KIVI: keys per channel over 32-token groups, values per token over 32-channel
@@ -35,6 +37,13 @@ __device__ __forceinline__ void load8(const void* base, size_t elem, float (&x)[
     x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
     x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
   }
+}
+
+// Two E5M2 codes, RN-even with saturation to +-57344: lo -> low byte, hi -> high byte.
+__device__ __forceinline__ uint32_t e5m2x2_rn(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 // Two E4M3 codes, RN-even with saturation: lo -> low byte, hi -> high byte.
@@ -93,7 +102,8 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(AppendParams p, uint3
   constexpr int kChunk = 256;
   const int side = blockIdx.z;
   const int scheme = side ? p.v_scheme : p.k_scheme;
-  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR;
+  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_FP8_E5M2_PER_TENSOR ||
+                          scheme == KVQ_INT8_SYM_PER_TENSOR;
   const bool per_channel = scheme == KVQ_INT8_SYM_PER_CHANNEL || scheme == KVQ_UINT8_ASYM_PER_CHANNEL;
   if (!per_tensor && !per_channel) return;
   const bool asym = scheme == KVQ_UINT8_ASYM_PER_CHANNEL;
@@ -169,10 +179,12 @@ __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
     float* scale = side ? p.v_scale : p.k_scale;
     uint8_t* zp = side ? p.v_zp : p.k_zp;
     const uint32_t* base = keys + 2 + side * 2 * hd;
-    if (scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR) {
+    if (scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_FP8_E5M2_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR) {
       if (threadIdx.x == 0) {
         const float amax = __uint_as_float(keys[side]);
-        scale[0] = __fdiv_rn(amax, scheme == KVQ_FP8_E4M3_PER_TENSOR ? 448.0f : 127.0f);
+        scale[0] = __fdiv_rn(amax, scheme == KVQ_FP8_E4M3_PER_TENSOR   ? 448.0f
+                                   : scheme == KVQ_FP8_E5M2_PER_TENSOR ? 57344.0f
+                                                                       : 127.0f);
       }
     } else if (scheme == KVQ_INT8_SYM_PER_CHANNEL) {
       for (int i = threadIdx.x; i < hd; i += blockDim.x)
@@ -248,6 +260,10 @@ __device__ __forceinline__ uint32_t code_of(float z, int zp, int scheme, int& sa
     sat += fabsf(z) > 448.0f;
     return e4m3x2_rn(z, 0.0f) & 0xFFu;
   }
+  if (scheme == KVQ_FP8_E5M2_PER_TENSOR) {
+    sat += fabsf(z) > 57344.0f;
+    return e5m2x2_rn(z, 0.0f) & 0xFFu;
+  }
   if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
     const float c = __fadd_rn(rintf(z), (float)zp);
     sat += c < 0.0f || c > 255.0f;
@@ -284,6 +300,7 @@ __device__ __forceinline__ uint2 careful_row(const float (&x)[8], const Scales8&
 }
 
 // Fast rows (s in range): false when a value may saturate or is out of range.
+template <bool kE5M2>
 __device__ __forceinline__ bool fp8_row(const float (&x)[8], const Scales8& sc, uint2& out) {
   uint32_t c[4];
   float amax = 0.0f;
@@ -291,11 +308,12 @@ __device__ __forceinline__ bool fp8_row(const float (&x)[8], const Scales8& sc, 
   for (int k = 0; k < 4; ++k) {
     float q0, q1;
     const float z0 = quot(x[2 * k], sc.s[0], sc.y[0], q0), z1 = quot(x[2 * k + 1], sc.s[0], sc.y[0], q1);
-    c[k] = e4m3x2_rn(z0, z1);
+    c[k] = kE5M2 ? e5m2x2_rn(z0, z1) : e4m3x2_rn(z0, z1);
     amax = fmaxf(amax, fmaxf(fabsf(q0), fabsf(q1)));
   }
   out = make_uint2(prmt(c[0], c[1], 0x5410u), prmt(c[2], c[3], 0x5410u));
-  return amax < 447.9f;  // |z| < 448: nothing saturates (q is within a few ulps of z)
+  return amax < (kE5M2 ? 57340.0f : 447.9f);  // |z| below the largest finite: nothing saturates
+                                              // (q is within a few ulps of z)
 }
 
 // symmetric: clamp(rne(z), -127, 127); z + 1.5 * 2^23 holds rne(z) (ties to even) in its low bits
@@ -346,7 +364,8 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   const int scheme = side ? VS : KS;  // compile-time per side
   const int lane8 = threadIdx.x & 15;
   const bool per_channel = side ? is_per_channel(VS) : is_per_channel(KS);
-  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR;
+  const bool per_tensor = scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_FP8_E5M2_PER_TENSOR ||
+                          scheme == KVQ_INT8_SYM_PER_TENSOR;
   float* scale = side ? p.v_scale : p.k_scale;
   const uint8_t* zp = side ? p.v_zp : p.k_zp;
   const void* src_base = side ? p.v_new : p.k_new;
@@ -459,7 +478,9 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
       bool ok = false;
       if (row_fast) {
         if (scheme == KVQ_FP8_E4M3_PER_TENSOR)
-          ok = fp8_row(x, sc, codes);
+          ok = fp8_row<false>(x, sc, codes);
+        else if (scheme == KVQ_FP8_E5M2_PER_TENSOR)
+          ok = fp8_row<true>(x, sc, codes);
         else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL)
           ok = asym_row(x, sc, codes);
         else
@@ -788,6 +809,12 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
               v = __fmul_rn(__half2float(__half(hr)), p.scale[0]);
               break;
             }
+            case KVQ_FP8_E5M2_PER_TENSOR: {  // an E5M2 byte is the high byte of the same-valued f16
+              __half_raw hr;
+              hr.x = (unsigned short)(q << 8);
+              v = __fmul_rn(__half2float(__half(hr)), p.scale[0]);
+              break;
+            }
             case KVQ_INT8_SYM_PER_TENSOR: v = __fmul_rn((float)(int8_t)q, p.scale[0]); break;
             case KVQ_INT8_SYM_PER_TOKEN: v = __fmul_rn((float)(int8_t)q, p.scale[row]); break;
             case KVQ_INT8_SYM_PER_CHANNEL: v = __fmul_rn((float)(int8_t)q, p.scale[h * kHeadDim + d]); break;
@@ -850,7 +877,8 @@ bool append_pair_supported(int ks, int vs) {
   if (is_kivi(ks) || is_kivi(vs)) return ks == vs;
   constexpr int F = KVQ_FP8_E4M3_PER_TENSOR, T = KVQ_INT8_SYM_PER_TENSOR, K = KVQ_INT8_SYM_PER_TOKEN,
                 C = KVQ_INT8_SYM_PER_CHANNEL, U = KVQ_UINT8_ASYM_PER_CHANNEL;
-  const int pairs[][2] = {{F, F}, {T, T}, {K, K}, {C, C}, {U, U}, {T, U}, {C, U}, {K, U}, {T, K}, {F, T}, {T, F}};
+  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR;
+  const int pairs[][2] = {{F, F}, {T, T}, {K, K}, {C, C}, {U, U}, {T, U}, {C, U}, {K, U}, {T, K}, {F, T}, {T, F}, {E, E}};
   for (const auto& pr : pairs)
     if (pr[0] == ks && pr[1] == vs) return true;
   return false;
@@ -864,6 +892,8 @@ cudaError_t launch_quantize_rows(const AppendParams& p, long long rows, cudaStre
   if (ks == A && vs == B) return launch_quantize_rows_pair<A, B>(p, rows, st);
   KVQ_PAIR(F, F) KVQ_PAIR(T, T) KVQ_PAIR(K, K) KVQ_PAIR(C, C) KVQ_PAIR(U, U)
   KVQ_PAIR(T, U) KVQ_PAIR(C, U) KVQ_PAIR(K, U) KVQ_PAIR(T, K) KVQ_PAIR(F, T) KVQ_PAIR(T, F)
+  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR;
+  KVQ_PAIR(E, E)
 #undef KVQ_PAIR
   return cudaErrorNotSupported;
 }

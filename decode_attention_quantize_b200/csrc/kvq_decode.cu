@@ -12,7 +12,7 @@
 //   S^T[tokens x heads] = codes(f16, exact) . Q'^T      (Q' = q * fold, split hi + lo f16)
 //   online softmax in the log2 domain, fp32
 //   O^T[d x heads]     += codes^T(f16, exact) . P'^T   (P' = p * fold, split hi + lo f16)
-// Codes stay exact (every E4M3, int8, uint8 - zp, INT4 and INT2 value is an f16 value);
+// Codes stay exact (every E4M3, E5M2, int8, uint8 - zp, INT4 and INT2 value is an f16 value);
 // scales are folded into the fp32 operand, which is split into two f16 halves (about 22
 // significant bits, range-normalised by a power of two) so the result stays well inside
 // 2e-4 of an fp64 reference. Each CTA writes one (m, l, O) partial per pair it touches;
@@ -41,18 +41,20 @@ constexpr int kRT = 32;                 // residual tile tokens (bf16 rows)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-enum { FMT_E4M3, FMT_S8, FMT_U8, FMT_U4, FMT_U2 };
+enum { FMT_E4M3, FMT_E5M2, FMT_S8, FMT_U8, FMT_U4, FMT_U2 };
 enum { FOLD_TENSOR, FOLD_TOKEN, FOLD_CHANNEL, FOLD_KIVI };
 
 __host__ __device__ constexpr int fmt_of(int s) {
   return s == KVQ_FP8_E4M3_PER_TENSOR      ? FMT_E4M3
+         : s == KVQ_FP8_E5M2_PER_TENSOR    ? FMT_E5M2
          : s == KVQ_UINT8_ASYM_PER_CHANNEL ? FMT_U8
          : s == KVQ_KIVI_INT4              ? FMT_U4
          : s == KVQ_KIVI_INT2              ? FMT_U2
                                            : FMT_S8;
 }
 __host__ __device__ constexpr int fold_of(int s) {
-  return (s == KVQ_FP8_E4M3_PER_TENSOR || s == KVQ_INT8_SYM_PER_TENSOR)        ? FOLD_TENSOR
+  return (s == KVQ_FP8_E4M3_PER_TENSOR || s == KVQ_FP8_E5M2_PER_TENSOR || s == KVQ_INT8_SYM_PER_TENSOR)
+             ? FOLD_TENSOR
          : s == KVQ_INT8_SYM_PER_TOKEN                                          ? FOLD_TOKEN
          : (s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL) ? FOLD_CHANNEL
                                                                                 : FOLD_KIVI;
@@ -328,6 +330,9 @@ __device__ __forceinline__ void cvt8x4(uint32_t w, uint32_t zlo, uint32_t zhi, u
     asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.rn.f16x2.e4m3x2 %0, l;\n cvt.rn.f16x2.e4m3x2 %1, h;\n}\n"
         : "=r"(lo), "=r"(hi)
         : "r"(w));
+  } else if constexpr (FMT == FMT_E5M2) {  // an E5M2 byte is the high byte of the equal f16
+    lo = prmt(w, 0u, 0x1404u);
+    hi = prmt(w, 0u, 0x3424u);
   } else if constexpr (FMT == FMT_S8) {  // word already XORed with 0x80808080: codes biased by 128
     lo = hsub2_u(prmt(w, 0x64646464u, 0x5150u), 0x64806480u);  // (1024 + 128 + q) - 1152
     hi = hsub2_u(prmt(w, 0x64646464u, 0x5352u), 0x64806480u);
@@ -1195,7 +1200,7 @@ Variant variant() {
   return Variant{KS, VS, PG ? 1 : 0, decode_kernel<KS, VS, PG>, C::kSmemBytes, C::kTS};
 }
 
-constexpr int kNumVariants = 24;
+constexpr int kNumVariants = 26;
 constexpr int kMaxDevices = 64;
 
 const Variant* variants() {
@@ -1222,6 +1227,8 @@ const Variant* variants() {
       variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_INT8_SYM_PER_TENSOR, true>(),
       variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, false>(),
       variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, true>(),
+      variant<KVQ_FP8_E5M2_PER_TENSOR, KVQ_FP8_E5M2_PER_TENSOR, false>(),
+      variant<KVQ_FP8_E5M2_PER_TENSOR, KVQ_FP8_E5M2_PER_TENSOR, true>(),
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
   };

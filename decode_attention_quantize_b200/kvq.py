@@ -26,6 +26,7 @@ INT8_SYM_PER_CHANNEL = 3
 UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
+FP8_E5M2_PER_TENSOR = 7
 KVQ_F32, KVQ_BF16 = 0, 1
 KVQ_DENSE, KVQ_PAGED = 0, 1
 KVQ_APPEND_CALIBRATE = 0x1
@@ -240,7 +241,7 @@ class QuantizedKVCache:
         rows = (s.num_pages, s.Hkv, s.page_size) if s.paged else (s.B, s.Hkv, s.capacity)
         for side, sch in (("k", s.k_scheme), ("v", s.v_scheme)):
             self.t[side + "_codes"] = torch.zeros(*rows, row_bytes(sch, s.D), dtype=torch.uint8, device=dev)
-            if sch in (FP8_E4M3_PER_TENSOR, INT8_SYM_PER_TENSOR):
+            if sch in (FP8_E4M3_PER_TENSOR, FP8_E5M2_PER_TENSOR, INT8_SYM_PER_TENSOR):
                 self.t[side + "_scale"] = torch.zeros(4, dtype=torch.float32, device=dev)
             elif sch == INT8_SYM_PER_TOKEN:
                 self.t[side + "_scale"] = torch.zeros(*rows, dtype=torch.float32, device=dev)

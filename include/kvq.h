@@ -60,6 +60,9 @@ typedef enum kvq_status {
  *                       s = (max - min)/(2^bits - 1), q = clamp(rne((x - min)/s)), fp32
  *                       scale and minimum, codes packed along head_dim (lower channel in
  *                       lower bits), recent tokens in a bf16 residual of 128 tokens.
+ *  FP8_E5M2_PER_TENSOR  OCP E5M2 codes of x/s, s = absmax/57344 over the calibrating append,
+ *                       saturating at +-57344 (llms.blog §1 compares E4M3 with E5M2; a format
+ *                       variant beyond the configurations the pages measure).
  * A zero range gives s = 0 and code 0. */
 typedef enum kvq_scheme {
   KVQ_FP8_E4M3_PER_TENSOR = 0,
@@ -68,7 +71,8 @@ typedef enum kvq_scheme {
   KVQ_INT8_SYM_PER_CHANNEL = 3,
   KVQ_UINT8_ASYM_PER_CHANNEL = 4,
   KVQ_KIVI_INT4 = 5,
-  KVQ_KIVI_INT2 = 6
+  KVQ_KIVI_INT2 = 6,
+  KVQ_FP8_E5M2_PER_TENSOR = 7
 } kvq_scheme;
 
 typedef enum kvq_dtype { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;

@@ -109,6 +109,7 @@ INT8_SYM_PER_CHANNEL = 3
 UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
+FP8_E5M2_PER_TENSOR = 7
 
 
 @dataclass
@@ -172,7 +173,8 @@ class Workload:
 
 
 def workloads() -> dict:
-    """The five workloads: tiny INT8, FP8 8B-shaped, KIVI-4 70B, KIVI-2 131K, paged INT8."""
+    """The six workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 70B, KIVI-2 131K,
+    paged INT8."""
     return {
         "tiny_int8": Workload(
             name="tiny_int8", seed=1, B=1, Hq=1, Hkv=1, D=128,
@@ -181,6 +183,10 @@ def workloads() -> dict:
         "fp8_8b": Workload(
             name="fp8_8b", seed=2, B=32, Hq=32, Hkv=8, D=128,
             k_scheme=FP8_E4M3_PER_TENSOR, v_scheme=FP8_E4M3_PER_TENSOR, bf16=True,
+            outlier_scale=20.0, rope_theta=500000.0, context=4096),
+        "e5m2_8b": Workload(
+            name="e5m2_8b", seed=6, B=32, Hq=32, Hkv=8, D=128,
+            k_scheme=FP8_E5M2_PER_TENSOR, v_scheme=FP8_E5M2_PER_TENSOR, bf16=True,
             outlier_scale=20.0, rope_theta=500000.0, context=4096),
         "kivi4_70b": Workload(
             name="kivi4_70b", seed=3, B=16, Hq=64, Hkv=8, D=128,

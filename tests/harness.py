@@ -16,7 +16,7 @@ import synth
 from oracle import OracleCache
 
 ATTN_RTOL = 2e-4          # max|out - ref| <= ATTN_RTOL * max|ref|
-CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
+CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
               synth.UINT8_ASYM_PER_CHANNEL)
 SCALE = np.float32(1.0 / math.sqrt(128.0))
 
@@ -75,7 +75,7 @@ def compare_dense(oc: OracleCache, gc, where=""):
             f"{where}: {side} codes differ"
         sch = oc.k_scheme if side == "k" else oc.v_scheme
         s_g, s_o = np_of(gc[side + "_scale"]), oc[side + "_scale"]
-        if sch in (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
+        if sch in (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
             assert s_g.view(np.uint32)[0] == s_o.view(np.uint32)[0], f"{where}: {side} scale differs"
         elif sch == synth.INT8_SYM_PER_TOKEN:
             assert np.array_equal(s_g[:, :, :L].view(np.uint32), s_o[:, :, :L].view(np.uint32)), \
@@ -115,7 +115,7 @@ def compare_paged(oc: OracleCache, gc, where=""):
                     assert np.array_equal(np_of(gc[side + "_scale"])[page, :, slot].view(np.uint32),
                                           oc[side + "_scale"][page, :, slot].view(np.uint32))
         s_g, s_o = np_of(gc[side + "_scale"]), oc[side + "_scale"]
-        if sch in (synth.FP8_E4M3_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
+        if sch in (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
             assert s_g.view(np.uint32)[0] == s_o.view(np.uint32)[0], f"{where}: {side} scale differs"
         elif sch in (synth.INT8_SYM_PER_CHANNEL, synth.UINT8_ASYM_PER_CHANNEL):
             assert np.array_equal(s_g.view(np.uint32), s_o.view(np.uint32)), f"{where}: {side} channel scales"

@@ -113,6 +113,10 @@ def test_fp8_8b_full():
     _dense_full("fp8_8b")
 
 
+def test_e5m2_8b_full():
+    _dense_full("e5m2_8b")
+
+
 def test_kivi4_70b_full():
     _dense_full("kivi4_70b")
 

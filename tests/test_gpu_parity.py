@@ -20,6 +20,7 @@ S = synth
 # ------------------------------------------------------------------ dense, 8-bit schemes
 @pytest.mark.parametrize("ks,vs", [
     (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR),
+    (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR),
     (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TENSOR),
     (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN),
     (S.INT8_SYM_PER_CHANNEL, S.INT8_SYM_PER_CHANNEL),
@@ -71,7 +72,7 @@ BULK_PAIRS = [
     (S.UINT8_ASYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL), (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
     (S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL), (S.INT8_SYM_PER_TOKEN, S.UINT8_ASYM_PER_CHANNEL),
     (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TOKEN), (S.FP8_E4M3_PER_TENSOR, S.INT8_SYM_PER_TENSOR),
-    (S.INT8_SYM_PER_TENSOR, S.FP8_E4M3_PER_TENSOR),
+    (S.INT8_SYM_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR),
 ]
 
 
@@ -121,6 +122,7 @@ def test_kivi_chunked_appends_match_bulk():
     (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL, 16),
     (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL, 32),
     (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR, 16),
+    (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR, 32),
     (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN, 64),
     (S.INT8_SYM_PER_CHANNEL, S.INT8_SYM_PER_CHANNEL, 16),
 ])
@@ -188,9 +190,33 @@ def test_saturation_is_counted():
     assert gc.status()[1] > 0
 
 
+@pytest.mark.parametrize("scheme", [S.FP8_E4M3_PER_TENSOR, S.FP8_E5M2_PER_TENSOR, S.INT8_SYM_PER_TENSOR])
+def test_saturated_codes_match_oracle(scheme):
+    # a per-tensor scale calibrated on a small prefill, then tokens up to 50x past its range:
+    # the saturated codes (largest finite of the format) must still match bit for bit
+    B, Hq, Hkv = 2, 8, 2
+    w = H.workload(B, Hq, Hkv, scheme, scheme, bf16=False)  # fp32 inputs, scaled below
+    K = synth.keys(w, 0, B, 0, Hkv, 0, 70)
+    V = synth.values(w, 0, B, 0, Hkv, 0, 70)
+    oc = H.OracleCache(B, Hq, Hkv, 128, scheme, scheme, cap=128)
+    gc = H.kvq().QuantizedKVCache(H.kvq().CacheSpec(B, Hq, Hkv, scheme, scheme, capacity=128))
+    oc.append(K[:, :, :64], V[:, :, :64], False, calibrate=True)
+    gc.append(H.dev(K[:, :, :64], False), H.dev(V[:, :, :64], False), calibrate=True)
+    for t, f in zip(range(64, 70), (1.5, 3.0, 7.0, 20.0, 50.0, -50.0)):
+        kk = np.ascontiguousarray(K[:, :, t:t + 1] * np.float32(f))
+        vv = np.ascontiguousarray(V[:, :, t:t + 1] * np.float32(f))
+        oc.append(kk, vv, False)
+        gc.append(H.dev(kk, False), H.dev(vv, False))
+    torch.cuda.synchronize()
+    H.compare_dense(oc, gc, "saturated tokens")
+    assert gc.status()[1] > 0
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), False, "decode over saturated codes")
+
+
 # ------------------------------------------------------------------ dequantize
 @pytest.mark.parametrize("ks,vs", [(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.KIVI_INT2, S.KIVI_INT2),
-                                   (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL)])
+                                   (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
+                                   (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR)])
 def test_dequantize_matches_oracle(ks, vs):
     oc, gc, _ = H.dense_case(B=2, Hq=8, Hkv=2, ks=ks, vs=vs, prefill=200, steps=1, cap=384)
     T = oc.tokens()
