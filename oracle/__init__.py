@@ -35,6 +35,7 @@ UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
+APPEND_CALIBRATE, APPEND_RESCALE = 1, 2  # append modes (oq_append)
 
 _lib = None
 
@@ -235,13 +236,18 @@ class OracleCache:
     def tokens(self, b=0):
         return int(lib().oq_tokens(ctypes.byref(self.c), b))
 
-    def append(self, k, v, bf16: bool, calibrate=False, new_lens=None):
+    def append(self, k, v, bf16: bool, calibrate=False, new_lens=None, rescale=False):
+        """calibrate: scales from this block; rescale: merge this block's scales into the
+        cached ones and requantize the cached codes whose scale grew (not both)."""
+        if calibrate and rescale:
+            raise ValueError("calibrate and rescale are exclusive")
         k = np.ascontiguousarray(k)
         v = np.ascontiguousarray(v)
         n_new = k.shape[2]
         nl = None if new_lens is None else np.ascontiguousarray(new_lens, np.int32)
+        mode = APPEND_CALIBRATE if calibrate else (APPEND_RESCALE if rescale else 0)
         rc = lib().oq_append(ctypes.byref(self.c), k.ctypes.data, v.ctypes.data, int(bf16), n_new,
-                             _ptr(nl), int(bool(calibrate)))
+                             _ptr(nl), mode)
         if rc != 0:
             raise ValueError("oracle append rejected the call (capacity or arguments)")
 

@@ -308,6 +308,23 @@ static void calibrate(const oq_cache* c, const block* k, int scheme, float* scal
   }
 }
 
+/* Code of value x under a fixed scale s (and zero point zp) of an 8-bit scheme with
+ * batch-wide scales. */
+static int code_for(int scheme, float x, float s, uint8_t zp) {
+  switch (scheme) {
+    case OQ_FP8_E4M3_PER_TENSOR:
+      return s == 0.0f ? 0 : oq_e4m3_encode(x / s);
+    case OQ_FP8_E5M2_PER_TENSOR:
+      return s == 0.0f ? 0 : oq_e5m2_encode(x / s);
+    case OQ_INT8_SYM_PER_TENSOR:
+    case OQ_INT8_SYM_PER_CHANNEL:
+      return oq_sym_code(x, s, 127);
+    case OQ_UINT8_ASYM_PER_CHANNEL:
+      return oq_asym_code(x, s, zp);
+  }
+  return 0;
+}
+
 /* Quantize token t of the block (b, h) into cache row `row` (8-bit schemes). */
 static void quantize_token(const oq_cache* c, const block* k, int scheme, uint8_t* codes,
                            float* scale, const uint8_t* zp, int b, int h, int t, size_t row) {
@@ -326,26 +343,12 @@ static void quantize_token(const oq_cache* c, const block* k, int scheme, uint8_
   for (int d = 0; d < D; ++d) {
     const float x = block_at(k, b, h, t, d);
     int q = 0;
-    switch (scheme) {
-      case OQ_FP8_E4M3_PER_TENSOR:
-        q = scale[0] == 0.0f ? 0 : oq_e4m3_encode(x / scale[0]);
-        break;
-      case OQ_FP8_E5M2_PER_TENSOR:
-        q = scale[0] == 0.0f ? 0 : oq_e5m2_encode(x / scale[0]);
-        break;
-      case OQ_INT8_SYM_PER_TENSOR:
-        q = oq_sym_code(x, scale[0], 127);
-        break;
-      case OQ_INT8_SYM_PER_TOKEN:
-        q = oq_sym_code(x, tok_scale, 127);
-        break;
-      case OQ_INT8_SYM_PER_CHANNEL:
-        q = oq_sym_code(x, scale[h * D + d], 127);
-        break;
-      case OQ_UINT8_ASYM_PER_CHANNEL:
-        q = oq_asym_code(x, scale[h * D + d], zp[h * D + d]);
-        break;
-    }
+    if (scheme == OQ_INT8_SYM_PER_TOKEN)
+      q = oq_sym_code(x, tok_scale, 127);
+    else if (scheme == OQ_INT8_SYM_PER_CHANNEL || scheme == OQ_UINT8_ASYM_PER_CHANNEL)
+      q = code_for(scheme, x, scale[h * D + d], zp ? zp[h * D + d] : 0);
+    else
+      q = code_for(scheme, x, scale[0], 0);
     put_code(codes, scheme, D, row, d, q);
   }
 }
@@ -434,6 +437,91 @@ static int append_kivi(oq_cache* c, const block* kb, const block* vb) {
   return 0;
 }
 
+/* Dequantized value of an 8-bit code with batch-wide scale s (and zero point zp). */
+static float fixed_value(int scheme, int q, float s, uint8_t zp) {
+  switch (scheme) {
+    case OQ_FP8_E4M3_PER_TENSOR:
+      return oq_e4m3_decode((uint8_t)q) * s;
+    case OQ_FP8_E5M2_PER_TENSOR:
+      return oq_e5m2_decode((uint8_t)q) * s;
+    case OQ_INT8_SYM_PER_TENSOR:
+    case OQ_INT8_SYM_PER_CHANNEL:
+      return (float)(int8_t)q * s;
+    case OQ_UINT8_ASYM_PER_CHANNEL:
+      return (float)(q - (int)zp) * s;
+  }
+  return 0.0f;
+}
+
+/* Rescaling append, one side (P4 Step 3 merges the scale of every new block into the
+ * cached one with a running maximum; P4 Step 7 wants scales that only grow, or are
+ * recomputed as the cache grows). Symmetric schemes: s' = max(s, s_block) per scale
+ * element, s_block as in calibration. Asymmetric: (s', zp') of the union of the range the
+ * cached (s, zp) represent, [(0 - zp) s, (255 - zp) s], and the block's range widened to
+ * hold 0; unchanged when the block's range lies inside. Each cached code whose scale
+ * element changed is requantized from its dequantized value (the page's snippet keeps the
+ * old codes, which then decode with the wrong scale). */
+static void rescale(oq_cache* c, const block* k, int which) {
+  const int scheme = which ? c->v_scheme : c->k_scheme;
+  float* scale = which ? c->v_scale : c->k_scale;
+  uint8_t* zp = which ? c->v_zp : c->k_zp;
+  uint8_t* codes = which ? c->v_codes : c->k_codes;
+  const int B = c->B, H = c->Hkv, D = c->D;
+  const int per_tensor = scheme == OQ_FP8_E4M3_PER_TENSOR || scheme == OQ_FP8_E5M2_PER_TENSOR ||
+                         scheme == OQ_INT8_SYM_PER_TENSOR;
+  const int per_channel = scheme == OQ_INT8_SYM_PER_CHANNEL || scheme == OQ_UINT8_ASYM_PER_CHANNEL;
+  if (!per_tensor && !per_channel) return;
+  const int n = per_tensor ? 1 : H * D;
+  float* s_old = (float*)malloc(sizeof(float) * n);
+  uint8_t* zp_old = (uint8_t*)calloc(n, 1);
+  float* s_blk = (float*)calloc(n, sizeof(float));
+  uint8_t* zp_blk = (uint8_t*)calloc(n, 1);
+  memcpy(s_old, scale, sizeof(float) * n);
+  if (zp) memcpy(zp_old, zp, n);
+  if (scheme != OQ_UINT8_ASYM_PER_CHANNEL) {
+    calibrate(c, k, scheme, s_blk, zp_blk);
+    for (int i = 0; i < n; ++i)
+      if (s_blk[i] > scale[i]) scale[i] = s_blk[i];
+  } else {
+    for (int h = 0; h < H; ++h)
+      for (int d = 0; d < D; ++d) {
+        float mn = 0.0f, mx = 0.0f;
+        int first = 1;
+        for (int b = 0; b < B; ++b)
+          for (int t = 0; t < block_len(k, b); ++t) {
+            float v = block_at(k, b, h, t, d);
+            if (first || v < mn) mn = v;
+            if (first || v > mx) mx = v;
+            first = 0;
+          }
+        const int i = h * D + d;
+        const float lo_b = mn < 0.0f ? mn : 0.0f, hi_b = mx > 0.0f ? mx : 0.0f;
+        const float lo_o = (float)(0 - (int)zp_old[i]) * s_old[i];
+        const float hi_o = (float)(255 - (int)zp_old[i]) * s_old[i];
+        if (lo_b < lo_o || hi_b > hi_o)
+          oq_asym_params(lo_b < lo_o ? lo_b : lo_o, hi_b > hi_o ? hi_b : hi_o, &scale[i], &zp[i]);
+      }
+  }
+  for (int b = 0; b < B; ++b) {
+    const int len = c->paged ? c->seq_lens[b] : c->len;
+    for (int h = 0; h < H; ++h)
+      for (int t = 0; t < len; ++t) {
+        const size_t row = row_of(c, b, h, t);
+        for (int d = 0; d < D; ++d) {
+          const int i = per_tensor ? 0 : h * D + d;
+          const uint8_t z_new = zp ? zp[i] : 0;
+          if (scale[i] == s_old[i] && z_new == zp_old[i]) continue;
+          const float x = fixed_value(scheme, get_code(codes, scheme, D, row, d), s_old[i], zp_old[i]);
+          put_code(codes, scheme, D, row, d, code_for(scheme, x, scale[i], z_new));
+        }
+      }
+  }
+  free(s_old);
+  free(zp_old);
+  free(s_blk);
+  free(zp_blk);
+}
+
 int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
               const int32_t* new_lens, int calibrate_flag) {
   block kb = {k_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
@@ -457,9 +545,14 @@ int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, in
       return -1;
     }
   }
-  if (calibrate_flag) {
+  if (calibrate_flag == OQ_APPEND_CALIBRATE) {
     calibrate(c, &kb, c->k_scheme, c->k_scale, c->k_zp);
     calibrate(c, &vb, c->v_scheme, c->v_scale, c->v_zp);
+  } else if (calibrate_flag == OQ_APPEND_RESCALE) {
+    rescale(c, &kb, 0);
+    rescale(c, &vb, 1);
+  } else if (calibrate_flag != 0) {
+    return -1;
   }
   for (int b = 0; b < c->B; ++b) {
     const int start = c->paged ? c->seq_lens[b] : c->len;

@@ -74,9 +74,15 @@ typedef struct {
   int32_t *page_table, *seq_lens;
 } oq_cache;
 
+/* Append modes (the `calibrate` argument of oq_append). */
+enum { OQ_APPEND_PLAIN = 0, OQ_APPEND_CALIBRATE = 1, OQ_APPEND_RESCALE = 2 };
+
 /* Append n_new tokens per sequence (new_lens: per-sequence counts, paged only).
  * k_new/v_new are [B,Hkv,n_new,D], bf16 bits when in_bf16 else fp32.
- * calibrate != 0 recomputes per-tensor / per-channel scales from these tokens.
+ * calibrate: OQ_APPEND_CALIBRATE recomputes per-tensor / per-channel scales from these
+ * tokens; OQ_APPEND_RESCALE merges the block's scales into the cached ones (they only
+ * grow) and requantizes the cached codes whose scale changed, before the block is
+ * quantized. KIVI and per-token schemes ignore both.
  * Returns 0, or -1 on a capacity / argument error. */
 int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
               const int32_t* new_lens, int calibrate);

@@ -48,6 +48,16 @@ MUTATIONS = [
     ("attention lse", "*lse = m + log(l);", "*lse = log(l);"),
     ("gqa mapping", "const int hq = hk * G + j;", "const int hq = j * c->Hkv + hk;"),
     ("bytes formula", "return 2.0 * bytes_per_elem *", "return bytes_per_elem *"),
+    ("rescale keeps the smaller scale", "if (s_blk[i] > scale[i]) scale[i] = s_blk[i];",
+     "if (s_blk[i] < scale[i]) scale[i] = s_blk[i];"),
+    ("rescale keeps old codes", "put_code(codes, scheme, D, row, d, code_for(scheme, x, scale[i], z_new));",
+     "(void)x;"),
+    ("rescale requantizes with the old scale", "code_for(scheme, x, scale[i], z_new)",
+     "code_for(scheme, x, s_old[i], z_new)"),
+    ("rescale old range top", "(float)(255 - (int)zp_old[i]) * s_old[i]", "(float)(255 + (int)zp_old[i]) * s_old[i]"),
+    ("rescale drops old low end", "lo_b < lo_o ? lo_b : lo_o", "lo_b"),
+    ("rescale paged length", "const int len = c->paged ? c->seq_lens[b] : c->len;",
+     "const int len = c->paged ? c->seq_lens[b] - 1 : c->len;"),
 ]
 
 

@@ -582,3 +582,206 @@ def test_calibrate_only_equals_calibrating_append():
     for name in ("k_scale", "v_scale", "v_zp"):
         assert np.array_equal(a[name], b[name]), name
     assert not b["k_codes"].any() and not b["seq_lens"].any()
+
+
+# --------------------------------------------------------------- rescaling append
+# n4n.ai Step 3 merges each new block's scale into the cached one with a running maximum;
+# Step 7 asks for scales that only grow, or are recomputed as the cache grows. The oracle's
+# rescaling append merges and requantizes the cached codes whose scale changed.
+BATCH_WIDE = [oracle.FP8_E4M3_PER_TENSOR, oracle.FP8_E5M2_PER_TENSOR, oracle.INT8_SYM_PER_TENSOR,
+              oracle.INT8_SYM_PER_CHANNEL, oracle.UINT8_ASYM_PER_CHANNEL]
+
+
+def _exact(x) -> Fraction:
+    return Fraction(float(x))
+
+
+def _nearest_sym(x: Fraction, s: Fraction, qmax=127):
+    """All integers k in [-qmax, qmax] at the least distance |x - k s| (brute force)."""
+    d = [abs(x - k * s) for k in range(-qmax, qmax + 1)]
+    m = min(d)
+    return [k - qmax for k, v in enumerate(d) if v == m], m
+
+
+@pytest.mark.parametrize("scheme", BATCH_WIDE)
+def test_rescale_on_empty_cache_equals_calibration(scheme):
+    # merging into the zero scale (or the empty range) of a fresh cache is a calibration
+    rng = np.random.default_rng(40 + scheme)
+    B, H, T, D = 2, 2, 5, 16
+    k = rng.normal(0, 2, (B, H, T, D)).astype(np.float32)
+    v = rng.normal(0.4, 1, (B, H, T, D)).astype(np.float32)
+    a = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, scheme, cap=8)
+    b = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, scheme, cap=8)
+    a.append(k, v, bf16=False, rescale=True)
+    b.append(k, v, bf16=False, calibrate=True)
+    for name in ("k_scale", "v_scale", "k_codes", "v_codes"):
+        assert np.array_equal(a[name], b[name]), name
+    if scheme == oracle.UINT8_ASYM_PER_CHANNEL:
+        assert np.array_equal(a["v_zp"], b["v_zp"])
+    assert a["v_scale"].any() and a["v_codes"].any()
+
+
+@pytest.mark.parametrize("scheme", BATCH_WIDE)
+def test_rescale_inside_range_changes_nothing(scheme):
+    rng = np.random.default_rng(50 + scheme)
+    B, H, T, D = 2, 2, 6, 16
+    x = rng.normal(0.2, 2, (B, H, T, D)).astype(np.float32)
+    y = (x[:, :, :2] * F32(0.5)).astype(np.float32)  # inside every per-channel / per-tensor range
+    a = OracleCache(B, H, H, D, scheme, scheme, cap=8)
+    b = OracleCache(B, H, H, D, scheme, scheme, cap=8)
+    for c in (a, b):
+        c.append(x, x, bf16=False, calibrate=True)
+    before = {n: a[n].copy() for n in ("k_scale", "k_codes", "v_zp") if a[n] is not None}
+    a.append(y, y, bf16=False, rescale=True)
+    b.append(y, y, bf16=False)  # plain append with the cached scales
+    for n, old in before.items():
+        assert np.array_equal(a[n][..., :T, :] if n == "k_codes" else a[n],
+                              old[..., :T, :] if n == "k_codes" else old), n
+    assert np.array_equal(a["k_codes"], b["k_codes"]) and np.array_equal(a["v_codes"], b["v_codes"])
+
+
+def test_rescale_per_tensor_int8_grows_and_requantizes_to_nearest():
+    rng = np.random.default_rng(60)
+    B, H, T, D = 1, 2, 6, 16
+    x = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    amax = F32(np.abs(x).max())
+    y = np.zeros((B, H, 1, D), np.float32)
+    y[0, 1, 0, 3] = F32(4) * amax
+    c = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.INT8_SYM_PER_TENSOR, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    s0 = c["k_scale"][0]
+    q0 = c["k_codes"][:, :, :T].view(np.int8).astype(int)
+    c.append(y, y, bf16=False, rescale=True)
+    s1 = c["k_scale"][0]
+    assert s1 == F32(F32(4) * amax) / F32(127) and s1 > s0  # the block's scale wins
+    q1 = c["k_codes"][:, :, :T].view(np.int8).astype(int)
+    assert c["k_codes"][0, 1, T, 3].view(np.int8) == 127
+    S1 = _exact(s1)
+    for old, new in zip(q0.ravel(), q1.ravel()):
+        xo = _exact(F32(old) * s0)                  # the cached value before the rescale
+        best, dist = _nearest_sym(xo, S1)
+        r = xo / S1
+        half = math.floor(r) + Fraction(1, 2)
+        if len(best) > 1:                           # an exact tie between two levels: the even one
+            assert new in best and new % 2 == 0
+        elif abs(r - half) <= abs(r) * Fraction(1, 2**24):
+            # within the fp32 rounding of x / s of a tie: the rounded quotient decides
+            assert new in (math.floor(r), math.floor(r) + 1)
+        else:
+            assert new == best[0]
+        assert abs(new) <= abs(old)
+
+
+def test_rescale_fp8_requantizes_like_torch_cast():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(61)
+    B, H, T, D = 1, 2, 8, 16
+    x = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    y = (x[:, :, :1] * F32(3)).astype(np.float32)
+    c = OracleCache(B, H, H, D, oracle.FP8_E4M3_PER_TENSOR, oracle.FP8_E4M3_PER_TENSOR, cap=16)
+    c.append(x, x, bf16=False, calibrate=True)
+    s0 = c["v_scale"][0]
+    old = c["v_codes"][:, :, :T].copy()
+    c.append(y, y, bf16=False, rescale=True)
+    s1 = c["v_scale"][0]
+    assert s1 == F32(np.abs(y).max()) / F32(448)
+    xo = torch.from_numpy(old.copy()).view(torch.float8_e4m3fn).float() * float(s0)   # fp32 product
+    want = (xo / float(s1)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(c["v_codes"][:, :, :T], want)
+
+
+def test_rescale_asym_union_of_ranges():
+    rng = np.random.default_rng(62)
+    B, H, T, D = 2, 1, 6, 8
+    x = rng.normal(0.5, 1, (B, H, T, D)).astype(np.float32)
+    y = np.zeros((B, H, 1, D), np.float32)
+    y[0, 0, 0, :4] = F32(5)                      # channels 0..3 grow upwards only
+    y[1, 0, 0, 4:6] = F32(-7)                    # channels 4, 5 grow downwards only
+    c = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    s0, z0 = c["v_scale"].copy(), c["v_zp"].copy()
+    old = c["v_codes"][:, :, :T].copy()
+    c.append(y, y, bf16=False, rescale=True)
+    s1, z1 = c["v_scale"], c["v_zp"]
+    for d in range(D):
+        lo_o = float(F32(0 - int(z0[0, d])) * s0[0, d])
+        hi_o = float(F32(255 - int(z0[0, d])) * s0[0, d])
+        col = y[:, 0, 0, d]
+        lo, hi = min(lo_o, float(col.min()), 0.0), max(hi_o, float(col.max()), 0.0)
+        if d >= 6:
+            assert s1[0, d] == s0[0, d] and z1[0, d] == z0[0, d]   # untouched channels
+            assert np.array_equal(c["v_codes"][:, :, :T, d], old[:, :, :, d])
+            continue
+        s, z = float(s1[0, d]), int(z1[0, d])
+        assert abs(s - (hi - lo) / 255) <= 1e-6 * s                 # 255 steps over the union
+        assert -z * s <= lo + s / 2 and (255 - z) * s >= hi - s / 2  # the union is represented
+        S1 = _exact(s1[0, d])
+        for b in range(B):
+            for t in range(T):
+                xo = _exact(F32(int(old[b, 0, t, d]) - int(z0[0, d])) * s0[0, d])
+                q = int(c["v_codes"][b, 0, t, d])
+                dist = [abs(xo - (k - z) * S1) for k in range(256)]
+                assert dist[q] == min(dist)                          # nearest representable level
+
+
+def test_rescale_per_channel_sym_only_grown_channels_move():
+    rng = np.random.default_rng(63)
+    B, H, T, D = 2, 2, 5, 8
+    x = rng.normal(0, 1, (B, H, T, D)).astype(np.float32)
+    y = np.zeros((B, H, 1, D), np.float32)
+    y[1, 1, 0, 2] = F32(9)
+    c = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_CHANNEL, oracle.INT8_SYM_PER_CHANNEL, cap=8)
+    c.append(x, x, bf16=False, calibrate=True)
+    s0, old = c["k_scale"].copy(), c["k_codes"][:, :, :T].copy()
+    c.append(y, y, bf16=False, rescale=True)
+    moved = c["k_scale"] != s0
+    assert moved.sum() == 1 and moved[1, 2] and c["k_scale"][1, 2] == F32(9) / F32(127)
+    keep = np.ones((H, D), bool)
+    keep[1, 2] = False
+    for h in range(H):
+        for d in range(D):
+            same = np.array_equal(c["k_codes"][:, h, :T, d], old[:, h, :, d])
+            assert same == bool(keep[h, d]) or (not keep[h, d] and same and not old[:, h, :, d].any())
+
+
+def test_rescale_scales_never_shrink():
+    rng = np.random.default_rng(64)
+    B, H, D = 1, 2, 16
+    c = OracleCache(B, H, H, D, oracle.FP8_E5M2_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, cap=64)
+    prev_k, prev_lo, prev_hi = 0.0, np.zeros((H, D)), np.zeros((H, D))
+    for i in range(8):
+        blk = rng.normal(0, float(rng.uniform(0.2, 3)), (B, H, 4, D)).astype(np.float32)
+        c.append(blk, blk, bf16=False, rescale=True)
+        sk = float(c["k_scale"][0])
+        lo = (0 - c["v_zp"].astype(float)) * c["v_scale"]
+        hi = (255 - c["v_zp"].astype(float)) * c["v_scale"]
+        assert sk >= prev_k
+        # the represented range only widens, up to the half step the integer zero point
+        # rounds away at one end
+        half = c["v_scale"] / 2 * (1 + 1e-5)
+        assert np.all(lo <= prev_lo + half) and np.all(hi >= prev_hi - half)
+        prev_k, prev_lo, prev_hi = sk, lo, hi
+
+
+def test_rescale_paged_matches_dense():
+    rng = np.random.default_rng(65)
+    B, H, D, ps, maxp = 2, 2, 16, 4, 3
+    table = rng.permutation(8)[:6].astype(np.int32).reshape(B, maxp)
+    k = rng.normal(0, 1, (B, H, 7, D)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, 7, D)).astype(np.float32)
+    y = (k[:, :, :2] * F32(2.5)).astype(np.float32)
+    w = (v[:, :, :2] * F32(-3)).astype(np.float32)
+    pg = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, paged=True,
+                     page_size=ps, max_pages=maxp, num_pages=8, page_table=table)
+    dn = OracleCache(B, H, H, D, oracle.INT8_SYM_PER_TENSOR, oracle.UINT8_ASYM_PER_CHANNEL, cap=12)
+    pg.append(k, v, bf16=False, calibrate=True, new_lens=np.array([7, 7], np.int32))
+    dn.append(k, v, bf16=False, calibrate=True)
+    pg.append(y, w, bf16=False, rescale=True, new_lens=np.array([2, 2], np.int32))
+    dn.append(y, w, bf16=False, rescale=True)
+    for n in ("k_scale", "v_scale", "v_zp"):
+        assert np.array_equal(pg[n], dn[n]), n
+    for b in range(B):
+        for t in range(9):
+            page, slot = table[b, t // ps], t % ps
+            assert np.array_equal(pg["k_codes"][page, :, slot], dn["k_codes"][b, :, t])
+            assert np.array_equal(pg["v_codes"][page, :, slot], dn["v_codes"][b, :, t])
