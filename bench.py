@@ -309,6 +309,36 @@ class GpuWorkload:
             self.cache.desc.num_quantized, self.cache.desc.num_residual = saved
         return sum(ms) / len(ms) / 1e3
 
+    def time_rescale(self, flush, stream, reps=3):
+        """Rescaling append of one token per sequence whose values are 2^(i+1) times the step
+        token's, so every repetition grows the batch-wide scales and requantizes every cached
+        code. Dense caches with batch-wide scales only; leaves the cache rescaled."""
+        torch = self.torch
+        d = self.cache.desc
+        ms = []
+        for i in range(reps):
+            f = float(2 ** (i + 1))
+            k = (self.k_new.float() * f).to(self.k_new.dtype)
+            v = (self.v_new.float() * f).to(self.v_new.dtype)
+            d.num_quantized, d.num_residual = self.saved
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                flush()
+                a.record(stream)
+                self.cache.append(k, v, rescale=True, stream=stream)
+                b.record(stream)
+            torch.cuda.synchronize()
+            ms.append(a.elapsed_time(b))
+        W = self.seed_w
+        cached = W.B * W.Hkv * self.saved[0]
+        nbytes = 0.0
+        for sch in (W.k_scheme, W.v_scheme):
+            if sch in CALIBRATED:
+                nbytes += 2.0 * cached * row_bytes(sch)  # every cached code read and written
+        nbytes += 2 * (W.B * W.Hkv * 128 * (2 if W.bf16 else 4)) * 2  # the token, read twice
+        nbytes += W.B * W.Hkv * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme))
+        return sum(ms) / len(ms) / 1e3, nbytes, cached
+
     def _build_paged(self, W):
         kvq, torch = self.kvq, self.torch
         lens = W.prefill_lengths()
@@ -758,6 +788,15 @@ def main():
         out["e2e"] = None
     if rank == 0:
         out["quant_error"] = quant_error(r["G"], W, torch.cuda.current_stream())
+        G = r["G"]
+        if not W.paged and not W.kivi and G.calib and G.append_token:
+            t_rs, b_rs, cached = G.time_rescale(L2Flush(G.dev), torch.cuda.current_stream())
+            gbs = b_rs / t_rs / 1e9
+            out["rescale"] = {"what": "rescaling append of one token per sequence that grows the batch-wide "
+                                      "scales: every cached code requantized, mean of 3, L2 flushed before each "
+                                      "(after the timed steps)",
+                              "ms": t_rs * 1e3, "algorithmic_bytes": b_rs, "cached_rows": cached, "GBps": gbs,
+                              "frac": gbs / peak}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         b, t, n, desc = oracle_time(W, args.cpu_seconds)
         out["cpu_baseline"] = {"value": b / t / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",

@@ -156,8 +156,11 @@ kvq_status kvq_cache_bytes(const kvq_cache_desc* d, kvq_footprint* out) {
 }
 
 size_t kvq_append_workspace_bytes(const kvq_cache_desc* d, uint32_t flags) {
-  if (!d || !(flags & KVQ_APPEND_CALIBRATE)) return 0;
-  return round_up((2 + 4 * (size_t)d->num_kv_heads * kHeadDim) * sizeof(uint32_t));
+  if (!d || d->num_kv_heads <= 0) return 0;
+  const size_t hd = (size_t)d->num_kv_heads * kHeadDim;
+  if (flags & KVQ_APPEND_RESCALE) return round_up(rescale_ws_offset(d->num_kv_heads) + 2 * hd * 5 + 16);
+  if (flags & KVQ_APPEND_CALIBRATE) return round_up((2 + 4 * hd) * sizeof(uint32_t));
+  return 0;
 }
 
 kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void* v_new, int32_t in_dtype,
@@ -166,7 +169,8 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   kvq_status st = kvq_validate(d);
   if (st != KVQ_OK) return st;
   if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
-  if (n_new < 0 || (flags & ~KVQ_APPEND_CALIBRATE)) return KVQ_ERR_INVALID_ARG;
+  if (n_new < 0 || (flags & ~(KVQ_APPEND_CALIBRATE | KVQ_APPEND_RESCALE))) return KVQ_ERR_INVALID_ARG;
+  if ((flags & KVQ_APPEND_CALIBRATE) && (flags & KVQ_APPEND_RESCALE)) return KVQ_ERR_INVALID_ARG;
   if (n_new == 0) return KVQ_OK;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
   const bool paged = d->layout == KVQ_PAGED;
@@ -176,8 +180,11 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   if (!append_pair_supported(d->k_scheme, d->v_scheme)) return KVQ_ERR_UNSUPPORTED;
   if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)n_new >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
   if (paged && n_new > seq_capacity(d)) return KVQ_ERR_CAPACITY;
-  const bool calibrate = (flags & KVQ_APPEND_CALIBRATE) != 0 && !kivi;
-  if (calibrate) {
+  const int mode = kivi                             ? kAppendPlain
+                   : (flags & KVQ_APPEND_CALIBRATE) ? kAppendCalibrate
+                   : (flags & KVQ_APPEND_RESCALE)   ? kAppendRescale
+                                                    : kAppendPlain;
+  if (mode != kAppendPlain) {
     if (!workspace || workspace_bytes < kvq_append_workspace_bytes(d, flags) || !aligned16(workspace))
       return KVQ_ERR_WORKSPACE;
   }
@@ -224,8 +231,7 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   p.page_table = d->page_table;
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
-  const cudaError_t e = launch_append(p, static_cast<uint32_t*>(workspace), calibrate, r_old, flushed, r_new,
-                                      static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_append(p, workspace, mode, r_old, flushed, r_new, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return from_cuda(e);
   if (!paged) {
     if (kivi) {

@@ -15,6 +15,8 @@
 //    (infra.bea.ai §3; llms.blog §3).
 #include <cuda_fp8.h>
 
+#include <algorithm>
+
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
 
@@ -171,6 +173,25 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(AppendParams p, uint3
   }
 }
 
+// Asymmetric parameters of the range [lo, hi] (lo <= 0 <= hi): s = (hi - lo) / 255,
+// zp = clamp(rne(-lo / s), 0, 255); a zero range gives s = 0 and zp = 0.
+__device__ __forceinline__ void asym_params(float lo, float hi, float& s, uint8_t& zp) {
+  s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
+  int z = 0;
+  if (s != 0.0f) {
+    float zf = rintf(__fdiv_rn(-lo, s));
+    zf = fminf(fmaxf(zf, 0.0f), 255.0f);
+    z = (int)zf;
+  }
+  zp = (uint8_t)z;
+}
+
+__device__ __forceinline__ float calib_scale(int scheme, float amax) {
+  return __fdiv_rn(amax, scheme == KVQ_FP8_E4M3_PER_TENSOR   ? 448.0f
+                         : scheme == KVQ_FP8_E5M2_PER_TENSOR ? 57344.0f
+                                                             : 127.0f);
+}
+
 // Turn the reduced statistics into scales (and zero points): one block.
 __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
   const int hd = p.H * kHeadDim;
@@ -180,29 +201,14 @@ __global__ void calib_finalize_kernel(AppendParams p, const uint32_t* keys) {
     uint8_t* zp = side ? p.v_zp : p.k_zp;
     const uint32_t* base = keys + 2 + side * 2 * hd;
     if (scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_FP8_E5M2_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR) {
-      if (threadIdx.x == 0) {
-        const float amax = __uint_as_float(keys[side]);
-        scale[0] = __fdiv_rn(amax, scheme == KVQ_FP8_E4M3_PER_TENSOR   ? 448.0f
-                                   : scheme == KVQ_FP8_E5M2_PER_TENSOR ? 57344.0f
-                                                                       : 127.0f);
-      }
+      if (threadIdx.x == 0) scale[0] = calib_scale(scheme, __uint_as_float(keys[side]));
     } else if (scheme == KVQ_INT8_SYM_PER_CHANNEL) {
       for (int i = threadIdx.x; i < hd; i += blockDim.x)
         scale[i] = __fdiv_rn(__uint_as_float(base[hd + i]), 127.0f);
     } else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
       for (int i = threadIdx.x; i < hd; i += blockDim.x) {
         const float mn = key_to_float(base[i]), mx = key_to_float(base[hd + i]);
-        const float lo = mn < 0.0f ? mn : 0.0f;
-        const float hi = mx > 0.0f ? mx : 0.0f;
-        const float s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
-        int z = 0;
-        if (s != 0.0f) {
-          float zf = rintf(__fdiv_rn(-lo, s));
-          zf = fminf(fmaxf(zf, 0.0f), 255.0f);
-          z = (int)zf;
-        }
-        scale[i] = s;
-        zp[i] = (uint8_t)z;
+        asym_params(mn < 0.0f ? mn : 0.0f, mx > 0.0f ? mx : 0.0f, scale[i], zp[i]);
       }
     }
   }
@@ -493,6 +499,171 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
   }
   if (sat && p.status) atomicAdd(p.status + 1, (uint32_t)sat);
 }
+
+// ------------------------------------------------------------------ rescaling append
+// Merge each block's scales into the cached ones (n4n.ai Step 3 keeps a running maximum;
+// Step 7 wants scales that only grow, or are recomputed as the cache grows) and requantize
+// the cached codes whose scale element changed. Symmetric schemes: s' = max(s, s_block).
+// uint8 asymmetric: the parameters of the union of the range the cached (s, zp) represent,
+// [(0 - zp) s, (255 - zp) s], and the block's range (with 0), unchanged when it lies inside.
+// Workspace after the calibration keys: old scales [2][H*D] fp32, old zero points
+// [2][H*D] uint8, and one changed flag per side.
+struct RescaleWs {
+  float* s_old;
+  uint8_t* zp_old;
+  uint32_t* changed;
+};
+
+__global__ void rescale_finalize_kernel(AppendParams p, const uint32_t* keys, RescaleWs ws) {
+  const int hd = p.H * kHeadDim;
+  __shared__ uint32_t grew[2];
+  if (threadIdx.x < 2) grew[threadIdx.x] = 0u;
+  __syncthreads();
+  for (int side = 0; side < 2; ++side) {
+    const int scheme = side ? p.v_scheme : p.k_scheme;
+    float* scale = side ? p.v_scale : p.k_scale;
+    uint8_t* zp = side ? p.v_zp : p.k_zp;
+    const uint32_t* base = keys + 2 + side * 2 * hd;
+    float* s_old = ws.s_old + side * hd;
+    uint8_t* z_old = ws.zp_old + side * hd;
+    if (scheme == KVQ_FP8_E4M3_PER_TENSOR || scheme == KVQ_FP8_E5M2_PER_TENSOR || scheme == KVQ_INT8_SYM_PER_TENSOR) {
+      if (threadIdx.x == 0) {
+        const float so = scale[0], sb = calib_scale(scheme, __uint_as_float(keys[side]));
+        s_old[0] = so;
+        z_old[0] = 0;
+        if (sb > so) {
+          scale[0] = sb;
+          grew[side] = 1u;
+        }
+      }
+    } else if (scheme == KVQ_INT8_SYM_PER_CHANNEL) {
+      for (int i = threadIdx.x; i < hd; i += blockDim.x) {
+        const float so = scale[i], sb = __fdiv_rn(__uint_as_float(base[hd + i]), 127.0f);
+        s_old[i] = so;
+        z_old[i] = 0;
+        if (sb > so) {
+          scale[i] = sb;
+          grew[side] = 1u;
+        }
+      }
+    } else if (scheme == KVQ_UINT8_ASYM_PER_CHANNEL) {
+      for (int i = threadIdx.x; i < hd; i += blockDim.x) {
+        const float so = scale[i];
+        const uint8_t zo = zp[i];
+        s_old[i] = so;
+        z_old[i] = zo;
+        const float mn = key_to_float(base[i]), mx = key_to_float(base[hd + i]);
+        const float lo_b = mn < 0.0f ? mn : 0.0f, hi_b = mx > 0.0f ? mx : 0.0f;
+        const float lo_o = __fmul_rn((float)(0 - (int)zo), so), hi_o = __fmul_rn((float)(255 - (int)zo), so);
+        if (lo_b < lo_o || hi_b > hi_o) {
+          asym_params(lo_b < lo_o ? lo_b : lo_o, hi_b > hi_o ? hi_b : hi_o, scale[i], zp[i]);
+          grew[side] = 1u;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 2) ws.changed[threadIdx.x] = grew[threadIdx.x];
+}
+
+// Value of an 8-bit code of a batch-wide scheme under (s, zp).
+template <int SCHEME>
+__device__ __forceinline__ float fixed_value(uint32_t q, float s, int zp) {
+  if constexpr (SCHEME == KVQ_FP8_E4M3_PER_TENSOR) {
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)q, __NV_E4M3);
+    return __fmul_rn(__half2float(__half(hr)), s);
+  } else if constexpr (SCHEME == KVQ_FP8_E5M2_PER_TENSOR) {
+    __half_raw hr;
+    hr.x = (unsigned short)(q << 8);
+    return __fmul_rn(__half2float(__half(hr)), s);
+  } else if constexpr (SCHEME == KVQ_UINT8_ASYM_PER_CHANNEL) {
+    return __fmul_rn((float)((int)q - zp), s);
+  } else {
+    return __fmul_rn((float)(int8_t)q, s);
+  }
+}
+
+// Requantize the cached rows of one side (blockIdx.y = kv head) when its scales changed:
+// 8 threads per 128-code row, 16 codes each; the thread's 16 channels keep their old and
+// new parameters in registers across the rows it visits.
+template <int SCHEME>
+__global__ void __launch_bounds__(256) requant_kernel(AppendParams p, RescaleWs ws, int side) {
+  if (ws.changed[side] == 0u) return;
+  constexpr bool kPerChannel = SCHEME == KVQ_INT8_SYM_PER_CHANNEL || SCHEME == KVQ_UINT8_ASYM_PER_CHANNEL;
+  const int h = blockIdx.y, lane8 = threadIdx.x & 7;
+  const int hd = p.H * kHeadDim;
+  const float* scale = side ? p.v_scale : p.k_scale;
+  const uint8_t* zp = side ? p.v_zp : p.k_zp;
+  uint8_t* codes = static_cast<uint8_t*>(side ? p.v_codes : p.k_codes);
+  float so[16], sn[16], yn[16];
+  int zo[16], zn[16];
+  uint32_t keep = 0u, fast = 0u;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int i = kPerChannel ? h * kHeadDim + lane8 * 16 + k : 0;
+    so[k] = ws.s_old[side * hd + i];
+    sn[k] = scale[i];
+    yn[k] = __frcp_rn(sn[k]);
+    zo[k] = SCHEME == KVQ_UINT8_ASYM_PER_CHANNEL ? (int)ws.zp_old[side * hd + i] : 0;
+    zn[k] = SCHEME == KVQ_UINT8_ASYM_PER_CHANNEL ? (int)zp[i] : 0;
+    if (sn[k] == so[k] && zn[k] == zo[k]) keep |= 1u << k;
+    if (quot_range(sn[k]) && quot_range(so[k])) fast |= 1u << k;
+  }
+  const int span = p.paged ? p.max_pages * p.page_size : p.pos0;
+  const long long rows = (long long)p.B * span;
+  for (long long r = (long long)blockIdx.x * 32 + (threadIdx.x >> 3); r < rows; r += (long long)gridDim.x * 32) {
+    const int b = (int)(r / span), pos = (int)(r % span);
+    if (p.paged && pos >= p.seq_lens[b]) continue;
+    size_t row;
+    if (!cache_row(p, b, h, pos, row)) continue;
+    uint4* ptr = reinterpret_cast<uint4*>(codes + row * kHeadDim + lane8 * 16);
+    const uint4 in = *ptr;
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t o[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t q = (w[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+      uint32_t c = q;
+      if (!((keep >> k) & 1u)) {
+        c = 0u;
+        if (sn[k] != 0.0f) {
+          const float x = fixed_value<SCHEME>(q, so[k], zo[k]);
+          float qq;
+          const float z = ((fast >> k) & 1u) ? quot(x, sn[k], yn[k], qq) : __fdiv_rn(x, sn[k]);
+          int sat = 0;
+          c = code_of(z, zn[k], SCHEME, sat);
+        }
+      }
+      o[k >> 2] |= c << (8 * (k & 3));
+    }
+    *ptr = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+int sm_count();
+
+template <int SCHEME>
+void launch_requant(const AppendParams& p, const RescaleWs& ws, int side, cudaStream_t st) {
+  const long long span = p.paged ? (long long)p.max_pages * p.page_size : p.pos0;
+  const long long chunks = ((long long)p.B * span + 31) / 32;
+  if (chunks == 0) return;
+  const long long cap = std::max(1LL, 16LL * sm_count() / p.H);
+  dim3 grid((unsigned)std::min(chunks, cap), p.H);
+  requant_kernel<SCHEME><<<grid, 256, 0, st>>>(p, ws, side);
+  count_launches(1);
+}
+
+void launch_requant_side(const AppendParams& p, const RescaleWs& ws, int side, cudaStream_t st) {
+  switch (side ? p.v_scheme : p.k_scheme) {
+    case KVQ_FP8_E4M3_PER_TENSOR: launch_requant<KVQ_FP8_E4M3_PER_TENSOR>(p, ws, side, st); break;
+    case KVQ_FP8_E5M2_PER_TENSOR: launch_requant<KVQ_FP8_E5M2_PER_TENSOR>(p, ws, side, st); break;
+    case KVQ_INT8_SYM_PER_TENSOR: launch_requant<KVQ_INT8_SYM_PER_TENSOR>(p, ws, side, st); break;
+    case KVQ_INT8_SYM_PER_CHANNEL: launch_requant<KVQ_INT8_SYM_PER_CHANNEL>(p, ws, side, st); break;
+    case KVQ_UINT8_ASYM_PER_CHANNEL: launch_requant<KVQ_UINT8_ASYM_PER_CHANNEL>(p, ws, side, st); break;
+    default: break;  // per-token scales: nothing to merge
+  }
+}
+
 
 __global__ void seq_lens_advance_kernel(AppendParams p) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
@@ -898,8 +1069,11 @@ cudaError_t launch_quantize_rows(const AppendParams& p, long long rows, cudaStre
   return cudaErrorNotSupported;
 }
 
-cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
-                          int flushed, int r_new, cudaStream_t st) {
+size_t rescale_ws_offset(int H) { return ((2 + 4 * (size_t)H * kHeadDim) * sizeof(uint32_t) + 255) & ~(size_t)255; }
+
+cudaError_t launch_append(const AppendParams& p, void* workspace, int mode, int r_old, int flushed, int r_new,
+                          cudaStream_t st) {
+  uint32_t* calib_keys = static_cast<uint32_t*>(workspace);
   const bool kivi = is_kivi(p.k_scheme);
   if (kivi) {
     if (flushed > 0) {
@@ -929,7 +1103,7 @@ cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool cali
     }
     return cudaGetLastError();
   }
-  if (calibrate) {
+  if (mode != kAppendPlain) {
     const int hd = p.H * kHeadDim;
     calib_init_kernel<<<(2 + 4 * hd + 255) / 256, 256, 0, st>>>(calib_keys, hd);
     dim3 grid((p.n_new + 255) / 256, p.B * p.H, 2);
@@ -937,8 +1111,21 @@ cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool cali
       calib_reduce_kernel<true><<<grid, 256, 0, st>>>(p, calib_keys);
     else
       calib_reduce_kernel<false><<<grid, 256, 0, st>>>(p, calib_keys);
-    calib_finalize_kernel<<<1, 256, 0, st>>>(p, calib_keys);
-    count_launches(3);
+    count_launches(2);
+    if (mode == kAppendCalibrate) {
+      calib_finalize_kernel<<<1, 256, 0, st>>>(p, calib_keys);
+      count_launches(1);
+    } else {
+      uint8_t* w = static_cast<uint8_t*>(workspace) + rescale_ws_offset(p.H);
+      RescaleWs ws;
+      ws.s_old = reinterpret_cast<float*>(w);
+      ws.zp_old = w + 2 * (size_t)hd * sizeof(float);
+      ws.changed = reinterpret_cast<uint32_t*>(w + 2 * (size_t)hd * (sizeof(float) + 1));
+      rescale_finalize_kernel<<<1, 256, 0, st>>>(p, calib_keys, ws);
+      count_launches(1);
+      launch_requant_side(p, ws, 0, st);
+      launch_requant_side(p, ws, 1, st);
+    }
   }
   const long long rows = (long long)p.B * p.H * p.n_new;
   const cudaError_t e = launch_quantize_rows(p, rows, st);

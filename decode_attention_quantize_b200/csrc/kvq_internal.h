@@ -87,8 +87,14 @@ constexpr int kMaxCtas = 1024;
 // Count of kernel launches issued by the library (reported by kvq_launch_count).
 void count_launches(int n);  // decode grid bound used to size the workspace
 
-cudaError_t launch_append(const AppendParams& p, uint32_t* calib_keys, bool calibrate, int r_old,
-                          int flushed, int r_new, cudaStream_t st);
+// Append modes: plain (the scales in the cache), calibrating (scales from the block), or
+// rescaling (the block's scales merged into the cached ones, cached codes requantized).
+enum { kAppendPlain = 0, kAppendCalibrate = 1, kAppendRescale = 2 };
+// Workspace: calibration keys, then (rescaling) the offset below: old scales [2][H*128]
+// fp32, old zero points [2][H*128] uint8, two changed flags.
+size_t rescale_ws_offset(int H);
+cudaError_t launch_append(const AppendParams& p, void* workspace, int mode, int r_old, int flushed, int r_new,
+                          cudaStream_t st);
 cudaError_t launch_dequantize(const DequantParams& p, cudaStream_t st);
 // Launch with programmatic dependent launch: the kernel may be scheduled while the previous
 // kernel in the stream is still running and must call griddepcontrol.wait before it touches

@@ -30,6 +30,7 @@ FP8_E5M2_PER_TENSOR = 7
 KVQ_F32, KVQ_BF16 = 0, 1
 KVQ_DENSE, KVQ_PAGED = 0, 1
 KVQ_APPEND_CALIBRATE = 0x1
+KVQ_APPEND_RESCALE = 0x2
 KVQ_DEV_BAD_PAGE, KVQ_DEV_BAD_LENGTH, KVQ_DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 EXPORTS = [
@@ -138,9 +139,11 @@ def row_bytes(scheme: int, D: int = 128) -> int:
 
 # ---------------------------------------------------------------- entry points
 def kvq_quantize_append(desc: KvqDesc, k_new, v_new, new_lens=None, calibrate=False, workspace=None,
-                        stream=None):
-    """Quantize [B, Hkv, n, D] K/V (bf16 or fp32) and append them to the cache."""
-    flags = KVQ_APPEND_CALIBRATE if calibrate else 0
+                        stream=None, rescale=False):
+    """Quantize [B, Hkv, n, D] K/V (bf16 or fp32) and append them to the cache.
+    calibrate: scales from this block; rescale: grow the scales to cover this block and
+    requantize the cached codes whose scale changed."""
+    flags = (KVQ_APPEND_CALIBRATE if calibrate else 0) | (KVQ_APPEND_RESCALE if rescale else 0)
     need = lib.kvq_append_workspace_bytes(ctypes.byref(desc), flags)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=k_new.device)
@@ -229,12 +232,36 @@ class CacheSpec:
     D: int = 128
 
 
-class QuantizedKVCache:
-    """One layer's quantized cache in caller-owned (torch) device memory plus its descriptor."""
+class RescaleSchedule:
+    """When to rescale: n4n.ai Step 7 recomputes the scales of a growing cache every 1024
+    new tokens. ``step(n)`` counts appended tokens and answers whether this append is the
+    one that rescales (the count restarts there, and at a calibration)."""
 
-    def __init__(self, spec: CacheSpec, device="cuda", page_table=None):
+    def __init__(self, every: int = 1024):
+        if every <= 0:
+            raise ValueError("every must be positive")
+        self.every = every
+        self.pending = 0
+
+    def step(self, n_new: int) -> bool:
+        self.pending += int(n_new)
+        if self.pending >= self.every:
+            self.pending = 0
+            return True
+        return False
+
+    def reset(self):
+        self.pending = 0
+
+
+class QuantizedKVCache:
+    """One layer's quantized cache in caller-owned (torch) device memory plus its descriptor.
+    ``rescale_every`` > 0 makes every append that completes that many tokens a rescaling one."""
+
+    def __init__(self, spec: CacheSpec, device="cuda", page_table=None, rescale_every: int = 0):
         s = spec
         self.spec = s
+        self.schedule = RescaleSchedule(rescale_every) if rescale_every > 0 else None
         dev = torch.device(device)
         self.t = {}
         kivi = s.k_scheme in (KIVI_INT4, KIVI_INT2)
@@ -285,9 +312,16 @@ class QuantizedKVCache:
     def num_residual(self):
         return self.desc.num_residual
 
-    def append(self, k, v, new_lens=None, calibrate=False, workspace=None, stream=None):
+    def append(self, k, v, new_lens=None, calibrate=False, workspace=None, stream=None, rescale=None):
+        """rescale: True / False, or None to follow ``rescale_every`` (never when calibrating)."""
+        if calibrate:
+            if self.schedule is not None:
+                self.schedule.reset()
+            rescale = False
+        elif rescale is None:
+            rescale = self.schedule.step(k.shape[2]) if self.schedule is not None else False
         kvq_quantize_append(self.desc, k, v, new_lens=new_lens, calibrate=calibrate, workspace=workspace,
-                            stream=stream)
+                            stream=stream, rescale=rescale)
 
     def dequantize(self, which: int, out_tokens: int, stream=None):
         return kvq_dequantize(self.desc, which, out_tokens, stream=stream, device=self.device)

@@ -80,6 +80,7 @@ typedef enum kvq_layout { KVQ_DENSE = 0, KVQ_PAGED = 1 } kvq_layout;
 
 /* kvq_quantize_append flags */
 #define KVQ_APPEND_CALIBRATE 0x1u  /* recompute per-tensor / per-channel scales from this block */
+#define KVQ_APPEND_RESCALE 0x2u    /* merge this block's scales into the cached ones, requantize */
 
 /* device status word bits (dev_status[0]); dev_status[1] counts saturated codes */
 #define KVQ_DEV_BAD_PAGE 0x1u
@@ -144,7 +145,8 @@ KVQ_API kvq_status kvq_validate(const kvq_cache_desc* desc);
 /* Bytes the cache arrays take (n4n.ai Step 6 "peak memory"; llms.blog memory-per-token). */
 KVQ_API kvq_status kvq_cache_bytes(const kvq_cache_desc* desc, kvq_footprint* out);
 
-/* Workspace kvq_quantize_append needs for `flags` (0 unless KVQ_APPEND_CALIBRATE). */
+/* Workspace kvq_quantize_append needs for `flags` (0 unless KVQ_APPEND_CALIBRATE or
+ * KVQ_APPEND_RESCALE). */
 KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t flags);
 
 /*
@@ -154,7 +156,15 @@ KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t f
  *   new_lens      paged only, device int32 [batch] or NULL: per-sequence counts <= n_new
  *   flags         KVQ_APPEND_CALIBRATE: per-tensor / per-channel scales from this block
  *                 (otherwise the scales already in the descriptor are used; values beyond
- *                 them saturate and are counted in dev_status[1])
+ *                 them saturate and are counted in dev_status[1]).
+ *                 KVQ_APPEND_RESCALE (not with CALIBRATE): the scales grow to cover this
+ *                 block and the cached codes whose scale changed are requantized first
+ *                 (n4n.ai Step 3 keeps a running maximum of the scales; Step 7 recomputes
+ *                 them as the cache grows, e.g. every 1024 tokens). Symmetric schemes take
+ *                 max(cached, block) per scale element; uint8 asymmetric takes the union
+ *                 of the cached representable range [(0 - zp) s, (255 - zp) s] and the
+ *                 block's range. A cached code is requantized from its dequantized value.
+ *                 Both flags are ignored for per-token and KIVI schemes.
  * Dense: tokens go to positions num_quantized.. of every row; the library updates
  * num_quantized / num_residual in *desc when the call is accepted. KIVI: tokens enter the
  * residual; when a token arrives at a full residual, its 128 tokens are quantized.

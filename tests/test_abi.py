@@ -124,3 +124,38 @@ def test_footprint_matches_the_pages_per_token_bytes():
     assert L.kvq_cache_bytes(ctypes.byref(d5), ctypes.byref(f)) == kvq.KVQ_OK
     assert f.code_bytes * 80 / 4096 == 81920  # INT4 codes: 80 KiB per token for 80 layers
     assert f.bytes_per_token == 2 * 64 + 2 * 8 * 4  # codes + fp32 (scale, min) per 32 elements
+
+
+def test_rescale_flag_is_checked_on_the_host():
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    d = _desc()
+    cal = L.kvq_append_workspace_bytes(ctypes.byref(d), kvq.KVQ_APPEND_CALIBRATE)
+    res = L.kvq_append_workspace_bytes(ctypes.byref(d), kvq.KVQ_APPEND_RESCALE)
+    assert L.kvq_append_workspace_bytes(ctypes.byref(d), 0) == 0
+    # the rescaling workspace holds the calibration keys plus the old scales, zero points and flags
+    assert res >= cal + 2 * 2 * 128 * 5 + 16 and res % 256 == 0
+    buf = 0x20000
+    both = kvq.KVQ_APPEND_CALIBRATE | kvq.KVQ_APPEND_RESCALE
+    assert L.kvq_quantize_append(ctypes.byref(d), buf, buf, kvq.KVQ_BF16, 4, None, both, buf, res,
+                                 None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_append(ctypes.byref(d), buf, buf, kvq.KVQ_BF16, 4, None, 0x4, buf, res,
+                                 None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_append(ctypes.byref(d), buf, buf, kvq.KVQ_BF16, 4, None, kvq.KVQ_APPEND_RESCALE,
+                                 buf, cal, None) == kvq.KVQ_ERR_WORKSPACE
+    assert d.num_quantized == 0  # nothing was accepted
+
+
+def test_rescale_schedule_counts_tokens():
+    # every 1024 appended tokens one append rescales (n4n.ai Step 7); a calibration restarts the count
+    from decode_attention_quantize_b200.kvq import RescaleSchedule
+    s = RescaleSchedule(1024)
+    fired = [s.step(1) for _ in range(3000)]
+    assert [i for i, f in enumerate(fired) if f] == [1023, 2047]
+    s = RescaleSchedule(1024)
+    assert not s.step(1000) and s.step(100) and s.pending == 0
+    s.step(500)
+    s.reset()
+    assert s.pending == 0 and not s.step(1023) and s.step(1)
+    with pytest.raises(ValueError):
+        RescaleSchedule(0)

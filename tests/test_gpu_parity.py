@@ -213,6 +213,88 @@ def test_saturated_codes_match_oracle(scheme):
     H.decode_both(oc, gc, synth.queries(w, 0, 0, B), False, "decode over saturated codes")
 
 
+# ------------------------------------------------------------------ rescaling append
+# Scales merged with each block's (they only grow) and the cached codes whose scale changed
+# requantized, bit for bit against the oracle; blocks inside the range, a grown single
+# token, a grown bulk block; dense and paged.
+RESCALE_PAIRS = [
+    (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR),
+    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL), (S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL),
+    (S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TOKEN),
+]
+RESCALE_SPANS = [(300, 340, 0.5), (340, 341, 3.0), (341, 345, 1.0), (345, 420, -1.75)]
+
+
+def _f32(a, bf16):
+    return synth.bf16_bits_to_f32(a) if bf16 else a
+
+
+@pytest.mark.parametrize("ks,vs", RESCALE_PAIRS)
+def test_rescale_dense(ks, vs):
+    B, Hq, Hkv = 2, 8, 2
+    w = H.workload(B, Hq, Hkv, ks, vs, bf16=False)
+    K = synth.keys(w, 0, B, 0, Hkv, 0, 420)
+    V = synth.values(w, 0, B, 0, Hkv, 0, 420)
+    oc = H.OracleCache(B, Hq, Hkv, 128, ks, vs, cap=512)
+    gc = H.kvq().QuantizedKVCache(H.kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=512))
+    # the first block rescales a fresh cache (zero scales): the same as a calibration
+    oc.append(K[:, :, :300], V[:, :, :300], False, rescale=True)
+    gc.append(H.dev(K[:, :, :300], False), H.dev(V[:, :, :300], False), rescale=True)
+    torch.cuda.synchronize()
+    H.compare_dense(oc, gc, "rescaling prefill")
+    for a, b, f in RESCALE_SPANS:
+        kk = np.ascontiguousarray(K[:, :, a:b] * np.float32(f))
+        vv = np.ascontiguousarray(V[:, :, a:b] * np.float32(-f))
+        oc.append(kk, vv, False, rescale=True)
+        gc.append(H.dev(kk, False), H.dev(vv, False), rescale=True)
+        torch.cuda.synchronize()
+        H.compare_dense(oc, gc, f"rescale at {a}")
+        H.decode_both(oc, gc, synth.queries(w, a, 0, B), False, f"decode after rescale at {a}")
+    assert gc.status()[0] == 0
+
+
+def test_rescale_paged():
+    B, Hq, Hkv, ks, vs = 4, 16, 4, S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, ks, vs, lens=[37, 100, 5, 64], page_size=16,
+                                                    steps=8)
+    oc.append(K, V, True, calibrate=True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
+    for s, f in enumerate((0.25, 4.0, 1.0, -3.0)):
+        kk = np.stack([_f32(synth.keys(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0], True)
+                       for b in range(B)]) * np.float32(f)
+        vv = np.stack([_f32(synth.values(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0], True)
+                       for b in range(B)]) * np.float32(-f)
+        kk, vv = np.ascontiguousarray(kk, np.float32), np.ascontiguousarray(vv, np.float32)
+        oc.append(kk, vv, False, rescale=True)
+        gc.append(H.dev(kk, False), H.dev(vv, False), rescale=True)
+        torch.cuda.synchronize()
+        H.compare_paged(oc, gc, f"paged rescale {s}")
+        H.decode_both(oc, gc, synth.queries(w, s, 0, B), True, f"paged decode after rescale {s}")
+    assert gc.status()[0] == 0
+
+
+def test_rescale_schedule_every_1024_tokens():
+    # a cache built token by token with rescale_every=64 (the policy's period, shortened)
+    B, Hq, Hkv, ks, vs = 1, 8, 2, S.INT8_SYM_PER_TENSOR, S.INT8_SYM_PER_TENSOR
+    w = H.workload(B, Hq, Hkv, ks, vs, bf16=False)
+    K = synth.keys(w, 0, B, 0, Hkv, 0, 200)
+    V = synth.values(w, 0, B, 0, Hkv, 0, 200)
+    oc = H.OracleCache(B, Hq, Hkv, 128, ks, vs, cap=256)
+    gc = H.kvq().QuantizedKVCache(H.kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=256), rescale_every=64)
+    oc.append(K[:, :, :8], V[:, :, :8], False, calibrate=True)
+    gc.append(H.dev(K[:, :, :8], False), H.dev(V[:, :, :8], False), calibrate=True)
+    growth = np.float32(1.0)
+    for t in range(8, 200):
+        growth *= np.float32(1.01)
+        kk = np.ascontiguousarray(K[:, :, t:t + 1] * growth)
+        vv = np.ascontiguousarray(V[:, :, t:t + 1] * growth)
+        oc.append(kk, vv, False, rescale=(t - 8 + 1) % 64 == 0)
+        gc.append(H.dev(kk, False), H.dev(vv, False))
+    torch.cuda.synchronize()
+    H.compare_dense(oc, gc, "scheduled rescales")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), False, "decode after scheduled rescales")
+
+
 # ------------------------------------------------------------------ dequantize
 @pytest.mark.parametrize("ks,vs", [(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.KIVI_INT2, S.KIVI_INT2),
                                    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
