@@ -35,6 +35,7 @@ UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
+INT4_SYM_PER_GROUP = 8
 APPEND_CALIBRATE, APPEND_RESCALE = 1, 2  # append modes (oq_append)
 
 _lib = None
@@ -87,6 +88,8 @@ def load(path: str):
     L.oq_e5m2_decode.restype = f32
     L.oq_sym_code.argtypes = [f32, f32, i32]
     L.oq_sym_code.restype = i32
+    L.oq_int4_code.argtypes = [f32, f32]
+    L.oq_int4_code.restype = i32
     L.oq_asym_params.argtypes = [f32, f32, vp, vp]
     L.oq_asym_code.argtypes = [f32, f32, ctypes.c_uint8]
     L.oq_asym_code.restype = i32
@@ -133,6 +136,10 @@ def sym_code(x: float, s: float, qmax: int = 127) -> int:
     return int(lib().oq_sym_code(float(x), float(s), qmax))
 
 
+def int4_code(x: float, s: float) -> int:
+    return int(lib().oq_int4_code(float(x), float(s)))
+
+
 def asym_params(mn: float, mx: float):
     s = np.zeros(1, np.float32)
     zp = np.zeros(1, np.uint8)
@@ -174,7 +181,7 @@ def kv_bytes_per_token(n_layers: int, n_kv_heads: int, d_head: int, bytes_per_el
 
 
 def _bits(scheme):
-    return {KIVI_INT4: 4, KIVI_INT2: 2}.get(scheme, 8)
+    return {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4}.get(scheme, 8)
 
 
 # ---------------------------------------------------------------- cache
@@ -204,6 +211,9 @@ class OracleCache:
                 scale = np.zeros((Hkv, D), np.float32)
                 if scheme == UINT8_ASYM_PER_CHANNEL:
                     zp = np.zeros((Hkv, D), np.uint8)
+            elif scheme == INT4_SYM_PER_GROUP:
+                rows = (num_pages, Hkv, page_size) if paged else (B, Hkv, cap)
+                scale = np.zeros((*rows, D // group), np.float32)
             else:
                 shape = (B, Hkv, cap // group, D) if side == "k" else (B, Hkv, cap, D // group)
                 scale = np.zeros(shape, np.float32)

@@ -16,6 +16,8 @@
  *  - per-tensor and per-channel scales are fixed by the calibrating append.
  *  - KIVI residual: 128 tokens, groups of 32, flush when a token arrives at a full
  *    residual.
+ *  - INT4 symmetric per group: groups of 32 consecutive channels of a token, s = absmax / 7,
+ *    q = clamp(rne(x / s), -8, 7), two's-complement nibbles, lower channel in the low bits.
  */
 #include "kvq_oracle.h"
 
@@ -128,6 +130,17 @@ int oq_sym_code(float x, float s, int qmax) {
   return (int)r;
 }
 
+/* INT4 group code (P3 §2 "INT4 Group-Wise"; the page code of P4 Step 3 divides by
+ * max|x| / 7 and clamps to the signed 4-bit range): clamp(rne(x / s), -8, 7); a zero
+ * range gives 0. */
+int oq_int4_code(float x, float s) {
+  if (s == 0.0f) return 0;
+  float r = rintf(x / s);
+  if (r > 7.0f) r = 7.0f;
+  if (r < -8.0f) r = -8.0f;
+  return (int)r;
+}
+
 /* Asymmetric uint8 parameters over [min(mn,0), max(mx,0)]: s = range / 255,
  * zp = clamp(rne(-lo / s), 0, 255)  (P4 Step 2 "per-channel asymmetric INT8",
  * Step 3 v_scale / v_zp). */
@@ -198,7 +211,7 @@ float oq_kivi_value(int code, float s, float mn) {
 static int is_kivi(int scheme) { return scheme == OQ_KIVI_INT4 || scheme == OQ_KIVI_INT2; }
 
 static int code_bits(int scheme) {
-  if (scheme == OQ_KIVI_INT4) return 4;
+  if (scheme == OQ_KIVI_INT4 || scheme == OQ_INT4_SYM_PER_GROUP) return 4;
   if (scheme == OQ_KIVI_INT2) return 2;
   return 8;
 }
@@ -325,10 +338,27 @@ static int code_for(int scheme, float x, float s, uint8_t zp) {
   return 0;
 }
 
-/* Quantize token t of the block (b, h) into cache row `row` (8-bit schemes). */
+/* Quantize token t of the block (b, h) into cache row `row` (8-bit schemes and INT4
+ * per group). */
 static void quantize_token(const oq_cache* c, const block* k, int scheme, uint8_t* codes,
                            float* scale, const uint8_t* zp, int b, int h, int t, size_t row) {
   const int D = c->D;
+  if (scheme == OQ_INT4_SYM_PER_GROUP) {
+    /* one scale per group of g consecutive channels of this token (P3 §2, P4 Step 2) */
+    const int g = c->group;
+    for (int j = 0; j < D / g; ++j) {
+      float amax = 0.0f;
+      for (int d = j * g; d < (j + 1) * g; ++d) {
+        float a = fabsf(block_at(k, b, h, t, d));
+        if (a > amax) amax = a;
+      }
+      const float s = amax / 7.0f;
+      scale[row * (size_t)(D / g) + (size_t)j] = s;
+      for (int d = j * g; d < (j + 1) * g; ++d)
+        put_code(codes, scheme, D, row, d, oq_int4_code(block_at(k, b, h, t, d), s) & 0xF);
+    }
+    return;
+  }
   float tok_scale = 0.0f;
   if (scheme == OQ_INT8_SYM_PER_TOKEN) {
     /* one scale per token row over head_dim (P3 §2 "INT8 Per-Token") */
@@ -623,6 +653,8 @@ static float value_at(const oq_cache* c, int which, int b, int h, int t, int d) 
       return (float)(int8_t)q * scale[h * D + d];
     case OQ_UINT8_ASYM_PER_CHANNEL:
       return (float)(q - (int)zp[h * D + d]) * scale[h * D + d];
+    case OQ_INT4_SYM_PER_GROUP:
+      return (float)(q >= 8 ? q - 16 : q) * scale[row * (size_t)(D / c->group) + (size_t)(d / c->group)];
   }
   return 0.0f;
 }

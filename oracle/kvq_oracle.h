@@ -42,7 +42,8 @@ enum {
   OQ_UINT8_ASYM_PER_CHANNEL = 4,
   OQ_KIVI_INT4 = 5,
   OQ_KIVI_INT2 = 6,
-  OQ_FP8_E5M2_PER_TENSOR = 7
+  OQ_FP8_E5M2_PER_TENSOR = 7,
+  OQ_INT4_SYM_PER_GROUP = 8
 };
 
 /* ---- element codecs ---- */
@@ -53,6 +54,7 @@ float oq_e4m3_decode(uint8_t code);
 uint8_t oq_e5m2_encode(float x);            /* round-to-nearest-even, saturate finite */
 float oq_e5m2_decode(uint8_t code);
 int oq_sym_code(float x, float s, int qmax); /* clamp(rne(x/s), -qmax, qmax); 0 if s == 0 */
+int oq_int4_code(float x, float s);         /* clamp(rne(x/s), -8, 7); 0 if s == 0 */
 void oq_asym_params(float mn, float mx, float* s, uint8_t* zp);
 int oq_asym_code(float x, float s, uint8_t zp);
 void oq_kivi_group(const float* x, int n, int stride, int bits, int* codes, float* s, float* mn);

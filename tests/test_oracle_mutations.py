@@ -56,6 +56,11 @@ MUTATIONS = [
      "code_for(scheme, x, s_old[i], z_new)"),
     ("rescale old range top", "(float)(255 - (int)zp_old[i]) * s_old[i]", "(float)(255 + (int)zp_old[i]) * s_old[i]"),
     ("rescale drops old low end", "lo_b < lo_o ? lo_b : lo_o", "lo_b"),
+    ("int4 qmax 8", "const float s = amax / 7.0f;", "const float s = amax / 8.0f;"),
+    ("int4 no sign extension", "(float)(q >= 8 ? q - 16 : q)", "(float)q"),
+    ("int4 clamp -7", "if (r < -8.0f) r = -8.0f;", "if (r < -7.0f) r = -7.0f;"),
+    ("int4 group amax from group 0", "for (int d = j * g; d < (j + 1) * g; ++d) {\n        float a = fabsf",
+     "for (int d = 0; d < g; ++d) {\n        float a = fabsf"),
     ("rescale paged length", "const int len = c->paged ? c->seq_lens[b] : c->len;",
      "const int len = c->paged ? c->seq_lens[b] - 1 : c->len;"),
 ]

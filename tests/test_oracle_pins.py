@@ -785,3 +785,97 @@ def test_rescale_paged_matches_dense():
             page, slot = table[b, t // ps], t % ps
             assert np.array_equal(pg["k_codes"][page, :, slot], dn["k_codes"][b, :, t])
             assert np.array_equal(pg["v_codes"][page, :, slot], dn["v_codes"][b, :, t])
+
+
+# --------------------------------------------------------------- INT4 symmetric per group
+# llms.blog §2 "INT4 Group-Wise": groups of 32-128 elements along the channel dimension;
+# n4n.ai Step 2 "Per-group INT4" and its Step 3 code: scale = max|x| / 7, codes clamped to the
+# signed 4-bit range. Groups here are 32 consecutive channels of one token.
+def _int4_cache(B, H, cap=8, **kw):
+    return OracleCache(B, H, H, 32 * 4, oracle.INT4_SYM_PER_GROUP, oracle.INT4_SYM_PER_GROUP, cap=cap, **kw)
+
+
+def test_int4_group_scale_exact_grid_and_packing():
+    s = 2.0**-3
+    x = np.zeros((1, 1, 1, 128), np.float32)
+    ks = np.array([(i % 15) - 7 for i in range(128)])
+    x[0, 0, 0] = ks * s                          # every group holds -7..7, so absmax = 7 s
+    c = _int4_cache(1, 1)
+    c.append(x, x, bf16=False)
+    assert np.all(c["k_scale"][0, 0, 0] == F32(s))   # (7 s) / 7 = s exactly
+    row = c["k_codes"][0, 0, 0]
+    assert row.shape == (64,)
+    for d in range(128):
+        nib = (int(row[d // 2]) >> (4 * (d % 2))) & 0xF  # lower channel in the low nibble
+        val = nib - 16 if nib >= 8 else nib          # two's complement
+        assert val == ks[d], d
+    assert np.array_equal(c.dequantize(0, 8)[0, 0, 0], x[0, 0, 0])
+
+
+def test_int4_code_is_nearest_level_and_clamped():
+    rng = np.random.default_rng(70)
+    for _ in range(300):
+        s = float(F32(rng.uniform(0.01, 3)))
+        v = float(F32(rng.normal(0, 6 * s)))
+        q = oracle.int4_code(v, s)
+        r = Fraction(v) / Fraction(s)
+        d = [abs(r - k) for k in range(-8, 8)]
+        m = min(d)
+        best = [k - 8 for k, e in enumerate(d) if e == m]
+        half = math.floor(r) + Fraction(1, 2)
+        if len(best) > 1:
+            assert q in best and q % 2 == 0
+        elif abs(r - half) <= abs(r) * Fraction(1, 2**24) and -8 < math.floor(r) < 7:
+            assert q in (math.floor(r), math.floor(r) + 1)
+        else:
+            assert q == best[0]
+    assert oracle.int4_code(100.0, 1.0) == 7 and oracle.int4_code(-100.0, 1.0) == -8
+    assert oracle.int4_code(3.0, 0.0) == 0
+
+
+def test_int4_groups_are_channel_slices_of_one_token():
+    rng = np.random.default_rng(71)
+    B, H, T = 2, 2, 5
+    x = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    y = x.copy()
+    y[1, 0, 3, 70] = 40.0                        # group 2 of token 3 of (b=1, h=0)
+    a, b = _int4_cache(B, H), _int4_cache(B, H)
+    a.append(x, x, bf16=False)
+    b.append(y, y, bf16=False)
+    diff = a["k_scale"] != b["k_scale"]
+    assert diff.sum() == 1 and diff[1, 0, 3, 2]
+    assert b["k_scale"][1, 0, 3, 2] == F32(40.0) / F32(7)
+    changed = np.argwhere(a["k_codes"] != b["k_codes"])
+    assert len(changed) and all((r[0], r[1], r[2]) == (1, 0, 3) and 64 <= 2 * r[3] < 96 for r in changed)
+    for g in range(4):                           # per-group scale is the group's absmax / 7
+        amax = np.abs(x[0, 1, 2, 32 * g:32 * (g + 1)]).max()
+        assert a["k_scale"][0, 1, 2, g] == F32(amax) / F32(7)
+
+
+def test_int4_dequant_within_half_step_and_zero_group():
+    rng = np.random.default_rng(72)
+    x = rng.normal(0, 2, (1, 2, 6, 128)).astype(np.float32)
+    x[0, 1, 4, 96:] = 0.0                        # an all-zero group
+    c = _int4_cache(1, 2)
+    c.append(x, x, bf16=False)
+    deq = c.dequantize(1, 8)[:, :, :6]
+    s = np.repeat(c["v_scale"][:, :, :6], 32, axis=-1)
+    assert np.all(np.abs(deq - x) <= s / 2 * (1 + 2**-20))
+    assert c["v_scale"][0, 1, 4, 3] == 0 and not deq[0, 1, 4, 96:].any()
+
+
+def test_int4_paged_matches_dense():
+    rng = np.random.default_rng(73)
+    B, H, ps, maxp = 2, 2, 4, 3
+    table = rng.permutation(8)[:6].astype(np.int32).reshape(B, maxp)
+    lens = np.array([7, 3], np.int32)
+    x = rng.normal(0, 1, (B, H, 7, 128)).astype(np.float32)
+    pg = _int4_cache(B, H, cap=0, paged=True, page_size=ps, max_pages=maxp, num_pages=8, page_table=table)
+    dn = _int4_cache(B, H, cap=8)
+    pg.append(x, x, bf16=False, new_lens=lens)
+    dn.append(x, x, bf16=False)
+    for b in range(B):
+        for t in range(lens[b]):
+            page, slot = table[b, t // ps], t % ps
+            assert np.array_equal(pg["k_codes"][page, :, slot], dn["k_codes"][b, :, t])
+            assert np.array_equal(pg["v_scale"][page, :, slot], dn["v_scale"][b, :, t])
