@@ -36,7 +36,8 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {synth.FP8_E4M3_PER_TENSOR: "fp8_e4m3", synth.FP8_E5M2_PER_TENSOR: "fp8_e5m2", synth.INT8_SYM_PER_TENSOR: "int8",
               synth.INT8_SYM_PER_TOKEN: "int8", synth.INT8_SYM_PER_CHANNEL: "int8",
-              synth.UINT8_ASYM_PER_CHANNEL: "uint8", synth.KIVI_INT4: "int4", synth.KIVI_INT2: "int2"}
+              synth.UINT8_ASYM_PER_CHANNEL: "uint8", synth.KIVI_INT4: "int4", synth.KIVI_INT2: "int2",
+              synth.INT4_SYM_PER_GROUP: "int4"}
 CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
               synth.UINT8_ASYM_PER_CHANNEL)
 KERNEL_SOURCES = ["decode_attention_quantize_b200/csrc/kvq_decode.cu",
@@ -57,7 +58,7 @@ def parse():
 
 # ---------------------------------------------------------------- algorithmic bytes
 def row_bytes(scheme):
-    return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2}.get(scheme, 8) // 8
+    return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2, synth.INT4_SYM_PER_GROUP: 4}.get(scheme, 8) // 8
 
 
 def meta_bytes_per_token(scheme, Hkv):
@@ -66,6 +67,8 @@ def meta_bytes_per_token(scheme, Hkv):
         return 4.0
     if scheme in (synth.KIVI_INT4, synth.KIVI_INT2):
         return 8.0 * 128 / 32  # fp32 (scale, min) per 32 elements
+    if scheme == synth.INT4_SYM_PER_GROUP:
+        return 4.0 * 128 / 32  # fp32 scale per 32 channels
     return 0.0
 
 

@@ -33,7 +33,7 @@ size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_FP8_E5M2_PER_TENSOR; }
+bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_INT4_SYM_PER_GROUP; }
 
 bool needs_scale(int s) { return true; }
 bool needs_zp(int s) { return s == KVQ_UINT8_ASYM_PER_CHANNEL; }
@@ -51,6 +51,8 @@ uint64_t scale_elems(const kvq_cache_desc* d, int side) {
       return paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity;
     case KVQ_INT8_SYM_PER_CHANNEL:
     case KVQ_UINT8_ASYM_PER_CHANNEL: return H * D;
+    case KVQ_INT4_SYM_PER_GROUP:
+      return (paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity) * (D / 32);
     default:
       return side == 0 ? B * H * (uint64_t)(d->capacity / 32) * D : B * H * (uint64_t)d->capacity * (D / 32);
   }
@@ -104,6 +106,8 @@ kvq_status kvq_validate(const kvq_cache_desc* d) {
       return KVQ_ERR_INVALID_ARG;
     if (d->num_residual < 0 || d->num_residual > d->residual_cap) return KVQ_ERR_INVALID_ARG;
   }
+  if ((d->k_scheme == KVQ_INT4_SYM_PER_GROUP || d->v_scheme == KVQ_INT4_SYM_PER_GROUP) && d->group_size != 32)
+    return KVQ_ERR_UNSUPPORTED;
   if (d->layout == KVQ_DENSE) {
     if (d->capacity < 128 || d->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;
     if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)d->capacity >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
@@ -143,6 +147,7 @@ kvq_status kvq_cache_bytes(const kvq_cache_desc* d, kvq_footprint* out) {
     if (needs_zp(s)) bytes += (uint64_t)d->num_kv_heads * d->head_dim;  // uint8 zero points
     meta += bytes;
     if (s == KVQ_INT8_SYM_PER_TOKEN) per_token_meta += 4.0;
+    if (s == KVQ_INT4_SYM_PER_GROUP) per_token_meta += 4.0 * d->head_dim / 32.0;  // fp32 scale per group
     if (is_kivi(s)) per_token_meta += 8.0 * d->head_dim / 32.0;  // (scale, min) per 32 tokens or channels
   }
   f.meta_bytes = meta;

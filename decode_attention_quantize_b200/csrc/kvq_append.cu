@@ -12,7 +12,9 @@
 //    ("How KV cache quantization reduces GPU memory", n4n.ai, Steps 2-3);
 //  - KIVI: keys per channel over 32-token groups, values per token over 32-channel
 //    groups, min-max with 2^bits - 1 steps, bf16 residual of 128 tokens
-//    (infra.bea.ai §3; llms.blog §3).
+//    (infra.bea.ai §3; llms.blog §3);
+//  - INT4 symmetric per group: s = absmax/7 over 32 consecutive channels of a token,
+//    q = clamp(rne(x/s), -8, 7) as two's-complement nibbles (llms.blog §2; n4n.ai Step 2).
 #include <cuda_fp8.h>
 
 #include <algorithm>
@@ -353,6 +355,23 @@ __device__ __forceinline__ bool asym_row(const float (&x)[8], const Scales8& sc,
 
 constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL; }
 
+// Eight INT4 codes of a thread's slice of one group: clamp(rne(x / s), -8, 7) as two's-
+// complement nibbles, lower channel in the low bits; a zero group gives zero codes.
+__device__ __forceinline__ uint32_t int4_codes(const float (&x)[8], float s) {
+  if (s == 0.0f) return 0u;
+  const float y = __frcp_rn(s);
+  const bool fast = quot_range(s);
+  uint32_t w = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float q;
+    const float z = fast ? quot(x[k], s, y, q) : __fdiv_rn(x[k], s);  // |z| <= 7 (1 + 2^-23)
+    const float c = fminf(fmaxf(rintf(z), -8.0f), 7.0f);
+    w |= ((uint32_t)(int)c & 0xFu) << (4 * k);
+  }
+  return w;
+}
+
 // Rows (b, h, i) of the new block; 16 threads per row, 8 channels each; blockIdx.z = side.
 // Bulk form (kR > 1): blockIdx.y = b * H + h and blockIdx.x a run of 16 * kR tokens of that
 // row, so no thread divides and every row of the block belongs to one head; each thread loads
@@ -450,6 +469,15 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
         for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         tok_s = __fdiv_rn(m, 127.0f);
       }
+      // INT4 per group: absmax over the four lanes (32 channels) of the group
+      if (scheme == KVQ_INT4_SYM_PER_GROUP) {
+        float m = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        tok_s = __fdiv_rn(m, 7.0f);
+      }
       if (!act[it]) continue;
       const int b = rb[it], h = rh[it];
       size_t row;
@@ -457,6 +485,12 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
         row = (size_t)rows_at[it];
       } else {
         if (!cache_row(p, b, h, (p.paged ? p.seq_lens[b] : p.pos0) + ri[it], row)) continue;
+      }
+      if (scheme == KVQ_INT4_SYM_PER_GROUP) {
+        uint8_t* dst = static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * (kHeadDim / 2);
+        *reinterpret_cast<uint32_t*>(dst + lane8 * 4) = int4_codes(x, tok_s);
+        if ((lane8 & 3) == 0) scale[row * (kHeadDim / 32) + (lane8 >> 2)] = tok_s;
+        continue;
       }
       if (per_channel && h != chan_head) {
         fixed_fast = true;
@@ -992,6 +1026,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
             case KVQ_UINT8_ASYM_PER_CHANNEL:
               v = __fmul_rn((float)(q - (int)p.zp[h * kHeadDim + d]), p.scale[h * kHeadDim + d]);
               break;
+            case KVQ_INT4_SYM_PER_GROUP:
+              v = __fmul_rn((float)(q >= 8 ? q - 16 : q), p.scale[row * (kHeadDim / 32) + d / 32]);
+              break;
             default: {  // KIVI
               size_t m;
               if (p.which == 0)
@@ -1048,8 +1085,9 @@ bool append_pair_supported(int ks, int vs) {
   if (is_kivi(ks) || is_kivi(vs)) return ks == vs;
   constexpr int F = KVQ_FP8_E4M3_PER_TENSOR, T = KVQ_INT8_SYM_PER_TENSOR, K = KVQ_INT8_SYM_PER_TOKEN,
                 C = KVQ_INT8_SYM_PER_CHANNEL, U = KVQ_UINT8_ASYM_PER_CHANNEL;
-  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR;
-  const int pairs[][2] = {{F, F}, {T, T}, {K, K}, {C, C}, {U, U}, {T, U}, {C, U}, {K, U}, {T, K}, {F, T}, {T, F}, {E, E}};
+  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR, G = KVQ_INT4_SYM_PER_GROUP;
+  const int pairs[][2] = {{F, F}, {T, T}, {K, K}, {C, C}, {U, U}, {T, U}, {C, U}, {K, U}, {T, K}, {F, T}, {T, F},
+                          {E, E}, {G, G}};
   for (const auto& pr : pairs)
     if (pr[0] == ks && pr[1] == vs) return true;
   return false;
@@ -1063,8 +1101,8 @@ cudaError_t launch_quantize_rows(const AppendParams& p, long long rows, cudaStre
   if (ks == A && vs == B) return launch_quantize_rows_pair<A, B>(p, rows, st);
   KVQ_PAIR(F, F) KVQ_PAIR(T, T) KVQ_PAIR(K, K) KVQ_PAIR(C, C) KVQ_PAIR(U, U)
   KVQ_PAIR(T, U) KVQ_PAIR(C, U) KVQ_PAIR(K, U) KVQ_PAIR(T, K) KVQ_PAIR(F, T) KVQ_PAIR(T, F)
-  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR;
-  KVQ_PAIR(E, E)
+  constexpr int E = KVQ_FP8_E5M2_PER_TENSOR, G = KVQ_INT4_SYM_PER_GROUP;
+  KVQ_PAIR(E, E) KVQ_PAIR(G, G)
 #undef KVQ_PAIR
   return cudaErrorNotSupported;
 }

@@ -41,8 +41,9 @@ constexpr int kRT = 32;                 // residual tile tokens (bf16 rows)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
 
-enum { FMT_E4M3, FMT_E5M2, FMT_S8, FMT_U8, FMT_U4, FMT_U2 };
-enum { FOLD_TENSOR, FOLD_TOKEN, FOLD_CHANNEL, FOLD_KIVI };
+enum { FMT_E4M3, FMT_E5M2, FMT_S8, FMT_U8, FMT_U4, FMT_U2, FMT_S4 };
+// FOLD_GROUP: one scale per (token, 32-channel group), for keys and values (INT4 per group)
+enum { FOLD_TENSOR, FOLD_TOKEN, FOLD_CHANNEL, FOLD_KIVI, FOLD_GROUP };
 
 __host__ __device__ constexpr int fmt_of(int s) {
   return s == KVQ_FP8_E4M3_PER_TENSOR      ? FMT_E4M3
@@ -50,6 +51,7 @@ __host__ __device__ constexpr int fmt_of(int s) {
          : s == KVQ_UINT8_ASYM_PER_CHANNEL ? FMT_U8
          : s == KVQ_KIVI_INT4              ? FMT_U4
          : s == KVQ_KIVI_INT2              ? FMT_U2
+         : s == KVQ_INT4_SYM_PER_GROUP     ? FMT_S4
                                            : FMT_S8;
 }
 __host__ __device__ constexpr int fold_of(int s) {
@@ -57,6 +59,7 @@ __host__ __device__ constexpr int fold_of(int s) {
              ? FOLD_TENSOR
          : s == KVQ_INT8_SYM_PER_TOKEN                                          ? FOLD_TOKEN
          : (s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL) ? FOLD_CHANNEL
+         : s == KVQ_INT4_SYM_PER_GROUP                                          ? FOLD_GROUP
                                                                                 : FOLD_KIVI;
 }
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -68,6 +71,8 @@ struct Cfg {
   static constexpr int kKFmt = fmt_of(KS), kVFmt = fmt_of(VS);
   static constexpr int kKFold = fold_of(KS), kVFold = fold_of(VS);
   static constexpr bool kKivi = kKFold == FOLD_KIVI;
+  // values with one scale per (token, 32-channel group): KIVI and INT4 per group
+  static constexpr bool kGroupV = kVFold == FOLD_KIVI || kVFold == FOLD_GROUP;
   // 32 tokens per consumer warp per tile: two independent 16-token MMA chains per warp, and
   // the per-tile bookkeeping and softmax reductions shared by twice the tokens
   static constexpr int kTPW = 32;
@@ -77,9 +82,11 @@ struct Cfg {
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTS * kKRow;     // multiple of 1024 (swizzle atom)
   static constexpr int kOffKM = kOffV + kTS * kVRow;
-  static constexpr int kKMeta = kKivi ? (kTS / 32) * kHeadDim * 4 * 2 : (kKFold == FOLD_TOKEN ? kTS * 4 : 0);
+  static constexpr int kKMeta = kKivi ? (kTS / 32) * kHeadDim * 4 * 2
+                                : (kKFold == FOLD_TOKEN ? kTS * 4 : (kKFold == FOLD_GROUP ? kTS * 16 : 0));
   static constexpr int kOffVM = kOffKM + kKMeta;
-  static constexpr int kVMeta = kKivi ? kTS * 4 * 4 * 2 : (kVFold == FOLD_TOKEN ? kTS * 4 : 0);
+  static constexpr int kVMeta = kKivi ? kTS * 4 * 4 * 2
+                                : (kVFold == FOLD_TOKEN ? kTS * 4 : (kVFold == FOLD_GROUP ? kTS * 16 : 0));
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
@@ -263,6 +270,8 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       } else {
         if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
         if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
+        if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * 4, C::kKMeta, bar);
+        if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * 4, C::kVMeta, bar);
       }
     } else {
       // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
@@ -291,6 +300,8 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       uint32_t per_page = ps * (C::kKRow + C::kVRow);
       if constexpr (C::kKFold == FOLD_TOKEN) per_page += ps * 4;
       if constexpr (C::kVFold == FOLD_TOKEN) per_page += ps * 4;
+      if constexpr (C::kKFold == FOLD_GROUP) per_page += ps * 16;
+      if constexpr (C::kVFold == FOLD_GROUP) per_page += ps * 16;
       mbar_arrive_expect_tx(bar, nvalid * per_page);
 #pragma unroll
       for (int i = 0; i < C::kTS / 16; ++i) {
@@ -300,6 +311,10 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
         tma_2d(sb + C::kOffV + i * ps * C::kVRow, tv, 0, (int)prow, bar);
         if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar);
         if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar);
+        if constexpr (C::kKFold == FOLD_GROUP)
+          bulk_g2s(sb + C::kOffKM + i * ps * 16, p.k_scale + prow * 4, ps * 16, bar);
+        if constexpr (C::kVFold == FOLD_GROUP)
+          bulk_g2s(sb + C::kOffVM + i * ps * 16, p.v_scale + prow * 4, ps * 16, bar);
       }
     }
   }
@@ -347,6 +362,21 @@ __device__ __forceinline__ uint32_t u4_pair(uint32_t w, int k) {
   const uint32_t x = (k & 2) ? (w >> 8) : w;
   if (k & 1) return hfma2_u(and_or(x, 0x00F000F0u, kF16Magic1024x2), 0x2C002C00u, 0xD400D400u);  // /16 - 64
   return hsub2_u(and_or(x, 0x000F000Fu, kF16Magic1024x2), kF16Magic1024x2);
+}
+
+// Signed (two's-complement) nibbles: XOR with 8 turns a code n into n + 8, which the LOP3 does
+// while it places the nibble under the f16 magic number; the offsets then remove 8 more than
+// in the unsigned form. Nibble pairs of a word as in u4_pair.
+__device__ __forceinline__ uint32_t s4_pair(uint32_t w, int k) {
+  const uint32_t x = (k & 2) ? (w >> 8) : w;
+  if (k & 1) return hfma2_u(and_xor(x, 0x00F000F0u, 0x64806480u), 0x2C002C00u, 0xD480D480u);  // /16 - 72
+  return hsub2_u(and_xor(x, 0x000F000Fu, 0x64086408u), 0x64086408u);                            // - 1032
+}
+
+// Byte `sel` selects (0x4040 + 0x101 c) of a word of signed nibbles -> f16x2 of its two
+// channels (low nibble, high nibble).
+__device__ __forceinline__ uint32_t s4_byte(uint32_t w, uint32_t sel) {
+  return hfma2_u(and_xor(prmt(w, 0u, sel), 0x00F0000Fu, 0x64806408u), 0x2C003C00u, 0xD480E408u);
 }
 
 // 2-bit field pairs of a 32-bit word: k = 0..7 -> (field k, field k + 8).
@@ -465,6 +495,31 @@ __device__ __forceinline__ int build_q(const float* q_s, const float* fold, cons
   return eq;
 }
 
+// Q' fragments for INT4 per-group keys: k-step ks covers channels 16 ks .. 16 ks + 15 (one
+// half of group ks / 2), slot pair h of column group c holding channels 16 ks + 8 h + 2 c and
+// + 1, so every MMA sums one group only. No fold: the group scales multiply the partial sums.
+__device__ __forceinline__ int build_q_s4(const float* q_s, int g, int c, uint32_t (&qh)[8][2], uint32_t (&ql)[8][2]) {
+  float pl[8][2][2];
+  float mx = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float2 v = *reinterpret_cast<const float2*>(q_s + q_off(g, 16 * ks + 8 * h + 2 * c));
+      pl[ks][h][0] = v.x;
+      pl[ks][h][1] = v.y;
+      mx = fmaxf(mx, fmaxf(fabsf(v.x), fabsf(v.y)));
+    }
+  mx = warp_max(mx);
+  const int eq = range_shift(mx);
+  const float sh = pow2i(eq);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) split_f16x2(pl[ks][h][0] * sh, pl[ks][h][1] * sh, qh[ks][h], ql[ks][h]);
+  return eq;
+}
+
 // ------------------------------------------------------------------ one tile, one warp
 // kMasked: the warp's tokens are not all valid (ragged tail or missing pages).
 template <class C, bool kMasked>
@@ -536,6 +591,38 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         const int i = ks >> 1, k0 = 2 * (ks & 1);
         const uint32_t u = word_of(x, i), v = word_of(y, i);
         mma2(ks, u4_pair(u, k0), u4_pair(v, k0), u4_pair(u, k0 + 1), u4_pair(v, k0 + 1), true);
+      }
+    } else if constexpr (C::kKFmt == FMT_S4) {
+      // whole 64-byte rows g and g + 8; lane c takes byte c of every word, so each k-step
+      // covers 16 channels of one 32-channel group and each group's partial sum takes the
+      // (token, group) scale before it joins the score
+      uint4 x[4], y[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        x[i] = lds<uint4>(base + C::kOffK + swz<64>(r0, i));
+        y[i] = lds<uint4>(base + C::kOffK + swz<64>(r1, i));
+      }
+      const float* ksc = reinterpret_cast<const float*>(base + C::kOffKM);
+      const uint32_t sel = 0x4040u + 0x101u * (uint32_t)c;
+      const bool split = S.qsplit;
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        float ag[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int ks = 2 * grp + h2;
+          const uint32_t f0 = s4_byte(word_of(x[grp], 2 * h2), sel), f1 = s4_byte(word_of(y[grp], 2 * h2), sel);
+          const uint32_t f2 = s4_byte(word_of(x[grp], 2 * h2 + 1), sel);
+          const uint32_t f3 = s4_byte(word_of(y[grp], 2 * h2 + 1), sel);
+          mma_16816(ag, f0, f1, f2, f3, S.qh[ks][0], S.qh[ks][1]);
+          if (split) mma_16816(ag, f0, f1, f2, f3, S.ql[ks][0], S.ql[ks][1]);
+        }
+        const float s0 = ksc[r0 * 4 + grp], s1 = ksc[r1 * 4 + grp];
+        float(&dst)[4] = (grp & 1) ? a1 : a0;
+        dst[0] = fmaf(s0, ag[0], dst[0]);
+        dst[1] = fmaf(s0, ag[1], dst[1]);
+        dst[2] = fmaf(s1, ag[2], dst[2]);
+        dst[3] = fmaf(s1, ag[3], dst[3]);
       }
     } else if constexpr (C::kKFmt == FMT_U2) {
       const uint2 x = lds<uint2>(base + C::kOffK + swz<32>(r0, c >> 1) + 8 * (c & 1));
@@ -636,12 +723,12 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
   }
 
   // (6) value-side fold and accumulator exponent
-  constexpr bool kVPerToken = C::kVFold == FOLD_TOKEN || C::kKivi;
+  constexpr bool kVPerToken = C::kVFold == FOLD_TOKEN || C::kGroupV;
   // folded value scale of token tok, group j (per-token fold: group 0); 0 for masked tokens.
   // Read from shared memory where it is used, so the 16 (KIVI: 32) values are not held live.
   auto vscale = [&](int tok, int j) -> float {
     if (!tok_ok(tok)) return 0.0f;
-    if constexpr (C::kKivi) return reinterpret_cast<const float*>(base + C::kOffVM)[tok * 4 + j];
+    if constexpr (C::kGroupV) return reinterpret_cast<const float*>(base + C::kOffVM)[tok * 4 + j];
     return reinterpret_cast<const float*>(base + C::kOffVM)[tok];
   };
   int evn = 15;
@@ -653,7 +740,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       for (int k = 0; k < 4; ++k) {
         const int tok = tok_base + sb * 16 + 2 * c + (k & 1) + 8 * (k >> 1);
         const bool ok = tok_ok(tok);
-        if constexpr (C::kKivi) {
+        if constexpr (C::kGroupV) {
           const float4 s4 = lds<float4>(base + C::kOffVM + tok * 16);
           const float m4 = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
           smax = fmaxf(smax, ok ? m4 : 0.0f);
@@ -702,7 +789,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     bool ok[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) ok[k] = tok_ok(tk[k]);
-    if constexpr (!C::kKivi) {
+    if constexpr (!C::kGroupV) {
       float pv[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) pv[k] = (C::kVFold == FOLD_TOKEN ? pt[sb][k] * vscale(tk[k], 0) : pt[sb][k]) * pscale;
@@ -736,7 +823,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         }
       }
     } else {
-      // KIVI: one B operand per 32-channel group; zero-point term on CUDA cores
+      // one B operand per 32-channel group; KIVI's zero-point term on CUDA cores
       uint32_t bh[4][2], bl[4][2];
       float4 s4[4];  // value scales of this thread's four tokens, groups 0..3
 #pragma unroll
@@ -755,7 +842,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
         split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
       }
-      if (!residual) {
+      if (C::kKivi && !residual) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (!ok[k]) continue;
@@ -769,7 +856,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       // INT4 codes: one transposed matrix load per 8 tokens gives every lane its (token 2c,
       // token 2c + 1) pair of 16-bit words (4 channels) for all four channel groups
       uint32_t v4[2][4];
-      if constexpr (C::kVFmt == FMT_U4) {
+      if constexpr (C::kVFmt == FMT_U4 || C::kVFmt == FMT_S4) {
         if (!residual) {
           const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -804,6 +891,11 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
           for (int pp = 0; pp < 2; ++pp)
 #pragma unroll
             for (int e = 0; e < 4; ++e) pr[pp][e] = u4_pair(v4[pp][j], e);
+        } else if constexpr (C::kVFmt == FMT_S4) {
+#pragma unroll
+          for (int pp = 0; pp < 2; ++pp)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[pp][e] = s4_pair(v4[pp][j], e);
         } else {
 #pragma unroll
           for (int pp = 0; pp < 2; ++pp) {
@@ -914,7 +1006,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
       if constexpr (!C::kKivi) {
         const float* fold = nullptr;
         if constexpr (C::kKFold == FOLD_CHANNEL) fold = p.k_scale + (size_t)d.hk * kHeadDim;
-        const int eq = build_q<C::kKFmt>(q_s, fold, nullptr, g, c, S.qh, S.ql);
+        int eq;
+        if constexpr (C::kKFmt == FMT_S4)
+          eq = build_q_s4(q_s, g, c, S.qh, S.ql);
+        else
+          eq = build_q<C::kKFmt>(q_s, fold, nullptr, g, c, S.qh, S.ql);
         S.qsplit = (C::kKFold == FOLD_CHANNEL) || !p.q_bf16;
         float mul = sc_log2 * pow2i(-eq);
         if constexpr (C::kKFold == FOLD_TENSOR) mul *= p.k_scale[0];
@@ -1000,9 +1096,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
           for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
             for (int rh = 0; rh < 2; ++rh) {
-              const int ch = dmap_v<C::kKivi>(g, mt, rh);
-              red_o[(w * kMH + 2 * c - kMH * half) * kHeadDim + red_col<C::kKivi>(ch, 2 * c)] = S.o[mt][2 * rh] * oscale;
-              red_o[(w * kMH + 2 * c + 1 - kMH * half) * kHeadDim + red_col<C::kKivi>(ch, 2 * c + 1)] =
+              const int ch = dmap_v<C::kGroupV>(g, mt, rh);
+              red_o[(w * kMH + 2 * c - kMH * half) * kHeadDim + red_col<C::kGroupV>(ch, 2 * c)] = S.o[mt][2 * rh] * oscale;
+              red_o[(w * kMH + 2 * c + 1 - kMH * half) * kHeadDim + red_col<C::kGroupV>(ch, 2 * c + 1)] =
                   S.o[mt][2 * rh + 1] * oscale;
             }
         }
@@ -1023,7 +1119,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
 #pragma unroll
             for (int ww = 0; ww < kCW; ++ww) {
               const float a = fast_exp2(red_m[ww * 8 + j] - M);
-              float x = red_o[(ww * kMH + j - kMH * half) * kHeadDim + red_col<C::kKivi>(dd, j)];
+              float x = red_o[(ww * kMH + j - kMH * half) * kHeadDim + red_col<C::kGroupV>(dd, j)];
               if constexpr (C::kKivi) x += red_z[(ww * kMH + j - kMH * half) * 4 + (dd >> 5)];
               ov = fmaf(a, x, ov);
               L = fmaf(a, red_l[ww * 8 + j], L);
@@ -1200,7 +1296,7 @@ Variant variant() {
   return Variant{KS, VS, PG ? 1 : 0, decode_kernel<KS, VS, PG>, C::kSmemBytes, C::kTS};
 }
 
-constexpr int kNumVariants = 26;
+constexpr int kNumVariants = 28;
 constexpr int kMaxDevices = 64;
 
 const Variant* variants() {
@@ -1229,6 +1325,8 @@ const Variant* variants() {
       variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, true>(),
       variant<KVQ_FP8_E5M2_PER_TENSOR, KVQ_FP8_E5M2_PER_TENSOR, false>(),
       variant<KVQ_FP8_E5M2_PER_TENSOR, KVQ_FP8_E5M2_PER_TENSOR, true>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, false>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, true>(),
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
   };

@@ -120,6 +120,13 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t mask, uint32_t b
   return r;
 }
 
+// (a & mask) ^ bits in one LOP3
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t mask, uint32_t bits) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(r) : "r"(a), "r"(mask), "r"(bits));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t hsub2_u(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
@@ -216,7 +223,7 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 // ------------------------------------------------------------------ scheme traits
 __host__ __device__ constexpr bool is_kivi(int s) { return s == KVQ_KIVI_INT4 || s == KVQ_KIVI_INT2; }
 __host__ __device__ constexpr int code_bits(int s) {
-  return s == KVQ_KIVI_INT4 ? 4 : (s == KVQ_KIVI_INT2 ? 2 : 8);
+  return (s == KVQ_KIVI_INT4 || s == KVQ_INT4_SYM_PER_GROUP) ? 4 : (s == KVQ_KIVI_INT2 ? 2 : 8);
 }
 __host__ __device__ constexpr int row_bytes(int s) { return kHeadDim * code_bits(s) / 8; }
 

@@ -27,6 +27,7 @@ UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
+INT4_SYM_PER_GROUP = 8
 KVQ_F32, KVQ_BF16 = 0, 1
 KVQ_DENSE, KVQ_PAGED = 0, 1
 KVQ_APPEND_CALIBRATE = 0x1
@@ -134,7 +135,7 @@ def _dtype_code(t):
 
 
 def row_bytes(scheme: int, D: int = 128) -> int:
-    return D * {KIVI_INT4: 4, KIVI_INT2: 2}.get(scheme, 8) // 8
+    return D * {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4}.get(scheme, 8) // 8
 
 
 # ---------------------------------------------------------------- entry points
@@ -272,6 +273,8 @@ class QuantizedKVCache:
                 self.t[side + "_scale"] = torch.zeros(4, dtype=torch.float32, device=dev)
             elif sch == INT8_SYM_PER_TOKEN:
                 self.t[side + "_scale"] = torch.zeros(*rows, dtype=torch.float32, device=dev)
+            elif sch == INT4_SYM_PER_GROUP:
+                self.t[side + "_scale"] = torch.zeros(*rows, s.D // 32, dtype=torch.float32, device=dev)
             elif sch in (INT8_SYM_PER_CHANNEL, UINT8_ASYM_PER_CHANNEL):
                 self.t[side + "_scale"] = torch.zeros(s.Hkv, s.D, dtype=torch.float32, device=dev)
                 if sch == UINT8_ASYM_PER_CHANNEL:

@@ -63,6 +63,11 @@ typedef enum kvq_status {
  *  FP8_E5M2_PER_TENSOR  OCP E5M2 codes of x/s, s = absmax/57344 over the calibrating append,
  *                       saturating at +-57344 (llms.blog §1 compares E4M3 with E5M2; a format
  *                       variant beyond the configurations the pages measure).
+ *  INT4_SYM_PER_GROUP   clamp(rne(x/s), -8, 7) with s = absmax/7 per group of 32 consecutive
+ *                       channels of one token (llms.blog §2 "INT4 Group-Wise"; n4n.ai Step 2
+ *                       "Per-group INT4"); two's-complement nibbles packed along head_dim,
+ *                       lower channel in the low bits (64-byte rows); fp32 scales
+ *                       [rows][4] beside the codes. group_size must be 32. K and V both.
  * A zero range gives s = 0 and code 0. */
 typedef enum kvq_scheme {
   KVQ_FP8_E4M3_PER_TENSOR = 0,
@@ -72,7 +77,8 @@ typedef enum kvq_scheme {
   KVQ_UINT8_ASYM_PER_CHANNEL = 4,
   KVQ_KIVI_INT4 = 5,
   KVQ_KIVI_INT2 = 6,
-  KVQ_FP8_E5M2_PER_TENSOR = 7
+  KVQ_FP8_E5M2_PER_TENSOR = 7,
+  KVQ_INT4_SYM_PER_GROUP = 8
 } kvq_scheme;
 
 typedef enum kvq_dtype { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
@@ -94,6 +100,8 @@ typedef enum kvq_layout { KVQ_DENSE = 0, KVQ_PAGED = 1 } kvq_layout;
  *   paged codes  [num_pages, kv_heads, page_size, row_bytes]
  *   per-tensor scale            float [1]
  *   per-token scale             float [batch, kv_heads, capacity]  (paged: [num_pages, kv_heads, page_size])
+ *   INT4 per-group scale        float [batch, kv_heads, capacity, head_dim/32] (paged: [num_pages,
+ *                               kv_heads, page_size, head_dim/32])
  *   per-channel scale           float [kv_heads, head_dim]; uint8 zero point (k_zp/v_zp) same shape
  *   KIVI key scale and minimum  float [batch, kv_heads, capacity/32, head_dim] (k_scale, k_zero)
  *   KIVI value scale and minimum float [batch, kv_heads, capacity, head_dim/32] (v_scale, v_zero)

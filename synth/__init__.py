@@ -110,6 +110,7 @@ UINT8_ASYM_PER_CHANNEL = 4
 KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
+INT4_SYM_PER_GROUP = 8
 
 
 @dataclass
@@ -173,8 +174,8 @@ class Workload:
 
 
 def workloads() -> dict:
-    """The six workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 70B, KIVI-2 131K,
-    paged INT8."""
+    """The seven workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4
+    per-group 70B-shaped, KIVI-2 131K, paged INT8."""
     return {
         "tiny_int8": Workload(
             name="tiny_int8", seed=1, B=1, Hq=1, Hkv=1, D=128,
@@ -193,6 +194,10 @@ def workloads() -> dict:
             k_scheme=KIVI_INT4, v_scheme=KIVI_INT4, bf16=True,
             outlier_scale=20.0, rope_theta=500000.0, context=32768,
             extra={"seeded_residual": True}),
+        "int4g_70b": Workload(
+            name="int4g_70b", seed=7, B=16, Hq=64, Hkv=8, D=128,
+            k_scheme=INT4_SYM_PER_GROUP, v_scheme=INT4_SYM_PER_GROUP, bf16=True,
+            outlier_scale=20.0, rope_theta=500000.0, context=32768),
         "kivi2_131k": Workload(
             name="kivi2_131k", seed=4, B=4, Hq=64, Hkv=8, D=128,
             k_scheme=KIVI_INT2, v_scheme=KIVI_INT2, bf16=True,

@@ -77,7 +77,7 @@ def compare_dense(oc: OracleCache, gc, where=""):
         s_g, s_o = np_of(gc[side + "_scale"]), oc[side + "_scale"]
         if sch in (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR):
             assert s_g.view(np.uint32)[0] == s_o.view(np.uint32)[0], f"{where}: {side} scale differs"
-        elif sch == synth.INT8_SYM_PER_TOKEN:
+        elif sch in (synth.INT8_SYM_PER_TOKEN, synth.INT4_SYM_PER_GROUP):
             assert np.array_equal(s_g[:, :, :L].view(np.uint32), s_o[:, :, :L].view(np.uint32)), \
                 f"{where}: {side} token scales differ"
         elif sch in (synth.INT8_SYM_PER_CHANNEL, synth.UINT8_ASYM_PER_CHANNEL):
@@ -111,7 +111,7 @@ def compare_paged(oc: OracleCache, gc, where=""):
                 page, slot = table[b, t // ps], t % ps
                 assert np.array_equal(pool_g[page, :, slot], pool_o[page, :, slot]), \
                     f"{where}: {side} codes differ at seq {b} token {t}"
-                if sch == synth.INT8_SYM_PER_TOKEN:
+                if sch in (synth.INT8_SYM_PER_TOKEN, synth.INT4_SYM_PER_GROUP):
                     assert np.array_equal(np_of(gc[side + "_scale"])[page, :, slot].view(np.uint32),
                                           oc[side + "_scale"][page, :, slot].view(np.uint32))
         s_g, s_o = np_of(gc[side + "_scale"]), oc[side + "_scale"]

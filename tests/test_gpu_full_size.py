@@ -51,7 +51,7 @@ def _check_pair_dense(w, gc, oc, b, h, out_gpu, q):
         got = H.np_of(gc[side + "_codes"][b, h, :L])
         assert np.array_equal(got, oc[side + "_codes"][0, 0, :L]), f"pair {(b, h)}: {side} codes"
         sch = w.k_scheme if side == "k" else w.v_scheme
-        if sch == synth.INT8_SYM_PER_TOKEN:
+        if sch in (synth.INT8_SYM_PER_TOKEN, synth.INT4_SYM_PER_GROUP):
             assert np.array_equal(H.np_of(gc[side + "_scale"][b, h, :L]).view(np.uint32),
                                   oc[side + "_scale"][0, 0, :L].view(np.uint32))
         if sch in (synth.KIVI_INT4, synth.KIVI_INT2):
@@ -115,6 +115,10 @@ def test_fp8_8b_full():
 
 def test_e5m2_8b_full():
     _dense_full("e5m2_8b")
+
+
+def test_int4g_70b_full():
+    _dense_full("int4g_70b")
 
 
 def test_kivi4_70b_full():

@@ -213,6 +213,48 @@ def test_saturated_codes_match_oracle(scheme):
     H.decode_both(oc, gc, synth.queries(w, 0, 0, B), False, "decode over saturated codes")
 
 
+# ------------------------------------------------------------------ INT4 symmetric per group
+# keys: every MMA sums one 32-channel group and takes its (token, group) scale afterwards;
+# values: one scaled P' per group; ragged tails, GQA group sizes, both input types, paged.
+@pytest.mark.parametrize("prefill", [1, 100, 128, 300, 9600])
+def test_int4_group_dense(prefill):
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=prefill, steps=2,
+                 outlier=100.0)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8, 16])
+def test_int4_group_gqa_sizes(G):
+    H.dense_case(B=2, Hq=2 * G, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=200, steps=1)
+
+
+def test_int4_group_fp32_inputs_and_queries():
+    H.dense_case(B=1, Hq=4, Hkv=1, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=257, steps=2,
+                 bf16=False, rope=0.0)
+    H.dense_case(B=2, Hq=8, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=130, steps=1,
+                 bf16=True, q_bf16=False)
+
+
+@pytest.mark.parametrize("ps", [16, 32, 64])
+def test_int4_group_paged(ps):
+    B, Hq, Hkv, sch = 4, 16, 4, S.INT4_SYM_PER_GROUP
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, sch, sch, lens=[37, 100, 5, 64], page_size=ps,
+                                                    steps=2)
+    oc.append(K, V, True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc, "int4 paged prefill")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), True, "int4 paged decode 0")
+    for s in range(2):
+        kk = np.stack([synth.keys(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(B)])
+        vv = np.stack([synth.values(w, b, b + 1, 0, Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(B)])
+        oc.append(kk, vv, True)
+        gc.append(H.dev(kk, True), H.dev(vv, True))
+        torch.cuda.synchronize()
+        H.compare_paged(oc, gc, f"int4 paged step {s}")
+        H.decode_both(oc, gc, synth.queries(w, s + 1, 0, B), True, f"int4 paged decode {s + 1}")
+    assert gc.status()[0] == 0
+
+
 # ------------------------------------------------------------------ rescaling append
 # Scales merged with each block's (they only grow) and the cached codes whose scale changed
 # requantized, bit for bit against the oracle; blocks inside the range, a grown single
@@ -298,7 +340,8 @@ def test_rescale_schedule_every_1024_tokens():
 # ------------------------------------------------------------------ dequantize
 @pytest.mark.parametrize("ks,vs", [(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.KIVI_INT2, S.KIVI_INT2),
                                    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
-                                   (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR)])
+                                   (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR),
+                                   (S.INT4_SYM_PER_GROUP, S.INT4_SYM_PER_GROUP)])
 def test_dequantize_matches_oracle(ks, vs):
     oc, gc, _ = H.dense_case(B=2, Hq=8, Hkv=2, ks=ks, vs=vs, prefill=200, steps=1, cap=384)
     T = oc.tokens()
