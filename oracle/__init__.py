@@ -64,6 +64,7 @@ class _Cache(ctypes.Structure):
         ("k_zp", ctypes.c_void_p), ("v_zp", ctypes.c_void_p),
         ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
+        ("rotate", ctypes.c_int),
     ]
 
 
@@ -99,6 +100,8 @@ def load(path: str):
     L.oq_append.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp, i32]
     L.oq_append.restype = i32
     L.oq_calibrate.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp]
+    L.oq_fwht.argtypes = [vp, i32]
+    L.oq_fwht.restype = None
     L.oq_calibrate.restype = i32
     L.oq_tokens.argtypes = [ctypes.POINTER(_Cache), i32]
     L.oq_tokens.restype = i32
@@ -138,6 +141,13 @@ def sym_code(x: float, s: float, qmax: int = 127) -> int:
 
 def int4_code(x: float, s: float) -> int:
     return int(lib().oq_int4_code(float(x), float(s)))
+
+
+def fwht(x) -> np.ndarray:
+    """Normalised Walsh-Hadamard transform of a float32 vector (length a power of two)."""
+    y = np.array(x, np.float32, copy=True)
+    lib().oq_fwht(y.ctypes.data, int(y.size))
+    return y
 
 
 def asym_params(mn: float, mx: float):
@@ -189,7 +199,7 @@ class OracleCache:
     """Oracle cache with numpy arrays in the library's layouts (see module docstring)."""
 
     def __init__(self, B, Hq, Hkv, D, k_scheme, v_scheme, cap=0, paged=False, page_size=16,
-                 max_pages=0, num_pages=0, page_table=None, group=32, rcap=128):
+                 max_pages=0, num_pages=0, page_table=None, group=32, rcap=128, rotate=False):
         self.B, self.Hq, self.Hkv, self.D = B, Hq, Hkv, D
         self.k_scheme, self.v_scheme = k_scheme, v_scheme
         self.paged, self.cap, self.page_size = paged, cap, page_size
@@ -231,6 +241,8 @@ class OracleCache:
                         max_pages, num_pages, group, rcap, 0, 0)
         for name, arr in self.arrays.items():
             setattr(self.c, name, _ptr(arr))
+        self.c.rotate = int(bool(rotate))
+        self.rotate = bool(rotate)
 
     def __getitem__(self, name):
         return self.arrays[name]

@@ -18,6 +18,9 @@
  *    residual.
  *  - INT4 symmetric per group: groups of 32 consecutive channels of a token, s = absmax / 7,
  *    q = clamp(rne(x / s), -8, 7), two's-complement nibbles, lower channel in the low bits.
+ *  - rotation (optional): the normalised Walsh-Hadamard transform of each K/V row before it
+ *    is quantized, of each query before attention, and of each attention output and
+ *    dequantized row after (P3 §5, QuaRot / RotateKV); fp32 butterflies in span order.
  */
 #include "kvq_oracle.h"
 
@@ -28,6 +31,33 @@
 /* ------------------------------------------------------------------------- */
 /* element codecs                                                            */
 /* ------------------------------------------------------------------------- */
+
+/* Normalised Walsh-Hadamard transform (Sylvester order): H_n with entries
+ * (-1)^popcount(i & j), scaled by 1/sqrt(n) so that it is orthogonal and symmetric, hence
+ * its own inverse; rotating q and k alike keeps q.k (P3 §5 "QuaRot / RotateKV"). */
+void oq_fwht(float* x, int n) {
+  for (int h = 1; h < n; h *= 2)
+    for (int i = 0; i < n; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        const float a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+  const float c = (float)(1.0 / sqrt((double)n));
+  for (int i = 0; i < n; ++i) x[i] = x[i] * c;
+}
+
+static void fwht_d(double* x, int n) {
+  for (int h = 1; h < n; h *= 2)
+    for (int i = 0; i < n; i += 2 * h)
+      for (int j = i; j < i + h; ++j) {
+        const double a = x[j], b = x[j + h];
+        x[j] = a + b;
+        x[j + h] = a - b;
+      }
+  const double c = 1.0 / sqrt((double)n);
+  for (int i = 0; i < n; ++i) x[i] *= c;
+}
 
 float oq_bf16_to_f32(uint16_t h) {
   uint32_t u = (uint32_t)h << 16;
@@ -552,15 +582,41 @@ static void rescale(oq_cache* c, const block* k, int which) {
   free(zp_blk);
 }
 
+static int append_rows(oq_cache* c, const block* kbp, const block* vbp, int calibrate_flag);
+
+/* fp32 copy of a [B, Hkv, n_new, D] block with every row rotated. */
+static float* rotated_rows(const oq_cache* c, const void* x, int in_bf16, int n_new) {
+  const size_t n = (size_t)c->B * (size_t)c->Hkv * (size_t)n_new * (size_t)c->D;
+  float* r = (float*)malloc(sizeof(float) * (n ? n : 1));
+  for (size_t i = 0; i < n; ++i) r[i] = input_at(x, in_bf16, i);
+  for (size_t row = 0; row < n / (size_t)c->D; ++row) oq_fwht(r + row * c->D, c->D);
+  return r;
+}
+
 int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
               const int32_t* new_lens, int calibrate_flag) {
   block kb = {k_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
   block vb = {v_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
   if (new_lens && !c->paged) return -1;
   if (is_kivi(c->k_scheme) || is_kivi(c->v_scheme)) {
-    if (!(is_kivi(c->k_scheme) && is_kivi(c->v_scheme)) || c->paged) return -1;
+    if (!(is_kivi(c->k_scheme) && is_kivi(c->v_scheme)) || c->paged || c->rotate) return -1;
     return append_kivi(c, &kb, &vb);
   }
+  if (!c->rotate) return append_rows(c, &kb, &vb, calibrate_flag);
+  /* rotate every row of the block first: statistics and codes are those of H x */
+  float* kr = rotated_rows(c, k_new, in_bf16, n_new);
+  float* vr = rotated_rows(c, v_new, in_bf16, n_new);
+  block kq = {kr, 0, n_new, new_lens, c->Hkv, c->D};
+  block vq = {vr, 0, n_new, new_lens, c->Hkv, c->D};
+  const int rc = append_rows(c, &kq, &vq, calibrate_flag);
+  free(kr);
+  free(vr);
+  return rc;
+}
+
+static int append_rows(oq_cache* c, const block* kbp, const block* vbp, int calibrate_flag) {
+  const block kb = *kbp, vb = *vbp;
+  const int n_new = kb.n_new;
   /* capacity */
   for (int b = 0; b < c->B; ++b) {
     const int start = c->paged ? c->seq_lens[b] : c->len;
@@ -602,11 +658,15 @@ int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, in
 
 int oq_calibrate(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
                  const int32_t* new_lens) {
-  block kb = {k_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
-  block vb = {v_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
   if (is_kivi(c->k_scheme) || is_kivi(c->v_scheme)) return -1;
+  float* kr = c->rotate ? rotated_rows(c, k_new, in_bf16, n_new) : NULL;
+  float* vr = c->rotate ? rotated_rows(c, v_new, in_bf16, n_new) : NULL;
+  block kb = {kr ? (const void*)kr : k_new, kr ? 0 : in_bf16, n_new, new_lens, c->Hkv, c->D};
+  block vb = {vr ? (const void*)vr : v_new, vr ? 0 : in_bf16, n_new, new_lens, c->Hkv, c->D};
   calibrate(c, &kb, c->k_scheme, c->k_scale, c->k_zp);
   calibrate(c, &vb, c->v_scheme, c->v_scale, c->v_zp);
+  free(kr);
+  free(vr);
   return 0;
 }
 
@@ -664,10 +724,11 @@ void oq_dequantize(const oq_cache* c, int which, float* out, int T_out) {
   for (int b = 0; b < c->B; ++b)
     for (int h = 0; h < c->Hkv; ++h) {
       const int T = oq_tokens(c, b);
-      for (int t = 0; t < T_out; ++t)
-        for (int d = 0; d < D; ++d)
-          out[(((size_t)b * c->Hkv + h) * (size_t)T_out + t) * D + d] =
-              t < T ? value_at(c, which, b, h, t, d) : 0.0f;
+      for (int t = 0; t < T_out; ++t) {
+        float* row = out + (((size_t)b * c->Hkv + h) * (size_t)T_out + t) * D;
+        for (int d = 0; d < D; ++d) row[d] = t < T ? value_at(c, which, b, h, t, d) : 0.0f;
+        if (c->rotate && t < T) oq_fwht(row, D);  /* back from the rotated domain */
+      }
     }
 }
 
@@ -717,8 +778,10 @@ static void decode_pair(const oq_cache* c, const void* q, int q_bf16, float scal
   for (int j = 0; j < G; ++j) {
     const int hq = hk * G + j; /* query head h reads kv head h / G */
     for (int d = 0; d < D; ++d) qr[d] = input_at(q, q_bf16, ((size_t)b * c->Hq + hq) * D + d);
+    if (c->rotate) oq_fwht(qr, D);  /* the cache holds H k and H v: attend with H q */
     double l;
     oq_attention_row(qr, k, v, T, D, scale, out + (size_t)j * D, &l);
+    if (c->rotate) fwht_d(out + (size_t)j * D, D);  /* sum p (H v) = H (sum p v) */
     if (lse) lse[j] = l;
   }
   free(k);

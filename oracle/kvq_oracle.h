@@ -74,6 +74,8 @@ typedef struct {
   uint8_t *k_zp, *v_zp;
   uint16_t *k_res, *v_res;       /* bf16 [B,Hkv,rcap,D] */
   int32_t *page_table, *seq_lens;
+  int rotate;                    /* 1: K/V rows and queries rotated by the normalised
+                                    Walsh-Hadamard transform over head_dim (not with KIVI) */
 } oq_cache;
 
 /* Append modes (the `calibrate` argument of oq_append). */
@@ -93,6 +95,11 @@ int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, in
  * cache from the block (same arguments), quantize nothing. */
 int oq_calibrate(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, int n_new,
                  const int32_t* new_lens);
+
+/* In-place normalised Walsh-Hadamard transform of n (a power of two) values: butterfly
+ * stages of span 1, 2, 4, ..., n/2, each (a, b) -> (a + b, a - b) in fp32, then every value
+ * times the fp32 constant nearest 1/sqrt(n). The transform is its own inverse. */
+void oq_fwht(float* x, int n);
 
 /* Tokens visible to decode for sequence b. */
 int oq_tokens(const oq_cache* c, int b);

@@ -61,6 +61,14 @@ MUTATIONS = [
     ("int4 clamp -7", "if (r < -8.0f) r = -8.0f;", "if (r < -7.0f) r = -7.0f;"),
     ("int4 group amax from group 0", "for (int d = j * g; d < (j + 1) * g; ++d) {\n        float a = fabsf",
      "for (int d = 0; d < g; ++d) {\n        float a = fabsf"),
+    ("fwht sign", "        x[j] = a + b;\n        x[j + h] = a - b;\n      }\n  const float c",
+     "        x[j] = a + b;\n        x[j + h] = b - a;\n      }\n  const float c"),
+    ("fwht unnormalised", "const float c = (float)(1.0 / sqrt((double)n));", "const float c = 1.0f;"),
+    ("fwht skips last stage", "  for (int h = 1; h < n; h *= 2)\n    for (int i = 0; i < n; i += 2 * h)\n      for (int j = i; j < i + h; ++j) {\n        const float a",
+     "  for (int h = 1; h < n / 2; h *= 2)\n    for (int i = 0; i < n; i += 2 * h)\n      for (int j = i; j < i + h; ++j) {\n        const float a"),
+    ("decode query not rotated", "    if (c->rotate) oq_fwht(qr, D);", "    (void)0;"),
+    ("decode output not rotated back", "    if (c->rotate) fwht_d(out + (size_t)j * D, D);", "    (void)0;"),
+    ("dequantize not rotated back", "        if (c->rotate && t < T) oq_fwht(row, D);", "        (void)row;"),
     ("rescale paged length", "const int len = c->paged ? c->seq_lens[b] : c->len;",
      "const int len = c->paged ? c->seq_lens[b] - 1 : c->len;"),
 ]

@@ -879,3 +879,73 @@ def test_int4_paged_matches_dense():
             page, slot = table[b, t // ps], t % ps
             assert np.array_equal(pg["k_codes"][page, :, slot], dn["k_codes"][b, :, t])
             assert np.array_equal(pg["v_scale"][page, :, slot], dn["v_scale"][b, :, t])
+
+
+# --------------------------------------------------------------- Walsh-Hadamard rotation
+# llms.blog §5 (QuaRot / RotateKV): an orthogonal Hadamard rotation of K, V and Q spreads
+# outlier channels before low-bit quantization and leaves q.k unchanged.
+def _walsh(n, j):
+    return np.array([(-1) ** bin(i & j).count("1") for i in range(n)], np.float64)
+
+
+def test_fwht_basis_vectors_are_walsh_functions():
+    c = F32(1.0 / math.sqrt(128.0))
+    for j in (0, 1, 5, 64, 77, 127):
+        e = np.zeros(128, np.float32)
+        e[j] = 1.0
+        assert np.array_equal(oracle.fwht(e), (_walsh(128, j) * float(c)).astype(np.float32)), j
+
+
+def test_fwht_matches_the_hadamard_matrix_and_is_orthogonal():
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    Hm = scipy_linalg.hadamard(128).astype(np.float64) / math.sqrt(128.0)
+    rng = np.random.default_rng(80)
+    for _ in range(20):
+        x = rng.normal(0, 3, 128).astype(np.float32)
+        y = oracle.fwht(x).astype(np.float64)
+        ref = Hm @ x.astype(np.float64)
+        assert np.max(np.abs(y - ref)) <= 1e-6 * np.abs(x).sum()
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) <= 1e-6 * np.linalg.norm(x)   # Parseval
+        z = oracle.fwht(oracle.fwht(x)).astype(np.float64)                              # own inverse
+        assert np.max(np.abs(z - x)) <= 1e-6 * np.abs(x).max()
+
+
+def test_rotated_cache_quantizes_the_rotated_rows():
+    # codes and scales of a rotating cache are those of a plain cache fed H x
+    rng = np.random.default_rng(81)
+    B, H, T = 2, 2, 9
+    k = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    k[..., 3] *= 30                              # an outlier channel
+    kr = np.apply_along_axis(oracle.fwht, -1, k)
+    vr = np.apply_along_axis(oracle.fwht, -1, v)
+    for sch in (oracle.INT8_SYM_PER_TOKEN, oracle.INT4_SYM_PER_GROUP, oracle.FP8_E4M3_PER_TENSOR):
+        a = OracleCache(B, H, H, 128, sch, sch, cap=16, rotate=True)
+        b = OracleCache(B, H, H, 128, sch, sch, cap=16)
+        a.append(k, v, bf16=False, calibrate=True)
+        b.append(kr, vr, bf16=False, calibrate=True)
+        for n in ("k_codes", "v_codes", "k_scale", "v_scale"):
+            assert np.array_equal(a[n], b[n]), (sch, n)
+        # dequantize returns the original domain: H applied to the rotated values
+        back = np.apply_along_axis(oracle.fwht, -1, b.dequantize(0, 16)[:, :, :T])
+        assert np.array_equal(a.dequantize(0, 16)[:, :, :T], back)
+
+
+def test_rotated_decode_equals_attention_in_the_original_domain():
+    rng = np.random.default_rng(82)
+    B, Hq, H, T = 1, 4, 2, 40
+    k = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    k[..., 7] *= 20
+    c = OracleCache(B, Hq, H, 128, oracle.INT8_SYM_PER_TOKEN, oracle.INT8_SYM_PER_TOKEN, cap=64, rotate=True)
+    c.append(k, v, bf16=False)
+    q = rng.normal(0, 1, (B, Hq, 128)).astype(np.float32)
+    out, lse = c.decode(q, bf16=False, scale=0.09)
+    K, V = c.dequantize(0, T).astype(np.float64), c.dequantize(1, T).astype(np.float64)
+    for h in range(Hq):
+        s = K[0, h // 2] @ q[0, h].astype(np.float64) * float(F32(0.09))
+        p = np.exp(s - s.max())
+        ref = (p / p.sum()) @ V[0, h // 2]
+        assert np.max(np.abs(out[0, h] - ref)) <= 1e-5 * np.abs(ref).max()
+        assert abs(lse[0, h] - (s.max() + math.log(p.sum()))) <= 1e-5
+
