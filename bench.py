@@ -251,7 +251,7 @@ class GpuWorkload:
         self.append_token = W.name != "tiny_int8"  # the tiny configuration decodes without appending
         pre = total - 1 if self.append_token else total
         cap = (total + 127) // 128 * 128
-        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap)
+        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap, rotate=W.rotate)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev)
         self.calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
         self.pre_k = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, 0, pre), W.bf16)
@@ -356,7 +356,7 @@ class GpuWorkload:
             table[b, :n] = perm[off:off + n]
             off += n
         spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, paged=True, page_size=W.page_size,
-                             max_pages=max_pages, num_pages=num_pages)
+                             max_pages=max_pages, num_pages=num_pages, rotate=W.rotate)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev, page_table=torch.from_numpy(table))
         n_max = int(lens.max())
         K = torch.zeros((W.B, W.Hkv, n_max, 128), dtype=torch.bfloat16, device=self.dev)
@@ -637,7 +637,7 @@ class OracleUnit:
         K = synth.keys(w, b, b + 1, h, h + 1, 0, pre + 1)
         V = synth.values(w, b, b + 1, h, h + 1, 0, pre + 1)
         cap = (pre + 1 + 127) // 128 * 128
-        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap)
+        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate)
         calib = w.k_scheme in CALIBRATED or w.v_scheme in CALIBRATED
         self.oc.append(K[:, :, :pre], V[:, :, :pre], w.bf16, calibrate=calib)
         self.saved = (self.oc.c.len, self.oc.c.res)
@@ -726,6 +726,7 @@ def main():
               "k_scheme": w.k_scheme, "v_scheme": w.v_scheme,
               "context": (f"uniform {w.len_lo}..{w.len_hi}" if w.paged else w.prefill_tokens()),
               "layout": "paged/16" if w.paged else "dense",
+              "rotation": "walsh-hadamard" if w.rotate else "none",
               "step": ("decode only" if w.name == "tiny_int8" else "append 1 token per sequence + decode"),
               "l2": "flushed before every timed step (256 MiB write, then 256 MiB read), outside the event interval",
               "parallelism": f"replicas x{args.gpus}"}

@@ -97,6 +97,8 @@ kvq_status kvq_validate(const kvq_cache_desc* d) {
   if (!valid_scheme(d->k_scheme) || !valid_scheme(d->v_scheme)) return KVQ_ERR_INVALID_ARG;
   if (d->layout != KVQ_DENSE && d->layout != KVQ_PAGED) return KVQ_ERR_INVALID_ARG;
   const bool kivi_k = is_kivi(d->k_scheme), kivi_v = is_kivi(d->v_scheme);
+  if (d->rotation != KVQ_ROTATE_NONE && d->rotation != KVQ_ROTATE_HADAMARD) return KVQ_ERR_INVALID_ARG;
+  if (d->rotation != KVQ_ROTATE_NONE && (kivi_k || kivi_v)) return KVQ_ERR_UNSUPPORTED;
   if (kivi_k || kivi_v) {
     if (d->k_scheme != d->v_scheme) return KVQ_ERR_UNSUPPORTED;
     if (d->layout == KVQ_PAGED) return KVQ_ERR_UNSUPPORTED;
@@ -236,6 +238,7 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   p.page_table = d->page_table;
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
+  p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
   const cudaError_t e = launch_append(p, workspace, mode, r_old, flushed, r_new, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return from_cuda(e);
   if (!paged) {
@@ -281,6 +284,7 @@ kvq_status kvq_dequantize(const kvq_cache_desc* d, int32_t which, float* out, in
   p.page_table = d->page_table;
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
+  p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
   p.out = out;
   return from_cuda(launch_dequantize(p, static_cast<cudaStream_t>(stream)));
 }
@@ -335,6 +339,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   p.page_table = d->page_table;
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
+  p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
   p.q = q;
   p.q_bf16 = q_dtype == KVQ_BF16;
   p.softmax_scale = softmax_scale;

@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(256) calib_reduce_kernel(AppendParams p, uint3
   for (int t = t_begin + rl; t < t_end; t += 16) {
     float v[8];
     load8<kBf16>(x, (((size_t)b * p.H + h) * (size_t)p.n_new + t) * kHeadDim + lane8 * 8, v);
+    if (p.rotate) fwht_row16(v, 0xFFFFu << (threadIdx.x & 16), lane8);  // the half warp shares t
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (asym) {
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
     for (int it = 0; it < kR; ++it) {
       float x[8];
       in[it].unpack(x);
+      if (p.rotate) fwht_row16(x, 0xFFFFu << (threadIdx.x & 16), lane8);
       // per-token scale: absmax over the 16 lanes of this row (a half warp)
       float tok_s = 0.0f;
       if (scheme == KVQ_INT8_SYM_PER_TOKEN) {
@@ -1043,6 +1045,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
       }
     }
   }
+  if (p.rotate) fwht_row16(y, 0xFFFFu << (threadIdx.x & 16), lane8);  // back from the rotated domain
   float4* o = reinterpret_cast<float4*>(p.out + (size_t)r * kHeadDim + lane8 * 8);
   o[0] = make_float4(y[0], y[1], y[2], y[3]);
   o[1] = make_float4(y[4], y[5], y[6], y[7]);

@@ -992,6 +992,20 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
         q_s[q_off(j, dd)] = v;
       }
       named_sync(1, kCW * 32);
+      if (p.rotate) {  // H q: butterflies of span 1 .. 64 over the staged rows, then 1/sqrt(128)
+        for (int h = 1; h < kHeadDim; h <<= 1) {
+          for (int idx = tid; idx < 8 * kHeadDim / 2; idx += kCW * 32) {
+            const int j = idx >> 6, i = idx & 63;
+            const int lo = ((i & ~(h - 1)) << 1) | (i & (h - 1));
+            const float a = q_s[q_off(j, lo)], b = q_s[q_off(j, lo + h)];
+            q_s[q_off(j, lo)] = a + b;
+            q_s[q_off(j, lo + h)] = a - b;
+          }
+          named_sync(1, kCW * 32);
+        }
+        for (int idx = tid; idx < 8 * kHeadDim; idx += kCW * 32) q_s[q_off(idx >> 7, idx & 127)] *= kInvSqrt128;
+        named_sync(1, kCW * 32);
+      }
 #pragma unroll
       for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
@@ -1011,7 +1025,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
           eq = build_q_s4(q_s, g, c, S.qh, S.ql);
         else
           eq = build_q<C::kKFmt>(q_s, fold, nullptr, g, c, S.qh, S.ql);
-        S.qsplit = (C::kKFold == FOLD_CHANNEL) || !p.q_bf16;
+        S.qsplit = (C::kKFold == FOLD_CHANNEL) || !p.q_bf16 || p.rotate;
         float mul = sc_log2 * pow2i(-eq);
         if constexpr (C::kKFold == FOLD_TENSOR) mul *= p.k_scale[0];
         S.kmul = mul;
@@ -1198,6 +1212,11 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
   if (M != kNegInf && L > 0.0f) {
     ov = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
     lse = (M + log2f(L)) * 0.69314718055994531f;
+  }
+  if (p.rotate) {  // sum p (H v) = H (sum p v): rotate the output back
+    float r[4] = {ov.x, ov.y, ov.z, ov.w};
+    fwht_row32(r, lane);
+    ov = make_float4(r[0], r[1], r[2], r[3]);
   }
   reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + hq) * kHeadDim)[lane] = ov;
   if (lane == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;

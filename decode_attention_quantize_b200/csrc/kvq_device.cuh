@@ -204,6 +204,61 @@ __device__ __forceinline__ float quot(float x, float s, float y, float& q) {
 // s with a normal reciprocal and room for the correction's residual: 2^-60 .. 2^60
 __device__ __forceinline__ bool quot_range(float s) { return s >= 8.67361738e-19f && s <= 1.15292150e+18f; }
 
+// ------------------------------------------------------------------ Walsh-Hadamard rotation
+// Normalised transform H/sqrt(128) of a 128-value row, as butterflies of span 1, 2, ..., 64
+// ((a, b) -> (a + b, a - b), a the lower index) and a final multiply by the fp32 value of
+// 1/sqrt(128): every output is the same sequence of fp32 operations in any thread layout.
+constexpr float kInvSqrt128 = 0.0883883476483184405f;
+
+// Row held by the 16 lanes of a half warp, lane l holding values 8l .. 8l + 7 (mask: the
+// half warp's lanes, which must all take part).
+__device__ __forceinline__ void fwht_row16(float (&x)[8], unsigned mask, int lane16) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (!(k & h)) {
+        const float a = x[k], b = x[k + h];
+        x[k] = a + b;
+        x[k + h] = a - b;
+      }
+#pragma unroll
+  for (int m = 1; m < 16; m <<= 1) {
+    const bool upper = (lane16 & m) != 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float y = __shfl_xor_sync(mask, x[k], m);
+      x[k] = upper ? y - x[k] : x[k] + y;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x[k] *= kInvSqrt128;
+}
+
+// Row held by a whole warp, lane l holding values 4l .. 4l + 3.
+__device__ __forceinline__ void fwht_row32(float (&x)[4], int lane) {
+#pragma unroll
+  for (int h = 1; h < 4; h <<= 1)
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (!(k & h)) {
+        const float a = x[k], b = x[k + h];
+        x[k] = a + b;
+        x[k + h] = a - b;
+      }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float y = __shfl_xor_sync(0xffffffffu, x[k], m);
+      x[k] = upper ? y - x[k] : x[k] + y;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] *= kInvSqrt128;
+}
+
 // ------------------------------------------------------------------ reductions
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

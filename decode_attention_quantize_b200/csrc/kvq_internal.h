@@ -32,6 +32,7 @@ struct AppendParams {
   const int32_t* page_table;
   int32_t* seq_lens;
   uint32_t* status;
+  int rotate;  // rows rotated by the normalised Walsh-Hadamard transform before quantization
 };
 
 struct DequantParams {
@@ -47,6 +48,7 @@ struct DequantParams {
   const int32_t* seq_lens;
   uint32_t* status;
   float* out;
+  int rotate;  // rotate each dequantized row back
 };
 
 struct DecodeParams {
@@ -80,6 +82,7 @@ struct DecodeParams {
   int n_pairs;
   int ts;                       // tokens per quantized tile of the chosen kernel
   int nq, nr;                   // dense: quantized / residual tiles per pair
+  int rotate;                   // rotate each query, and each output back
 };
 
 constexpr int kMaxCtas = 1024;

@@ -30,6 +30,7 @@ FP8_E5M2_PER_TENSOR = 7
 INT4_SYM_PER_GROUP = 8
 KVQ_F32, KVQ_BF16 = 0, 1
 KVQ_DENSE, KVQ_PAGED = 0, 1
+KVQ_ROTATE_NONE, KVQ_ROTATE_HADAMARD = 0, 1
 KVQ_APPEND_CALIBRATE = 0x1
 KVQ_APPEND_RESCALE = 0x2
 KVQ_DEV_BAD_PAGE, KVQ_DEV_BAD_LENGTH, KVQ_DEV_TIMEOUT = 0x1, 0x2, 0x4
@@ -58,6 +59,7 @@ class KvqDesc(ctypes.Structure):
         ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("dev_status", ctypes.c_void_p),
+        ("rotation", ctypes.c_int32),
     ]
 
 
@@ -231,6 +233,7 @@ class CacheSpec:
     max_pages: int = 0
     num_pages: int = 0
     D: int = 128
+    rotate: bool = False         # Walsh-Hadamard rotation of K, V and Q (not with KIVI)
 
 
 class RescaleSchedule:
@@ -298,6 +301,7 @@ class QuantizedKVCache:
         d.capacity = s.capacity
         d.page_size, d.max_pages_per_seq, d.num_pages = s.page_size, s.max_pages, s.num_pages
         d.group_size, d.residual_cap = 32, 128
+        d.rotation = KVQ_ROTATE_HADAMARD if s.rotate else KVQ_ROTATE_NONE
         for name, tensor in self.t.items():
             setattr(d, name, tensor.data_ptr())
         self.desc = d

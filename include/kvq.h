@@ -28,7 +28,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 1
+#define KVQ_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define KVQ_API __attribute__((visibility("default")))
@@ -84,6 +84,13 @@ typedef enum kvq_scheme {
 typedef enum kvq_dtype { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
 typedef enum kvq_layout { KVQ_DENSE = 0, KVQ_PAGED = 1 } kvq_layout;
 
+/* Online rotation of K, V and Q ("KV Cache Quantization in Production LLM Serving",
+ * llms.blog §5, QuaRot / RotateKV): the normalised Walsh-Hadamard transform H/sqrt(128) over
+ * head_dim, orthogonal and symmetric, so (H q).(H k) = q.k and H (sum p H v) = sum p v. Rows
+ * are transformed in fp32 by butterflies of span 1, 2, ..., 64 and a final multiply by the
+ * fp32 value of 1/sqrt(128). */
+typedef enum kvq_rotation { KVQ_ROTATE_NONE = 0, KVQ_ROTATE_HADAMARD = 1 } kvq_rotation;
+
 /* kvq_quantize_append flags */
 #define KVQ_APPEND_CALIBRATE 0x1u  /* recompute per-tensor / per-channel scales from this block */
 #define KVQ_APPEND_RESCALE 0x2u    /* merge this block's scales into the cached ones, requantize */
@@ -134,6 +141,9 @@ typedef struct kvq_cache_desc {
   int32_t* page_table;
   int32_t* seq_lens;
   uint32_t* dev_status;
+  int32_t rotation;          /* kvq_rotation: KVQ_ROTATE_HADAMARD rotates every K/V row before it
+                                is quantized, each query before attention and each output and
+                                dequantized row back (not with KIVI schemes) */
 } kvq_cache_desc;
 
 typedef struct kvq_footprint {

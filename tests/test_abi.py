@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol():
     for name in _declared():
         assert hasattr(lib, name), name
     assert sorted(kvq.EXPORTS) == _declared()
-    assert lib.kvq_abi_version() == 1
+    assert lib.kvq_abi_version() == 2
 
 
 def _desc(**kw):
@@ -55,6 +55,9 @@ def test_validation_is_host_side():
         (dict(capacity=200), kvq.KVQ_ERR_INVALID_ARG),
         (dict(k_scheme=9), kvq.KVQ_ERR_INVALID_ARG),
         (dict(k_scheme=5, v_scheme=6), kvq.KVQ_ERR_UNSUPPORTED),
+        (dict(rotation=2), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(rotation=1, k_scheme=5, v_scheme=5), kvq.KVQ_ERR_UNSUPPORTED),   # no rotation with KIVI
+        (dict(rotation=1, k_scheme=8, v_scheme=8, group_size=64), kvq.KVQ_ERR_UNSUPPORTED),
         (dict(k_codes=None), kvq.KVQ_ERR_INVALID_ARG),
         (dict(k_codes=0x10004), kvq.KVQ_ERR_INVALID_ARG),   # not 16-byte aligned
         (dict(layout=1, page_size=16, max_pages_per_seq=4, num_pages=8), kvq.KVQ_ERR_INVALID_ARG),

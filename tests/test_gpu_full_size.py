@@ -74,7 +74,8 @@ def _dense_full(name):
     cap = (total + 127) // 128 * 128
     K = synth.keys(w, 0, w.B, 0, w.Hkv, 0, total)
     V = synth.values(w, 0, w.B, 0, w.Hkv, 0, total)
-    gc = kvq.QuantizedKVCache(kvq.CacheSpec(w.B, w.Hq, w.Hkv, w.k_scheme, w.v_scheme, capacity=cap))
+    gc = kvq.QuantizedKVCache(kvq.CacheSpec(w.B, w.Hq, w.Hkv, w.k_scheme, w.v_scheme, capacity=cap,
+                                            rotate=w.rotate))
     calib = w.k_scheme in CAL or w.v_scheme in CAL
     gc.append(H.dev(K[:, :, :pre], w.bf16), H.dev(V[:, :, :pre], w.bf16), calibrate=calib)
     if append:
@@ -86,14 +87,14 @@ def _dense_full(name):
     assert gc.status()[0] == 0
     full_cal = None
     if calib:
-        full_cal = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, cap=128)
+        full_cal = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, cap=128, rotate=w.rotate)
         full_cal.calibrate(K[:, :, :pre], V[:, :, :pre], w.bf16)
         for side in ("k", "v"):
             assert np.array_equal(H.np_of(gc[side + "_scale"]).reshape(-1)[:full_cal[side + "_scale"].size]
                                   .view(np.uint32), full_cal[side + "_scale"].reshape(-1).view(np.uint32))
     refs, gots = [], []
     for b, h in _pairs(w):
-        oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap)
+        oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate)
         if full_cal is not None:
             _copy_scales(oc, full_cal, h)
         oc.append(K[b:b + 1, h:h + 1, :pre], V[b:b + 1, h:h + 1, :pre], w.bf16)
@@ -119,6 +120,10 @@ def test_e5m2_8b_full():
 
 def test_int4g_70b_full():
     _dense_full("int4g_70b")
+
+
+def test_int4g_rot_70b_full():
+    _dense_full("int4g_rot_70b")
 
 
 def test_kivi4_70b_full():

@@ -255,6 +255,41 @@ def test_int4_group_paged(ps):
     assert gc.status()[0] == 0
 
 
+# ------------------------------------------------------------------ Walsh-Hadamard rotation
+# K/V rows rotated before quantization (codes and scales bit for bit), the query rotated and
+# the output rotated back in decode, dequantized rows rotated back.
+@pytest.mark.parametrize("ks,vs", [
+    (S.INT4_SYM_PER_GROUP, S.INT4_SYM_PER_GROUP), (S.INT8_SYM_PER_TOKEN, S.INT8_SYM_PER_TOKEN),
+    (S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.INT8_SYM_PER_CHANNEL, S.UINT8_ASYM_PER_CHANNEL),
+])
+def test_rotation_dense(ks, vs):
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=ks, vs=vs, prefill=300, steps=2, outlier=100.0, rotate=True)
+
+
+def test_rotation_bulk_fp32_and_gqa():
+    H.dense_case(B=4, Hq=8, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=9600, steps=1,
+                 rotate=True)
+    H.dense_case(B=1, Hq=4, Hkv=1, ks=S.INT8_SYM_PER_TOKEN, vs=S.INT8_SYM_PER_TOKEN, prefill=257, steps=1,
+                 bf16=False, rope=0.0, rotate=True)
+    H.dense_case(B=2, Hq=32, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=130, steps=1,
+                 rotate=True)
+
+
+def test_rotation_paged_and_dequantize():
+    B, Hq, Hkv, sch = 4, 16, 4, S.INT4_SYM_PER_GROUP
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, sch, sch, lens=[37, 100, 5, 64], page_size=16,
+                                                    steps=0, rotate=True)
+    oc.append(K, V, True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc, "rotated paged prefill")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), True, "rotated paged decode")
+    for which in (0, 1):
+        got = gc.dequantize(which, 101).cpu().numpy()
+        ref = oc.dequantize(which, 101)
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), f"rotated dequantize side {which}"
+
+
 # ------------------------------------------------------------------ rescaling append
 # Scales merged with each block's (they only grow) and the cached codes whose scale changed
 # requantized, bit for bit against the oracle; blocks inside the range, a grown single
