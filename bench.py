@@ -61,14 +61,14 @@ def row_bytes(scheme):
     return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2, synth.INT4_SYM_PER_GROUP: 4}.get(scheme, 8) // 8
 
 
-def meta_bytes_per_token(scheme, Hkv):
+def meta_bytes_per_token(scheme, Hkv, group=32):
     """Per-token-row metadata bytes that decode must read (K or V side)."""
     if scheme == synth.INT8_SYM_PER_TOKEN:
         return 4.0
     if scheme in (synth.KIVI_INT4, synth.KIVI_INT2):
         return 8.0 * 128 / 32  # fp32 (scale, min) per 32 elements
     if scheme == synth.INT4_SYM_PER_GROUP:
-        return 4.0 * 128 / 32  # fp32 scale per 32 channels
+        return 4.0 * 128 / group  # fp32 scale per group of channels
     return 0.0
 
 
@@ -86,7 +86,7 @@ def decode_bytes(w, lens_q, len_res=0):
     """Algorithmic bytes of one decode call: codes + metadata + residual + Q + out."""
     rows = int(np.sum(lens_q)) * w.Hkv
     b = rows * (row_bytes(w.k_scheme) + row_bytes(w.v_scheme))
-    b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv) + meta_bytes_per_token(w.v_scheme, w.Hkv))
+    b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv, w.group) + meta_bytes_per_token(w.v_scheme, w.Hkv, w.group))
     b += fixed_meta_bytes(w.k_scheme, w.Hkv) + fixed_meta_bytes(w.v_scheme, w.Hkv)
     b += w.B * w.Hkv * len_res * 128 * 2 * 2
     b += w.B * w.Hq * 128 * (2 if w.bf16 else 4)  # Q
@@ -103,7 +103,7 @@ def append_bytes(w, n=1):
         b += rows * 128 * 2 * 2  # bf16 residual write
     else:
         b += rows * (row_bytes(w.k_scheme) + row_bytes(w.v_scheme))
-        b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv) + meta_bytes_per_token(w.v_scheme, w.Hkv))
+        b += rows * (meta_bytes_per_token(w.k_scheme, w.Hkv, w.group) + meta_bytes_per_token(w.v_scheme, w.Hkv, w.group))
     return float(b)
 
 
@@ -251,7 +251,7 @@ class GpuWorkload:
         self.append_token = W.name != "tiny_int8"  # the tiny configuration decodes without appending
         pre = total - 1 if self.append_token else total
         cap = (total + 127) // 128 * 128
-        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap, rotate=W.rotate)
+        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap, rotate=W.rotate, group=W.group)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev)
         self.calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
         self.pre_k = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, 0, pre), W.bf16)
@@ -290,7 +290,7 @@ class GpuWorkload:
             b += W.B * W.Hkv * self.cache.desc.num_residual * 128 * 2 * 2
         else:
             b += rows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme))
-            b += rows * (meta_bytes_per_token(W.k_scheme, W.Hkv) + meta_bytes_per_token(W.v_scheme, W.Hkv))
+            b += rows * (meta_bytes_per_token(W.k_scheme, W.Hkv, W.group) + meta_bytes_per_token(W.v_scheme, W.Hkv, W.group))
         return float(b)
 
     def time_prefill(self, flush, stream, reps=3):
@@ -356,7 +356,7 @@ class GpuWorkload:
             table[b, :n] = perm[off:off + n]
             off += n
         spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, paged=True, page_size=W.page_size,
-                             max_pages=max_pages, num_pages=num_pages, rotate=W.rotate)
+                             max_pages=max_pages, num_pages=num_pages, rotate=W.rotate, group=W.group)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev, page_table=torch.from_numpy(table))
         n_max = int(lens.max())
         K = torch.zeros((W.B, W.Hkv, n_max, 128), dtype=torch.bfloat16, device=self.dev)
@@ -637,7 +637,7 @@ class OracleUnit:
         K = synth.keys(w, b, b + 1, h, h + 1, 0, pre + 1)
         V = synth.values(w, b, b + 1, h, h + 1, 0, pre + 1)
         cap = (pre + 1 + 127) // 128 * 128
-        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate)
+        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group)
         calib = w.k_scheme in CALIBRATED or w.v_scheme in CALIBRATED
         self.oc.append(K[:, :, :pre], V[:, :, :pre], w.bf16, calibrate=calib)
         self.saved = (self.oc.c.len, self.oc.c.res)
@@ -727,6 +727,7 @@ def main():
               "context": (f"uniform {w.len_lo}..{w.len_hi}" if w.paged else w.prefill_tokens()),
               "layout": "paged/16" if w.paged else "dense",
               "rotation": "walsh-hadamard" if w.rotate else "none",
+              "group": w.group,
               "step": ("decode only" if w.name == "tiny_int8" else "append 1 token per sequence + decode"),
               "l2": "flushed before every timed step (256 MiB write, then 256 MiB read), outside the event interval",
               "parallelism": f"replicas x{args.gpus}"}

@@ -52,7 +52,8 @@ uint64_t scale_elems(const kvq_cache_desc* d, int side) {
     case KVQ_INT8_SYM_PER_CHANNEL:
     case KVQ_UINT8_ASYM_PER_CHANNEL: return H * D;
     case KVQ_INT4_SYM_PER_GROUP:
-      return (paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity) * (D / 32);
+      return (paged ? (uint64_t)d->num_pages * H * d->page_size : B * H * (uint64_t)d->capacity) *
+             (D / (uint64_t)d->group_size);
     default:
       return side == 0 ? B * H * (uint64_t)(d->capacity / 32) * D : B * H * (uint64_t)d->capacity * (D / 32);
   }
@@ -108,7 +109,8 @@ kvq_status kvq_validate(const kvq_cache_desc* d) {
       return KVQ_ERR_INVALID_ARG;
     if (d->num_residual < 0 || d->num_residual > d->residual_cap) return KVQ_ERR_INVALID_ARG;
   }
-  if ((d->k_scheme == KVQ_INT4_SYM_PER_GROUP || d->v_scheme == KVQ_INT4_SYM_PER_GROUP) && d->group_size != 32)
+  if ((d->k_scheme == KVQ_INT4_SYM_PER_GROUP || d->v_scheme == KVQ_INT4_SYM_PER_GROUP) &&
+      d->group_size != 32 && d->group_size != 64 && d->group_size != 128)
     return KVQ_ERR_UNSUPPORTED;
   if (d->layout == KVQ_DENSE) {
     if (d->capacity < 128 || d->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;
@@ -149,7 +151,7 @@ kvq_status kvq_cache_bytes(const kvq_cache_desc* d, kvq_footprint* out) {
     if (needs_zp(s)) bytes += (uint64_t)d->num_kv_heads * d->head_dim;  // uint8 zero points
     meta += bytes;
     if (s == KVQ_INT8_SYM_PER_TOKEN) per_token_meta += 4.0;
-    if (s == KVQ_INT4_SYM_PER_GROUP) per_token_meta += 4.0 * d->head_dim / 32.0;  // fp32 scale per group
+    if (s == KVQ_INT4_SYM_PER_GROUP) per_token_meta += 4.0 * d->head_dim / d->group_size;  // fp32 per group
     if (is_kivi(s)) per_token_meta += 8.0 * d->head_dim / 32.0;  // (scale, min) per 32 tokens or channels
   }
   f.meta_bytes = meta;
@@ -239,6 +241,7 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
   p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
+  p.group = d->group_size;
   const cudaError_t e = launch_append(p, workspace, mode, r_old, flushed, r_new, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return from_cuda(e);
   if (!paged) {
@@ -285,6 +288,7 @@ kvq_status kvq_dequantize(const kvq_cache_desc* d, int32_t which, float* out, in
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
   p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
+  p.group = d->group_size;
   p.out = out;
   return from_cuda(launch_dequantize(p, static_cast<cudaStream_t>(stream)));
 }
@@ -307,7 +311,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   const size_t need = kvq_decode_workspace_bytes(d);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KVQ_ERR_WORKSPACE;
   const bool paged = d->layout == KVQ_PAGED;
-  if (!decode_supported(d->k_scheme, d->v_scheme, paged)) return KVQ_ERR_UNSUPPORTED;
+  if (!decode_supported(d->k_scheme, d->v_scheme, paged, d->group_size)) return KVQ_ERR_UNSUPPORTED;
   const int G = d->num_q_heads / d->num_kv_heads;
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
@@ -340,6 +344,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   p.seq_lens = d->seq_lens;
   p.status = d->dev_status;
   p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
+  p.group = d->group_size;
   p.q = q;
   p.q_bf16 = q_dtype == KVQ_BF16;
   p.softmax_scale = softmax_scale;

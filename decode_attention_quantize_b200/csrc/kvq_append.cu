@@ -356,19 +356,62 @@ __device__ __forceinline__ bool asym_row(const float (&x)[8], const Scales8& sc,
 
 constexpr bool is_per_channel(int s) { return s == KVQ_INT8_SYM_PER_CHANNEL || s == KVQ_UINT8_ASYM_PER_CHANNEL; }
 
+// Two fp32 lanes in one 64-bit register for the packed f32x2 arithmetic of sm_100 (each lane is
+// the same correctly rounded IEEE operation as its scalar form).
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Eight INT4 codes of a thread's slice of one group: clamp(rne(x / s), -8, 7) as two's-
-// complement nibbles, lower channel in the low bits; a zero group gives zero codes.
+// complement nibbles, lower channel in the low bits; a zero group gives zero codes. Since
+// s = absmax / 7 rounded, |x / s| <= 7 (1 + 2^-23), so rne never leaves [-7, 7] and the clamp
+// never acts; RN(z + 1.5 * 2^23) holds rne(z) in its low bits, whose low four bits are the
+// two's-complement nibble. The quotients are the fma-corrected ones, two per packed op.
 __device__ __forceinline__ uint32_t int4_codes(const float (&x)[8], float s) {
   if (s == 0.0f) return 0u;
-  const float y = __frcp_rn(s);
-  const bool fast = quot_range(s);
   uint32_t w = 0u;
+  if (quot_range(s)) {
+    const float y = __frcp_rn(s);
+    const f32x2 y2 = pk2(y, y), ns2 = pk2(-s, -s), m2 = pk2(kRoundMagic, kRoundMagic);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const f32x2 x2 = pk2(x[2 * k], x[2 * k + 1]);
+      const f32x2 q = mul2(x2, y2);
+      const f32x2 t = add2(fma2(fma2(q, ns2, x2), y2, q), m2);  // RN(q - e y) + magic
+      float t0, t1;
+      upk2(t, t0, t1);
+      w |= ((__float_as_uint(t0) & 0xFu) << (8 * k)) | ((__float_as_uint(t1) & 0xFu) << (8 * k + 4));
+    }
+    return w;
+  }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    float q;
-    const float z = fast ? quot(x[k], s, y, q) : __fdiv_rn(x[k], s);  // |z| <= 7 (1 + 2^-23)
-    const float c = fminf(fmaxf(rintf(z), -8.0f), 7.0f);
-    w |= ((uint32_t)(int)c & 0xFu) << (4 * k);
+    const float z = __fdiv_rn(x[k], s);
+    w |= (__float_as_uint(__fadd_rn(z, kRoundMagic)) & 0xFu) << (4 * k);
   }
   return w;
 }
@@ -471,13 +514,12 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
         for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         tok_s = __fdiv_rn(m, 127.0f);
       }
-      // INT4 per group: absmax over the four lanes (32 channels) of the group
+      // INT4 per group: absmax over the group / 8 lanes (4, 8 or 16) of the group
       if (scheme == KVQ_INT4_SYM_PER_GROUP) {
         float m = 0.0f;
 #pragma unroll
         for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(x[k]));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        for (int o = 1; o < p.group / 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         tok_s = __fdiv_rn(m, 7.0f);
       }
       if (!act[it]) continue;
@@ -491,7 +533,8 @@ __global__ void __launch_bounds__(256, (is_per_channel(KS) || is_per_channel(VS)
       if (scheme == KVQ_INT4_SYM_PER_GROUP) {
         uint8_t* dst = static_cast<uint8_t*>(side ? p.v_codes : p.k_codes) + row * (kHeadDim / 2);
         *reinterpret_cast<uint32_t*>(dst + lane8 * 4) = int4_codes(x, tok_s);
-        if ((lane8 & 3) == 0) scale[row * (kHeadDim / 32) + (lane8 >> 2)] = tok_s;
+        const int lanes = p.group / 8;  // lanes per group
+        if ((lane8 & (lanes - 1)) == 0) scale[row * (kHeadDim / p.group) + lane8 / lanes] = tok_s;
         continue;
       }
       if (per_channel && h != chan_head) {
@@ -720,35 +763,6 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
   return r;
 }
 
-// Two fp32 lanes in one 64-bit register for the packed f32x2 arithmetic of sm_100 (each lane is
-// the same correctly rounded IEEE operation as its scalar form).
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pk2(float a, float b) {
-  f32x2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void upk2(f32x2 v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
-__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
-  f32x2 r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-  f32x2 r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-  f32x2 r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
-  f32x2 r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
 
 // Two KIVI codes at once: d = RN(v - min), then the division-free quotient of `quot` in its
 // residual form r = RN(d - q * s) (the same values; zero signs do not reach integer codes),
@@ -1029,7 +1043,7 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
               v = __fmul_rn((float)(q - (int)p.zp[h * kHeadDim + d]), p.scale[h * kHeadDim + d]);
               break;
             case KVQ_INT4_SYM_PER_GROUP:
-              v = __fmul_rn((float)(q >= 8 ? q - 16 : q), p.scale[row * (kHeadDim / 32) + d / 32]);
+              v = __fmul_rn((float)(q >= 8 ? q - 16 : q), p.scale[row * (kHeadDim / p.group) + d / p.group]);
               break;
             default: {  // KIVI
               size_t m;

@@ -65,9 +65,11 @@ __host__ __device__ constexpr int fold_of(int s) {
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 __host__ __device__ constexpr int rup(int a, int m) { return (a + m - 1) / m * m; }
 
-template <int KS, int VS, bool PAGED>
+// NG: scales per token row of an INT4 per-group side (4, 2 or 1 for groups of 32, 64, 128)
+template <int KS, int VS, bool PAGED, int NG = 4>
 struct Cfg {
   static constexpr bool kPaged = PAGED;
+  static constexpr int kNG = NG;
   static constexpr int kKFmt = fmt_of(KS), kVFmt = fmt_of(VS);
   static constexpr int kKFold = fold_of(KS), kVFold = fold_of(VS);
   static constexpr bool kKivi = kKFold == FOLD_KIVI;
@@ -83,10 +85,10 @@ struct Cfg {
   static constexpr int kOffV = kTS * kKRow;     // multiple of 1024 (swizzle atom)
   static constexpr int kOffKM = kOffV + kTS * kVRow;
   static constexpr int kKMeta = kKivi ? (kTS / 32) * kHeadDim * 4 * 2
-                                : (kKFold == FOLD_TOKEN ? kTS * 4 : (kKFold == FOLD_GROUP ? kTS * 16 : 0));
+                                : (kKFold == FOLD_TOKEN ? kTS * 4 : (kKFold == FOLD_GROUP ? kTS * NG * 4 : 0));
   static constexpr int kOffVM = kOffKM + kKMeta;
   static constexpr int kVMeta = kKivi ? kTS * 4 * 4 * 2
-                                : (kVFold == FOLD_TOKEN ? kTS * 4 : (kVFold == FOLD_GROUP ? kTS * 16 : 0));
+                                : (kVFold == FOLD_TOKEN ? kTS * 4 : (kVFold == FOLD_GROUP ? kTS * NG * 4 : 0));
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
@@ -270,8 +272,8 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       } else {
         if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
         if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
-        if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * 4, C::kKMeta, bar);
-        if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * 4, C::kVMeta, bar);
+        if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * C::kNG, C::kKMeta, bar);
+        if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * C::kNG, C::kVMeta, bar);
       }
     } else {
       // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
@@ -300,8 +302,8 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       uint32_t per_page = ps * (C::kKRow + C::kVRow);
       if constexpr (C::kKFold == FOLD_TOKEN) per_page += ps * 4;
       if constexpr (C::kVFold == FOLD_TOKEN) per_page += ps * 4;
-      if constexpr (C::kKFold == FOLD_GROUP) per_page += ps * 16;
-      if constexpr (C::kVFold == FOLD_GROUP) per_page += ps * 16;
+      if constexpr (C::kKFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
+      if constexpr (C::kVFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
       mbar_arrive_expect_tx(bar, nvalid * per_page);
 #pragma unroll
       for (int i = 0; i < C::kTS / 16; ++i) {
@@ -312,9 +314,9 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
         if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar);
         if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar);
         if constexpr (C::kKFold == FOLD_GROUP)
-          bulk_g2s(sb + C::kOffKM + i * ps * 16, p.k_scale + prow * 4, ps * 16, bar);
+          bulk_g2s(sb + C::kOffKM + i * ps * C::kNG * 4, p.k_scale + prow * C::kNG, ps * C::kNG * 4, bar);
         if constexpr (C::kVFold == FOLD_GROUP)
-          bulk_g2s(sb + C::kOffVM + i * ps * 16, p.v_scale + prow * 4, ps * 16, bar);
+          bulk_g2s(sb + C::kOffVM + i * ps * C::kNG * 4, p.v_scale + prow * C::kNG, ps * C::kNG * 4, bar);
       }
     }
   }
@@ -520,6 +522,21 @@ __device__ __forceinline__ int build_q_s4(const float* q_s, int g, int c, uint32
   return eq;
 }
 
+// The value scales of token tok for the four 32-channel blocks of a row (KIVI, INT4 per group;
+// groups of 64 or 128 channels repeat each scale over the blocks they cover).
+template <class C>
+__device__ __forceinline__ float4 vscale4(const uint8_t* base, int tok) {
+  if constexpr (C::kKivi || C::kNG == 4) {
+    return lds<float4>(base + C::kOffVM + tok * 16);
+  } else if constexpr (C::kNG == 2) {
+    const float2 s = lds<float2>(base + C::kOffVM + tok * 8);
+    return make_float4(s.x, s.x, s.y, s.y);
+  } else {
+    const float s = lds<float>(base + C::kOffVM + tok * 4);
+    return make_float4(s, s, s, s);
+  }
+}
+
 // ------------------------------------------------------------------ one tile, one warp
 // kMasked: the warp's tokens are not all valid (ragged tail or missing pages).
 template <class C, bool kMasked>
@@ -605,19 +622,25 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       const float* ksc = reinterpret_cast<const float*>(base + C::kOffKM);
       const uint32_t sel = 0x4040u + 0x101u * (uint32_t)c;
       const bool split = S.qsplit;
+      constexpr int kSteps = 8 / C::kNG;  // 16-channel k-steps per group
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
-        float ag[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int grp = 0; grp < C::kNG; ++grp) {
+        float ag[4] = {0.f, 0.f, 0.f, 0.f}, ah[4] = {0.f, 0.f, 0.f, 0.f};  // two chains per group
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int ks = 2 * grp + h2;
-          const uint32_t f0 = s4_byte(word_of(x[grp], 2 * h2), sel), f1 = s4_byte(word_of(y[grp], 2 * h2), sel);
-          const uint32_t f2 = s4_byte(word_of(x[grp], 2 * h2 + 1), sel);
-          const uint32_t f3 = s4_byte(word_of(y[grp], 2 * h2 + 1), sel);
-          mma_16816(ag, f0, f1, f2, f3, S.qh[ks][0], S.qh[ks][1]);
-          if (split) mma_16816(ag, f0, f1, f2, f3, S.ql[ks][0], S.ql[ks][1]);
+        for (int st2 = 0; st2 < kSteps; ++st2) {
+          const int ks = grp * kSteps + st2, ch = ks >> 1, h2 = ks & 1;  // 32-channel chunk, half
+          const uint32_t f0 = s4_byte(word_of(x[ch], 2 * h2), sel), f1 = s4_byte(word_of(y[ch], 2 * h2), sel);
+          const uint32_t f2 = s4_byte(word_of(x[ch], 2 * h2 + 1), sel);
+          const uint32_t f3 = s4_byte(word_of(y[ch], 2 * h2 + 1), sel);
+          float(&acc_k)[4] = (kSteps > 2 && (st2 & 1)) ? ah : ag;
+          mma_16816(acc_k, f0, f1, f2, f3, S.qh[ks][0], S.qh[ks][1]);
+          if (split) mma_16816(acc_k, f0, f1, f2, f3, S.ql[ks][0], S.ql[ks][1]);
         }
-        const float s0 = ksc[r0 * 4 + grp], s1 = ksc[r1 * 4 + grp];
+        if constexpr (kSteps > 2) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ag[k] += ah[k];
+        }
+        const float s0 = ksc[r0 * C::kNG + grp], s1 = ksc[r1 * C::kNG + grp];
         float(&dst)[4] = (grp & 1) ? a1 : a0;
         dst[0] = fmaf(s0, ag[0], dst[0]);
         dst[1] = fmaf(s0, ag[1], dst[1]);
@@ -728,7 +751,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
   // Read from shared memory where it is used, so the 16 (KIVI: 32) values are not held live.
   auto vscale = [&](int tok, int j) -> float {
     if (!tok_ok(tok)) return 0.0f;
-    if constexpr (C::kGroupV) return reinterpret_cast<const float*>(base + C::kOffVM)[tok * 4 + j];
+    if constexpr (C::kGroupV) return reinterpret_cast<const float*>(base + C::kOffVM)[tok * C::kNG + j * C::kNG / 4];
     return reinterpret_cast<const float*>(base + C::kOffVM)[tok];
   };
   int evn = 15;
@@ -741,7 +764,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         const int tok = tok_base + sb * 16 + 2 * c + (k & 1) + 8 * (k >> 1);
         const bool ok = tok_ok(tok);
         if constexpr (C::kGroupV) {
-          const float4 s4 = lds<float4>(base + C::kOffVM + tok * 16);
+          const float4 s4 = vscale4<C>(base, tok);
           const float m4 = fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w));
           smax = fmaxf(smax, ok ? m4 : 0.0f);
         } else {
@@ -829,7 +852,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         s4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (!residual && ok[k]) s4[k] = lds<float4>(base + C::kOffVM + tk[k] * 16);
+        if (!residual && ok[k]) s4[k] = vscale4<C>(base, tk[k]);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -923,11 +946,11 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int KS, int VS, bool PAGED>
-__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED>::kMinBlocks)
+template <int KS, int VS, bool PAGED, int NG>
+__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
-  using C = Cfg<KS, VS, PAGED>;
+  using C = Cfg<KS, VS, PAGED, NG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   grid_dependency_wait();    // the cache, the queries and the plan come from earlier kernels
@@ -1304,18 +1327,18 @@ bool make_map(CUtensorMap* map, const void* base, int row_bytes_, uint64_t rows,
 }
 
 struct Variant {
-  int k, v, paged;
+  int k, v, paged, ng;
   void (*kernel)(const DecodeParams, const CUtensorMap, const CUtensorMap);
   int smem, ts;
 };
 
-template <int KS, int VS, bool PG>
+template <int KS, int VS, bool PG, int NG = 4>
 Variant variant() {
-  using C = Cfg<KS, VS, PG>;
-  return Variant{KS, VS, PG ? 1 : 0, decode_kernel<KS, VS, PG>, C::kSmemBytes, C::kTS};
+  using C = Cfg<KS, VS, PG, NG>;
+  return Variant{KS, VS, PG ? 1 : 0, NG, decode_kernel<KS, VS, PG, NG>, C::kSmemBytes, C::kTS};
 }
 
-constexpr int kNumVariants = 28;
+constexpr int kNumVariants = 32;
 constexpr int kMaxDevices = 64;
 
 const Variant* variants() {
@@ -1346,6 +1369,10 @@ const Variant* variants() {
       variant<KVQ_FP8_E5M2_PER_TENSOR, KVQ_FP8_E5M2_PER_TENSOR, true>(),
       variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, false>(),
       variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, true>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, false, 2>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, true, 2>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, false, 1>(),
+      variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, true, 1>(),
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
   };
@@ -1353,11 +1380,16 @@ const Variant* variants() {
   return table;
 }
 
-const Variant* find_variant(int k, int v, int paged) {
+// ng: scales per row of an INT4 per-group scheme (128 / group size); 4 for the others
+const Variant* find_variant(int k, int v, int paged, int ng) {
   const Variant* table = variants();
   for (int i = 0; i < kNumVariants; ++i)
-    if (table[i].k == k && table[i].v == v && table[i].paged == paged) return &table[i];
+    if (table[i].k == k && table[i].v == v && table[i].paged == paged && table[i].ng == ng) return &table[i];
   return nullptr;
+}
+
+int groups_per_row(int k_scheme, int group) {
+  return (k_scheme == KVQ_INT4_SYM_PER_GROUP && group > 0) ? kHeadDim / group : 4;
 }
 
 int sm_count() {
@@ -1374,12 +1406,12 @@ int sm_count() {
 
 }  // namespace
 
-bool decode_supported(int k_scheme, int v_scheme, int paged) {
-  return find_variant(k_scheme, v_scheme, paged) != nullptr;
+bool decode_supported(int k_scheme, int v_scheme, int paged, int group) {
+  return find_variant(k_scheme, v_scheme, paged, groups_per_row(k_scheme, group)) != nullptr;
 }
 
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
-  const Variant* var = find_variant(p.k_scheme, p.v_scheme, p.paged);
+  const Variant* var = find_variant(p.k_scheme, p.v_scheme, p.paged, groups_per_row(p.k_scheme, p.group));
   if (!var) return cudaErrorNotSupported;
   p.ts = var->ts;
   if (!p.paged) {

@@ -33,6 +33,7 @@ struct AppendParams {
   int32_t* seq_lens;
   uint32_t* status;
   int rotate;  // rows rotated by the normalised Walsh-Hadamard transform before quantization
+  int group;   // INT4 per-group: channels per group (32, 64 or 128)
 };
 
 struct DequantParams {
@@ -49,6 +50,7 @@ struct DequantParams {
   uint32_t* status;
   float* out;
   int rotate;  // rotate each dequantized row back
+  int group;   // INT4 per-group: channels per group
 };
 
 struct DecodeParams {
@@ -83,6 +85,7 @@ struct DecodeParams {
   int ts;                       // tokens per quantized tile of the chosen kernel
   int nq, nr;                   // dense: quantized / residual tiles per pair
   int rotate;                   // rotate each query, and each output back
+  int group;                    // INT4 per-group: channels per group (selects the kernel)
 };
 
 constexpr int kMaxCtas = 1024;
@@ -120,7 +123,7 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 
 // Returns cudaErrorNotSupported when the (k_scheme, v_scheme, layout) pair has no kernel.
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st);
-bool decode_supported(int k_scheme, int v_scheme, int paged);
+bool decode_supported(int k_scheme, int v_scheme, int paged, int group);
 bool append_pair_supported(int k_scheme, int v_scheme);
 
 }  // namespace kvq

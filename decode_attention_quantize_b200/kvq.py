@@ -234,6 +234,7 @@ class CacheSpec:
     num_pages: int = 0
     D: int = 128
     rotate: bool = False         # Walsh-Hadamard rotation of K, V and Q (not with KIVI)
+    group: int = 32              # INT4 per group: channels per group (32, 64 or 128); KIVI: 32
 
 
 class RescaleSchedule:
@@ -277,7 +278,7 @@ class QuantizedKVCache:
             elif sch == INT8_SYM_PER_TOKEN:
                 self.t[side + "_scale"] = torch.zeros(*rows, dtype=torch.float32, device=dev)
             elif sch == INT4_SYM_PER_GROUP:
-                self.t[side + "_scale"] = torch.zeros(*rows, s.D // 32, dtype=torch.float32, device=dev)
+                self.t[side + "_scale"] = torch.zeros(*rows, s.D // s.group, dtype=torch.float32, device=dev)
             elif sch in (INT8_SYM_PER_CHANNEL, UINT8_ASYM_PER_CHANNEL):
                 self.t[side + "_scale"] = torch.zeros(s.Hkv, s.D, dtype=torch.float32, device=dev)
                 if sch == UINT8_ASYM_PER_CHANNEL:
@@ -300,7 +301,7 @@ class QuantizedKVCache:
         d.layout = KVQ_PAGED if s.paged else KVQ_DENSE
         d.capacity = s.capacity
         d.page_size, d.max_pages_per_seq, d.num_pages = s.page_size, s.max_pages, s.num_pages
-        d.group_size, d.residual_cap = 32, 128
+        d.group_size, d.residual_cap = s.group, 128
         d.rotation = KVQ_ROTATE_HADAMARD if s.rotate else KVQ_ROTATE_NONE
         for name, tensor in self.t.items():
             setattr(d, name, tensor.data_ptr())

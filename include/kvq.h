@@ -63,11 +63,11 @@ typedef enum kvq_status {
  *  FP8_E5M2_PER_TENSOR  OCP E5M2 codes of x/s, s = absmax/57344 over the calibrating append,
  *                       saturating at +-57344 (llms.blog §1 compares E4M3 with E5M2; a format
  *                       variant beyond the configurations the pages measure).
- *  INT4_SYM_PER_GROUP   clamp(rne(x/s), -8, 7) with s = absmax/7 per group of 32 consecutive
- *                       channels of one token (llms.blog §2 "INT4 Group-Wise"; n4n.ai Step 2
- *                       "Per-group INT4"); two's-complement nibbles packed along head_dim,
- *                       lower channel in the low bits (64-byte rows); fp32 scales
- *                       [rows][4] beside the codes. group_size must be 32. K and V both.
+ *  INT4_SYM_PER_GROUP   clamp(rne(x/s), -8, 7) with s = absmax/7 per group of group_size (32,
+ *                       64 or 128) consecutive channels of one token (llms.blog §2 "INT4
+ *                       Group-Wise"; n4n.ai Step 2 "Per-group INT4"); two's-complement nibbles
+ *                       packed along head_dim, lower channel in the low bits (64-byte rows);
+ *                       fp32 scales [rows][head_dim / group_size]. K and V both.
  * A zero range gives s = 0 and code 0. */
 typedef enum kvq_scheme {
   KVQ_FP8_E4M3_PER_TENSOR = 0,
@@ -107,8 +107,8 @@ typedef enum kvq_rotation { KVQ_ROTATE_NONE = 0, KVQ_ROTATE_HADAMARD = 1 } kvq_r
  *   paged codes  [num_pages, kv_heads, page_size, row_bytes]
  *   per-tensor scale            float [1]
  *   per-token scale             float [batch, kv_heads, capacity]  (paged: [num_pages, kv_heads, page_size])
- *   INT4 per-group scale        float [batch, kv_heads, capacity, head_dim/32] (paged: [num_pages,
- *                               kv_heads, page_size, head_dim/32])
+ *   INT4 per-group scale        float [batch, kv_heads, capacity, head_dim/group_size] (paged:
+ *                               [num_pages, kv_heads, page_size, head_dim/group_size])
  *   per-channel scale           float [kv_heads, head_dim]; uint8 zero point (k_zp/v_zp) same shape
  *   KIVI key scale and minimum  float [batch, kv_heads, capacity/32, head_dim] (k_scale, k_zero)
  *   KIVI value scale and minimum float [batch, kv_heads, capacity, head_dim/32] (v_scale, v_zero)
@@ -124,7 +124,7 @@ typedef struct kvq_cache_desc {
   int32_t capacity;          /* dense: tokens per (batch, kv_head); multiple of 128 */
   int32_t page_size;         /* paged: 16, 32 or 64 tokens */
   int32_t max_pages_per_seq, num_pages;
-  int32_t group_size;        /* KIVI: 32 */
+  int32_t group_size;        /* KIVI: 32; INT4 per group: 32, 64 or 128 */
   int32_t residual_cap;      /* KIVI: 128 */
   int32_t num_quantized;     /* dense: quantized tokens per row (library-maintained) */
   int32_t num_residual;      /* KIVI: tokens in the bf16 residual (library-maintained) */

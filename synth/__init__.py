@@ -175,9 +175,9 @@ class Workload:
 
 
 def workloads() -> dict:
-    """The eight workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4
-    per-group 70B-shaped (the latter also with the Walsh-Hadamard rotation, same inputs),
-    KIVI-2 131K, paged INT8."""
+    """The nine workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4
+    per-group 70B-shaped (INT4 with groups of 32, also with the Walsh-Hadamard rotation, and
+    with groups of 128; same inputs), KIVI-2 131K, paged INT8."""
     return {
         "tiny_int8": Workload(
             name="tiny_int8", seed=1, B=1, Hq=1, Hkv=1, D=128,
@@ -204,6 +204,10 @@ def workloads() -> dict:
             name="int4g_rot_70b", seed=7, B=16, Hq=64, Hkv=8, D=128,
             k_scheme=INT4_SYM_PER_GROUP, v_scheme=INT4_SYM_PER_GROUP, bf16=True,
             outlier_scale=20.0, rope_theta=500000.0, context=32768, rotate=True),
+        "int4g128_70b": Workload(
+            name="int4g128_70b", seed=7, B=16, Hq=64, Hkv=8, D=128,
+            k_scheme=INT4_SYM_PER_GROUP, v_scheme=INT4_SYM_PER_GROUP, bf16=True,
+            outlier_scale=20.0, rope_theta=500000.0, context=32768, group=128),
         "kivi2_131k": Workload(
             name="kivi2_131k", seed=4, B=4, Hq=64, Hkv=8, D=128,
             k_scheme=KIVI_INT2, v_scheme=KIVI_INT2, bf16=True,

@@ -133,7 +133,7 @@ def decode_both(oc: OracleCache, gc, q: np.ndarray, bf16: bool, where=""):
 
 
 def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16=None, seed=11, outlier=20.0,
-               rope=500000.0, chunks=None, rotate=False):
+               rope=500000.0, chunks=None, rotate=False, group=32):
     """Prefill (calibrating when the scheme needs it), then `steps` one-token appends each
     followed by a decode; codes and attention compared after every call."""
     q_bf16 = bf16 if q_bf16 is None else q_bf16
@@ -143,8 +143,8 @@ def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16
         cap = max(128, (total + 127) // 128 * 128)
     K = synth.keys(w, 0, B, 0, Hkv, 0, total)
     V = synth.values(w, 0, B, 0, Hkv, 0, total)
-    oc = OracleCache(B, Hq, Hkv, 128, ks, vs, cap=cap, rotate=rotate)
-    gc = kvq().QuantizedKVCache(kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=cap, rotate=rotate))
+    oc = OracleCache(B, Hq, Hkv, 128, ks, vs, cap=cap, rotate=rotate, group=group)
+    gc = kvq().QuantizedKVCache(kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=cap, rotate=rotate, group=group))
     calib = ks in CALIBRATED or vs in CALIBRATED
     bounds = [0, prefill] if chunks is None else [0, *chunks, prefill]
     for i, (a, b) in enumerate(zip(bounds, bounds[1:])):
@@ -169,7 +169,7 @@ def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16
 
 
 def paged_case(B, Hq, Hkv, ks, vs, lens, page_size=16, steps=2, seed=21, extra_pages=5, bad_page=None,
-               rotate=False):
+               rotate=False, group=32):
     w = workload(B, Hq, Hkv, ks, vs, bf16=True, seed=seed)
     lens = np.asarray(lens, np.int32)
     n_max = int(lens.max()) if len(lens) else 0
@@ -193,9 +193,9 @@ def paged_case(B, Hq, Hkv, ks, vs, lens, page_size=16, steps=2, seed=21, extra_p
             V[b:b + 1, :, :lens[b]] = synth.values(w, b, b + 1, 0, Hkv, 0, int(lens[b]))
     oc = OracleCache(B, Hq, Hkv, 128, ks, vs, paged=True, page_size=page_size, max_pages=max_pages,
                      num_pages=num_pages, page_table=table if bad_page is None else _clean(table, num_pages),
-                     rotate=rotate)
+                     rotate=rotate, group=group)
     spec = kvq().CacheSpec(B, Hq, Hkv, ks, vs, paged=True, page_size=page_size, max_pages=max_pages,
-                           num_pages=num_pages, rotate=rotate)
+                           num_pages=num_pages, rotate=rotate, group=group)
     gc = kvq().QuantizedKVCache(spec, page_table=torch.from_numpy(table))
     calib = ks in CALIBRATED or vs in CALIBRATED
     nl = torch.from_numpy(lens).cuda()

@@ -57,7 +57,7 @@ def test_validation_is_host_side():
         (dict(k_scheme=5, v_scheme=6), kvq.KVQ_ERR_UNSUPPORTED),
         (dict(rotation=2), kvq.KVQ_ERR_INVALID_ARG),
         (dict(rotation=1, k_scheme=5, v_scheme=5), kvq.KVQ_ERR_UNSUPPORTED),   # no rotation with KIVI
-        (dict(rotation=1, k_scheme=8, v_scheme=8, group_size=64), kvq.KVQ_ERR_UNSUPPORTED),
+        (dict(k_scheme=8, v_scheme=8, group_size=16), kvq.KVQ_ERR_UNSUPPORTED),   # INT4 groups: 32, 64, 128
         (dict(k_codes=None), kvq.KVQ_ERR_INVALID_ARG),
         (dict(k_codes=0x10004), kvq.KVQ_ERR_INVALID_ARG),   # not 16-byte aligned
         (dict(layout=1, page_size=16, max_pages_per_seq=4, num_pages=8), kvq.KVQ_ERR_INVALID_ARG),

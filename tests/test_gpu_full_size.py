@@ -75,7 +75,7 @@ def _dense_full(name):
     K = synth.keys(w, 0, w.B, 0, w.Hkv, 0, total)
     V = synth.values(w, 0, w.B, 0, w.Hkv, 0, total)
     gc = kvq.QuantizedKVCache(kvq.CacheSpec(w.B, w.Hq, w.Hkv, w.k_scheme, w.v_scheme, capacity=cap,
-                                            rotate=w.rotate))
+                                            rotate=w.rotate, group=w.group))
     calib = w.k_scheme in CAL or w.v_scheme in CAL
     gc.append(H.dev(K[:, :, :pre], w.bf16), H.dev(V[:, :, :pre], w.bf16), calibrate=calib)
     if append:
@@ -94,7 +94,7 @@ def _dense_full(name):
                                   .view(np.uint32), full_cal[side + "_scale"].reshape(-1).view(np.uint32))
     refs, gots = [], []
     for b, h in _pairs(w):
-        oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate)
+        oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group)
         if full_cal is not None:
             _copy_scales(oc, full_cal, h)
         oc.append(K[b:b + 1, h:h + 1, :pre], V[b:b + 1, h:h + 1, :pre], w.bf16)
@@ -124,6 +124,10 @@ def test_int4g_70b_full():
 
 def test_int4g_rot_70b_full():
     _dense_full("int4g_rot_70b")
+
+
+def test_int4g128_70b_full():
+    _dense_full("int4g128_70b")
 
 
 def test_kivi4_70b_full():

@@ -234,6 +234,28 @@ def test_int4_group_fp32_inputs_and_queries():
                  bf16=True, q_bf16=False)
 
 
+@pytest.mark.parametrize("group", [64, 128])
+def test_int4_larger_groups(group):
+    # groups of 64 and 128 channels (128: one scale per token): dense with ragged tails, paged,
+    # rotated, and dequantize
+    H.dense_case(B=2, Hq=16, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=300, steps=2,
+                 outlier=100.0, group=group)
+    oc, gc, _ = H.dense_case(B=2, Hq=8, Hkv=2, ks=S.INT4_SYM_PER_GROUP, vs=S.INT4_SYM_PER_GROUP, prefill=9600,
+                             steps=1, group=group, rotate=True)
+    for which in (0, 1):
+        got = gc.dequantize(which, 9601).cpu().numpy()
+        assert np.array_equal(got.view(np.uint32), oc.dequantize(which, 9601).view(np.uint32))
+    B, Hq, Hkv, sch = 4, 16, 4, S.INT4_SYM_PER_GROUP
+    w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, sch, sch, lens=[37, 100, 5, 64], page_size=32,
+                                                    steps=0, group=group)
+    oc.append(K, V, True, new_lens=lens)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl)
+    torch.cuda.synchronize()
+    H.compare_paged(oc, gc, f"paged, groups of {group}")
+    H.decode_both(oc, gc, synth.queries(w, 0, 0, B), True, f"paged decode, groups of {group}")
+    assert gc.status()[0] == 0
+
+
 @pytest.mark.parametrize("ps", [16, 32, 64])
 def test_int4_group_paged(ps):
     B, Hq, Hkv, sch = 4, 16, 4, S.INT4_SYM_PER_GROUP

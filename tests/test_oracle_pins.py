@@ -949,3 +949,22 @@ def test_rotated_decode_equals_attention_in_the_original_domain():
         assert np.max(np.abs(out[0, h] - ref)) <= 1e-5 * np.abs(ref).max()
         assert abs(lse[0, h] - (s.max() + math.log(p.sum()))) <= 1e-5
 
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_int4_larger_groups_share_one_scale(group):
+    # groups of 64 or 128 channels (128: one scale per token, the page code's default)
+    rng = np.random.default_rng(74 + group)
+    B, H, T = 1, 2, 4
+    x = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    c = OracleCache(B, H, H, 128, oracle.INT4_SYM_PER_GROUP, oracle.INT4_SYM_PER_GROUP, cap=8, group=group)
+    c.append(x, x, bf16=False)
+    assert c["k_scale"].shape == (B, H, 8, 128 // group)
+    for h in range(H):
+        for t in range(T):
+            for j in range(128 // group):
+                amax = np.abs(x[0, h, t, group * j:group * (j + 1)]).max()
+                assert c["k_scale"][0, h, t, j] == F32(amax) / F32(7)
+    d = c.dequantize(0, 8)[:, :, :T]
+    s = np.repeat(c["k_scale"][:, :, :T], group, axis=-1)
+    assert np.all(np.abs(d - x) <= s / 2 * (1 + 2**-20))
