@@ -36,6 +36,8 @@ KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
 INT4_SYM_PER_GROUP = 8
+KIVI_INT4_F16 = 9   # KIVI with fp16 scale and minimum
+KIVI_INT2_F16 = 10
 APPEND_CALIBRATE, APPEND_RESCALE = 1, 2  # append modes (oq_append)
 
 _lib = None
@@ -95,6 +97,11 @@ def load(path: str):
     L.oq_asym_code.argtypes = [f32, f32, ctypes.c_uint8]
     L.oq_asym_code.restype = i32
     L.oq_kivi_group.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    L.oq_kivi_group_f16.argtypes = [vp, i32, i32, i32, vp, vp, vp]
+    L.oq_f16_encode.argtypes = [f32]
+    L.oq_f16_encode.restype = ctypes.c_uint16
+    L.oq_f16_decode.argtypes = [ctypes.c_uint16]
+    L.oq_f16_decode.restype = f32
     L.oq_kivi_value.argtypes = [i32, f32, f32]
     L.oq_kivi_value.restype = f32
     L.oq_append.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp, i32]
@@ -161,13 +168,22 @@ def asym_code(x: float, s: float, zp: int) -> int:
     return int(lib().oq_asym_code(float(x), float(s), int(zp)))
 
 
-def kivi_group(x: np.ndarray, bits: int):
+def kivi_group(x: np.ndarray, bits: int, f16_meta: bool = False):
     x = np.ascontiguousarray(x, dtype=np.float32)
     codes = np.zeros(x.size, np.int32)
     s = np.zeros(1, np.float32)
     mn = np.zeros(1, np.float32)
-    lib().oq_kivi_group(x.ctypes.data, x.size, 1, bits, codes.ctypes.data, s.ctypes.data, mn.ctypes.data)
+    fn = lib().oq_kivi_group_f16 if f16_meta else lib().oq_kivi_group
+    fn(x.ctypes.data, x.size, 1, bits, codes.ctypes.data, s.ctypes.data, mn.ctypes.data)
     return codes, s[0], mn[0]
+
+
+def f16_encode(x: float) -> int:
+    return int(lib().oq_f16_encode(float(x)))
+
+
+def f16_decode(h: int) -> float:
+    return float(lib().oq_f16_decode(int(h)))
 
 
 def kivi_value(code: int, s: float, mn: float) -> float:
@@ -191,7 +207,7 @@ def kv_bytes_per_token(n_layers: int, n_kv_heads: int, d_head: int, bytes_per_el
 
 
 def _bits(scheme):
-    return {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4}.get(scheme, 8)
+    return {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4, KIVI_INT4_F16: 4, KIVI_INT2_F16: 2}.get(scheme, 8)
 
 
 # ---------------------------------------------------------------- cache
@@ -231,7 +247,7 @@ class OracleCache:
             self.arrays[side + "_scale"] = scale
             self.arrays[side + "_zero"] = zero
             self.arrays[side + "_zp"] = zp
-        kivi = k_scheme in (KIVI_INT4, KIVI_INT2)
+        kivi = k_scheme in (KIVI_INT4, KIVI_INT2, KIVI_INT4_F16, KIVI_INT2_F16)
         self.arrays["k_res"] = np.zeros((B, Hkv, rcap, D), np.uint16) if kivi else None
         self.arrays["v_res"] = np.zeros((B, Hkv, rcap, D), np.uint16) if kivi else None
         self.arrays["page_table"] = (np.ascontiguousarray(page_table, np.int32)

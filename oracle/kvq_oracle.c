@@ -228,6 +228,66 @@ void oq_kivi_group(const float* x, int n, int stride, int bits, int* codes, floa
   *mn = lo;
 }
 
+/* IEEE binary16 (sign, 5 exponent bits with bias 15, 10 mantissa bits; subnormals
+ * M * 2^-24): nearest value, ties to even mantissa. Values beyond the largest finite
+ * 65504 saturate to it (a scale or minimum must stay finite). NaN stays NaN. */
+uint16_t oq_f16_encode(float x) {
+  const uint16_t sign = signbit(x) ? 0x8000 : 0x0000;
+  const float a = fabsf(x);
+  if (isnan(x)) return (uint16_t)(sign | 0x7E00);
+  if (a >= 65504.0f) return (uint16_t)(sign | 0x7BFF);
+  if (a < ldexpf(1.0f, -14)) {
+    /* subnormal grid: multiples of 2^-24; 1024 * 2^-24 is the smallest normal (0x0400) */
+    const float m = rintf(ldexpf(a, 24));
+    return (uint16_t)(sign | (uint16_t)m);
+  }
+  int e2;
+  frexpf(a, &e2);                        /* a in [2^(e2-1), 2^e2) */
+  int E = e2 - 1;                        /* unbiased exponent, -14..15 */
+  float m = rintf(ldexpf(a, 10 - E));    /* significand * 1024, in [1024, 2048] */
+  if (m == 2048.0f) {
+    m = 1024.0f;
+    E += 1;
+  }
+  if (E > 15) return (uint16_t)(sign | 0x7BFF);
+  return (uint16_t)(sign | (uint16_t)(((E + 15) << 10) | ((int)m - 1024)));
+}
+
+float oq_f16_decode(uint16_t h) {
+  const int s = h >> 15, E = (h >> 10) & 0x1F, M = h & 0x3FF;
+  float v;
+  if (E == 31)
+    v = M == 0 ? INFINITY : NAN;
+  else if (E == 0)
+    v = ldexpf((float)M, -24);
+  else
+    v = ldexpf(1.0f + (float)M / 1024.0f, E - 15);
+  return s ? -v : v;
+}
+
+/* KIVI group with its scale and minimum stored in fp16 (the precision of the tensors the
+ * pages' cache code works in, P4 Step 3; half the metadata bytes, so INT2 takes 3 bits per
+ * element): the fp32 scale and minimum of oq_kivi_group rounded to fp16, and the codes of
+ * the stored values, q = clamp(rne((x - mn16) / s16), 0, qmax); s16 == 0 gives code 0. */
+void oq_kivi_group_f16(const float* x, int n, int stride, int bits, int* codes, float* s, float* mn) {
+  float sc, lo;
+  oq_kivi_group(x, n, stride, bits, codes, &sc, &lo);
+  const float s16 = oq_f16_decode(oq_f16_encode(sc)), mn16 = oq_f16_decode(oq_f16_encode(lo));
+  const int qmax = (1 << bits) - 1;
+  for (int i = 0; i < n; ++i) {
+    if (s16 == 0.0f) {
+      codes[i] = 0;
+      continue;
+    }
+    float r = rintf((x[(size_t)i * stride] - mn16) / s16);
+    if (r < 0.0f) r = 0.0f;
+    if (r > (float)qmax) r = (float)qmax;
+    codes[i] = (int)r;
+  }
+  *s = s16;
+  *mn = mn16;
+}
+
 /* x_hat = fl(fl(q * s) + min): two roundings, no fused multiply-add. */
 float oq_kivi_value(int code, float s, float mn) {
   float a = (float)code * s;
@@ -238,11 +298,13 @@ float oq_kivi_value(int code, float s, float mn) {
 /* cache layout helpers                                                      */
 /* ------------------------------------------------------------------------- */
 
-static int is_kivi(int scheme) { return scheme == OQ_KIVI_INT4 || scheme == OQ_KIVI_INT2; }
+static int is_kivi(int scheme) {
+  return scheme == OQ_KIVI_INT4 || scheme == OQ_KIVI_INT2 || scheme == OQ_KIVI_INT4_F16 || scheme == OQ_KIVI_INT2_F16;
+}
 
 static int code_bits(int scheme) {
-  if (scheme == OQ_KIVI_INT4 || scheme == OQ_INT4_SYM_PER_GROUP) return 4;
-  if (scheme == OQ_KIVI_INT2) return 2;
+  if (scheme == OQ_KIVI_INT4 || scheme == OQ_INT4_SYM_PER_GROUP || scheme == OQ_KIVI_INT4_F16) return 4;
+  if (scheme == OQ_KIVI_INT2 || scheme == OQ_KIVI_INT2_F16) return 2;
   return 8;
 }
 
@@ -421,12 +483,14 @@ static void kivi_flush(oq_cache* c, int b, int h, int pos0, const float* xk, con
                        int R) {
   const int D = c->D, g = c->group, H = c->Hkv;
   const int kb = code_bits(c->k_scheme), vb = code_bits(c->v_scheme);
+  const int kh = c->k_scheme == OQ_KIVI_INT4_F16 || c->k_scheme == OQ_KIVI_INT2_F16;
+  const int vh = c->v_scheme == OQ_KIVI_INT4_F16 || c->v_scheme == OQ_KIVI_INT2_F16;
   int* codes = (int*)malloc(sizeof(int) * (size_t)(g > D ? g : D));
   for (int gi = 0; gi < R / g; ++gi) {
     const size_t meta = (((size_t)b * H + h) * (size_t)(c->cap / g) + (size_t)(pos0 / g + gi)) * D;
     for (int d = 0; d < D; ++d) {
       float s, mn;
-      oq_kivi_group(xk + (size_t)gi * g * D + d, g, D, kb, codes, &s, &mn);
+      (kh ? oq_kivi_group_f16 : oq_kivi_group)(xk + (size_t)gi * g * D + d, g, D, kb, codes, &s, &mn);
       c->k_scale[meta + d] = s;
       c->k_zero[meta + d] = mn;
       for (int j = 0; j < g; ++j)
@@ -437,7 +501,7 @@ static void kivi_flush(oq_cache* c, int b, int h, int pos0, const float* xk, con
     const size_t row = row_of(c, b, h, pos0 + t);
     for (int j = 0; j < D / g; ++j) {
       float s, mn;
-      oq_kivi_group(xv + (size_t)t * D + (size_t)j * g, g, 1, vb, codes, &s, &mn);
+      (vh ? oq_kivi_group_f16 : oq_kivi_group)(xv + (size_t)t * D + (size_t)j * g, g, 1, vb, codes, &s, &mn);
       c->v_scale[row * (size_t)(D / g) + j] = s;
       c->v_zero[row * (size_t)(D / g) + j] = mn;
       for (int i = 0; i < g; ++i) put_code(c->v_codes, c->v_scheme, D, row, j * g + i, codes[i]);

@@ -43,7 +43,9 @@ enum {
   OQ_KIVI_INT4 = 5,
   OQ_KIVI_INT2 = 6,
   OQ_FP8_E5M2_PER_TENSOR = 7,
-  OQ_INT4_SYM_PER_GROUP = 8
+  OQ_INT4_SYM_PER_GROUP = 8,
+  OQ_KIVI_INT4_F16 = 9,  /* KIVI with fp16 scale and minimum */
+  OQ_KIVI_INT2_F16 = 10
 };
 
 /* ---- element codecs ---- */
@@ -55,6 +57,11 @@ uint8_t oq_e5m2_encode(float x);            /* round-to-nearest-even, saturate f
 float oq_e5m2_decode(uint8_t code);
 int oq_sym_code(float x, float s, int qmax); /* clamp(rne(x/s), -qmax, qmax); 0 if s == 0 */
 int oq_int4_code(float x, float s);         /* clamp(rne(x/s), -8, 7); 0 if s == 0 */
+uint16_t oq_f16_encode(float x);            /* IEEE half, RN-even, saturating at +-65504 */
+float oq_f16_decode(uint16_t h);
+/* KIVI group with fp16 parameters: s and min in fp32, stored rounded to fp16, codes from
+ * the stored values; *s and *mn receive the stored (fp16) values. */
+void oq_kivi_group_f16(const float* x, int n, int stride, int bits, int* codes, float* s, float* mn);
 void oq_asym_params(float mn, float mx, float* s, uint8_t* zp);
 int oq_asym_code(float x, float s, uint8_t zp);
 void oq_kivi_group(const float* x, int n, int stride, int bits, int* codes, float* s, float* mn);

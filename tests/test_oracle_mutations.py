@@ -69,6 +69,11 @@ MUTATIONS = [
     ("decode query not rotated", "    if (c->rotate) oq_fwht(qr, D);", "    (void)0;"),
     ("decode output not rotated back", "    if (c->rotate) fwht_d(out + (size_t)j * D, D);", "    (void)0;"),
     ("dequantize not rotated back", "        if (c->rotate && t < T) oq_fwht(row, D);", "        (void)row;"),
+    ("f16 exponent bias", "return (uint16_t)(sign | (uint16_t)(((E + 15) << 10) | ((int)m - 1024)));",
+     "return (uint16_t)(sign | (uint16_t)(((E + 14) << 10) | ((int)m - 1024)));"),
+    ("f16 subnormal grid", "    v = ldexpf((float)M, -24);", "    v = ldexpf((float)M, -23);"),
+    ("kivi f16 codes from fp32 parameters", "float r = rintf((x[(size_t)i * stride] - mn16) / s16);",
+     "float r = rintf((x[(size_t)i * stride] - lo) / sc);"),
     ("rescale paged length", "const int len = c->paged ? c->seq_lens[b] : c->len;",
      "const int len = c->paged ? c->seq_lens[b] - 1 : c->len;"),
 ]

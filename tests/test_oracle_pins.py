@@ -968,3 +968,60 @@ def test_int4_larger_groups_share_one_scale(group):
     d = c.dequantize(0, 8)[:, :, :T]
     s = np.repeat(c["k_scale"][:, :, :T], group, axis=-1)
     assert np.all(np.abs(d - x) <= s / 2 * (1 + 2**-20))
+
+
+# --------------------------------------------------------------- KIVI with fp16 metadata
+# Scale and minimum stored in fp16 (the tensor precision of the pages' cache code, n4n.ai
+# Step 3), which halves KIVI's metadata: INT2 then takes 2 + 2 * 16 / 32 = 3 bits per element.
+def test_f16_codec_matches_numpy():
+    rng = np.random.default_rng(90)
+    vals = np.concatenate([rng.normal(0, 1, 3000), rng.normal(0, 1e-5, 1000), rng.uniform(-65000, 65000, 1000),
+                           [0.0, -0.0, 2.0**-24, 2.0**-25, 3 * 2.0**-26, 65504.0, 2.0**-14, 1 + 2.0**-11]])
+    for v in vals.astype(np.float32):
+        want = np.array([v], np.float32).astype(np.float16).view(np.uint16)[0]
+        assert oracle.f16_encode(float(v)) == want, v
+        assert oracle.f16_decode(int(want)) == np.float32(np.array([want], np.uint16).view(np.float16)[0])
+    assert oracle.f16_encode(1e6) == 0x7BFF and oracle.f16_encode(-65520.0) == 0xFBFF  # saturating
+
+
+@pytest.mark.parametrize("bits", [4, 2])
+def test_kivi_f16_meta_is_the_rounded_fp32_meta_with_nearest_codes(bits):
+    qmax = 2**bits - 1
+    rng = np.random.default_rng(91 + bits)
+    for _ in range(200):
+        x = (rng.normal(0.3, 1.5, 32) * rng.uniform(0.01, 50)).astype(np.float32)
+        _, s32, mn32 = oracle.kivi_group(x, bits)
+        codes, s16, mn16 = oracle.kivi_group(x, bits, f16_meta=True)
+        assert s16 == np.float32(np.float16(s32)) and mn16 == np.float32(np.float16(mn32))
+        S, M = Fraction(float(s16)), Fraction(float(mn16))
+        for v, q in zip(x, codes):
+            d = [abs(Fraction(float(v)) - (k * S + M)) for k in range(qmax + 1)]
+            # nearest level of the stored grid, up to the fp32 rounding of (x - min) / s
+            assert d[q] <= min(d) + S * Fraction(1, 2**20), (v, q)
+
+
+def test_kivi_f16_cache_layout_and_dequant():
+    rng = np.random.default_rng(93)
+    B, H = 1, 2
+    x = rng.normal(0, 1, (B, H, 200, 128)).astype(np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16)          # bf16 bits (truncated; any bf16 will do)
+    a = OracleCache(B, 4, H, 128, oracle.KIVI_INT2_F16, oracle.KIVI_INT2_F16, cap=256)
+    b = OracleCache(B, 4, H, 128, oracle.KIVI_INT2, oracle.KIVI_INT2, cap=256)
+    a.append(xb, xb, bf16=True)
+    b.append(xb, xb, bf16=True)
+    assert a.length == b.length == 128 and a.residual == b.residual == 72
+    for side in ("k", "v"):
+        s16, s32 = a[side + "_scale"], b[side + "_scale"]
+        assert np.array_equal(s16, s32.astype(np.float16).astype(np.float32))
+        z16, z32 = a[side + "_zero"], b[side + "_zero"]
+        assert np.array_equal(z16, z32.astype(np.float16).astype(np.float32))
+    # the residual (bf16) is untouched by the metadata precision
+    assert np.array_equal(a["k_res"], b["k_res"])
+    d = a.dequantize(1, 256)[:, :, :128].astype(np.float64)
+    xf = synth_bf16(xb)[:, :, :128]
+    s = np.repeat(a["v_scale"][:, :, :128], 32, axis=-1)
+    assert np.all(np.abs(d - xf) <= s * 0.5 + np.abs(xf) * 2.0**-10 + 2.0**-24)
+
+
+def synth_bf16(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
