@@ -35,8 +35,9 @@ MUTATIONS = [
     ("kivi dequant sign", "  return a + mn;", "  return a - mn;"),
     ("kivi no min shift", "float diff = x[(size_t)i * stride] - lo;", "float diff = x[(size_t)i * stride];"),
     ("kivi key axis transposed",
-     "oq_kivi_group(xk + (size_t)gi * g * D + d, g, D, kb, codes, &s, &mn);",
-     "oq_kivi_group(xk + (size_t)gi * g * D + (size_t)d * g % (g * D), g, 1, kb, codes, &s, &mn);"),
+     "(kh ? oq_kivi_group_f16 : oq_kivi_group)(xk + (size_t)gi * g * D + d, g, D, kb, codes, &s, &mn);",
+     "(kh ? oq_kivi_group_f16 : oq_kivi_group)(xk + (size_t)gi * g * D + (size_t)d * g % (g * D), g, 1, kb, codes, "
+     "&s, &mn);"),
     ("kivi flush rule", "const int r_new = ((total - 1) % R) + 1;", "const int r_new = total % R;"),
     ("kivi pack order", "const int byte = d / per, sh = (d % per) * bits;",
      "const int byte = d / per, sh = (per - 1 - d % per) * bits;"),
