@@ -67,6 +67,7 @@ class _Cache(ctypes.Structure):
         ("k_res", ctypes.c_void_p), ("v_res", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("rotate", ctypes.c_int),
+        ("rope_theta", ctypes.c_float),
     ]
 
 
@@ -108,6 +109,8 @@ def load(path: str):
     L.oq_append.restype = i32
     L.oq_calibrate.argtypes = [ctypes.POINTER(_Cache), vp, vp, i32, i32, vp]
     L.oq_fwht.argtypes = [vp, i32]
+    L.oq_rope.argtypes = [vp, i32, i32, ctypes.c_double]
+    L.oq_rope.restype = None
     L.oq_fwht.restype = None
     L.oq_calibrate.restype = i32
     L.oq_tokens.argtypes = [ctypes.POINTER(_Cache), i32]
@@ -148,6 +151,13 @@ def sym_code(x: float, s: float, qmax: int = 127) -> int:
 
 def int4_code(x: float, s: float) -> int:
     return int(lib().oq_int4_code(float(x), float(s)))
+
+
+def rope(x, pos: int, theta: float) -> np.ndarray:
+    """Rotate-half RoPE of a row at position pos (fp64)."""
+    y = np.array(x, np.float64, copy=True)
+    lib().oq_rope(y.ctypes.data, int(y.size), int(pos), float(theta))
+    return y
 
 
 def fwht(x) -> np.ndarray:
@@ -215,7 +225,8 @@ class OracleCache:
     """Oracle cache with numpy arrays in the library's layouts (see module docstring)."""
 
     def __init__(self, B, Hq, Hkv, D, k_scheme, v_scheme, cap=0, paged=False, page_size=16,
-                 max_pages=0, num_pages=0, page_table=None, group=32, rcap=128, rotate=False):
+                 max_pages=0, num_pages=0, page_table=None, group=32, rcap=128, rotate=False,
+                 rope_theta=0.0):
         self.B, self.Hq, self.Hkv, self.D = B, Hq, Hkv, D
         self.k_scheme, self.v_scheme = k_scheme, v_scheme
         self.paged, self.cap, self.page_size = paged, cap, page_size
@@ -259,6 +270,7 @@ class OracleCache:
             setattr(self.c, name, _ptr(arr))
         self.c.rotate = int(bool(rotate))
         self.rotate = bool(rotate)
+        self.c.rope_theta = float(rope_theta)
 
     def __getitem__(self, name):
         return self.arrays[name]

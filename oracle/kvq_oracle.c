@@ -21,6 +21,9 @@
  *  - rotation (optional): the normalised Walsh-Hadamard transform of each K/V row before it
  *    is quantized, of each query before attention, and of each attention output and
  *    dequantized row after (P3 §5, QuaRot / RotateKV); fp32 butterflies in span order.
+ *  - pre-RoPE keys (optional, P3 §4 KVQuant): keys are quantized as given (before RoPE)
+ *    and decode applies rotate-half RoPE in fp64 to each dequantized key at its position
+ *    in the sequence; queries arrive with RoPE applied.
  */
 #include "kvq_oracle.h"
 
@@ -662,6 +665,7 @@ int oq_append(oq_cache* c, const void* k_new, const void* v_new, int in_bf16, in
   block kb = {k_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
   block vb = {v_new, in_bf16, n_new, new_lens, c->Hkv, c->D};
   if (new_lens && !c->paged) return -1;
+  if (c->rotate && c->rope_theta > 0.0f) return -1;  /* one of the two rotations at a time */
   if (is_kivi(c->k_scheme) || is_kivi(c->v_scheme)) {
     if (!(is_kivi(c->k_scheme) && is_kivi(c->v_scheme)) || c->paged || c->rotate) return -1;
     return append_kivi(c, &kb, &vb);
@@ -802,8 +806,9 @@ void oq_dequantize(const oq_cache* c, int which, float* out, int T_out) {
 
 /* softmax(scale * q.k_t) over t, then the probability-weighted sum of v_t; scores
  * and the sums are fp64, t ascending. T == 0 gives zeros and lse = -inf. */
-void oq_attention_row(const float* q, const float* k, const float* v, int T, int D,
-                      float scale, double* out, double* lse) {
+/* Scores against fp64 keys (kd) when given, else the fp32 keys k. */
+static void attention_row(const float* q, const float* k, const double* kd, const float* v, int T, int D,
+                          float scale, double* out, double* lse) {
   for (int d = 0; d < D; ++d) out[d] = 0.0;
   if (T == 0) {
     *lse = -INFINITY;
@@ -813,7 +818,8 @@ void oq_attention_row(const float* q, const float* k, const float* v, int T, int
   double m = -INFINITY;
   for (int t = 0; t < T; ++t) {
     double acc = 0.0;
-    for (int d = 0; d < D; ++d) acc += (double)q[d] * (double)k[(size_t)t * D + d];
+    for (int d = 0; d < D; ++d)
+      acc += (double)q[d] * (kd ? kd[(size_t)t * D + d] : (double)k[(size_t)t * D + d]);
     s[t] = acc * (double)scale;
     if (s[t] > m) m = s[t];
   }
@@ -828,6 +834,23 @@ void oq_attention_row(const float* q, const float* k, const float* v, int T, int
   free(s);
 }
 
+void oq_attention_row(const float* q, const float* k, const float* v, int T, int D,
+                      float scale, double* out, double* lse) {
+  attention_row(q, k, NULL, v, T, D, scale, out, lse);
+}
+
+void oq_rope(double* x, int D, int pos, double theta) {
+  const int half = D / 2;
+  for (int i = 0; i < half; ++i) {
+    const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
+    const double ang = (double)pos * inv_freq;
+    const double c = cos(ang), s = sin(ang);
+    const double a = x[i], b = x[i + half];
+    x[i] = a * c - b * s;
+    x[i + half] = b * c + a * s;
+  }
+}
+
 static void decode_pair(const oq_cache* c, const void* q, int q_bf16, float scale, int b,
                         int hk, double* out, double* lse) {
   const int D = c->D, G = c->Hq / c->Hkv, T = oq_tokens(c, b);
@@ -839,16 +862,25 @@ static void decode_pair(const oq_cache* c, const void* q, int q_bf16, float scal
       k[(size_t)t * D + d] = value_at(c, 0, b, hk, t, d);
       v[(size_t)t * D + d] = value_at(c, 1, b, hk, t, d);
     }
+  double* kd = NULL;
+  if (c->rope_theta > 0.0f) {  /* pre-RoPE keys: token t sits at position t of the sequence */
+    kd = (double*)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1) * D);
+    for (int t = 0; t < T; ++t) {
+      for (int d = 0; d < D; ++d) kd[(size_t)t * D + d] = (double)k[(size_t)t * D + d];
+      oq_rope(kd + (size_t)t * D, D, t, (double)c->rope_theta);
+    }
+  }
   for (int j = 0; j < G; ++j) {
     const int hq = hk * G + j; /* query head h reads kv head h / G */
     for (int d = 0; d < D; ++d) qr[d] = input_at(q, q_bf16, ((size_t)b * c->Hq + hq) * D + d);
     if (c->rotate) oq_fwht(qr, D);  /* the cache holds H k and H v: attend with H q */
     double l;
-    oq_attention_row(qr, k, v, T, D, scale, out + (size_t)j * D, &l);
+    attention_row(qr, k, kd, v, T, D, scale, out + (size_t)j * D, &l);
     if (c->rotate) fwht_d(out + (size_t)j * D, D);  /* sum p (H v) = H (sum p v) */
     if (lse) lse[j] = l;
   }
   free(k);
+  free(kd);
   free(v);
   free(qr);
 }

@@ -83,6 +83,8 @@ typedef struct {
   int32_t *page_table, *seq_lens;
   int rotate;                    /* 1: K/V rows and queries rotated by the normalised
                                     Walsh-Hadamard transform over head_dim (not with KIVI) */
+  float rope_theta;              /* > 0: keys are cached before RoPE and decode rotates each
+                                    dequantized key at its position (KVQuant pre-RoPE keys) */
 } oq_cache;
 
 /* Append modes (the `calibrate` argument of oq_append). */
@@ -107,6 +109,11 @@ int oq_calibrate(oq_cache* c, const void* k_new, const void* v_new, int in_bf16,
  * stages of span 1, 2, 4, ..., n/2, each (a, b) -> (a + b, a - b) in fp32, then every value
  * times the fp32 constant nearest 1/sqrt(n). The transform is its own inverse. */
 void oq_fwht(float* x, int n);
+
+/* Rotate-half RoPE of one row in fp64 at position pos: for i < D/2, with inverse
+ * frequency theta^(-2i/D) and angle pos * that, (x_i, x_{i+D/2}) becomes
+ * (x_i cos - x_{i+D/2} sin, x_{i+D/2} cos + x_i sin). */
+void oq_rope(double* x, int D, int pos, double theta);
 
 /* Tokens visible to decode for sequence b. */
 int oq_tokens(const oq_cache* c, int b);

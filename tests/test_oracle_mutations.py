@@ -75,6 +75,13 @@ MUTATIONS = [
     ("f16 subnormal grid", "    v = ldexpf((float)M, -24);", "    v = ldexpf((float)M, -23);"),
     ("kivi f16 codes from fp32 parameters", "float r = rintf((x[(size_t)i * stride] - mn16) / s16);",
      "float r = rintf((x[(size_t)i * stride] - lo) / sc);"),
+    ("rope sine sign", "    x[i] = a * c - b * s;\n    x[i + half] = b * c + a * s;",
+     "    x[i] = a * c + b * s;\n    x[i + half] = b * c - a * s;"),
+    ("rope frequency exponent", "const double inv_freq = pow(theta, -2.0 * (double)i / (double)D);\n    const double ang = (double)pos",
+     "const double inv_freq = pow(theta, -1.0 * (double)i / (double)D);\n    const double ang = (double)pos"),
+    ("pre-rope position off by one", "oq_rope(kd + (size_t)t * D, D, t, (double)c->rope_theta);",
+     "oq_rope(kd + (size_t)t * D, D, t + 1, (double)c->rope_theta);"),
+    ("pre-rope keys not rotated", "  if (c->rope_theta > 0.0f) {  /* pre-RoPE keys", "  if (0) {  /* pre-RoPE keys"),
     ("rescale paged length", "const int len = c->paged ? c->seq_lens[b] : c->len;",
      "const int len = c->paged ? c->seq_lens[b] - 1 : c->len;"),
 ]

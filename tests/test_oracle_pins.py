@@ -1025,3 +1025,55 @@ def test_kivi_f16_cache_layout_and_dequant():
 
 def synth_bf16(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------- pre-RoPE keys (KVQuant)
+# llms.blog §4: KVQuant quantizes keys before the rotary embedding, whose position-dependent
+# rotation would otherwise mix the outlier channels; decode rotates each dequantized key.
+def test_rope_equals_the_complex_rotation():
+    rng = np.random.default_rng(100)
+    theta = 500000.0
+    for pos in (0, 1, 7, 4095, 131071):
+        x = rng.normal(0, 1, 128)
+        z = (x[:64] + 1j * x[64:]) * np.exp(1j * pos * theta ** (-np.arange(64) * 2.0 / 128))
+        y = oracle.rope(x, pos, theta)
+        assert np.max(np.abs(y - np.concatenate([z.real, z.imag]))) <= 1e-12 * np.abs(x).sum()
+        assert abs(np.linalg.norm(y) - np.linalg.norm(x)) <= 1e-12 * np.linalg.norm(x)
+    assert np.array_equal(oracle.rope(np.arange(128.0), 0, theta), np.arange(128.0))   # position 0
+
+
+def test_rope_scores_depend_on_relative_position():
+    rng = np.random.default_rng(101)
+    q, k = rng.normal(0, 1, 128), rng.normal(0, 1, 128)
+    a = oracle.rope(q, 1000, 10000.0) @ oracle.rope(k, 990, 10000.0)
+    b = oracle.rope(q, 10, 10000.0) @ oracle.rope(k, 0, 10000.0)
+    assert abs(a - b) <= 1e-9 * np.abs(q).sum() * np.abs(k).sum()
+
+
+@pytest.mark.parametrize("scheme", [oracle.INT8_SYM_PER_CHANNEL, oracle.KIVI_INT4])
+def test_pre_rope_decode_rotates_each_dequantized_key_at_its_position(scheme):
+    rng = np.random.default_rng(102)
+    B, Hq, H, T = 1, 4, 2, 150
+    k = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    v = rng.normal(0, 1, (B, H, T, 128)).astype(np.float32)
+    k[..., 5] *= 20
+    bf16 = scheme == oracle.KIVI_INT4
+    if bf16:  # KIVI takes bf16 inputs
+        k = (k.view(np.uint32) >> 16).astype(np.uint16)
+        v = (v.view(np.uint32) >> 16).astype(np.uint16)
+    c = OracleCache(B, Hq, H, 128, scheme, scheme, cap=256, rope_theta=10000.0)
+    c.append(k, v, bf16=bf16, calibrate=scheme != oracle.KIVI_INT4)
+    q = rng.normal(0, 1, (B, Hq, 128)).astype(np.float32)
+    out, lse = c.decode(q, bf16=False, scale=0.09)
+    K, V = c.dequantize(0, T).astype(np.float64), c.dequantize(1, T).astype(np.float64)
+    Kr = np.stack([np.stack([oracle.rope(K[0, h, t], t, 10000.0) for t in range(T)]) for h in range(H)])
+    for h in range(Hq):
+        s = Kr[h // 2] @ q[0, h].astype(np.float64) * float(F32(0.09))
+        p = np.exp(s - s.max())
+        ref = (p / p.sum()) @ V[0, h // 2]
+        assert np.max(np.abs(out[0, h] - ref)) <= 1e-9 * np.abs(ref).max()
+        assert abs(lse[0, h] - (s.max() + math.log(p.sum()))) <= 1e-9
+    # the cache itself holds the keys as given (dequantize returns pre-RoPE values)
+    plain = OracleCache(B, Hq, H, 128, scheme, scheme, cap=256)
+    plain.append(k, v, bf16=bf16, calibrate=scheme != oracle.KIVI_INT4)
+    assert np.array_equal(plain["k_codes"], c["k_codes"])
