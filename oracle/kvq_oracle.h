@@ -14,9 +14,12 @@
  *  [P3] "KV Cache Quantization in Production LLM Serving: Comparing FP8, INT8, INT4,
  *       KIVI, and KVQuant" (llms.blog): memory-per-token formula, §1 FP8 E4M3 (and
  *       E5M2, the other OCP FP8 format the section compares it with), §2 INT8 symmetric
- *       [-127,127], §3 KIVI.
+ *       [-127,127] and INT4 group-wise, §3 KIVI, §4 KVQuant (pre-RoPE keys), §5 QuaRot /
+ *       RotateKV (Hadamard rotation).
  *  [P4] "How KV cache quantization reduces GPU memory" (n4n.ai): Step 1 tensor shape,
- *       Step 2 schemes, Step 3 QuantizedKVCache (quantize / dequantize / append).
+ *       Step 2 schemes (per-group INT4), Step 3 QuantizedKVCache (quantize / dequantize /
+ *       append, running-max scale merge), Step 7 edge cases (scales that grow or are
+ *       recomputed as the cache grows).
  *
  * Parity status: every function here is pinned by a CPU test (worked examples,
  * closed forms, invariants, brute force). End-to-end model quality (perplexity,
