@@ -193,6 +193,8 @@ kvq_status kvq_quantize_append(kvq_cache_desc* d, const void* k_new, const void*
                    : (flags & KVQ_APPEND_CALIBRATE) ? kAppendCalibrate
                    : (flags & KVQ_APPEND_RESCALE)   ? kAppendRescale
                                                     : kAppendPlain;
+  // the statistics and KIVI flush grids take one block row per (sequence, kv head)
+  if ((kivi || mode != kAppendPlain) && (int64_t)d->batch * d->num_kv_heads > 65535) return KVQ_ERR_UNSUPPORTED;
   if (mode != kAppendPlain) {
     if (!workspace || workspace_bytes < kvq_append_workspace_bytes(d, flags) || !aligned16(workspace))
       return KVQ_ERR_WORKSPACE;

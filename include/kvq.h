@@ -183,6 +183,8 @@ KVQ_API size_t kvq_append_workspace_bytes(const kvq_cache_desc* desc, uint32_t f
  *                 of the cached representable range [(0 - zp) s, (255 - zp) s] and the
  *                 block's range. A cached code is requantized from its dequantized value.
  *                 Both flags are ignored for per-token and KIVI schemes.
+ *                 Calibrating, rescaling and KIVI appends need batch * kv_heads <= 65535
+ *                 (else KVQ_ERR_UNSUPPORTED, before anything is launched).
  * Dense: tokens go to positions num_quantized.. of every row; the library updates
  * num_quantized / num_residual in *desc when the call is accepted. KIVI: tokens enter the
  * residual; when a token arrives at a full residual, its 128 tokens are quantized.

@@ -147,6 +147,11 @@ def test_rescale_flag_is_checked_on_the_host():
     assert L.kvq_quantize_append(ctypes.byref(d), buf, buf, kvq.KVQ_BF16, 4, None, kvq.KVQ_APPEND_RESCALE,
                                  buf, cal, None) == kvq.KVQ_ERR_WORKSPACE
     assert d.num_quantized == 0  # nothing was accepted
+    # statistics need one block row per (sequence, kv head): refused on the host past 65535
+    big = _desc(batch=40000, num_q_heads=4, num_kv_heads=2, capacity=128)
+    need = L.kvq_append_workspace_bytes(ctypes.byref(big), kvq.KVQ_APPEND_CALIBRATE)
+    assert L.kvq_quantize_append(ctypes.byref(big), buf, buf, kvq.KVQ_BF16, 1, None, kvq.KVQ_APPEND_CALIBRATE,
+                                 buf, need, None) == kvq.KVQ_ERR_UNSUPPORTED
 
 
 def test_rescale_schedule_counts_tokens():
