@@ -37,7 +37,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_plumbing():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a process that already runs threads
     out = mgr.dict()
     mp.start_processes(_worker, args=(world, _free_port(), out), nprocs=world, start_method="spawn", join=True)
     s0, k0, t0, v0 = out[0]
