@@ -37,6 +37,7 @@ FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {synth.FP8_E4M3_PER_TENSOR: "fp8_e4m3", synth.FP8_E5M2_PER_TENSOR: "fp8_e5m2", synth.INT8_SYM_PER_TENSOR: "int8",
               synth.INT8_SYM_PER_TOKEN: "int8", synth.INT8_SYM_PER_CHANNEL: "int8",
               synth.UINT8_ASYM_PER_CHANNEL: "uint8", synth.KIVI_INT4: "int4", synth.KIVI_INT2: "int2",
+              synth.KIVI_INT4_F16: "int4 (fp16 meta)", synth.KIVI_INT2_F16: "int2 (fp16 meta)",
               synth.INT4_SYM_PER_GROUP: "int4"}
 CALIBRATED = (synth.FP8_E4M3_PER_TENSOR, synth.FP8_E5M2_PER_TENSOR, synth.INT8_SYM_PER_TENSOR, synth.INT8_SYM_PER_CHANNEL,
               synth.UINT8_ASYM_PER_CHANNEL)
@@ -52,13 +53,15 @@ def parse():
     ap.add_argument("--workload", default="fp8_8b", choices=list(synth.workloads()))
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
 
 # ---------------------------------------------------------------- algorithmic bytes
 def row_bytes(scheme):
-    return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2, synth.INT4_SYM_PER_GROUP: 4}.get(scheme, 8) // 8
+    return 128 * {synth.KIVI_INT4: 4, synth.KIVI_INT2: 2, synth.INT4_SYM_PER_GROUP: 4, synth.KIVI_INT4_F16: 4,
+                  synth.KIVI_INT2_F16: 2}.get(scheme, 8) // 8
 
 
 def meta_bytes_per_token(scheme, Hkv, group=32):
@@ -67,6 +70,8 @@ def meta_bytes_per_token(scheme, Hkv, group=32):
         return 4.0
     if scheme in (synth.KIVI_INT4, synth.KIVI_INT2):
         return 8.0 * 128 / 32  # fp32 (scale, min) per 32 elements
+    if scheme in (synth.KIVI_INT4_F16, synth.KIVI_INT2_F16):
+        return 4.0 * 128 / 32  # fp16 (scale, min) per 32 elements
     if scheme == synth.INT4_SYM_PER_GROUP:
         return 4.0 * 128 / group  # fp32 scale per group of channels
     return 0.0
@@ -251,7 +256,8 @@ class GpuWorkload:
         self.append_token = W.name != "tiny_int8"  # the tiny configuration decodes without appending
         pre = total - 1 if self.append_token else total
         cap = (total + 127) // 128 * 128
-        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap, rotate=W.rotate, group=W.group)
+        spec = kvq.CacheSpec(W.B, W.Hq, W.Hkv, W.k_scheme, W.v_scheme, capacity=cap, rotate=W.rotate, group=W.group,
+                             rope_theta=W.prerope_theta)
         self.cache = kvq.QuantizedKVCache(spec, device=self.dev)
         self.calib = W.k_scheme in CALIBRATED or W.v_scheme in CALIBRATED
         self.pre_k = self._dev(synth.keys(W, 0, W.B, 0, W.Hkv, 0, pre), W.bf16)
@@ -276,17 +282,21 @@ class GpuWorkload:
         else:
             d.num_quantized, d.num_residual = 0, 0
 
-    def prefill_bytes(self):
+    def prefill_bytes(self, reads=None):
         """Algorithmic bytes of the prefill append: the block is read once (twice when it
-        calibrates a per-tensor / per-channel scale) and codes, metadata and residual written."""
+        calibrates a per-tensor / per-channel scale: the 2R + W count; reads=1 gives R + W) and
+        codes, metadata and residual written."""
         W = self.seed_w
         rows = self.prefill_rows
         elem = 2 if W.bf16 else 4
-        b = rows * 128 * elem * 2 * (2 if self.calib else 1)
+        if reads is None:
+            reads = 2 if self.calib else 1
+        b = rows * 128 * elem * 2 * reads
         if W.kivi:
             nq = (self.cache.desc.num_quantized if not W.paged else 0)
             qrows = W.B * W.Hkv * nq
-            b += qrows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme)) + qrows * 2 * 8.0 * 128 / 32
+            b += qrows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme))
+            b += qrows * (meta_bytes_per_token(W.k_scheme, W.Hkv) + meta_bytes_per_token(W.v_scheme, W.Hkv))
             b += W.B * W.Hkv * self.cache.desc.num_residual * 128 * 2 * 2
         else:
             b += rows * (row_bytes(W.k_scheme) + row_bytes(W.v_scheme))
@@ -383,7 +393,7 @@ class GpuWorkload:
         self.q_host = [synth.queries(W, s, 0, W.B) for s in range(2)]
         self.q = self._dev(self.q_host[0], W.bf16)
         self.out = torch.empty((W.B, W.Hq, 128), dtype=torch.float32, device=self.dev)
-        self.ws = torch.empty(kvq.kvq_decode_workspace_bytes(self.cache.desc), dtype=torch.uint8, device=self.dev)
+        self.ws = kvq.decode_workspace(self.cache.desc, self.dev)
         self.scale = 1.0 / math.sqrt(128.0)
 
     def paged_token(self, step):
@@ -415,20 +425,19 @@ class GpuWorkload:
         return np.full(W.B, nq), (nr if W.kivi else 0)
 
 
-def run_gpu(args, rank, world, local_rank):
+def measure_workload(name, rank, world, dev, steps, warmup, stream, flush, e2e=True):
+    """Build one workload's cache, time its bulk prefill append, then `steps` graph-replayed
+    steps (append + decode) and up to 400 decode calls, L2 flushed before each; device time by
+    CUDA events on the launching stream."""
     import torch
     import torch.distributed as dist
     from decode_attention_quantize_b200 import kvq
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = synth.workloads()[args.workload]
+    w = synth.workloads()[name]
     G = GpuWorkload(w, rank, dev)
     W = G.seed_w
-    stream = torch.cuda.Stream(device=dev)
-    flush = L2Flush(dev)
     t_prefill = G.time_prefill(flush, stream)
-    prefill = {"ms": t_prefill * 1e3, "bytes": G.prefill_bytes(), "tokens": G.prefill_rows // W.Hkv,
-               "calibrating": bool(G.calib)}
+    prefill = {"ms": t_prefill * 1e3, "bytes": G.prefill_bytes(), "bytes_r_plus_w": G.prefill_bytes(reads=1),
+               "tokens": G.prefill_rows // W.Hkv, "calibrating": bool(G.calib)}
     G.pre_k = G.pre_v = None  # release the prefill block before timing the steps
     torch.cuda.empty_cache()
 
@@ -450,16 +459,11 @@ def run_gpu(args, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def run_step(i):
-        if graph is not None:
-            graph.replay()
-        else:
-            k, v = G.paged_token(i)
-            with torch.cuda.stream(stream):
-                G.step(stream, k_new=k, v_new=v)
+        graph.replay()
 
     # paged: pre-generate the step tokens (host generation is outside timing)
     if W.paged:
-        total_steps = args.warmup + args.steps
+        total_steps = warmup + steps
         if total_steps + 200 > G.extra:
             raise SystemExit("too many steps for the page pool")
         toks = [G.paged_token(i) for i in range(total_steps)]
@@ -468,58 +472,103 @@ def run_gpu(args, rank, world, local_rank):
             with torch.cuda.stream(stream):
                 G.step(stream, k_new=toks[i][0], v_new=toks[i][1])
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         flush()
         run_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     launches0 = kvq.kvq_launch_count()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local_rank)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     torch.cuda.synchronize()
-    with sampler:
-        for i in range(args.steps):
-            with torch.cuda.stream(stream):
-                flush()
-                ev[i][0].record(stream)
-                if graph is not None:
-                    graph.replay()
-                else:
-                    run_step(args.warmup + i)
-                ev[i][1].record(stream)
-        torch.cuda.synchronize()
+    for i in range(steps):
+        with torch.cuda.stream(stream):
+            flush()
+            ev[i][0].record(stream)
+            run_step(warmup + i)
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     launches = kvq.kvq_launch_count() - launches0
     if graph is not None:
-        launches = args.steps * launches_per_replay
+        launches = steps * launches_per_replay
     # decode-only timing (the dominant kernel's call: split-KV kernel + merge), eager
-    dec_ms = []
-    for i in range(min(args.steps, 400)):
+    n_dec = min(steps, 400)
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_dec)]
+    for i in range(n_dec):
         with torch.cuda.stream(stream):
             flush()
             dec_ev[i][0].record(stream)
             G.cache.decode(G.q, G.scale, out=G.out, workspace=G.ws, stream=stream)
             dec_ev[i][1].record(stream)
     torch.cuda.synchronize()
-    dec_ms = [a.elapsed_time(b) for a, b in dec_ev[:min(args.steps, 400)]]
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
 
     t_step = sum(step_ms) / len(step_ms) / 1e3  # seconds (mean)
     t_dec = sum(dec_ms) / len(dec_ms) / 1e3
-    lens_q, len_res = G.decode_lens(args.warmup + args.steps // 2 + 1)
+    lens_q, len_res = G.decode_lens(warmup + steps // 2 + 1)
     dbytes = decode_bytes(W, lens_q, len_res)
-    lens_d, res_d = G.decode_lens(args.warmup + args.steps)  # state seen by the decode-only timing
+    lens_d, res_d = G.decode_lens(warmup + steps)  # state seen by the decode-only timing
     dbytes_dec = decode_bytes(W, lens_d, res_d)
     abytes = append_bytes(W) if G.append_token else 0.0
-    t_max = max_over_ranks(sum(step_ms) / 1e3, world, device=dev) / args.steps
+    t_max = max_over_ranks(sum(step_ms) / 1e3, world, device=dev) / steps
 
     # end to end through the public API: host inputs (pinned) -> device -> step -> host out
-    e2e = run_e2e(G, W, stream, flush, n=min(200, args.steps), step0=args.warmup + args.steps)
+    e2e_r = run_e2e(G, W, stream, flush, n=min(200, steps), step0=warmup + steps) if e2e else None
     status = G.cache.status()
     return dict(t_step=t_step, t_max=t_max, t_dec=t_dec, dbytes=dbytes, dbytes_dec=dbytes_dec, abytes=abytes,
-                launches=launches, prefill=prefill,
-                clocks=sampler.summary(), e2e=e2e, status=status, W=W, G=G)
+                launches=launches, prefill=prefill, e2e=e2e_r, status=status, W=W, G=G)
+
+
+# every workload the library measures; the headline line is `--workload`, the rest go into
+# `per_config` (one process, one GPU, shorter runs)
+PER_CONFIG = ["tiny_int8", "fp8_8b", "e5m2_8b", "fp8_8b_prerope", "kivi4_70b", "kivi4f16_70b", "int4g_70b",
+              "int4g_rot_70b", "int4g128_70b", "kivi2_131k", "kivi2f16_131k", "paged_int8"]
+NOMINAL_HBM_GBS = 8000.0  # the ~8 TB/s B200 figure the targets are stated against
+
+
+def config_summary(r, peak):
+    """One workload's line of `per_config`: the decode call, the step and the bulk append."""
+    W = r["W"]
+    gbs = r["dbytes_dec"] / r["t_dec"] / 1e9
+    pf = r["prefill"]
+    t_pf = pf["ms"] / 1e3
+    return {"workload": W.name, "dtype": dtype_of(W), "layout": "paged/16" if W.paged else "dense",
+            "decode_ms": r["t_dec"] * 1e3, "decode_GBps": gbs, "frac": gbs / peak,
+            "frac_nominal_8TBps": gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": r["dbytes_dec"],
+            "traffic": kernel_traffic(W.name), "step_ms": r["t_step"] * 1e3, "tokens_per_s": W.B / r["t_step"],
+            "append_bulk": {"ms": pf["ms"], "calibrating": pf["calibrating"],
+                            "GBps_2R_plus_W": pf["bytes"] / t_pf / 1e9, "frac_2R_plus_W": pf["bytes"] / t_pf / 1e9 / peak,
+                            "GBps_R_plus_W": pf["bytes_r_plus_w"] / t_pf / 1e9,
+                            "frac_R_plus_W": pf["bytes_r_plus_w"] / t_pf / 1e9 / peak},
+            "device_status": list(r["status"])}
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    flush = L2Flush(dev)
+    sampler = ClockSampler(local_rank)  # samples the whole GPU section, every workload
+    with sampler:
+        r = measure_workload(args.workload, rank, world, dev, args.steps, args.warmup, stream, flush)
+        per_config = None
+        if world == 1 and not args.no_per_config:
+            peak, _ = measured_peak()
+            per_config = []
+            for name in PER_CONFIG:
+                if name == args.workload:
+                    per_config.append(config_summary(r, peak))
+                    continue
+                rc = measure_workload(name, rank, world, dev, min(args.steps, 30), 3, stream, flush, e2e=False)
+                per_config.append(config_summary(rc, peak))
+                del rc
+                torch.cuda.empty_cache()
+        torch.cuda.synchronize()
+    r["clocks"] = sampler.summary()
+    r["per_config"] = per_config
+    return r
 
 
 def run_e2e(G, W, stream, flush, n, step0):
@@ -563,6 +612,17 @@ def run_e2e(G, W, stream, flush, n, step0):
 
 
 # ---------------------------------------------------------------- quantization error
+def _rope_rows(K, theta):
+    """Rotate-half RoPE of key rows K [T, 128] at positions 0..T-1 (fp64), for the error reference
+    of caches that hold keys before RoPE."""
+    T, D = K.shape
+    inv = theta ** (-2.0 * np.arange(D // 2) / D)
+    ang = np.arange(T)[:, None] * inv[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = K[:, :D // 2], K[:, D // 2:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=1)
+
+
 def _f64(a, bf16):
     a = np.asarray(a)
     if bf16:
@@ -598,7 +658,8 @@ def quant_error(G, W, stream, n_pairs=8):
         K = _f64(synth.keys(W, b, b + 1, h, h + 1, 0, L)[0, 0], W.bf16)
         V = _f64(synth.values(W, b, b + 1, h, h + 1, 0, L)[0, 0], W.bf16)
         qs = q[b, h * W.G:(h + 1) * W.G]
-        sc = qs @ K.T * scale
+        Kr = _rope_rows(K, W.prerope_theta) if W.prerope_theta > 0 else K
+        sc = qs @ Kr.T * scale
         pr = np.exp(sc - sc.max(axis=1, keepdims=True))
         ref = (pr @ V) / pr.sum(axis=1, keepdims=True)
         diffs.append(out[b, h * W.G:(h + 1) * W.G] - ref)
@@ -637,7 +698,8 @@ class OracleUnit:
         K = synth.keys(w, b, b + 1, h, h + 1, 0, pre + 1)
         V = synth.values(w, b, b + 1, h, h + 1, 0, pre + 1)
         cap = (pre + 1 + 127) // 128 * 128
-        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group)
+        self.oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group,
+                              rope_theta=w.prerope_theta)
         calib = w.k_scheme in CALIBRATED or w.v_scheme in CALIBRATED
         self.oc.append(K[:, :, :pre], V[:, :, :pre], w.bf16, calibrate=calib)
         self.saved = (self.oc.c.len, self.oc.c.res)
@@ -711,6 +773,10 @@ def oracle_time(w, seconds, max_units=8):
     return tb, tt, steps, desc
 
 
+def dtype_of(w):
+    return DTYPE_NAME[w.k_scheme] + ("/" + DTYPE_NAME[w.v_scheme] if w.v_scheme != w.k_scheme else "")
+
+
 def emit(obj):
     print(json.dumps(obj), flush=True)
 
@@ -721,12 +787,14 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = synth.workloads()[args.workload]
-    dtype = DTYPE_NAME[w.k_scheme] + ("/" + DTYPE_NAME[w.v_scheme] if w.v_scheme != w.k_scheme else "")
+    dtype = dtype_of(w)
     config = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,
               "k_scheme": w.k_scheme, "v_scheme": w.v_scheme,
               "context": (f"uniform {w.len_lo}..{w.len_hi}" if w.paged else w.prefill_tokens()),
               "layout": "paged/16" if w.paged else "dense",
               "rotation": "walsh-hadamard" if w.rotate else "none",
+              "keys": (f"cached before RoPE, RoPE (base {w.prerope_theta:g}) applied at decode" if w.prerope_theta > 0
+                       else "cached as given"),
               "group": w.group,
               "step": ("decode only" if w.name == "tiny_int8" else "append 1 token per sequence + decode"),
               "l2": "flushed before every timed step (256 MiB write, then 256 MiB read), outside the event interval",
@@ -769,6 +837,7 @@ def main():
     roofline = {"bound": "hbm", "kernel": "decode attention call (split-KV kernel + LSE merge)",
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "frac_nominal_8TBps": achieved / NOMINAL_HBM_GBS,
                 "algorithmic_bytes_per_launch": r["dbytes_dec"], "launch_ms": r["t_dec"] * 1e3,
                 "traffic": kernel_traffic(W.name)}
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -783,6 +852,10 @@ def main():
     out["append_bulk"] = {"what": "prefill quantize-append of the whole context (calibrating when the scheme "
                                   "has batch-wide scales), mean of 3, L2 flushed before each",
                           "ms": pf["ms"], "algorithmic_bytes": pf["bytes"], "GBps": pf_gbs, "frac": pf_gbs / peak,
+                          "count": "2R+W when calibrating (the block is read for the statistics, then to quantize)",
+                          "algorithmic_bytes_r_plus_w": pf["bytes_r_plus_w"],
+                          "GBps_r_plus_w": pf["bytes_r_plus_w"] / (pf["ms"] / 1e3) / 1e9,
+                          "frac_r_plus_w": pf["bytes_r_plus_w"] / (pf["ms"] / 1e3) / 1e9 / peak,
                           "tokens_per_seq": pf["tokens"] if not W.paged else "variable",
                           "calibrating": pf["calibrating"]}
     if r["e2e"]:
@@ -808,6 +881,8 @@ def main():
                                "sample": desc}
         rate, ncores, desc_all = oracle_time_all_cores(W, args.cpu_seconds / 2)
         out["cpu_baseline"]["all_cores"] = {"value": rate / 1e9, "unit": UNIT, "cores": ncores, "sample": desc_all}
+    if r["per_config"] is not None:
+        out["per_config"] = r["per_config"]
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -29,11 +29,12 @@ __global__ void bounded_wait_check_kernel(uint32_t* status) {
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int kMaxQHeads = 8192;  // query heads per sequence the decode accepts
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_INT4_SYM_PER_GROUP; }
+bool valid_scheme(int s) { return s >= KVQ_FP8_E4M3_PER_TENSOR && s <= KVQ_KIVI_INT2_F16; }
 
 bool needs_scale(int s) { return true; }
 bool needs_zp(int s) { return s == KVQ_UINT8_ASYM_PER_CHANNEL; }
@@ -100,6 +101,10 @@ kvq_status kvq_validate(const kvq_cache_desc* d) {
   const bool kivi_k = is_kivi(d->k_scheme), kivi_v = is_kivi(d->v_scheme);
   if (d->rotation != KVQ_ROTATE_NONE && d->rotation != KVQ_ROTATE_HADAMARD) return KVQ_ERR_INVALID_ARG;
   if (d->rotation != KVQ_ROTATE_NONE && (kivi_k || kivi_v)) return KVQ_ERR_UNSUPPORTED;
+  // pre-RoPE keys: a finite base >= 0; with 8-bit key codes, without the Hadamard rotation
+  if (!(d->rope_theta >= 0.0f) || d->rope_theta > 3.0e38f) return KVQ_ERR_INVALID_ARG;
+  if (d->rope_theta > 0.0f && (d->rotation != KVQ_ROTATE_NONE || code_bits(d->k_scheme) != 8))
+    return KVQ_ERR_UNSUPPORTED;
   if (kivi_k || kivi_v) {
     if (d->k_scheme != d->v_scheme) return KVQ_ERR_UNSUPPORTED;
     if (d->layout == KVQ_PAGED) return KVQ_ERR_UNSUPPORTED;
@@ -112,15 +117,26 @@ kvq_status kvq_validate(const kvq_cache_desc* d) {
   if ((d->k_scheme == KVQ_INT4_SYM_PER_GROUP || d->v_scheme == KVQ_INT4_SYM_PER_GROUP) &&
       d->group_size != 32 && d->group_size != 64 && d->group_size != 128)
     return KVQ_ERR_UNSUPPORTED;
+  // The decode's split plan counts (sequence, kv head, head group) pairs and their tiles in
+  // 32-bit integers: bound the pair count, and below the tile count of a full cache.
+  if (d->num_q_heads > kMaxQHeads) return KVQ_ERR_UNSUPPORTED;
+  const uint64_t pairs = (uint64_t)d->batch * d->num_kv_heads * (uint64_t)((d->num_q_heads / d->num_kv_heads + 7) / 8);
+  if (pairs >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
   if (d->layout == KVQ_DENSE) {
     if (d->capacity < 128 || d->capacity % 128 != 0) return KVQ_ERR_INVALID_ARG;
     if ((uint64_t)d->batch * d->num_kv_heads * (uint64_t)d->capacity >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    // quantized tiles of 128 tokens plus at most four residual tiles of 32 per pair
+    if (pairs * (uint64_t)(d->capacity / 128 + 4) >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
     if (d->num_quantized < 0 || d->num_quantized > d->capacity) return KVQ_ERR_INVALID_ARG;
     if ((kivi_k) && d->num_quantized % 128 != 0) return KVQ_ERR_INVALID_ARG;
   } else {
     if (d->page_size != 16 && d->page_size != 32 && d->page_size != 64) return KVQ_ERR_UNSUPPORTED;
     if (d->max_pages_per_seq < 1 || d->num_pages < 1) return KVQ_ERR_INVALID_ARG;
     if ((uint64_t)d->num_pages * d->num_kv_heads * (uint64_t)d->page_size >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    // a sequence's longest length, and every sequence at that length in 128-token tiles
+    const uint64_t maxlen = (uint64_t)d->max_pages_per_seq * (uint64_t)d->page_size;
+    if (maxlen >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
+    if (pairs * ((maxlen + 127) / 128) >= (1ull << 31)) return KVQ_ERR_UNSUPPORTED;
     if (!d->page_table || !d->seq_lens) return KVQ_ERR_INVALID_ARG;
   }
   if (!d->k_codes || !d->v_codes || !d->k_scale || !d->v_scale || !d->dev_status) return KVQ_ERR_INVALID_ARG;
@@ -146,13 +162,13 @@ kvq_status kvq_cache_bytes(const kvq_cache_desc* d, kvq_footprint* out) {
   for (int side = 0; side < 2; ++side) {
     const int s = side ? d->v_scheme : d->k_scheme;
     const uint64_t n = scale_elems(d, side);
-    uint64_t bytes = n * 4;
+    uint64_t bytes = n * (kivi_f16(s) ? 2 : 4);     // fp16 or fp32 elements
     if (is_kivi(s)) bytes *= 2;                       // scale + minimum
     if (needs_zp(s)) bytes += (uint64_t)d->num_kv_heads * d->head_dim;  // uint8 zero points
     meta += bytes;
     if (s == KVQ_INT8_SYM_PER_TOKEN) per_token_meta += 4.0;
     if (s == KVQ_INT4_SYM_PER_GROUP) per_token_meta += 4.0 * d->head_dim / d->group_size;  // fp32 per group
-    if (is_kivi(s)) per_token_meta += 8.0 * d->head_dim / 32.0;  // (scale, min) per 32 tokens or channels
+    if (is_kivi(s)) per_token_meta += (kivi_f16(s) ? 4.0 : 8.0) * d->head_dim / 32.0;  // (scale, min) per 32 elements
   }
   f.meta_bytes = meta;
   f.residual_bytes = is_kivi(d->k_scheme)
@@ -295,6 +311,7 @@ kvq_status kvq_dequantize(const kvq_cache_desc* d, int32_t which, float* out, in
   return from_cuda(launch_dequantize(p, static_cast<cudaStream_t>(stream)));
 }
 
+
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* d) {
   if (!d || d->num_kv_heads < 1 || d->batch < 1 || d->num_q_heads < d->num_kv_heads) return 0;
   const int G = d->num_q_heads / d->num_kv_heads;
@@ -313,7 +330,8 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   const size_t need = kvq_decode_workspace_bytes(d);
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return KVQ_ERR_WORKSPACE;
   const bool paged = d->layout == KVQ_PAGED;
-  if (!decode_supported(d->k_scheme, d->v_scheme, paged, d->group_size)) return KVQ_ERR_UNSUPPORTED;
+  const bool rope = d->rope_theta > 0.0f;
+  if (!decode_supported(d->k_scheme, d->v_scheme, paged, d->group_size, rope)) return KVQ_ERR_UNSUPPORTED;
   const int G = d->num_q_heads / d->num_kv_heads;
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
@@ -347,6 +365,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   p.status = d->dev_status;
   p.rotate = d->rotation == KVQ_ROTATE_HADAMARD;
   p.group = d->group_size;
+  p.rope_theta = d->rope_theta;
   p.q = q;
   p.q_bf16 = q_dtype == KVQ_BF16;
   p.softmax_scale = softmax_scale;

@@ -18,6 +18,7 @@
 #include <cuda_fp8.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kvq_device.cuh"
 #include "kvq_internal.h"
@@ -719,8 +720,6 @@ __global__ void __launch_bounds__(256) requant_kernel(AppendParams p, RescaleWs 
   }
 }
 
-int sm_count();
-
 template <int SCHEME>
 void launch_requant(const AppendParams& p, const RescaleWs& ws, int side, cudaStream_t st) {
   const long long span = p.paged ? (long long)p.max_pages * p.page_size : p.pos0;
@@ -744,9 +743,26 @@ void launch_requant_side(const AppendParams& p, const RescaleWs& ws, int side, c
 }
 
 
+// A sequence's length grows by its new tokens only when every page they land on is a page of
+// the pool: an append that met a bad page or ran past the page table (flagged by the store) is
+// refused for that sequence, which keeps its length and so never shows rows that were not
+// written. The rows the store did write past the kept length stay invisible to decode.
 __global__ void seq_lens_advance_kernel(AppendParams p) {
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < p.B) p.seq_lens[b] += new_count(p, b);
+  if (b >= p.B) return;
+  const int n = new_count(p, b);
+  if (n == 0) return;
+  const int L = p.seq_lens[b];
+  const long long last = (long long)L + n - 1;
+  bool ok = L >= 0 && last / p.page_size < p.max_pages;
+  for (int pi = L / p.page_size; ok && pi <= (int)(last / p.page_size); ++pi) {
+    const int page = p.page_table[(size_t)b * p.max_pages + pi];
+    ok = page >= 0 && page < p.num_pages;
+  }
+  if (ok)
+    p.seq_lens[b] = L + n;
+  else
+    flag(p.status, L < 0 || last / p.page_size >= p.max_pages ? KVQ_DEV_BAD_LENGTH : KVQ_DEV_BAD_PAGE);
 }
 
 // ------------------------------------------------------------------ KIVI
@@ -764,14 +780,32 @@ __device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
 }
 
 
+// clamp(rne(z), 0, qmax) for any finite quotient z (the stored fp16 minimum may lie above a
+// value, and a saturated or underflowing fp16 scale may make z large): z is first bounded to
+// [-1, qmax + 1], where RN(z + 1.5 * 2^23) holds rne(z) in its low bits, then the code clamped.
+template <int kQmax>
+__device__ __forceinline__ uint32_t signed_code(float z) {
+  z = fminf(fmaxf(z, -1.0f), (float)kQmax + 1.0f);
+  const int c = (int)(__float_as_uint(__fadd_rn(z, kRoundMagic)) - (uint32_t)kRoundMagicBits);
+  return (uint32_t)(c < 0 ? 0 : (c > kQmax ? kQmax : c));
+}
+
 // Two KIVI codes at once: d = RN(v - min), then the division-free quotient of `quot` in its
 // residual form r = RN(d - q * s) (the same values; zero signs do not reach integer codes),
 // then rne. v2 holds the two values; lo2, s2, ns2 (= -s), y2 (= RN(1/s)) the lanes' group terms.
-template <int kQmax>
+// kSigned: the minimum is the stored fp16 one, so d may be negative (or the quotient large).
+template <int kQmax, bool kSigned = false>
 __device__ __forceinline__ void kivi_code2(f32x2 v2, f32x2 lo2, f32x2 s2n, f32x2 y2, uint32_t& c0, uint32_t& c1) {
   const f32x2 d = sub2(v2, lo2);
   const f32x2 q = mul2(d, y2);
   const f32x2 r = fma2(q, s2n, d);
+  if constexpr (kSigned) {
+    float z0, z1;
+    upk2(fma2(r, y2, q), z0, z1);
+    c0 = signed_code<kQmax>(z0);
+    c1 = signed_code<kQmax>(z1);
+    return;
+  }
   const f32x2 t = add2(fma2(r, y2, q), pk2(kRoundMagic, kRoundMagic));
   float t0, t1;
   upk2(t, t0, t1);
@@ -781,18 +815,30 @@ __device__ __forceinline__ void kivi_code2(f32x2 v2, f32x2 lo2, f32x2 s2n, f32x2
   c1 = c1 < (uint32_t)kQmax ? c1 : (uint32_t)kQmax;
 }
 
-// Code of d = RN(x - min) >= 0 with step s: rne(RN(d / s)); d <= max - min keeps it <= qmax.
-template <int kQmax>
+// Code of d = RN(x - min) with step s: rne(RN(d / s)); with the exact fp32 minimum d >= 0 and
+// d <= max - min keeps it in [0, qmax]; with the stored fp16 minimum it is clamped (kSigned).
+template <int kQmax, bool kSigned = false>
 __device__ __forceinline__ uint32_t kivi_code(float d, float s, float y, bool fast) {
   float q;
   const float z = fast ? quot(d, s, y, q) : __fdiv_rn(d, s);
+  if constexpr (kSigned) return signed_code<kQmax>(z);
   const uint32_t c = __float_as_uint(__fadd_rn(z, kRoundMagic)) - (uint32_t)kRoundMagicBits;
   return c < (uint32_t)kQmax ? c : (uint32_t)kQmax;
 }
 
+// fp16 storage of a KIVI scale or minimum: nearest-even, saturating at +-65504 (the value must
+// stay finite); returns the stored bits and the stored value as fp32 (exact).
+__device__ __forceinline__ uint32_t f16_store(float x, float& stored) {
+  const __half h = __float2half_rn(fminf(fmaxf(x, -65504.0f), 65504.0f));
+  stored = __half2float(h);
+  return (uint32_t)__half_as_ushort(h);
+}
+
 // One block per (R-token chunk, b*H + h): quantize R consecutive tokens of the combined
 // stream (old residual tokens, then the new block) into the cache at pos0 + chunk*R.
-template <int kBits>
+// kF16: scales and minima stored as fp16 (KIVI_INT4_F16 / KIVI_INT2_F16), codes from the stored
+// values.
+template <int kBits, bool kF16>
 __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int r_old) {
   constexpr int R = 128, G = 32, kQmax = (1 << kBits) - 1, kPer = 8 / kBits;
   constexpr int kRowBytes = kHeadDim * kBits / 8;
@@ -858,6 +904,7 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
     }
     float lo[2], sc[2], yr[2];
     bool fast[2];
+    uint32_t s16[2], m16[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       lo[k] = __uint_as_float(k ? (mn2 & 0xFFFF0000u) : (mn2 << 16));
@@ -865,10 +912,19 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
       if (lo[k] == 0.0f) lo[k] = 0.0f;
       if (hi == 0.0f) hi = 0.0f;
       sc[k] = __fdiv_rn(__fsub_rn(hi, lo[k]), (float)kQmax);
+      if constexpr (kF16) {  // the stored values take over
+        s16[k] = f16_store(sc[k], sc[k]);
+        m16[k] = f16_store(lo[k], lo[k]);
+      } else {
+        p.k_scale[meta + c0 + k] = sc[k];
+        p.k_zero[meta + c0 + k] = lo[k];
+      }
       yr[k] = __frcp_rn(sc[k]);
       fast[k] = sc[k] != 0.0f && quot_range(sc[k]);
-      p.k_scale[meta + c0 + k] = sc[k];
-      p.k_zero[meta + c0 + k] = lo[k];
+    }
+    if constexpr (kF16) {  // channels c0, c0 + 1: one 32-bit word of halves per array
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.k_scale) + meta + c0) = s16[0] | (s16[1] << 16);
+      *reinterpret_cast<uint32_t*>(reinterpret_cast<uint16_t*>(p.k_zero) + meta + c0) = m16[0] | (m16[1] << 16);
     }
     if (fast[0] && fast[1]) {
       // both channels of a token in one packed operation
@@ -876,7 +932,8 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
 #pragma unroll
       for (int j = 0; j < G; ++j) {
         uint32_t a, bb;
-        kivi_code2<kQmax>(pk2(__uint_as_float(raw[j] << 16), __uint_as_float(raw[j] & 0xFFFF0000u)), lo2, s2n, y2, a, bb);
+        kivi_code2<kQmax, kF16>(pk2(__uint_as_float(raw[j] << 16), __uint_as_float(raw[j] & 0xFFFF0000u)), lo2, s2n,
+                                y2, a, bb);
         bits[j / 4] |= (a << (8 * (j % 4) + shift0)) | (bb << (8 * (j % 4) + shift0 + kBits));
       }
     } else {
@@ -886,7 +943,7 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
         auto val = [&](int j) { return __uint_as_float(k ? (raw[j] & 0xFFFF0000u) : (raw[j] << 16)); };
 #pragma unroll
         for (int j = 0; j < G; ++j)
-          bits[j / 4] |= kivi_code<kQmax>(__fsub_rn(val(j), lo[k]), sc[k], yr[k], fast[k])
+          bits[j / 4] |= kivi_code<kQmax, kF16>(__fsub_rn(val(j), lo[k]), sc[k], yr[k], fast[k])
                          << (8 * (j % 4) + shift0 + k * kBits);
       }
     }
@@ -924,7 +981,12 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
     float hi = fmaxf(__uint_as_float(mx2 << 16), __uint_as_float(mx2 & 0xFFFF0000u));
     if (lo == 0.0f) lo = 0.0f;
     if (hi == 0.0f) hi = 0.0f;
-    const float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+    float sc = __fdiv_rn(__fsub_rn(hi, lo), (float)kQmax);
+    uint32_t s16 = 0u, m16 = 0u;
+    if constexpr (kF16) {  // the stored values take over
+      s16 = f16_store(sc, sc);
+      m16 = f16_store(lo, lo);
+    }
     uint32_t words[G * kBits / 32];
 #pragma unroll
     for (int w = 0; w < G * kBits / 32; ++w) words[w] = 0u;
@@ -936,13 +998,14 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
 #pragma unroll
         for (int i = 0; i < G / 2; ++i) {
           uint32_t a, bb;
-          kivi_code2<kQmax>(pk2(__uint_as_float(raw[i] << 16), __uint_as_float(raw[i] & 0xFFFF0000u)), lo2, s2n, y2, a, bb);
+          kivi_code2<kQmax, kF16>(pk2(__uint_as_float(raw[i] << 16), __uint_as_float(raw[i] & 0xFFFF0000u)), lo2, s2n,
+                                  y2, a, bb);
           words[(2 * i * kBits) / 32] |= (a << ((2 * i * kBits) % 32)) | (bb << ((2 * i * kBits) % 32 + kBits));
         }
       } else {
 #pragma unroll
         for (int i = 0; i < G; ++i)
-          words[(i * kBits) / 32] |= kivi_code<kQmax>(__fsub_rn(val(i), lo), sc, y, false) << ((i * kBits) % 32);
+          words[(i * kBits) / 32] |= kivi_code<kQmax, kF16>(__fsub_rn(val(i), lo), sc, y, false) << ((i * kBits) % 32);
       }
     }
     const size_t crow = ((size_t)b * p.H + h) * (size_t)p.cap + (size_t)(pos0 + tok);
@@ -952,8 +1015,13 @@ __global__ void __launch_bounds__(256, 3) kivi_flush_kernel(AppendParams p, int 
     } else {
       *reinterpret_cast<uint2*>(dst) = make_uint2(words[0], words[1]);
     }
-    p.v_scale[crow * (kHeadDim / G) + j] = sc;
-    p.v_zero[crow * (kHeadDim / G) + j] = lo;
+    if constexpr (kF16) {
+      reinterpret_cast<uint16_t*>(p.v_scale)[crow * (kHeadDim / G) + j] = (uint16_t)s16;
+      reinterpret_cast<uint16_t*>(p.v_zero)[crow * (kHeadDim / G) + j] = (uint16_t)m16;
+    } else {
+      p.v_scale[crow * (kHeadDim / G) + j] = sc;
+      p.v_zero[crow * (kHeadDim / G) + j] = lo;
+    }
   }
   __syncthreads();
   // key codes: R rows x kRowBytes, contiguous in the cache
@@ -1045,13 +1113,21 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
             case KVQ_INT4_SYM_PER_GROUP:
               v = __fmul_rn((float)(q >= 8 ? q - 16 : q), p.scale[row * (kHeadDim / p.group) + d / p.group]);
               break;
-            default: {  // KIVI
+            default: {  // KIVI: fl(fl(q * s) + min), s and min as stored (fp32 or fp16)
               size_t m;
               if (p.which == 0)
                 m = (((size_t)b * p.H + h) * (size_t)(p.cap / 32) + (size_t)(t / 32)) * kHeadDim + d;
               else
                 m = row * (kHeadDim / 32) + d / 32;
-              v = __fadd_rn(__fmul_rn((float)q, p.scale[m]), p.zero[m]);
+              float sm, mn;
+              if (kivi_f16(scheme)) {
+                sm = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(p.scale)[m]));
+                mn = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(p.zero)[m]));
+              } else {
+                sm = p.scale[m];
+                mn = p.zero[m];
+              }
+              v = __fadd_rn(__fmul_rn((float)q, sm), mn);
             }
           }
           y[k] = v;
@@ -1066,18 +1142,19 @@ __global__ void __launch_bounds__(256) dequantize_kernel(DequantParams p) {
 }
 
 // ------------------------------------------------------------------ launchers
-// Streaming multiprocessors of the current device (queried once per device).
+// Streaming multiprocessors of the current device, queried once per device ordinal (devices
+// past the cache are queried on every call).
 int sm_count() {
-  static int cached[64] = {0};
+  constexpr int kCached = 64;
+  static std::atomic<int> cached[kCached];
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (cached[dev] == 0) {
-    int n = 0;
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = (dev >= 0 && dev < kCached) ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    if (dev >= 0 && dev < kCached) cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 template <int KS, int VS>
@@ -1135,15 +1212,13 @@ cudaError_t launch_append(const AppendParams& p, void* workspace, int mode, int 
       const int bits = code_bits(p.k_scheme);
       const size_t smem = 2 * 128 * kHeadDim * 2 + 128 * (kHeadDim * bits / 8);
       dim3 grid(flushed / 128, p.B * p.H);
-      if (bits == 4) {
-        cudaFuncSetAttribute(kivi_flush_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kivi_flush_kernel<4><<<grid, 256, smem, st>>>(p, r_old);
-        count_launches(1);
-      } else {
-        cudaFuncSetAttribute(kivi_flush_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kivi_flush_kernel<2><<<grid, 256, smem, st>>>(p, r_old);
-        count_launches(1);
-      }
+      void (*kern)(AppendParams, int) =
+          kivi_f16(p.k_scheme) ? (bits == 4 ? kivi_flush_kernel<4, true> : kivi_flush_kernel<2, true>)
+                               : (bits == 4 ? kivi_flush_kernel<4, false> : kivi_flush_kernel<2, false>);
+      const cudaError_t ea = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (ea != cudaSuccess) return ea;
+      kern<<<grid, 256, smem, st>>>(p, r_old);
+      count_launches(1);
     }
     // residual update: only new tokens ever move into it
     const int count = flushed > 0 ? r_new : p.n_new;

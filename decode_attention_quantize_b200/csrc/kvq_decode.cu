@@ -49,8 +49,8 @@ __host__ __device__ constexpr int fmt_of(int s) {
   return s == KVQ_FP8_E4M3_PER_TENSOR      ? FMT_E4M3
          : s == KVQ_FP8_E5M2_PER_TENSOR    ? FMT_E5M2
          : s == KVQ_UINT8_ASYM_PER_CHANNEL ? FMT_U8
-         : s == KVQ_KIVI_INT4              ? FMT_U4
-         : s == KVQ_KIVI_INT2              ? FMT_U2
+         : (s == KVQ_KIVI_INT4 || s == KVQ_KIVI_INT4_F16) ? FMT_U4
+         : (s == KVQ_KIVI_INT2 || s == KVQ_KIVI_INT2_F16) ? FMT_U2
          : s == KVQ_INT4_SYM_PER_GROUP     ? FMT_S4
                                            : FMT_S8;
 }
@@ -66,13 +66,19 @@ __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 __host__ __device__ constexpr int rup(int a, int m) { return (a + m - 1) / m * m; }
 
 // NG: scales per token row of an INT4 per-group side (4, 2 or 1 for groups of 32, 64, 128)
-template <int KS, int VS, bool PAGED, int NG = 4>
+// ROPE: keys cached before RoPE (8-bit codes), rotated at their positions in the kernel
+template <int KS, int VS, bool PAGED, int NG = 4, bool ROPE = false>
 struct Cfg {
   static constexpr bool kPaged = PAGED;
   static constexpr int kNG = NG;
+  static constexpr bool kRope = ROPE;
+  static_assert(!ROPE || (row_bytes(KS) == kHeadDim && fold_of(KS) != FOLD_GROUP), "RoPE keys: 8-bit codes");
   static constexpr int kKFmt = fmt_of(KS), kVFmt = fmt_of(VS);
   static constexpr int kKFold = fold_of(KS), kVFold = fold_of(VS);
   static constexpr bool kKivi = kKFold == FOLD_KIVI;
+  // KIVI scale and minimum stored as fp16 (2 bytes per element instead of 4)
+  static constexpr bool kHalfMeta = kivi_f16(KS);
+  static constexpr int kMetaElem = kHalfMeta ? 2 : 4;
   // values with one scale per (token, 32-channel group): KIVI and INT4 per group
   static constexpr bool kGroupV = kVFold == FOLD_KIVI || kVFold == FOLD_GROUP;
   // 32 tokens per consumer warp per tile: two independent 16-token MMA chains per warp, and
@@ -84,20 +90,23 @@ struct Cfg {
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTS * kKRow;     // multiple of 1024 (swizzle atom)
   static constexpr int kOffKM = kOffV + kTS * kVRow;
-  static constexpr int kKMeta = kKivi ? (kTS / 32) * kHeadDim * 4 * 2
+  static constexpr int kKMeta = kKivi ? (kTS / 32) * kHeadDim * kMetaElem * 2
                                 : (kKFold == FOLD_TOKEN ? kTS * 4 : (kKFold == FOLD_GROUP ? kTS * NG * 4 : 0));
   static constexpr int kOffVM = kOffKM + kKMeta;
-  static constexpr int kVMeta = kKivi ? kTS * 4 * 4 * 2
+  static constexpr int kVMeta = kKivi ? kTS * 4 * kMetaElem * 2
                                 : (kVFold == FOLD_TOKEN ? kTS * 4 : (kVFold == FOLD_GROUP ? kTS * NG * 4 : 0));
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
   // heads staged per pass of the per-pair warp merge: all eight for INT4 KIVI (whose register
   // allocation suffers from the two-pass form), else four (half the staging, room for a stage)
-  static constexpr int kMergeHeads = KS == KVQ_KIVI_INT4 ? 8 : 4;
+  static constexpr int kMergeHeads = (kKivi && kKFmt == FMT_U4) ? 8 : 4;
   // 128-token stages: three when three still fit next to a second CTA on the SM
-  static constexpr int kFixedBytes =
-      2048 + kCW * kMergeHeads * kHeadDim * 4 + kCW * 8 * 4 * 2 + kCW * kMergeHeads * 4 * 4 + 8 * 144 * 4 + 1024;
+  // RoPE: the inverse frequencies (64 fp64), each warp's (base angle, frequency) pairs (64 float2)
+  // and the kv head's per-channel key scales (128 fp32)
+  static constexpr int kRopeBytes = ROPE ? 64 * 8 + kCW * 64 * 8 + kHeadDim * 4 : 0;
+  static constexpr int kFixedBytes = 2048 + kCW * kMergeHeads * kHeadDim * 4 + kCW * 8 * 4 * 2 +
+                                     kCW * kMergeHeads * 4 * 4 + 8 * 144 * 4 + kRopeBytes + 1024;
   static constexpr int kStages = (3 * kStageBytes + kFixedBytes <= 112 * 1024) ? 3 : 2;
   static constexpr int kMinBlocks = 2;  // resident CTAs per SM the registers (168) are sized for
   static constexpr int kOffDesc = kStages * kStageBytes;
@@ -108,7 +117,8 @@ struct Cfg {
   static constexpr int kOffRedZ = kOffRedL + kCW * 8 * 4;
   static constexpr int kOffQ = kOffRedZ + kCW * kMergeHeads * 4 * 4;
   static constexpr int kQStride = 144;          // q row stride (floats): see q_off
-  static constexpr int kSmemBytes = kOffQ + 8 * kQStride * 4 + 1024;  // + alignment slack
+  static constexpr int kOffRope = kOffQ + 8 * kQStride * 4;  // 8-byte aligned
+  static constexpr int kSmemBytes = kOffRope + kRopeBytes + 1024;  // + alignment slack
   static_assert(kMinBlocks * (kSmemBytes + 1024) <= 227 * 1024, "the resident CTAs must fit in shared memory");
 };
 
@@ -265,10 +275,15 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar);
       if constexpr (C::kKivi) {
         const size_t g0 = (pair_row * (p.cap / 32) + d.t0 / 32) * kHeadDim;
-        bulk_g2s(sb + C::kOffKM, p.k_scale + g0, C::kKMeta / 2, bar);
-        bulk_g2s(sb + C::kOffKM + C::kKMeta / 2, p.k_zero + g0, C::kKMeta / 2, bar);
-        bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * 4, C::kVMeta / 2, bar);
-        bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, p.v_zero + row0 * 4, C::kVMeta / 2, bar);
+        // element offsets in bytes: fp32 or fp16 metadata
+        const uint8_t* ks8 = reinterpret_cast<const uint8_t*>(p.k_scale);
+        const uint8_t* kz8 = reinterpret_cast<const uint8_t*>(p.k_zero);
+        const uint8_t* vs8 = reinterpret_cast<const uint8_t*>(p.v_scale);
+        const uint8_t* vz8 = reinterpret_cast<const uint8_t*>(p.v_zero);
+        bulk_g2s(sb + C::kOffKM, ks8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
+        bulk_g2s(sb + C::kOffKM + C::kKMeta / 2, kz8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
+        bulk_g2s(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
+        bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
       } else {
         if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
         if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
@@ -396,6 +411,30 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return float2_to_f16x2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
 
+// Two bf16 values times the power of two f, as f16x2 (exact when the products lie in the f16
+// range with their 8 significant bits).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float f) {
+  return float2_to_f16x2(__uint_as_float(w << 16) * f, __uint_as_float(w & 0xFFFF0000u) * f);
+}
+
+// Power-of-two exponent that brings a bf16 residual row into the f16 range: lane i scans row i
+// (256-byte rows of 128 bf16 values at `row0`; rows >= n are empty) and returns the range shift
+// of the row's largest magnitude (0 for a zero row). Each lane starts at its own 16-byte chunk
+// so the 32 rows' loads spread over the banks.
+__device__ __forceinline__ int residual_row_shift(const uint8_t* row0, int n, int lane) {
+  uint32_t m = 0u;
+  if (lane < n) {
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row0 + lane * 256 + (((q + lane) & 15) << 4));
+      m = __vmaxu2(m, __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu));
+      m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    }
+  }
+  const uint32_t top = max(m & 0xFFFFu, m >> 16);  // bf16 magnitudes order like their bits
+  return top ? range_shift(bf16_bits_to_float(top)) : 0;
+}
+
 template <class T>
 __device__ __forceinline__ T lds(const uint8_t* p) {
   return *reinterpret_cast<const T*>(p);
@@ -446,21 +485,46 @@ struct Consumer {
 // lanes of a quarter warp (two heads, four blocks) cover all 32 banks.
 __device__ __forceinline__ int q_off(int j, int d) { return j * 144 + d + 4 * (d >> 5); }
 
+// Shared memory after the query staging, in kernels for keys cached before RoPE: the 64 inverse
+// frequencies (fp64), each consumer warp's 64 (base angle, frequency) pairs of its current tile,
+// and the kv head's 128 per-channel key scales.
+__device__ __forceinline__ double* rope_theta_s(const float* q_s) {
+  return reinterpret_cast<double*>(const_cast<float*>(q_s) + 8 * 144);
+}
+__device__ __forceinline__ float2* rope_angles(const float* q_s) {
+  return reinterpret_cast<float2*>(rope_theta_s(q_s) + 64);
+}
+__device__ __forceinline__ float* rope_key_scales(const float* q_s) {
+  return reinterpret_cast<float*>(rope_angles(q_s) + kCW * 64);
+}
+
+// Elements 4i .. 4i + 3 of a metadata array of fp32 or (kHalf) fp16 values, as fp32.
+template <bool kHalf>
+__device__ __forceinline__ float4 meta4(const void* base, int i) {
+  if constexpr (kHalf) {
+    const uint2 u = reinterpret_cast<const uint2*>(base)[i];
+    const float2 a = f16x2_to_float2(u.x), b = f16x2_to_float2(u.y);
+    return make_float4(a.x, a.y, b.x, b.y);
+  } else {
+    return reinterpret_cast<const float4*>(base)[i];
+  }
+}
+
 // Build Q' fragments (head g, this thread's 32 channels 32c..32c+31) from q_s, optionally
 // multiplied by a per-channel fold; with `zmin` also returns sum_d q_d * zmin_d over those
-// channels (the KIVI key-minimum term). Returns the power-of-two shift applied to Q'.
-template <int FMT>
-__device__ __forceinline__ int build_q(const float* q_s, const float* fold, const float* zmin, int g, int c,
+// channels (the KIVI key-minimum term). fold and zmin hold fp32, or fp16 when kHalf. Returns the
+// power-of-two shift applied to Q'.
+template <int FMT, bool kHalf = false>
+__device__ __forceinline__ int build_q(const float* q_s, const void* fold, const void* zmin, int g, int c,
                                        uint32_t (&qh)[8][2], uint32_t (&ql)[8][2], float* bias = nullptr) {
   const float4* qrow = reinterpret_cast<const float4*>(q_s + q_off(g, 32 * c));
-  const float4* frow = fold ? reinterpret_cast<const float4*>(fold + 32 * c) : nullptr;
   // pass 1: the largest |q'| of the warp sets the range shift
   float mx = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float4 q4 = qrow[i];
-    if (frow) {
-      const float4 f4 = frow[i];
+    if (fold) {
+      const float4 f4 = meta4<kHalf>(fold, 8 * c + i);
       q4.x *= f4.x; q4.y *= f4.y; q4.z *= f4.z; q4.w *= f4.w;
     }
     mx = fmaxf(mx, fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w))));
@@ -475,12 +539,12 @@ __device__ __forceinline__ int build_q(const float* q_s, const float* fold, cons
   for (int i = 0; i < 8; ++i) {
     const float4 q4 = qrow[i];
     float4 m4 = make_float4(sh, sh, sh, sh);
-    if (frow) {
-      const float4 f4 = frow[i];
+    if (fold) {
+      const float4 f4 = meta4<kHalf>(fold, 8 * c + i);
       m4 = make_float4(f4.x * sh, f4.y * sh, f4.z * sh, f4.w * sh);
     }
     if (zmin) {
-      const float4 z4 = reinterpret_cast<const float4*>(zmin + 32 * c)[i];
+      const float4 z4 = meta4<kHalf>(zmin, 8 * c + i);
       bs = fmaf(q4.x, z4.x, fmaf(q4.y, z4.y, fmaf(q4.z, z4.z, fmaf(q4.w, z4.w, bs))));
     }
     pl[4 * i] = q4.x * m4.x;
@@ -522,11 +586,62 @@ __device__ __forceinline__ int build_q_s4(const float* q_s, int g, int c, uint32
   return eq;
 }
 
+// Q fragments for keys cached before RoPE: lane c holds the rotation pairs i = 16c .. 16c + 15,
+// k-step ks and slot pair h holding the two channels (i, i + 64) of pair i = 16c + 2ks + h, so a
+// lane rotates a key pair without exchanging values. No fold (per-channel key scales are applied
+// to the keys before the rotation). Returns the power-of-two shift applied to Q.
+__device__ __forceinline__ int build_q_rope(const float* q_s, int g, int c, uint32_t (&qh)[8][2],
+                                            uint32_t (&ql)[8][2]) {
+  float pl[8][2][2];
+  float mx = 0.0f;
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 16 * c + 2 * ks + h;
+      pl[ks][h][0] = q_s[q_off(g, i)];
+      pl[ks][h][1] = q_s[q_off(g, i + 64)];
+      mx = fmaxf(mx, fmaxf(fabsf(pl[ks][h][0]), fabsf(pl[ks][h][1])));
+    }
+  mx = warp_max(mx);
+  const int eq = range_shift(mx);
+  const float sh = pow2i(eq);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) split_f16x2(pl[ks][h][0] * sh, pl[ks][h][1] * sh, qh[ks][h], ql[ks][h]);
+  return eq;
+}
+
+// 2 pi as a double-double and 1 / (2 pi): angle reduction of position * frequency
+constexpr double kTwoPiHi = 6.283185307179586;
+constexpr double kTwoPiLo = 2.4492935982947064e-16;
+constexpr double kInvTwoPi = 0.15915494309189535;
+
+// A warp's RoPE angles for one tile: for pair i (frequency theta_i = base^(-2i/128), fp64 in
+// shared memory), the angle at the warp's first position pos0 is reduced modulo 2 pi in fp64
+// (positions up to 2^31 keep it accurate to ~1e-11 rad at 131072) and kept as fp32 with theta_i
+// in fp32; the angle at pos0 + j (j < 32) is then fma(j, theta_i, base_i), within ~2e-6 rad.
+__device__ __forceinline__ void rope_warp_angles(const double* theta, float2* rw, int pos0, int lane) {
+  __syncwarp();  // the previous tile's reads of rw are done
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int i = 2 * lane + k;
+    const double a = (double)pos0 * theta[i];
+    const double n = rint(a * kInvTwoPi);
+    const double r = fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, a));
+    rw[i] = make_float2((float)r, (float)theta[i]);
+  }
+  __syncwarp();
+}
+
 // The value scales of token tok for the four 32-channel blocks of a row (KIVI, INT4 per group;
 // groups of 64 or 128 channels repeat each scale over the blocks they cover).
 template <class C>
 __device__ __forceinline__ float4 vscale4(const uint8_t* base, int tok) {
-  if constexpr (C::kKivi || C::kNG == 4) {
+  if constexpr (C::kKivi) {
+    return meta4<C::kHalfMeta>(base + C::kOffVM, tok);
+  } else if constexpr (C::kNG == 4) {
     return lds<float4>(base + C::kOffVM + tok * 16);
   } else if constexpr (C::kNG == 2) {
     const float2 s = lds<float2>(base + C::kOffVM + tok * 8);
@@ -552,13 +667,24 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     return ok;
   };
 
-  // (1) query fragments that change per tile (KIVI key groups, residual rows)
+  // bf16 residual rows (warp 0 alone) are brought into the f16 range row by row: lane i holds the
+  // power-of-two exponents of key row i and value row i; scores and probabilities take the
+  // inverse factors, so the products are unchanged and every bf16 value stays exact
+  int res_kx = 0, res_vx = 0;
+  if (C::kKivi && residual) {
+    res_kx = residual_row_shift(base, d.n, 4 * g + c);
+    res_vx = residual_row_shift(base + kRT * kHeadDim * 2, d.n, 4 * g + c);
+  }
+
+  // (1) per-tile state: RoPE angles at the warp's positions; query fragments that change per
+  // tile (KIVI key groups, residual rows)
+  if constexpr (C::kRope) rope_warp_angles(rope_theta_s(q_s), rope_angles(q_s) + w * 64, d.t0 + tok_base, 4 * g + c);
   if constexpr (C::kKivi) {
     if (!residual) {
-      const float* ksm = reinterpret_cast<const float*>(base + C::kOffKM) + w * kHeadDim;
-      const float* kzm = reinterpret_cast<const float*>(base + C::kOffKM + C::kKMeta / 2) + w * kHeadDim;
+      const uint8_t* ksm = base + C::kOffKM + w * kHeadDim * C::kMetaElem;
+      const uint8_t* kzm = base + C::kOffKM + C::kKMeta / 2 + w * kHeadDim * C::kMetaElem;
       float bs;
-      const int eq = build_q<C::kKFmt>(q_s, ksm, kzm, g, c, S.qh, S.ql, &bs);
+      const int eq = build_q<C::kKFmt, C::kHalfMeta>(q_s, ksm, kzm, g, c, S.qh, S.ql, &bs);
       bs += __shfl_xor_sync(0xffffffffu, bs, 1);
       bs += __shfl_xor_sync(0xffffffffu, bs, 2);
       S.bias[0] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c));
@@ -576,6 +702,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 
   // (2) S^T = K . Q'^T for kNSub blocks of 16 tokens; two accumulators halve the MMA chain
   float acc[C::kNSub][4];
+  float res_kinv[C::kNSub][2];  // residual: 2^-shift of the lane's key rows g and g + 8
 #pragma unroll
   for (int sb = 0; sb < C::kNSub; ++sb) {
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -596,10 +723,14 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         w1[4 * i] = y.x; w1[4 * i + 1] = y.y; w1[4 * i + 2] = y.z; w1[4 * i + 3] = y.w;
       }
       const bool split = S.qsplit;
+      const int x0 = __shfl_sync(0xffffffffu, res_kx, r0), x1 = __shfl_sync(0xffffffffu, res_kx, r1);
+      const float f0 = pow2i(x0), f1 = pow2i(x1);
+      res_kinv[sb][0] = pow2i(-x0);
+      res_kinv[sb][1] = pow2i(-x1);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        mma2(ks, bf16x2_to_f16x2(w0[2 * ks]), bf16x2_to_f16x2(w1[2 * ks]), bf16x2_to_f16x2(w0[2 * ks + 1]),
-             bf16x2_to_f16x2(w1[2 * ks + 1]), split);
+        mma2(ks, bf16x2_to_f16x2_scaled(w0[2 * ks], f0), bf16x2_to_f16x2_scaled(w1[2 * ks], f1),
+             bf16x2_to_f16x2_scaled(w0[2 * ks + 1], f0), bf16x2_to_f16x2_scaled(w1[2 * ks + 1], f1), split);
     } else if constexpr (C::kKFmt == FMT_U4) {
       const uint4 x = lds<uint4>(base + C::kOffK + swz<64>(r0, c));
       const uint4 y = lds<uint4>(base + C::kOffK + swz<64>(r1, c));
@@ -656,6 +787,62 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         const uint32_t u = i ? x.y : x.x, v = i ? y.y : y.x;
         mma2(ks, u2_pair(u, k0), u2_pair(v, k0), u2_pair(u, k0 + 1), u2_pair(v, k0 + 1), true);
       }
+    } else if constexpr (C::kRope) {
+      // keys cached before RoPE: chunk c (channels 16c .. 16c + 15) and chunk 4 + c (their RoPE
+      // partners 64 + 16c ..) of rows g and g + 8; each pair is dequantized (per-channel scales
+      // here; per-tensor and per-token scales multiply the score), rotated at its position in
+      // fp32 and split into f16 hi + lo, which both meet the exact query fragments
+      const uint4 xa = lds<uint4>(base + C::kOffK + swz<128>(r0, c));
+      const uint4 xb = lds<uint4>(base + C::kOffK + swz<128>(r0, 4 + c));
+      const uint4 ya = lds<uint4>(base + C::kOffK + swz<128>(r1, c));
+      const uint4 yb = lds<uint4>(base + C::kOffK + swz<128>(r1, 4 + c));
+      const float2* rw = rope_angles(q_s) + w * 64;
+      const float* kch = rope_key_scales(q_s);
+      const float j0 = (float)(r0 - tok_base), j1 = (float)(r1 - tok_base);
+      const bool split = S.qsplit;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t wa0 = word_of(xa, q), wb0 = word_of(xb, q), wa1 = word_of(ya, q), wb1 = word_of(yb, q);
+        if constexpr (C::kKFmt == FMT_S8) {
+          wa0 ^= 0x80808080u; wb0 ^= 0x80808080u; wa1 ^= 0x80808080u; wb1 ^= 0x80808080u;
+        }
+        uint32_t h[4][2];  // [row r0 A, r0 B, r1 A, r1 B][bytes 0-1, bytes 2-3] as f16x2
+        cvt8x4<C::kKFmt>(wa0, S.zpk[q][0], S.zpk[q][1], h[0][0], h[0][1]);
+        cvt8x4<C::kKFmt>(wb0, S.zpk[4 + q][0], S.zpk[4 + q][1], h[1][0], h[1][1]);
+        cvt8x4<C::kKFmt>(wa1, S.zpk[q][0], S.zpk[q][1], h[2][0], h[2][1]);
+        cvt8x4<C::kKFmt>(wb1, S.zpk[4 + q][0], S.zpk[4 + q][1], h[3][0], h[3][1]);
+        uint32_t ahi[2][2][2], alo[2][2][2];  // [row][pair of the k-step slot h][...]: f16x2 (i, i + 64)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 16 * c + 4 * q + e;
+          const float2 bt = rw[i];
+          const float2 fa0 = f16x2_to_float2(h[0][e >> 1]), fb0 = f16x2_to_float2(h[1][e >> 1]);
+          const float2 fa1 = f16x2_to_float2(h[2][e >> 1]), fb1 = f16x2_to_float2(h[3][e >> 1]);
+          // key pair (x, y) = (channel i, channel i + 64) of rows g and g + 8
+          float x0 = (e & 1) ? fa0.y : fa0.x, y0 = (e & 1) ? fb0.y : fb0.x;
+          float x1 = (e & 1) ? fa1.y : fa1.x, y1 = (e & 1) ? fb1.y : fb1.x;
+          if constexpr (C::kKFold == FOLD_CHANNEL) {
+            const float sx = kch[i], sy = kch[i + 64];
+            x0 *= sx; x1 *= sx; y0 *= sy; y1 *= sy;
+          }
+          float sn0, cs0, sn1, cs1;
+          __sincosf(fmaf(j0, bt.y, bt.x), &sn0, &cs0);
+          __sincosf(fmaf(j1, bt.y, bt.x), &sn1, &cs1);
+          // (x, y) -> (x cos - y sin, y cos + x sin)
+          const int ks_h = e & 1, kk = e >> 1;  // slot pair h and k-step 2q + kk of this pair
+          split_f16x2(fmaf(x0, cs0, -y0 * sn0), fmaf(y0, cs0, x0 * sn0), ahi[0][kk][ks_h], alo[0][kk][ks_h]);
+          split_f16x2(fmaf(x1, cs1, -y1 * sn1), fmaf(y1, cs1, x1 * sn1), ahi[1][kk][ks_h], alo[1][kk][ks_h]);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const int ks = 2 * q + kk;
+          float(&acc_k)[4] = kk ? a1 : a0;
+          mma_16816(acc_k, ahi[0][kk][0], ahi[1][kk][0], ahi[0][kk][1], ahi[1][kk][1], S.qh[ks][0], S.qh[ks][1]);
+          mma_16816(acc_k, alo[0][kk][0], alo[1][kk][0], alo[0][kk][1], alo[1][kk][1], S.qh[ks][0], S.qh[ks][1]);
+          if (split)
+            mma_16816(acc_k, ahi[0][kk][0], ahi[1][kk][0], ahi[0][kk][1], ahi[1][kk][1], S.ql[ks][0], S.ql[ks][1]);
+        }
+      }
     } else {
       // 8-bit codes, 128-byte rows: chunks 2c and 2c+1 of rows g and g+8 (swizzled)
       const uint4 x0 = lds<uint4>(base + C::kOffK + swz<128>(r0, 2 * c));
@@ -690,6 +877,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       const bool ok = tok_ok(tok);
       float mul = S.kmul;
       if constexpr (C::kKFold == FOLD_TOKEN) mul *= reinterpret_cast<const float*>(base + C::kOffKM)[tok];
+      if (C::kKivi && residual) mul *= res_kinv[sb][r];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         float sv;
@@ -775,6 +963,10 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
     smax = warp_max(smax);
     evn = smax > 0.0f ? range_shift(smax) : (S.ev_set ? S.ev : 15);
   }
+  if (C::kKivi && residual) {  // each value row's inverse factor plays the role of its scale
+    const float smax = warp_max(4 * g + c < d.n ? pow2i(-res_vx) : 0.0f);
+    evn = smax > 0.0f ? range_shift(smax) : (S.ev_set ? S.ev : 15);
+  }
   // rescale the accumulator only when some head's max moved or the exponent changed
   const bool moved = (alpha[0] != 1.0f) || (alpha[1] != 1.0f) || (S.ev_set && evn != S.ev);
   if (__any_sync(0xffffffffu, moved)) {
@@ -849,10 +1041,17 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       // one B operand per 32-channel group; KIVI's zero-point term on CUDA cores
       uint32_t bh[4][2], bl[4][2];
       float4 s4[4];  // value scales of this thread's four tokens, groups 0..3
+      float rv[4];   // residual: the power of two each of the four tokens' value rows is scaled by
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         s4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        rv[k] = 1.0f;
         if (!residual && ok[k]) s4[k] = vscale4<C>(base, tk[k]);
+        if (C::kKivi && residual) {
+          const int x = __shfl_sync(0xffffffffu, res_vx, tk[k] & 31);
+          rv[k] = pow2i(x);
+          s4[k] = make_float4(pow2i(-x), 0.f, 0.f, 0.f);
+        }
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -860,7 +1059,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float sj = j == 0 ? s4[k].x : j == 1 ? s4[k].y : j == 2 ? s4[k].z : s4[k].w;
-          pv[k] = residual ? pt[sb][k] * pscale : pt[sb][k] * sj * pscale;
+          pv[k] = residual ? pt[sb][k] * s4[k].x * pscale : pt[sb][k] * sj * pscale;
         }
         split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
         split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
@@ -869,7 +1068,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (!ok[k]) continue;
-          const float4 z4 = lds<float4>(base + C::kOffVM + C::kVMeta / 2 + tk[k] * 16);
+          const float4 z4 = meta4<C::kHalfMeta>(base + C::kOffVM + C::kVMeta / 2, tk[k]);
           S.zacc[0] = fmaf(pt[sb][k], z4.x, S.zacc[0]);
           S.zacc[1] = fmaf(pt[sb][k], z4.y, S.zacc[1]);
           S.zacc[2] = fmaf(pt[sb][k], z4.z, S.zacc[2]);
@@ -904,10 +1103,11 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
             uint2 u1 = lds<uint2>(vr + tk[2 * pp + 1] * 256 + (32 * j + 4 * g) * 2);
             if (!ok[2 * pp]) u0 = make_uint2(0u, 0u);
             if (!ok[2 * pp + 1]) u1 = make_uint2(0u, 0u);
-            pr[pp][0] = float2_to_f16x2(bf16_bits_to_float(u0.x & 0xFFFFu), bf16_bits_to_float(u1.x & 0xFFFFu));
-            pr[pp][1] = float2_to_f16x2(bf16_bits_to_float(u0.x >> 16), bf16_bits_to_float(u1.x >> 16));
-            pr[pp][2] = float2_to_f16x2(bf16_bits_to_float(u0.y & 0xFFFFu), bf16_bits_to_float(u1.y & 0xFFFFu));
-            pr[pp][3] = float2_to_f16x2(bf16_bits_to_float(u0.y >> 16), bf16_bits_to_float(u1.y >> 16));
+            const float fa = rv[2 * pp], fb = rv[2 * pp + 1];
+            pr[pp][0] = float2_to_f16x2(bf16_bits_to_float(u0.x & 0xFFFFu) * fa, bf16_bits_to_float(u1.x & 0xFFFFu) * fb);
+            pr[pp][1] = float2_to_f16x2(bf16_bits_to_float(u0.x >> 16) * fa, bf16_bits_to_float(u1.x >> 16) * fb);
+            pr[pp][2] = float2_to_f16x2(bf16_bits_to_float(u0.y & 0xFFFFu) * fa, bf16_bits_to_float(u1.y & 0xFFFFu) * fb);
+            pr[pp][3] = float2_to_f16x2(bf16_bits_to_float(u0.y >> 16) * fa, bf16_bits_to_float(u1.y >> 16) * fb);
           }
         } else if constexpr (C::kVFmt == FMT_U4) {
 #pragma unroll
@@ -946,11 +1146,11 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int KS, int VS, bool PAGED, int NG>
-__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
+template <int KS, int VS, bool PAGED, int NG, bool ROPE>
+__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBlocks)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
-  using C = Cfg<KS, VS, PAGED, NG>;
+  using C = Cfg<KS, VS, PAGED, NG, ROPE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
   grid_dependency_wait();    // the cache, the queries and the plan come from earlier kernels
@@ -988,6 +1188,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
   float* red_z = reinterpret_cast<float*>(smem + C::kOffRedZ);
   float* q_s = reinterpret_cast<float*>(smem + C::kOffQ);
   const float sc_log2 = p.softmax_scale * kLog2e;
+  if constexpr (C::kRope) {  // inverse frequencies base^(-2i/128) in fp64 (visible after the first pair start)
+    if (threadIdx.x < 64)
+      rope_theta_s(q_s)[threadIdx.x] = pow((double)p.rope_theta, -2.0 * (double)threadIdx.x / (double)kHeadDim);
+  }
   bool dead = false;
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) S.zpk[ks][0] = S.zpk[ks][1] = S.zpv[ks][0] = S.zpv[ks][1] = 0u;
@@ -1014,6 +1218,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
         }
         q_s[q_off(j, dd)] = v;
       }
+      if constexpr (C::kRope && C::kKFold == FOLD_CHANNEL)  // per-channel key scales, applied before the rotation
+        rope_key_scales(q_s)[tid] = p.k_scale[(size_t)d.hk * kHeadDim + tid];
       named_sync(1, kCW * 32);
       if (p.rotate) {  // H q: butterflies of span 1 .. 64 over the staged rows, then 1/sqrt(128)
         for (int h = 1; h < kHeadDim; h <<= 1) {
@@ -1044,11 +1250,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
         const float* fold = nullptr;
         if constexpr (C::kKFold == FOLD_CHANNEL) fold = p.k_scale + (size_t)d.hk * kHeadDim;
         int eq;
-        if constexpr (C::kKFmt == FMT_S4)
+        if constexpr (C::kRope)
+          eq = build_q_rope(q_s, g, c, S.qh, S.ql);
+        else if constexpr (C::kKFmt == FMT_S4)
           eq = build_q_s4(q_s, g, c, S.qh, S.ql);
         else
           eq = build_q<C::kKFmt>(q_s, fold, nullptr, g, c, S.qh, S.ql);
-        S.qsplit = (C::kKFold == FOLD_CHANNEL) || !p.q_bf16 || p.rotate;
+        // bf16 queries are exact in f16 (after the power-of-two shift) unless a fold multiplies them
+        S.qsplit = (!C::kRope && C::kKFold == FOLD_CHANNEL) || !p.q_bf16 || p.rotate;
         float mul = sc_log2 * pow2i(-eq);
         if constexpr (C::kKFold == FOLD_TENSOR) mul *= p.k_scale[0];
         S.kmul = mul;
@@ -1058,7 +1267,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG>::kMinBlocks)
           for (int ks = 0; ks < 8; ++ks)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int d0 = dmap_k<C::kKFmt>(c, ks, h, 0);
+              // RoPE keys: word ks & 3 of chunk c (ks < 4) or of chunk 4 + c, bytes 2h, 2h + 1
+              const int d0 = C::kRope ? (ks >> 2) * 64 + 16 * c + 4 * (ks & 3) + 2 * h : dmap_k<C::kKFmt>(c, ks, h, 0);
               const float z0 = 1024.0f + p.k_zp[d.hk * kHeadDim + d0];
               const float z1 = 1024.0f + p.k_zp[d.hk * kHeadDim + d0 + 1];
               S.zpk[ks][h] = float2_to_f16x2(z0, z1);
@@ -1327,18 +1537,18 @@ bool make_map(CUtensorMap* map, const void* base, int row_bytes_, uint64_t rows,
 }
 
 struct Variant {
-  int k, v, paged, ng;
+  int k, v, paged, ng, rope;
   void (*kernel)(const DecodeParams, const CUtensorMap, const CUtensorMap);
   int smem, ts;
 };
 
-template <int KS, int VS, bool PG, int NG = 4>
+template <int KS, int VS, bool PG, int NG = 4, bool ROPE = false>
 Variant variant() {
-  using C = Cfg<KS, VS, PG, NG>;
-  return Variant{KS, VS, PG ? 1 : 0, NG, decode_kernel<KS, VS, PG, NG>, C::kSmemBytes, C::kTS};
+  using C = Cfg<KS, VS, PG, NG, ROPE>;
+  return Variant{KS, VS, PG ? 1 : 0, NG, ROPE ? 1 : 0, decode_kernel<KS, VS, PG, NG, ROPE>, C::kSmemBytes, C::kTS};
 }
 
-constexpr int kNumVariants = 32;
+constexpr int kNumVariants = 40;
 constexpr int kMaxDevices = 64;
 
 const Variant* variants() {
@@ -1375,16 +1585,27 @@ const Variant* variants() {
       variant<KVQ_INT4_SYM_PER_GROUP, KVQ_INT4_SYM_PER_GROUP, true, 1>(),
       variant<KVQ_KIVI_INT4, KVQ_KIVI_INT4, false>(),
       variant<KVQ_KIVI_INT2, KVQ_KIVI_INT2, false>(),
+      variant<KVQ_KIVI_INT4_F16, KVQ_KIVI_INT4_F16, false>(),
+      variant<KVQ_KIVI_INT2_F16, KVQ_KIVI_INT2_F16, false>(),
+      // keys cached before RoPE
+      variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, false, 4, true>(),
+      variant<KVQ_FP8_E4M3_PER_TENSOR, KVQ_FP8_E4M3_PER_TENSOR, true, 4, true>(),
+      variant<KVQ_INT8_SYM_PER_CHANNEL, KVQ_UINT8_ASYM_PER_CHANNEL, false, 4, true>(),
+      variant<KVQ_INT8_SYM_PER_CHANNEL, KVQ_UINT8_ASYM_PER_CHANNEL, true, 4, true>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_UINT8_ASYM_PER_CHANNEL, false, 4, true>(),
+      variant<KVQ_INT8_SYM_PER_TENSOR, KVQ_UINT8_ASYM_PER_CHANNEL, true, 4, true>(),
   };
   static_assert(sizeof(table) / sizeof(table[0]) == kNumVariants, "variant count");
   return table;
 }
 
 // ng: scales per row of an INT4 per-group scheme (128 / group size); 4 for the others
-const Variant* find_variant(int k, int v, int paged, int ng) {
+const Variant* find_variant(int k, int v, int paged, int ng, bool rope) {
   const Variant* table = variants();
   for (int i = 0; i < kNumVariants; ++i)
-    if (table[i].k == k && table[i].v == v && table[i].paged == paged && table[i].ng == ng) return &table[i];
+    if (table[i].k == k && table[i].v == v && table[i].paged == paged && table[i].ng == ng &&
+        table[i].rope == (rope ? 1 : 0))
+      return &table[i];
   return nullptr;
 }
 
@@ -1392,26 +1613,17 @@ int groups_per_row(int k_scheme, int group) {
   return (k_scheme == KVQ_INT4_SYM_PER_GROUP && group > 0) ? kHeadDim / group : 4;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 
 }  // namespace
 
-bool decode_supported(int k_scheme, int v_scheme, int paged, int group) {
-  return find_variant(k_scheme, v_scheme, paged, groups_per_row(k_scheme, group)) != nullptr;
+bool decode_supported(int k_scheme, int v_scheme, int paged, int group, bool rope) {
+  return find_variant(k_scheme, v_scheme, paged, groups_per_row(k_scheme, group), rope) != nullptr;
 }
 
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
-  const Variant* var = find_variant(p.k_scheme, p.v_scheme, p.paged, groups_per_row(p.k_scheme, p.group));
+  const Variant* var =
+      find_variant(p.k_scheme, p.v_scheme, p.paged, groups_per_row(p.k_scheme, p.group), p.rope_theta > 0.0f);
   if (!var) return cudaErrorNotSupported;
   p.ts = var->ts;
   if (!p.paged) {

@@ -276,9 +276,14 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 }
 
 // ------------------------------------------------------------------ scheme traits
-__host__ __device__ constexpr bool is_kivi(int s) { return s == KVQ_KIVI_INT4 || s == KVQ_KIVI_INT2; }
+__host__ __device__ constexpr bool kivi_f16(int s) { return s == KVQ_KIVI_INT4_F16 || s == KVQ_KIVI_INT2_F16; }
+__host__ __device__ constexpr bool is_kivi(int s) {
+  return s == KVQ_KIVI_INT4 || s == KVQ_KIVI_INT2 || kivi_f16(s);
+}
 __host__ __device__ constexpr int code_bits(int s) {
-  return (s == KVQ_KIVI_INT4 || s == KVQ_INT4_SYM_PER_GROUP) ? 4 : (s == KVQ_KIVI_INT2 ? 2 : 8);
+  return (s == KVQ_KIVI_INT4 || s == KVQ_KIVI_INT4_F16 || s == KVQ_INT4_SYM_PER_GROUP) ? 4
+         : (s == KVQ_KIVI_INT2 || s == KVQ_KIVI_INT2_F16)                              ? 2
+                                                                                        : 8;
 }
 __host__ __device__ constexpr int row_bytes(int s) { return kHeadDim * code_bits(s) / 8; }
 

@@ -86,6 +86,7 @@ struct DecodeParams {
   int nq, nr;                   // dense: quantized / residual tiles per pair
   int rotate;                   // rotate each query, and each output back
   int group;                    // INT4 per-group: channels per group (selects the kernel)
+  float rope_theta;             // > 0: keys cached before RoPE, rotated at their positions here
 };
 
 constexpr int kMaxCtas = 1024;
@@ -123,7 +124,9 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 
 // Returns cudaErrorNotSupported when the (k_scheme, v_scheme, layout) pair has no kernel.
 cudaError_t launch_decode(DecodeParams p, cudaStream_t st);
-bool decode_supported(int k_scheme, int v_scheme, int paged, int group);
+bool decode_supported(int k_scheme, int v_scheme, int paged, int group, bool rope);
 bool append_pair_supported(int k_scheme, int v_scheme);
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
 
 }  // namespace kvq

@@ -1,5 +1,7 @@
 // Allocation-free decode attention: the existing decode path with its workspace taken
 // from a static device array instead of caller memory.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kvq_device.cuh"
@@ -7,25 +9,51 @@
 
 namespace {
 
-// Split partials and the paged plan of kvq_decode_attention, for callers that cannot
-// allocate. Held by every GPU that loads the library until the process exits.
+// Split partials and the paged plan of kvq_decode_attention, for callers that cannot allocate.
+// Held by every GPU that loads the library until the process exits.
 static __device__ __align__(256) uint8_t g_decode_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 128;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices];  // device address of g_decode_scratch, per device ordinal
+// Device address of g_decode_scratch per device ordinal, and the CUDA context it was looked up
+// in: the address belongs to that context, so a different current context (after a device
+// reset, or a caller's own driver context) looks it up again.
+void* g_scratch_ptr[kMaxDevices];
+CUcontext g_scratch_ctx[kMaxDevices];
 
-// Device address of the array on the current device, looked up once per device. In host
-// code g_decode_scratch names a host-side stand-in, never the device memory itself.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  });
+  return fn;
+}
+
+// Device address of the array on the current device, looked up once per (device, context).
+// In host code g_decode_scratch names a host-side stand-in, never the device memory itself.
 kvq_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  CtxGetCurrentFn get = ctx_get_current();
+  if (!get) return KVQ_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return KVQ_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
+    // the look-up makes the runtime's context current when no context is yet
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return KVQ_ERR_CUDA;
+    if (!ctx && (get(&ctx) != CUDA_SUCCESS || !ctx)) return KVQ_ERR_CUDA;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   *out = g_scratch_ptr[dev];
   return KVQ_OK;

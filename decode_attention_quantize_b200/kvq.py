@@ -28,6 +28,9 @@ KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
 INT4_SYM_PER_GROUP = 8
+KIVI_INT4_F16 = 9    # KIVI with fp16 scale and minimum
+KIVI_INT2_F16 = 10
+KIVI_SCHEMES = (KIVI_INT4, KIVI_INT2, KIVI_INT4_F16, KIVI_INT2_F16)
 KVQ_F32, KVQ_BF16 = 0, 1
 KVQ_DENSE, KVQ_PAGED = 0, 1
 KVQ_ROTATE_NONE, KVQ_ROTATE_HADAMARD = 0, 1
@@ -60,6 +63,7 @@ class KvqDesc(ctypes.Structure):
         ("page_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
         ("dev_status", ctypes.c_void_p),
         ("rotation", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
     ]
 
 
@@ -136,8 +140,24 @@ def _dtype_code(t):
     raise ValueError(f"unsupported dtype {t.dtype}: bf16 or fp32")
 
 
+def _need(cond: bool, what: str):
+    if not cond:
+        raise ValueError(what)
+
+
+def _check_shape(t, shape, name):
+    _need(t is not None and tuple(t.shape) == tuple(shape), f"{name}: shape {None if t is None else tuple(t.shape)}, "
+                                                           f"expected {tuple(shape)}")
+
+
+def _check_device(tensors, device):
+    for name, t in tensors:
+        if t is not None and t.is_cuda and device is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
 def row_bytes(scheme: int, D: int = 128) -> int:
-    return D * {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4}.get(scheme, 8) // 8
+    return D * {KIVI_INT4: 4, KIVI_INT2: 2, INT4_SYM_PER_GROUP: 4, KIVI_INT4_F16: 4, KIVI_INT2_F16: 2}.get(scheme, 8) // 8
 
 
 # ---------------------------------------------------------------- entry points
@@ -147,6 +167,16 @@ def kvq_quantize_append(desc: KvqDesc, k_new, v_new, new_lens=None, calibrate=Fa
     calibrate: scales from this block; rescale: grow the scales to cover this block and
     requantize the cached codes whose scale changed."""
     flags = (KVQ_APPEND_CALIBRATE if calibrate else 0) | (KVQ_APPEND_RESCALE if rescale else 0)
+    # the kernels index k_new / v_new / new_lens by the descriptor's shape: check them first
+    _need(k_new is not None and v_new is not None and k_new.dim() == 4, "k_new, v_new: [B, Hkv, n, D] tensors")
+    n = int(k_new.shape[2])
+    _check_shape(k_new, (desc.batch, desc.num_kv_heads, n, desc.head_dim), "k_new")
+    _check_shape(v_new, (desc.batch, desc.num_kv_heads, n, desc.head_dim), "v_new")
+    _need(k_new.dtype == v_new.dtype, f"k_new and v_new dtypes differ ({k_new.dtype}, {v_new.dtype})")
+    if new_lens is not None:
+        _check_shape(new_lens, (desc.batch,), "new_lens")
+        _need(new_lens.dtype == torch.int32, "new_lens: int32")
+    _check_device([("v_new", v_new), ("new_lens", new_lens), ("workspace", workspace)], k_new.device)
     need = lib.kvq_append_workspace_bytes(ctypes.byref(desc), flags)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=k_new.device)
@@ -160,6 +190,8 @@ def kvq_dequantize(desc: KvqDesc, which: int, out_tokens: int, out=None, stream=
     if out is None:
         out = torch.empty((desc.batch, desc.num_kv_heads, out_tokens, desc.head_dim), dtype=torch.float32,
                           device=device)
+    _check_shape(out, (desc.batch, desc.num_kv_heads, out_tokens, desc.head_dim), "out")
+    _need(out.dtype == torch.float32, "out: float32")
     _check(lib.kvq_dequantize(ctypes.byref(desc), which, _ptr(out), out_tokens, _stream(stream)),
            "kvq_dequantize")
     return out
@@ -169,14 +201,32 @@ def kvq_decode_workspace_bytes(desc: KvqDesc) -> int:
     return int(lib.kvq_decode_workspace_bytes(ctypes.byref(desc)))
 
 
+def decode_workspace(desc: KvqDesc, device) -> torch.Tensor:
+    """A decode workspace for this descriptor (split partials and the paged plan; no contents
+    need to be kept between calls)."""
+    return torch.empty(kvq_decode_workspace_bytes(desc), dtype=torch.uint8, device=device)
+
+
+def _check_decode_args(desc: KvqDesc, q, out, lse):
+    _check_shape(q, (desc.batch, desc.num_q_heads, desc.head_dim), "q")
+    _check_shape(out, (desc.batch, desc.num_q_heads, desc.head_dim), "out")
+    _need(out.dtype == torch.float32, "out: float32")
+    if lse is not None:
+        _check_shape(lse, (desc.batch, desc.num_q_heads), "lse")
+        _need(lse.dtype == torch.float32, "lse: float32")
+    _check_device([("out", out), ("lse", lse)], q.device)
+
+
 def kvq_decode_attention(desc: KvqDesc, q, softmax_scale: float, out=None, lse=None, workspace=None,
                          stream=None):
     """Decode attention of q [B, Hq, D] over the quantized cache; returns (out, lse)."""
-    B, Hq, D = q.shape
+    _need(q is not None and q.dim() == 3, "q: [B, Hq, D] tensor")
     if out is None:
-        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        out = torch.empty(tuple(q.shape), dtype=torch.float32, device=q.device)
+    _check_decode_args(desc, q, out, lse)
     if workspace is None:
-        workspace = torch.empty(kvq_decode_workspace_bytes(desc), dtype=torch.uint8, device=q.device)
+        workspace = decode_workspace(desc, q.device)
+    _check_device([("workspace", workspace)], q.device)
     _check(lib.kvq_decode_attention(ctypes.byref(desc), _ptr(q), _dtype_code(q), float(softmax_scale),
                                     _ptr(out), _ptr(lse), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -187,9 +237,10 @@ def kvq_decode_attention(desc: KvqDesc, q, softmax_scale: float, out=None, lse=N
 def kvq_decode_attention_noalloc(desc: KvqDesc, q, softmax_scale: float, out=None, lse=None, stream=None):
     """kvq_decode_attention without a workspace: for callers that cannot allocate device
     memory (the library's static scratch array holds the partials; see include/kvq.h)."""
-    B, Hq, D = q.shape
+    _need(q is not None and q.dim() == 3, "q: [B, Hq, D] tensor")
     if out is None:
-        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        out = torch.empty(tuple(q.shape), dtype=torch.float32, device=q.device)
+    _check_decode_args(desc, q, out, lse)
     _check(lib.kvq_decode_attention_noalloc(ctypes.byref(desc), _ptr(q), _dtype_code(q), float(softmax_scale),
                                             _ptr(out), _ptr(lse), _stream(stream)),
            "kvq_decode_attention_noalloc")
@@ -235,6 +286,7 @@ class CacheSpec:
     D: int = 128
     rotate: bool = False         # Walsh-Hadamard rotation of K, V and Q (not with KIVI)
     group: int = 32              # INT4 per group: channels per group (32, 64 or 128); KIVI: 32
+    rope_theta: float = 0.0      # > 0: keys cached before RoPE, rotated at decode (8-bit key schemes)
 
 
 class RescaleSchedule:
@@ -269,7 +321,7 @@ class QuantizedKVCache:
         self.schedule = RescaleSchedule(rescale_every) if rescale_every > 0 else None
         dev = torch.device(device)
         self.t = {}
-        kivi = s.k_scheme in (KIVI_INT4, KIVI_INT2)
+        kivi = s.k_scheme in KIVI_SCHEMES
         rows = (s.num_pages, s.Hkv, s.page_size) if s.paged else (s.B, s.Hkv, s.capacity)
         for side, sch in (("k", s.k_scheme), ("v", s.v_scheme)):
             self.t[side + "_codes"] = torch.zeros(*rows, row_bytes(sch, s.D), dtype=torch.uint8, device=dev)
@@ -285,8 +337,9 @@ class QuantizedKVCache:
                     self.t[side + "_zp"] = torch.zeros(s.Hkv, s.D, dtype=torch.uint8, device=dev)
             else:
                 shape = (s.B, s.Hkv, s.capacity // 32, s.D) if side == "k" else (s.B, s.Hkv, s.capacity, s.D // 32)
-                self.t[side + "_scale"] = torch.zeros(*shape, dtype=torch.float32, device=dev)
-                self.t[side + "_zero"] = torch.zeros(*shape, dtype=torch.float32, device=dev)
+                meta = torch.float16 if sch in (KIVI_INT4_F16, KIVI_INT2_F16) else torch.float32
+                self.t[side + "_scale"] = torch.zeros(*shape, dtype=meta, device=dev)
+                self.t[side + "_zero"] = torch.zeros(*shape, dtype=meta, device=dev)
         if kivi:
             self.t["k_res"] = torch.zeros(s.B, s.Hkv, 128, s.D, dtype=torch.bfloat16, device=dev)
             self.t["v_res"] = torch.zeros(s.B, s.Hkv, 128, s.D, dtype=torch.bfloat16, device=dev)
@@ -303,10 +356,12 @@ class QuantizedKVCache:
         d.page_size, d.max_pages_per_seq, d.num_pages = s.page_size, s.max_pages, s.num_pages
         d.group_size, d.residual_cap = s.group, 128
         d.rotation = KVQ_ROTATE_HADAMARD if s.rotate else KVQ_ROTATE_NONE
+        d.rope_theta = float(s.rope_theta)
         for name, tensor in self.t.items():
             setattr(d, name, tensor.data_ptr())
         self.desc = d
         self.device = dev
+        self._decode_ws = None
         _check(lib.kvq_validate(ctypes.byref(d)), "kvq_validate")
 
     def __getitem__(self, name):
@@ -335,8 +390,13 @@ class QuantizedKVCache:
         return kvq_dequantize(self.desc, which, out_tokens, stream=stream, device=self.device)
 
     def decode(self, q, softmax_scale=None, out=None, lse=None, workspace=None, stream=None):
+        """Without a workspace the cache's own (allocated at the first decode, kept) is used."""
         if softmax_scale is None:
             softmax_scale = 1.0 / math.sqrt(self.spec.D)
+        if workspace is None:
+            if self._decode_ws is None:
+                self._decode_ws = decode_workspace(self.desc, self.device)
+            workspace = self._decode_ws
         return kvq_decode_attention(self.desc, q, softmax_scale, out=out, lse=lse, workspace=workspace,
                                     stream=stream)
 

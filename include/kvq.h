@@ -28,7 +28,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 2
+#define KVQ_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define KVQ_API __attribute__((visibility("default")))
@@ -68,6 +68,13 @@ typedef enum kvq_status {
  *                       Group-Wise"; n4n.ai Step 2 "Per-group INT4"); two's-complement nibbles
  *                       packed along head_dim, lower channel in the low bits (64-byte rows);
  *                       fp32 scales [rows][head_dim / group_size]. K and V both.
+ *  KIVI_INT4_F16 / KIVI_INT2_F16  KIVI with the scale and minimum of every group stored as IEEE
+ *                       fp16 (the precision of the tensors n4n.ai Step 3's cache code works
+ *                       in; half the metadata bytes, so INT2 takes 3 bits per element): the fp32
+ *                       s and min of a group rounded to nearest-even fp16, saturating at +-65504,
+ *                       and the codes taken from the stored values, q = clamp(rne((x - min16) /
+ *                       s16), 0, 2^bits - 1); s16 == 0 gives code 0. The scale and minimum
+ *                       arrays (k_scale, k_zero, v_scale, v_zero) then hold fp16 elements.
  * A zero range gives s = 0 and code 0. */
 typedef enum kvq_scheme {
   KVQ_FP8_E4M3_PER_TENSOR = 0,
@@ -78,7 +85,9 @@ typedef enum kvq_scheme {
   KVQ_KIVI_INT4 = 5,
   KVQ_KIVI_INT2 = 6,
   KVQ_FP8_E5M2_PER_TENSOR = 7,
-  KVQ_INT4_SYM_PER_GROUP = 8
+  KVQ_INT4_SYM_PER_GROUP = 8,
+  KVQ_KIVI_INT4_F16 = 9,
+  KVQ_KIVI_INT2_F16 = 10
 } kvq_scheme;
 
 typedef enum kvq_dtype { KVQ_F32 = 0, KVQ_BF16 = 1 } kvq_dtype;
@@ -112,6 +121,7 @@ typedef enum kvq_rotation { KVQ_ROTATE_NONE = 0, KVQ_ROTATE_HADAMARD = 1 } kvq_r
  *   per-channel scale           float [kv_heads, head_dim]; uint8 zero point (k_zp/v_zp) same shape
  *   KIVI key scale and minimum  float [batch, kv_heads, capacity/32, head_dim] (k_scale, k_zero)
  *   KIVI value scale and minimum float [batch, kv_heads, capacity, head_dim/32] (v_scale, v_zero)
+ *                               (fp16 elements, same shapes, for KIVI_INT4_F16 / KIVI_INT2_F16)
  *   KIVI residual               bf16  [batch, kv_heads, residual_cap, head_dim] (k_res, v_res)
  *   paged page_table            int32 [batch, max_pages_per_seq]; seq_lens int32 [batch]
  *   dev_status                  uint32 [2]
@@ -144,6 +154,14 @@ typedef struct kvq_cache_desc {
   int32_t rotation;          /* kvq_rotation: KVQ_ROTATE_HADAMARD rotates every K/V row before it
                                 is quantized, each query before attention and each output and
                                 dequantized row back (not with KIVI schemes) */
+  float rope_theta;          /* 0: keys are cached as given (after RoPE). > 0: keys are cached
+                                before RoPE (KVQuant's pre-RoPE key quantization, "KV Cache
+                                Quantization in Production LLM Serving", llms.blog §4) and decode
+                                rotates each dequantized key at its position t in the sequence
+                                (0-based): pairs (i, i + 64), angle t * rope_theta^(-2i/128),
+                                (a, b) -> (a cos - b sin, b cos + a sin); queries arrive rotated.
+                                8-bit key schemes, not with KVQ_ROTATE_HADAMARD. Dequantize returns
+                                the stored (pre-RoPE) keys. */
 } kvq_cache_desc;
 
 typedef struct kvq_footprint {
@@ -252,7 +270,9 @@ KVQ_API uint64_t kvq_launch_count(void);
  * kvq_decode_workspace_bytes exceeds that size is rejected with KVQ_ERR_WORKSPACE
  * before any launch. The first call on a device looks up the array's device address
  * (with that device current), so make the first call on each device before any stream
- * capture. Every call shares the one array: calls that overlap on the GPU (different
+ * capture. The address is kept per device and CUDA context: a call from another context on
+ * the same device (a caller's own driver context, or the new primary context after a device
+ * reset) looks it up again. Every call shares the one array: calls that overlap on the GPU (different
  * streams, or devices sharing a context) race, so serialise them. The array keeps the
  * previous call's contents; nothing in it needs to start at zero. Arguments and results
  * are those of kvq_decode_attention.

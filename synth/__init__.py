@@ -111,6 +111,9 @@ KIVI_INT4 = 5
 KIVI_INT2 = 6
 FP8_E5M2_PER_TENSOR = 7
 INT4_SYM_PER_GROUP = 8
+KIVI_INT4_F16 = 9   # KIVI with fp16 scale and minimum
+KIVI_INT2_F16 = 10
+KIVI_SCHEMES = (KIVI_INT4, KIVI_INT2, KIVI_INT4_F16, KIVI_INT2_F16)
 
 
 @dataclass
@@ -138,6 +141,8 @@ class Workload:
     residual_cap: int = 128
     group: int = 32
     rotate: bool = False            # Walsh-Hadamard rotation of K, V and Q
+    prerope_theta: float = 0.0      # > 0: keys cached before RoPE (generated with rope_theta = 0),
+                                    # RoPE with this base applied at decode
     extra: dict = field(default_factory=dict)
 
     @property
@@ -146,7 +151,7 @@ class Workload:
 
     @property
     def kivi(self) -> bool:
-        return self.k_scheme in (KIVI_INT4, KIVI_INT2)
+        return self.k_scheme in KIVI_SCHEMES
 
     def prefill_lengths(self) -> np.ndarray:
         """Prefill tokens per sequence."""
@@ -175,9 +180,11 @@ class Workload:
 
 
 def workloads() -> dict:
-    """The nine workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4
-    per-group 70B-shaped (INT4 with groups of 32, also with the Walsh-Hadamard rotation, and
-    with groups of 128; same inputs), KIVI-2 131K, paged INT8."""
+    """The workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4 per-group
+    70B-shaped (INT4 with groups of 32, also with the Walsh-Hadamard rotation, and with groups
+    of 128; same inputs), KIVI-2 131K, the two KIVI shapes with fp16 scale and minimum (same
+    inputs as their fp32-metadata twins), the FP8 8B shape with keys cached before RoPE (RoPE
+    applied at decode), paged INT8."""
     return {
         "tiny_int8": Workload(
             name="tiny_int8", seed=1, B=1, Hq=1, Hkv=1, D=128,
@@ -191,6 +198,10 @@ def workloads() -> dict:
             name="e5m2_8b", seed=6, B=32, Hq=32, Hkv=8, D=128,
             k_scheme=FP8_E5M2_PER_TENSOR, v_scheme=FP8_E5M2_PER_TENSOR, bf16=True,
             outlier_scale=20.0, rope_theta=500000.0, context=4096),
+        "fp8_8b_prerope": Workload(
+            name="fp8_8b_prerope", seed=2, B=32, Hq=32, Hkv=8, D=128,
+            k_scheme=FP8_E4M3_PER_TENSOR, v_scheme=FP8_E4M3_PER_TENSOR, bf16=True,
+            outlier_scale=20.0, rope_theta=0.0, prerope_theta=500000.0, context=4096),
         "kivi4_70b": Workload(
             name="kivi4_70b", seed=3, B=16, Hq=64, Hkv=8, D=128,
             k_scheme=KIVI_INT4, v_scheme=KIVI_INT4, bf16=True,
@@ -208,6 +219,16 @@ def workloads() -> dict:
             name="int4g128_70b", seed=7, B=16, Hq=64, Hkv=8, D=128,
             k_scheme=INT4_SYM_PER_GROUP, v_scheme=INT4_SYM_PER_GROUP, bf16=True,
             outlier_scale=20.0, rope_theta=500000.0, context=32768, group=128),
+        "kivi4f16_70b": Workload(
+            name="kivi4f16_70b", seed=3, B=16, Hq=64, Hkv=8, D=128,
+            k_scheme=KIVI_INT4_F16, v_scheme=KIVI_INT4_F16, bf16=True,
+            outlier_scale=20.0, rope_theta=500000.0, context=32768,
+            extra={"seeded_residual": True}),
+        "kivi2f16_131k": Workload(
+            name="kivi2f16_131k", seed=4, B=4, Hq=64, Hkv=8, D=128,
+            k_scheme=KIVI_INT2_F16, v_scheme=KIVI_INT2_F16, bf16=True,
+            outlier_scale=100.0, rope_theta=500000.0, context=131072,
+            extra={"prefill_extra": 128}),
         "kivi2_131k": Workload(
             name="kivi2_131k", seed=4, B=4, Hq=64, Hkv=8, D=128,
             k_scheme=KIVI_INT2, v_scheme=KIVI_INT2, bf16=True,

@@ -85,13 +85,16 @@ def compare_dense(oc: OracleCache, gc, where=""):
             if sch == synth.UINT8_ASYM_PER_CHANNEL:
                 assert np.array_equal(np_of(gc[side + "_zp"]), oc[side + "_zp"]), f"{where}: {side} zero points"
         else:
+            # KIVI: fp32 scale and minimum, or fp16 ones (the oracle holds the stored fp16 values
+            # as fp32, exactly)
             rows = L // 32 if side == "k" else L
             z_g = np_of(gc[side + "_zero"])
+            s_g, z_g = s_g.astype(np.float32), z_g.astype(np.float32)
             assert np.array_equal(s_g[:, :, :rows].view(np.uint32), s_o[:, :, :rows].view(np.uint32)), \
                 f"{where}: {side} KIVI scales differ"
             assert np.array_equal(z_g[:, :, :rows].view(np.uint32), oc[side + "_zero"][:, :, :rows].view(np.uint32)), \
                 f"{where}: {side} KIVI minima differ"
-    if oc.k_scheme in (synth.KIVI_INT4, synth.KIVI_INT2):
+    if oc.k_scheme in synth.KIVI_SCHEMES:
         r = oc.residual
         for side in ("k", "v"):
             got = np_of(gc[side + "_res"]).view(np.uint16)[:, :, :r]
@@ -123,19 +126,21 @@ def compare_paged(oc: OracleCache, gc, where=""):
                 assert np.array_equal(np_of(gc[side + "_zp"]), oc[side + "_zp"])
 
 
-def decode_both(oc: OracleCache, gc, q: np.ndarray, bf16: bool, where=""):
+def decode_both(oc: OracleCache, gc, q: np.ndarray, bf16: bool, where="", allow_zero=False):
     qd = dev(q, bf16)
     lse = torch.empty(q.shape[:2], dtype=torch.float32, device="cuda")
     out, _ = gc.decode(qd, float(SCALE), lse=lse)
     ref, ref_lse = oc.decode(q, bf16, float(SCALE))
     torch.cuda.synchronize()
-    return attn_check(out, ref, lse, ref_lse, where)
+    return attn_check(out, ref, lse, ref_lse, where, allow_zero=allow_zero)
 
 
 def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16=None, seed=11, outlier=20.0,
-               rope=500000.0, chunks=None, rotate=False, group=32):
+               rope=500000.0, chunks=None, rotate=False, group=32, prerope=0.0):
     """Prefill (calibrating when the scheme needs it), then `steps` one-token appends each
-    followed by a decode; codes and attention compared after every call."""
+    followed by a decode; codes and attention compared after every call. rope: RoPE the input
+    generator applies to the keys; prerope > 0: the cache holds keys before RoPE and decode
+    applies RoPE with this base (pass rope=0 for such keys)."""
     q_bf16 = bf16 if q_bf16 is None else q_bf16
     w = workload(B, Hq, Hkv, ks, vs, bf16=bf16, seed=seed, outlier=outlier, rope=rope)
     total = prefill + steps
@@ -143,8 +148,9 @@ def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16
         cap = max(128, (total + 127) // 128 * 128)
     K = synth.keys(w, 0, B, 0, Hkv, 0, total)
     V = synth.values(w, 0, B, 0, Hkv, 0, total)
-    oc = OracleCache(B, Hq, Hkv, 128, ks, vs, cap=cap, rotate=rotate, group=group)
-    gc = kvq().QuantizedKVCache(kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=cap, rotate=rotate, group=group))
+    oc = OracleCache(B, Hq, Hkv, 128, ks, vs, cap=cap, rotate=rotate, group=group, rope_theta=prerope)
+    gc = kvq().QuantizedKVCache(kvq().CacheSpec(B, Hq, Hkv, ks, vs, capacity=cap, rotate=rotate, group=group,
+                                                rope_theta=prerope))
     calib = ks in CALIBRATED or vs in CALIBRATED
     bounds = [0, prefill] if chunks is None else [0, *chunks, prefill]
     for i, (a, b) in enumerate(zip(bounds, bounds[1:])):
@@ -169,8 +175,8 @@ def dense_case(B, Hq, Hkv, ks, vs, prefill, steps=2, cap=None, bf16=True, q_bf16
 
 
 def paged_case(B, Hq, Hkv, ks, vs, lens, page_size=16, steps=2, seed=21, extra_pages=5, bad_page=None,
-               rotate=False, group=32):
-    w = workload(B, Hq, Hkv, ks, vs, bf16=True, seed=seed)
+               rotate=False, group=32, prerope=0.0):
+    w = workload(B, Hq, Hkv, ks, vs, bf16=True, seed=seed, rope=0.0 if prerope else 500000.0)
     lens = np.asarray(lens, np.int32)
     n_max = int(lens.max()) if len(lens) else 0
     need = [(int(L) + steps + page_size - 1) // page_size for L in lens]
@@ -193,9 +199,9 @@ def paged_case(B, Hq, Hkv, ks, vs, lens, page_size=16, steps=2, seed=21, extra_p
             V[b:b + 1, :, :lens[b]] = synth.values(w, b, b + 1, 0, Hkv, 0, int(lens[b]))
     oc = OracleCache(B, Hq, Hkv, 128, ks, vs, paged=True, page_size=page_size, max_pages=max_pages,
                      num_pages=num_pages, page_table=table if bad_page is None else _clean(table, num_pages),
-                     rotate=rotate, group=group)
+                     rotate=rotate, group=group, rope_theta=prerope)
     spec = kvq().CacheSpec(B, Hq, Hkv, ks, vs, paged=True, page_size=page_size, max_pages=max_pages,
-                           num_pages=num_pages, rotate=rotate, group=group)
+                           num_pages=num_pages, rotate=rotate, group=group, rope_theta=prerope)
     gc = kvq().QuantizedKVCache(spec, page_table=torch.from_numpy(table))
     calib = ks in CALIBRATED or vs in CALIBRATED
     nl = torch.from_numpy(lens).cuda()

@@ -26,7 +26,7 @@ def test_library_exports_every_declared_symbol():
     for name in _declared():
         assert hasattr(lib, name), name
     assert sorted(kvq.EXPORTS) == _declared()
-    assert lib.kvq_abi_version() == 2
+    assert lib.kvq_abi_version() == 3
 
 
 def _desc(**kw):
@@ -53,7 +53,7 @@ def test_validation_is_host_side():
         (dict(head_dim=64), kvq.KVQ_ERR_UNSUPPORTED),
         (dict(num_q_heads=7), kvq.KVQ_ERR_INVALID_ARG),
         (dict(capacity=200), kvq.KVQ_ERR_INVALID_ARG),
-        (dict(k_scheme=9), kvq.KVQ_ERR_INVALID_ARG),
+        (dict(k_scheme=11), kvq.KVQ_ERR_INVALID_ARG),
         (dict(k_scheme=5, v_scheme=6), kvq.KVQ_ERR_UNSUPPORTED),
         (dict(rotation=2), kvq.KVQ_ERR_INVALID_ARG),
         (dict(rotation=1, k_scheme=5, v_scheme=5), kvq.KVQ_ERR_UNSUPPORTED),   # no rotation with KIVI
@@ -167,3 +167,99 @@ def test_rescale_schedule_counts_tokens():
     assert s.pending == 0 and not s.step(1023) and s.step(1)
     with pytest.raises(ValueError):
         RescaleSchedule(0)
+
+
+def test_validation_bounds_the_decode_plan_integers():
+    # the decode's split plan counts pairs and tiles in 32-bit integers: refused on the host
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    buf = 0x10000
+    paged = dict(layout=1, page_table=buf, seq_lens=buf, num_pages=8)
+    cases = [
+        dict(num_q_heads=16384, num_kv_heads=2),                                   # > 8192 query heads
+        dict(batch=1000, num_q_heads=8192, num_kv_heads=1, capacity=1 << 20),     # 2^20 pairs x 8196 tiles
+        dict(page_size=64, max_pages_per_seq=(1 << 25) + 1, **paged),              # longest length >= 2^31
+        dict(batch=65535, num_q_heads=8, num_kv_heads=8, page_size=64, max_pages_per_seq=8200, **paged),
+    ]
+    for kw in cases:
+        assert L.kvq_validate(ctypes.byref(_desc(**kw))) == kvq.KVQ_ERR_UNSUPPORTED, kw
+    assert L.kvq_validate(ctypes.byref(_desc(num_q_heads=8192, num_kv_heads=1))) == kvq.KVQ_OK
+
+
+def test_binding_checks_shapes_before_any_device_call():
+    # a wrong-shaped tensor would make the kernels read or write past a buffer: the binding
+    # refuses it on the host (CPU tensors here; nothing reaches the library)
+    import torch
+    from decode_attention_quantize_b200 import kvq
+    cache = kvq.QuantizedKVCache(kvq.CacheSpec(2, 8, 2, kvq.FP8_E4M3_PER_TENSOR, kvq.FP8_E4M3_PER_TENSOR,
+                                               capacity=256), device="cpu")
+    good_kv = torch.zeros(2, 2, 4, 128, dtype=torch.bfloat16)
+    bad = [
+        (torch.zeros(2, 2, 4, 64, dtype=torch.bfloat16), good_kv),      # head_dim
+        (torch.zeros(1, 2, 4, 128, dtype=torch.bfloat16), good_kv),     # batch
+        (good_kv, torch.zeros(2, 2, 5, 128, dtype=torch.bfloat16)),     # v_new tokens differ
+        (good_kv, torch.zeros(2, 2, 4, 128, dtype=torch.float32)),      # dtypes differ
+        (torch.zeros(2, 4, 128, dtype=torch.bfloat16), good_kv),        # not 4-D
+    ]
+    for k, v in bad:
+        with pytest.raises(ValueError):
+            cache.append(k, v)
+    with pytest.raises(ValueError):
+        cache.append(good_kv, good_kv, new_lens=torch.zeros(2, dtype=torch.int32))  # dense: counts refused
+    for q in (torch.zeros(2, 4, 128, dtype=torch.bfloat16), torch.zeros(2, 8, 64, dtype=torch.bfloat16),
+              torch.zeros(3, 8, 128, dtype=torch.bfloat16)):
+        with pytest.raises(ValueError, match="q: shape"):
+            cache.decode(q)
+    q = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="out: shape"):
+        cache.decode(q, out=torch.zeros(2, 8, 127))
+    with pytest.raises(ValueError, match="out: float32"):
+        cache.decode(q, out=torch.zeros(2, 8, 128, dtype=torch.float64))
+    with pytest.raises(ValueError, match="lse: shape"):
+        cache.decode(q, lse=torch.zeros(2, 4))
+    with pytest.raises(ValueError, match="out: shape"):
+        kvq.kvq_dequantize(cache.desc, 0, 10, out=torch.zeros(2, 2, 9, 128))
+    paged = kvq.QuantizedKVCache(kvq.CacheSpec(2, 8, 2, kvq.INT8_SYM_PER_TENSOR, kvq.INT8_SYM_PER_TENSOR, paged=True,
+                                               max_pages=4, num_pages=8), device="cpu")
+    with pytest.raises(ValueError, match="new_lens"):
+        paged.append(good_kv, good_kv, new_lens=torch.zeros(3, dtype=torch.int32))
+    with pytest.raises(ValueError, match="new_lens: int32"):
+        paged.append(good_kv, good_kv, new_lens=torch.zeros(2, dtype=torch.int64))
+
+
+def test_fp16_kivi_metadata_halves_the_metadata_bytes():
+    # fp16 scale and minimum per 32 elements: KIVI INT2 takes 2 + 16 * 2 / 32 = 3 bits per element
+    # and INT4 takes 5, against 4 and 6 with fp32 metadata
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    buf = 0x30000
+    f = kvq.KvqFootprint()
+    bits = {}
+    for sch in (kvq.KIVI_INT2, kvq.KIVI_INT2_F16, kvq.KIVI_INT4, kvq.KIVI_INT4_F16):
+        d = _desc(batch=1, num_q_heads=64, num_kv_heads=8, capacity=4096, k_scheme=sch, v_scheme=sch, k_zero=buf,
+                  v_zero=buf, k_res=buf, v_res=buf)
+        assert L.kvq_cache_bytes(ctypes.byref(d), ctypes.byref(f)) == kvq.KVQ_OK
+        bits[sch] = f.bytes_per_token * 8 / (2 * 128)
+        meta_elems = 2 * 2 * 8 * (4096 // 32) * 128  # (K + V) x (scale + min)
+        assert f.meta_bytes == meta_elems * (2 if sch in (kvq.KIVI_INT2_F16, kvq.KIVI_INT4_F16) else 4)
+    assert bits == {kvq.KIVI_INT2: 4.0, kvq.KIVI_INT2_F16: 3.0, kvq.KIVI_INT4: 6.0, kvq.KIVI_INT4_F16: 5.0}
+
+
+def test_prerope_validation():
+    # keys cached before RoPE: a finite base >= 0, 8-bit key codes, not with the Hadamard rotation
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    buf = 0x30000
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=500000.0))) == kvq.KVQ_OK
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=-1.0))) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=float("nan")))) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=float("inf")))) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=1e4, rotation=1))) == kvq.KVQ_ERR_UNSUPPORTED
+    kivi = dict(k_scheme=5, v_scheme=5, k_zero=buf, v_zero=buf, k_res=buf, v_res=buf)
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=1e4, **kivi))) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_validate(ctypes.byref(_desc(rope_theta=1e4, k_scheme=8, v_scheme=8))) == kvq.KVQ_ERR_UNSUPPORTED
+    # a pair with no pre-RoPE decode kernel is refused before anything is launched
+    d = _desc(rope_theta=1e4, k_scheme=2, v_scheme=2)
+    need = L.kvq_decode_workspace_bytes(ctypes.byref(d))
+    assert L.kvq_decode_attention(ctypes.byref(d), buf, 1, ctypes.c_float(0.088), buf, None, buf, need,
+                                  None) == kvq.KVQ_ERR_UNSUPPORTED

@@ -11,7 +11,8 @@ from decode_attention_quantize_b200 import kvq
 PAIRS = [(kvq.FP8_E4M3_PER_TENSOR, kvq.FP8_E4M3_PER_TENSOR), (kvq.FP8_E5M2_PER_TENSOR, kvq.FP8_E5M2_PER_TENSOR),
          (kvq.INT8_SYM_PER_TENSOR, kvq.UINT8_ASYM_PER_CHANNEL), (kvq.INT8_SYM_PER_TOKEN, kvq.INT8_SYM_PER_TOKEN),
          (kvq.INT8_SYM_PER_CHANNEL, kvq.INT8_SYM_PER_CHANNEL), (kvq.INT4_SYM_PER_GROUP, kvq.INT4_SYM_PER_GROUP),
-         (kvq.KIVI_INT4, kvq.KIVI_INT4), (kvq.KIVI_INT2, kvq.KIVI_INT2)]
+         (kvq.KIVI_INT4, kvq.KIVI_INT4), (kvq.KIVI_INT2, kvq.KIVI_INT2),
+         (kvq.KIVI_INT4_F16, kvq.KIVI_INT4_F16), (kvq.KIVI_INT2_F16, kvq.KIVI_INT2_F16)]
 
 
 def _bytes(t):
@@ -41,7 +42,7 @@ def test_dense_allocation_matches_footprint(ks, vs):
     assert cache.desc.capacity == 256 and cache.desc.rotation == kvq.KVQ_ROTATE_NONE
 
 
-@pytest.mark.parametrize("ks,vs", [p for p in PAIRS if p[0] not in (kvq.KIVI_INT4, kvq.KIVI_INT2)])
+@pytest.mark.parametrize("ks,vs", [p for p in PAIRS if p[0] not in kvq.KIVI_SCHEMES])
 def test_paged_allocation_matches_footprint(ks, vs):
     cache = kvq.QuantizedKVCache(kvq.CacheSpec(3, 8, 2, ks, vs, paged=True, page_size=32, max_pages=4,
                                                num_pages=10), device="cpu")

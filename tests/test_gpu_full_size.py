@@ -1,11 +1,15 @@
-"""Full-size parity at the five workload shapes.
+"""Full-size parity at the benchmark workloads' shapes.
 
 The CUDA library builds each workload's cache exactly as the benchmark does (same shapes,
-calibration, one streamed token, the library's own grid choice) and the oracle recomputes
-sampled (sequence, kv_head) pairs one by one: their codes, scales, minima and residual
-tokens must match bit for bit and their attention rows must be within 2e-4 * max|ref|.
-Scales that span the whole batch (per-tensor, per-channel) come from an oracle calibration
-over the full prefill block.
+calibration, the streamed tokens, the library's own grid choice) and the oracle builds the
+same cache from the same inputs. Codes, scales, zero points, minima and residual tokens of
+EVERY (sequence, kv head) pair must match bit for bit; attention rows of sampled pairs (the
+oracle's fp64 attention costs seconds per pair at these lengths) must be within 2e-4 * max|ref|.
+
+The paged workload streams all of its 128 steps (one token per sequence appended, then a
+decode): attention is compared on steps 0, 1, 63 and 127 for sampled sequences and on every
+step for four seeded sequences (drawn among the shortest quarter, so the oracle keeps up), and
+every sequence's codes at every position after the last step.
 """
 import math
 
@@ -13,7 +17,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 import synth
 from oracle import OracleCache
 from tests import harness as H
@@ -27,42 +30,7 @@ def _pairs(w, n=6, seed=0):
     rng = np.random.default_rng(seed + w.seed)
     allp = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     idx = rng.choice(len(allp), size=min(n, len(allp)), replace=False)
-    return [allp[i] for i in sorted(idx)] + [allp[0], allp[-1]]
-
-
-def _copy_scales(dst: OracleCache, src: OracleCache, h: int):
-    """Give a one-head oracle cache the batch-wide scales an oracle calibration computed:
-    the per-tensor scale, or kv head h's row of a per-channel scale (and zero point)."""
-    for side in ("k", "v"):
-        s = src[side + "_scale"]
-        if s.size == 1:
-            dst[side + "_scale"][...] = s
-        elif s.ndim == 2 and s.shape[1] == 128:  # [Hkv, D]
-            dst[side + "_scale"][...] = s[h:h + 1]
-            if src[side + "_zp"] is not None:
-                dst[side + "_zp"][...] = src[side + "_zp"][h:h + 1]
-
-
-def _check_pair_dense(w, gc, oc, b, h, out_gpu, q):
-    """Bit-exact slice comparison and attention for one (b, h) pair."""
-    L = oc.length
-    G = w.G
-    for side in ("k", "v"):
-        got = H.np_of(gc[side + "_codes"][b, h, :L])
-        assert np.array_equal(got, oc[side + "_codes"][0, 0, :L]), f"pair {(b, h)}: {side} codes"
-        sch = w.k_scheme if side == "k" else w.v_scheme
-        if sch in (synth.INT8_SYM_PER_TOKEN, synth.INT4_SYM_PER_GROUP):
-            assert np.array_equal(H.np_of(gc[side + "_scale"][b, h, :L]).view(np.uint32),
-                                  oc[side + "_scale"][0, 0, :L].view(np.uint32))
-        if sch in (synth.KIVI_INT4, synth.KIVI_INT2):
-            rows = L // 32 if side == "k" else L
-            for name in ("_scale", "_zero"):
-                assert np.array_equal(H.np_of(gc[side + name][b, h, :rows]).view(np.uint32),
-                                      oc[side + name][0, 0, :rows].view(np.uint32)), f"pair {(b, h)} {side}{name}"
-            r = oc.residual
-            assert np.array_equal(H.np_of(gc[side + "_res"][b, h, :r]).view(np.uint16), oc[side + "_res"][0, 0, :r])
-    ref, ref_lse = oc.decode(q[b:b + 1, h * G:(h + 1) * G], w.bf16, SCALE)
-    return ref[0]
+    return sorted(set([allp[i] for i in idx] + [allp[0], allp[-1]]))
 
 
 def _dense_full(name):
@@ -75,35 +43,28 @@ def _dense_full(name):
     K = synth.keys(w, 0, w.B, 0, w.Hkv, 0, total)
     V = synth.values(w, 0, w.B, 0, w.Hkv, 0, total)
     gc = kvq.QuantizedKVCache(kvq.CacheSpec(w.B, w.Hq, w.Hkv, w.k_scheme, w.v_scheme, capacity=cap,
-                                            rotate=w.rotate, group=w.group))
+                                            rotate=w.rotate, group=w.group, rope_theta=w.prerope_theta))
+    oc = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group,
+                     rope_theta=w.prerope_theta)
     calib = w.k_scheme in CAL or w.v_scheme in CAL
     gc.append(H.dev(K[:, :, :pre], w.bf16), H.dev(V[:, :, :pre], w.bf16), calibrate=calib)
+    oc.append(K[:, :, :pre], V[:, :, :pre], w.bf16, calibrate=calib)
     if append:
         gc.append(H.dev(K[:, :, pre:], w.bf16), H.dev(V[:, :, pre:], w.bf16))
+        oc.append(K[:, :, pre:], V[:, :, pre:], w.bf16)
+    del K, V
     q = synth.queries(w, 0, 0, w.B)
-    out, _ = gc.decode(H.dev(q, w.bf16), SCALE)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    out, _ = gc.decode(H.dev(q, w.bf16), SCALE, lse=lse)
     torch.cuda.synchronize()
-    out = out.cpu().numpy()
     assert gc.status()[0] == 0
-    full_cal = None
-    if calib:
-        full_cal = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, cap=128, rotate=w.rotate)
-        full_cal.calibrate(K[:, :, :pre], V[:, :, :pre], w.bf16)
-        for side in ("k", "v"):
-            assert np.array_equal(H.np_of(gc[side + "_scale"]).reshape(-1)[:full_cal[side + "_scale"].size]
-                                  .view(np.uint32), full_cal[side + "_scale"].reshape(-1).view(np.uint32))
-    refs, gots = [], []
-    for b, h in _pairs(w):
-        oc = OracleCache(1, w.G, 1, 128, w.k_scheme, w.v_scheme, cap=cap, rotate=w.rotate, group=w.group)
-        if full_cal is not None:
-            _copy_scales(oc, full_cal, h)
-        oc.append(K[b:b + 1, h:h + 1, :pre], V[b:b + 1, h:h + 1, :pre], w.bf16)
-        if append:
-            oc.append(K[b:b + 1, h:h + 1, pre:], V[b:b + 1, h:h + 1, pre:], w.bf16)
-        assert gc.num_quantized == oc.length and gc.num_residual == oc.residual
-        refs.append(_check_pair_dense(w, gc, oc, b, h, None, q))
-        gots.append(out[b, h * w.G:(h + 1) * w.G])
-    H.attn_check(torch.from_numpy(np.stack(gots)), np.stack(refs), where=f"{name} sampled pairs")
+    H.compare_dense(oc, gc, f"{name}: every pair")
+    pairs = _pairs(w)
+    ref, ref_lse = oc.decode_pairs(q, w.bf16, SCALE, pairs)
+    G = w.G
+    got = torch.stack([out[b, h * G:(h + 1) * G] for b, h in pairs])
+    got_lse = torch.stack([lse[b, h * G:(h + 1) * G] for b, h in pairs])
+    H.attn_check(got, ref, got_lse, ref_lse, where=f"{name} sampled pairs")
 
 
 def test_tiny_int8_full():
@@ -116,6 +77,10 @@ def test_fp8_8b_full():
 
 def test_e5m2_8b_full():
     _dense_full("e5m2_8b")
+
+
+def test_fp8_8b_prerope_full():
+    _dense_full("fp8_8b_prerope")
 
 
 def test_int4g_70b_full():
@@ -138,15 +103,29 @@ def test_kivi2_131k_full():
     _dense_full("kivi2_131k")
 
 
+def test_kivi4f16_70b_full():
+    _dense_full("kivi4f16_70b")
+
+
+def test_kivi2f16_131k_full():
+    _dense_full("kivi2f16_131k")
+
+
+def _step_tokens(w, lens, s):
+    kk = np.stack([synth.keys(w, b, b + 1, 0, w.Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(w.B)])
+    vv = np.stack([synth.values(w, b, b + 1, 0, w.Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0]
+                   for b in range(w.B)])
+    return kk, vv
+
+
 def test_paged_int8_full():
-    """64 sequences of 1k..32k tokens in 16-token pages; calibrating prefill over all of
-    them, then 3 streamed tokens per sequence; sampled sequences recomputed by the oracle."""
+    """64 sequences of 1k..32k tokens in 16-token pages; a calibrating prefill over all of them,
+    then the workload's 128 streamed steps."""
     w = synth.workloads()["paged_int8"]
     kvq = H.kvq()
-    steps = 3
+    steps = w.steps
     lens = w.prefill_lengths()
-    table, pool = w.page_table(max_pages=(int(lens.max()) + w.steps + 15) // 16 + 1)
-    # the workload's table covers prefill + its 128 streamed steps
+    table, pool = w.page_table(max_pages=(int(lens.max()) + steps + 15) // 16 + 1)
     n_max = int(lens.max())
     K = np.zeros((w.B, w.Hkv, n_max, 128), np.uint16)
     V = np.zeros_like(K)
@@ -157,48 +136,42 @@ def test_paged_int8_full():
     spec = kvq.CacheSpec(w.B, w.Hq, w.Hkv, w.k_scheme, w.v_scheme, paged=True, page_size=16,
                          max_pages=table.shape[1], num_pages=pool)
     gc = kvq.QuantizedKVCache(spec, page_table=torch.from_numpy(table))
-    nl = torch.from_numpy(lens).cuda()
-    gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
-    toks = []
+    oc = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, paged=True, page_size=16,
+                     max_pages=table.shape[1], num_pages=pool, page_table=table)
+    gc.append(H.dev(K, True), H.dev(V, True), new_lens=torch.from_numpy(lens).cuda(), calibrate=True)
+    oc.append(K, V, True, calibrate=True, new_lens=lens)
+    del K, V
+    rng = np.random.default_rng(5)
+    sampled = sorted(set(rng.choice(w.B, 5, replace=False).tolist() + [int(np.argmax(lens))]))
+    shorter = np.argsort(lens)[: w.B // 4]
+    every = sorted(rng.choice(shorter, 4, replace=False).tolist())
+    checkpoints = {0, 1, 63, steps - 1}
+    G = w.G
     for s in range(steps):
-        kk = np.stack([synth.keys(w, b, b + 1, 0, w.Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(w.B)])
-        vv = np.stack([synth.values(w, b, b + 1, 0, w.Hkv, int(lens[b]) + s, int(lens[b]) + s + 1)[0] for b in range(w.B)])
-        toks.append((kk, vv))
+        kk, vv = _step_tokens(w, lens, s)
         gc.append(H.dev(kk, True), H.dev(vv, True))
-    q = synth.queries(w, steps, 0, w.B)
-    out, _ = gc.decode(H.dev(q, True), SCALE)
-    torch.cuda.synchronize()
-    out = out.cpu().numpy()
+        oc.append(kk, vv, True)
+        q = synth.queries(w, s, 0, w.B)
+        lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+        out, _ = gc.decode(H.dev(q, True), SCALE, lse=lse)
+        seqs = sorted(set(every) | (set(sampled) if s in checkpoints else set()))
+        pairs = [(b, h) for b in seqs for h in range(w.Hkv)]
+        ref, ref_lse = oc.decode_pairs(q, True, SCALE, pairs)
+        torch.cuda.synchronize()
+        got = torch.stack([out[b, h * G:(h + 1) * G] for b, h in pairs])
+        got_lse = torch.stack([lse[b, h * G:(h + 1) * G] for b, h in pairs])
+        H.attn_check(got, ref, got_lse, ref_lse, where=f"paged_int8 step {s}, sequences {seqs}")
     assert gc.status()[0] == 0
     assert np.array_equal(H.np_of(gc["seq_lens"]), lens + steps)
-    cal = OracleCache(w.B, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, paged=True, page_size=16,
-                      max_pages=table.shape[1], num_pages=1, page_table=table)
-    cal.calibrate(K, V, True, new_lens=lens)
-    del K, V
+    # every sequence's codes at every position, and the batch-wide scales and zero points
     for side in ("k", "v"):
-        assert np.array_equal(H.np_of(gc[side + "_scale"]).reshape(-1)[:cal[side + "_scale"].size].view(np.uint32),
-                              cal[side + "_scale"].reshape(-1).view(np.uint32)), side
-    assert np.array_equal(H.np_of(gc["v_zp"]), cal["v_zp"])
-    refs, gots = [], []
-    seqs = sorted(set(np.random.default_rng(5).choice(w.B, 5, replace=False).tolist() + [int(np.argmax(lens))]))
-    pool_k, pool_v = H.np_of(gc["k_codes"]), H.np_of(gc["v_codes"])
-    for b in seqs:
-        L = int(lens[b])
-        npg = (L + steps + 15) // 16
-        own = np.arange(npg, dtype=np.int32)[None]  # the oracle keeps this sequence in a compact pool
-        oc = OracleCache(1, w.Hq, w.Hkv, 128, w.k_scheme, w.v_scheme, paged=True, page_size=16,
-                         max_pages=npg, num_pages=npg, page_table=own)
-        for side in ("k", "v"):
-            oc[side + "_scale"][...] = cal[side + "_scale"]
-        oc["v_zp"][...] = cal["v_zp"]
-        oc.append(synth.keys(w, b, b + 1, 0, w.Hkv, 0, L), synth.values(w, b, b + 1, 0, w.Hkv, 0, L), True)
-        for kk, vv in toks:
-            oc.append(kk[b:b + 1], vv[b:b + 1], True)
-        for t in range(L + steps):
-            page, slot = table[b, t // 16], t % 16
-            assert np.array_equal(pool_k[page, :, slot], oc["k_codes"][t // 16, :, slot]), (b, t)
-            assert np.array_equal(pool_v[page, :, slot], oc["v_codes"][t // 16, :, slot]), (b, t)
-        ref, _ = oc.decode(q[b:b + 1], True, SCALE)
-        refs.append(ref[0])
-        gots.append(out[b])
-    H.attn_check(torch.from_numpy(np.stack(gots)), np.stack(refs), where="paged_int8 sampled sequences")
+        pool_g, pool_o = H.np_of(gc[side + "_codes"]), oc[side + "_codes"]
+        for b in range(w.B):
+            L = int(lens[b]) + steps
+            pages = table[b, :(L + 15) // 16]
+            g = pool_g[pages].transpose(0, 2, 1, 3).reshape(-1, w.Hkv, 128)[:L]
+            o = pool_o[pages].transpose(0, 2, 1, 3).reshape(-1, w.Hkv, 128)[:L]
+            assert np.array_equal(g, o), f"{side} codes of sequence {b}"
+        assert np.array_equal(H.np_of(gc[side + "_scale"]).reshape(-1)[:oc[side + "_scale"].size].view(np.uint32),
+                              oc[side + "_scale"].reshape(-1).view(np.uint32)), side
+    assert np.array_equal(H.np_of(gc["v_zp"]), oc["v_zp"])

@@ -99,13 +99,13 @@ def test_bulk_prefill_paged():
 
 
 # ------------------------------------------------------------------ KIVI
-@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2])
+@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2, S.KIVI_INT4_F16, S.KIVI_INT2_F16])
 @pytest.mark.parametrize("prefill", [44, 128, 129, 300, 384, 385])
 def test_kivi_prefill_and_stream(scheme, prefill):
     H.dense_case(B=2, Hq=16, Hkv=2, ks=scheme, vs=scheme, prefill=prefill, steps=2, cap=640)
 
 
-@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2])
+@pytest.mark.parametrize("scheme", [S.KIVI_INT4, S.KIVI_INT2, S.KIVI_INT4_F16, S.KIVI_INT2_F16])
 def test_kivi_flush_on_stream_boundary(scheme):
     # 127 + 1 fills the residual; the next token flushes 128 tokens into 4 key groups
     H.dense_case(B=1, Hq=8, Hkv=1, ks=scheme, vs=scheme, prefill=127, steps=3, cap=256)
@@ -165,15 +165,27 @@ def test_paged_empty_sequence_and_variable_lengths():
 
 
 def test_bad_page_id_is_flagged_not_dereferenced():
+    # sequence 1's second page is outside the pool: its append is refused on the device (its
+    # length stays 0, the rows written to its good pages stay invisible), sequence 0 is appended
     B, Hq, Hkv = 2, 8, 2
     w, oc, gc, K, V, lens, calib, nl = H.paged_case(B, Hq, Hkv, S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL,
                                                     lens=[40, 40], steps=0, bad_page=(1, 1))
     gc.append(H.dev(K, True), H.dev(V, True), new_lens=nl, calibrate=True)
-    out, _ = gc.decode(H.dev(synth.queries(w, 0, 0, B), True), float(H.SCALE))
+    q = synth.queries(w, 0, 0, B)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+    out, _ = gc.decode(H.dev(q, True), float(H.SCALE), lse=lse)
     torch.cuda.synchronize()
     st = gc.status(clear=True)
     assert st[0] & H.kvq().KVQ_DEV_BAD_PAGE
-    assert torch.isfinite(out).all()
+    assert H.np_of(gc["seq_lens"]).tolist() == [40, 0]
+    assert torch.all(out[1] == 0) and torch.all(torch.isneginf(lse[1]))
+    # the oracle over the same statistics, with sequence 1 holding no tokens (the calibration
+    # reads the whole block: the device saw both sequences' rows)
+    oc.calibrate(K, V, True, new_lens=lens)
+    oc.append(K, V, True, new_lens=np.array([40, 0], np.int32))  # the calibrated scales, sequence 0 only
+    H.compare_paged(oc, gc, "after a refused sequence")
+    ref, ref_lse = oc.decode(q, True, float(H.SCALE))
+    H.attn_check(out, ref, lse, ref_lse, "decode after a refused sequence")
     assert gc.status()[0] == 0
 
 
@@ -396,6 +408,7 @@ def test_rescale_schedule_every_1024_tokens():
 
 # ------------------------------------------------------------------ dequantize
 @pytest.mark.parametrize("ks,vs", [(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR), (S.KIVI_INT2, S.KIVI_INT2),
+                                   (S.KIVI_INT4_F16, S.KIVI_INT4_F16), (S.KIVI_INT2_F16, S.KIVI_INT2_F16),
                                    (S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL),
                                    (S.FP8_E5M2_PER_TENSOR, S.FP8_E5M2_PER_TENSOR),
                                    (S.INT4_SYM_PER_GROUP, S.INT4_SYM_PER_GROUP)])
