@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="measure the headline workload only")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="run the workload with this batch instead of its own (a reduced case for profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     return ap.parse_args()
 
@@ -786,6 +788,10 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.batch:
+        base = synth.workloads()[args.workload]
+        synth.register_workload(synth.Workload(**{**base.__dict__, "B": args.batch}))
+        args.no_per_config = True
     w = synth.workloads()[args.workload]
     dtype = dtype_of(w)
     config = {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.D,

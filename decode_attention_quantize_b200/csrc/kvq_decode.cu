@@ -653,11 +653,14 @@ __device__ __forceinline__ float4 vscale4(const uint8_t* base, int tok) {
 }
 
 // ------------------------------------------------------------------ one tile, one warp
-// kMasked: the warp's tokens are not all valid (ragged tail or missing pages).
-template <class C, bool kMasked>
+// kMasked: the warp's tokens are not all valid (ragged tail or missing pages). kResidual: a tile
+// of KIVI's bf16 residual rows (a separate instantiation, so the code tiles' path carries none
+// of the residual work).
+template <class C, bool kMasked, bool kResidual>
 __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p, const uint8_t* base,
-                                          const TileDesc& d, uint32_t valid, bool residual, int tok_base,
-                                          float sc_log2, const float* q_s) {
+                                          const TileDesc& d, uint32_t valid, int tok_base, float sc_log2,
+                                          const float* q_s) {
+  constexpr bool residual = kResidual;
   const int g = S.g, c = S.c, w = S.w;
   // validity of a token of this warp's range (tile-relative index)
   auto tok_ok = [&](int tok) -> bool {
@@ -1295,10 +1298,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBl
                                                        ((valid >> (tok_base / p.page_size)) &
                                                         ((1u << (C::kTPW + p.page_size - 1) / p.page_size) - 1u)) ==
                                                            ((1u << (C::kTPW + p.page_size - 1) / p.page_size) - 1u));
-      if (full)
-        warp_tile<C, false>(S, p, base, d, valid, residual, tok_base, sc_log2, q_s);
+      if (C::kKivi && residual)
+        warp_tile<C, true, C::kKivi>(S, p, base, d, valid, tok_base, sc_log2, q_s);
+      else if (full)
+        warp_tile<C, false, false>(S, p, base, d, valid, tok_base, sc_log2, q_s);
       else
-        warp_tile<C, true>(S, p, base, d, valid, residual, tok_base, sc_log2, q_s);
+        warp_tile<C, true, false>(S, p, base, d, valid, tok_base, sc_log2, q_s);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * st);

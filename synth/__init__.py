@@ -179,7 +179,21 @@ class Workload:
         return table, pool
 
 
+_OVERRIDES: dict = {}
+
+
+def register_workload(w: "Workload") -> None:
+    """Replace a named workload's shape for this process (e.g. a reduced batch for profiling)."""
+    _OVERRIDES[w.name] = w
+
+
 def workloads() -> dict:
+    table = _base_workloads()
+    table.update(_OVERRIDES)
+    return table
+
+
+def _base_workloads() -> dict:
     """The workloads: tiny INT8, FP8 E4M3 and FP8 E5M2 8B-shaped, KIVI-4 and INT4 per-group
     70B-shaped (INT4 with groups of 32, also with the Walsh-Hadamard rotation, and with groups
     of 128; same inputs), KIVI-2 131K, the two KIVI shapes with fp16 scale and minimum (same
