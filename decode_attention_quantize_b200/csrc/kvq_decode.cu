@@ -36,7 +36,6 @@ namespace kvq {
 namespace {
 
 constexpr int kCW = 4;                  // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kRT = 32;                 // residual tile tokens (bf16 rows)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -107,8 +106,15 @@ struct Cfg {
   static constexpr int kRopeBytes = ROPE ? 64 * 8 + kCW * 64 * 8 + kHeadDim * 4 : 0;
   static constexpr int kFixedBytes = 2048 + kCW * kMergeHeads * kHeadDim * 4 + kCW * 8 * 4 * 2 +
                                      kCW * kMergeHeads * 4 * 4 + 8 * 144 * 4 + kRopeBytes + 1024;
-  static constexpr int kStages = (3 * kStageBytes + kFixedBytes <= 112 * 1024) ? 3 : 2;
-  static constexpr int kMinBlocks = 2;  // resident CTAs per SM the registers (168) are sized for
+  // Dense KIVI: no producer warp. The consumer warps refill the stages themselves (the last warp
+  // to release a stage issues its next tile), so three CTAs of four warps fit on an SM at the
+  // same 168 registers a thread; the others keep a producer warp and two CTAs per SM.
+  static constexpr bool kSelfFed = kKivi && !PAGED;
+  static constexpr int kThreadsCta = kSelfFed ? kCW * 32 : (kCW + 1) * 32;
+  static constexpr int kMinBlocks = kSelfFed ? 3 : 2;  // resident CTAs per SM the registers are sized for
+  static constexpr int kStages =
+      kSelfFed ? ((3 * (3 * kStageBytes + kFixedBytes + 1024) <= 227 * 1024) ? 3 : 2)
+               : ((3 * kStageBytes + kFixedBytes <= 112 * 1024) ? 3 : 2);
   static constexpr int kOffDesc = kStages * kStageBytes;
   static constexpr int kOffBar = kOffDesc + kStages * 64;
   static constexpr int kOffRedO = kOffBar + 2 * kStages * 8 + 64;
@@ -240,6 +246,96 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 }
 
 // ------------------------------------------------------------------ producer
+// Issue the copies of tile d into stage `cur`: its descriptor, the expected transaction bytes
+// on the stage's full barrier, then 2-D TMA boxes of codes and 1-D bulk copies of metadata (or
+// the bf16 residual rows).
+template <class C>
+__device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, uint8_t* stages,
+                           TileDesc* descs, uint32_t full0, int cur, TileDesc d) {
+  const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
+  const uint32_t bar = full0 + 8 * cur;
+  const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
+  if (d.kind == 1) {  // KIVI residual: bf16 rows, whole 32-token slab (inside rcap)
+    const size_t r0 = (pair_row * p.rcap + d.t0) * kHeadDim;
+    descs[cur] = d;
+    mbar_arrive_expect_tx(bar, 2 * kRT * kHeadDim * 2);
+    bulk_g2s(sb, p.k_res + r0, kRT * kHeadDim * 2, bar);
+    bulk_g2s(sb + kRT * kHeadDim * 2, p.v_res + r0, kRT * kHeadDim * 2, bar);
+    return;
+  }
+  if constexpr (!C::kPaged) {
+    // whole tile: capacity is a multiple of 128 tokens, so the tile lies inside the row
+    const size_t row0 = pair_row * p.cap + d.t0;
+    const uint32_t bytes = C::kTS * (C::kKRow + C::kVRow) + C::kKMeta + C::kVMeta;
+    descs[cur] = d;
+    mbar_arrive_expect_tx(bar, bytes);
+    tma_2d(sb + C::kOffK, tk, 0, (int)row0, bar);
+    tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar);
+    if constexpr (C::kKivi) {
+      const size_t g0 = (pair_row * (p.cap / 32) + d.t0 / 32) * kHeadDim;
+      // element offsets in bytes: fp32 or fp16 metadata
+      const uint8_t* ks8 = reinterpret_cast<const uint8_t*>(p.k_scale);
+      const uint8_t* kz8 = reinterpret_cast<const uint8_t*>(p.k_zero);
+      const uint8_t* vs8 = reinterpret_cast<const uint8_t*>(p.v_scale);
+      const uint8_t* vz8 = reinterpret_cast<const uint8_t*>(p.v_zero);
+      bulk_g2s(sb + C::kOffKM, ks8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
+      bulk_g2s(sb + C::kOffKM + C::kKMeta / 2, kz8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
+      bulk_g2s(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
+      bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
+    } else {
+      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
+      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
+      if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * C::kNG, C::kKMeta, bar);
+      if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * C::kNG, C::kVMeta, bar);
+    }
+  } else {
+    // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
+    const int ps = p.page_size;
+    const int npg = (d.n + ps - 1) / ps;
+    const int pi0 = d.t0 / ps;
+    int page[C::kTS / 16];
+    uint32_t valid = 0, nvalid = 0;
+#pragma unroll
+    for (int i = 0; i < C::kTS / 16; ++i) {
+      page[i] = -1;
+      if (i < npg) {
+        const int pi = pi0 + i;
+        const int id = pi < p.max_pages ? p.page_table[(size_t)d.b * p.max_pages + pi] : -1;
+        page[i] = id;
+        if (id >= 0 && id < p.num_pages) {
+          valid |= 1u << i;
+          ++nvalid;
+        } else {
+          flag(p.status, KVQ_DEV_BAD_PAGE);
+        }
+      }
+    }
+    d.valid = valid;
+    descs[cur] = d;
+    uint32_t per_page = ps * (C::kKRow + C::kVRow);
+    if constexpr (C::kKFold == FOLD_TOKEN) per_page += ps * 4;
+    if constexpr (C::kVFold == FOLD_TOKEN) per_page += ps * 4;
+    if constexpr (C::kKFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
+    if constexpr (C::kVFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
+    mbar_arrive_expect_tx(bar, nvalid * per_page);
+#pragma unroll
+    for (int i = 0; i < C::kTS / 16; ++i) {
+      if (i >= npg || !((valid >> i) & 1u)) continue;
+      const size_t prow = ((size_t)page[i] * p.Hkv + d.hk) * ps;
+      tma_2d(sb + C::kOffK + i * ps * C::kKRow, tk, 0, (int)prow, bar);
+      tma_2d(sb + C::kOffV + i * ps * C::kVRow, tv, 0, (int)prow, bar);
+      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar);
+      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar);
+      if constexpr (C::kKFold == FOLD_GROUP)
+        bulk_g2s(sb + C::kOffKM + i * ps * C::kNG * 4, p.k_scale + prow * C::kNG, ps * C::kNG * 4, bar);
+      if constexpr (C::kVFold == FOLD_GROUP)
+        bulk_g2s(sb + C::kOffVM + i * ps * C::kNG * 4, p.v_scale + prow * C::kNG, ps * C::kNG * 4, bar);
+    }
+  }
+}
+
+// The producer warp's loop (one elected lane): each stage is refilled once the consumer warps
+// have released it.
 template <class C>
 __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                          uint8_t* stages, TileDesc* descs, uint32_t full0, uint32_t empty0,
@@ -248,92 +344,13 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
   ti.init(p, s, tb, te);
   for (int it = 0, st = 0, phase = 0; ti.t < te; ti.next(p, s), ++it) {
     if (it >= C::kStages && !mbar_wait(empty0 + 8 * st, phase ^ 1, p.status)) return;
-    TileDesc d = ti.desc(p, s);
+    const TileDesc d = ti.desc(p, s);
     const int cur = st;
     if (++st == C::kStages) {
       st = 0;
       phase ^= 1;
     }
-    const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
-    const uint32_t bar = full0 + 8 * cur;
-    const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
-    if (d.kind == 1) {  // KIVI residual: bf16 rows, whole 32-token slab (inside rcap)
-      const size_t r0 = (pair_row * p.rcap + d.t0) * kHeadDim;
-      descs[cur] = d;
-      mbar_arrive_expect_tx(bar, 2 * kRT * kHeadDim * 2);
-      bulk_g2s(sb, p.k_res + r0, kRT * kHeadDim * 2, bar);
-      bulk_g2s(sb + kRT * kHeadDim * 2, p.v_res + r0, kRT * kHeadDim * 2, bar);
-      continue;
-    }
-    if constexpr (!C::kPaged) {
-      // whole tile: capacity is a multiple of 128 tokens, so the tile lies inside the row
-      const size_t row0 = pair_row * p.cap + d.t0;
-      const uint32_t bytes = C::kTS * (C::kKRow + C::kVRow) + C::kKMeta + C::kVMeta;
-      descs[cur] = d;
-      mbar_arrive_expect_tx(bar, bytes);
-      tma_2d(sb + C::kOffK, tk, 0, (int)row0, bar);
-      tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar);
-      if constexpr (C::kKivi) {
-        const size_t g0 = (pair_row * (p.cap / 32) + d.t0 / 32) * kHeadDim;
-        // element offsets in bytes: fp32 or fp16 metadata
-        const uint8_t* ks8 = reinterpret_cast<const uint8_t*>(p.k_scale);
-        const uint8_t* kz8 = reinterpret_cast<const uint8_t*>(p.k_zero);
-        const uint8_t* vs8 = reinterpret_cast<const uint8_t*>(p.v_scale);
-        const uint8_t* vz8 = reinterpret_cast<const uint8_t*>(p.v_zero);
-        bulk_g2s(sb + C::kOffKM, ks8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
-        bulk_g2s(sb + C::kOffKM + C::kKMeta / 2, kz8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
-        bulk_g2s(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
-        bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
-      } else {
-        if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
-        if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
-        if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * C::kNG, C::kKMeta, bar);
-        if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * C::kNG, C::kVMeta, bar);
-      }
-    } else {
-      // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
-      const int ps = p.page_size;
-      const int npg = (d.n + ps - 1) / ps;
-      const int pi0 = d.t0 / ps;
-      int page[C::kTS / 16];
-      uint32_t valid = 0, nvalid = 0;
-#pragma unroll
-      for (int i = 0; i < C::kTS / 16; ++i) {
-        page[i] = -1;
-        if (i < npg) {
-          const int pi = pi0 + i;
-          const int id = pi < p.max_pages ? p.page_table[(size_t)d.b * p.max_pages + pi] : -1;
-          page[i] = id;
-          if (id >= 0 && id < p.num_pages) {
-            valid |= 1u << i;
-            ++nvalid;
-          } else {
-            flag(p.status, KVQ_DEV_BAD_PAGE);
-          }
-        }
-      }
-      d.valid = valid;
-      descs[cur] = d;
-      uint32_t per_page = ps * (C::kKRow + C::kVRow);
-      if constexpr (C::kKFold == FOLD_TOKEN) per_page += ps * 4;
-      if constexpr (C::kVFold == FOLD_TOKEN) per_page += ps * 4;
-      if constexpr (C::kKFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
-      if constexpr (C::kVFold == FOLD_GROUP) per_page += ps * C::kNG * 4;
-      mbar_arrive_expect_tx(bar, nvalid * per_page);
-#pragma unroll
-      for (int i = 0; i < C::kTS / 16; ++i) {
-        if (i >= npg || !((valid >> i) & 1u)) continue;
-        const size_t prow = ((size_t)page[i] * p.Hkv + d.hk) * ps;
-        tma_2d(sb + C::kOffK + i * ps * C::kKRow, tk, 0, (int)prow, bar);
-        tma_2d(sb + C::kOffV + i * ps * C::kVRow, tv, 0, (int)prow, bar);
-        if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar);
-        if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar);
-        if constexpr (C::kKFold == FOLD_GROUP)
-          bulk_g2s(sb + C::kOffKM + i * ps * C::kNG * 4, p.k_scale + prow * C::kNG, ps * C::kNG * 4, bar);
-        if constexpr (C::kVFold == FOLD_GROUP)
-          bulk_g2s(sb + C::kOffVM + i * ps * C::kNG * 4, p.v_scale + prow * C::kNG, ps * C::kNG * 4, bar);
-      }
-    }
+    issue_tile<C>(p, tk, tv, stages, descs, full0, cur, d);
   }
 }
 
@@ -1150,7 +1167,7 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 
 // ------------------------------------------------------------------ the kernel
 template <int KS, int VS, bool PAGED, int NG, bool ROPE>
-__global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBlocks)
+__global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBlocks)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_v) {
   using C = Cfg<KS, VS, PAGED, NG, ROPE>;
@@ -1165,16 +1182,26 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBl
   TileDesc* descs = reinterpret_cast<TileDesc*>(smem + C::kOffDesc);
   const uint32_t full0 = smem_addr(smem + C::kOffBar);
   const uint32_t empty0 = full0 + 8 * C::kStages;
+  // self-fed pipeline: releases of each stage counted in the slack after the barriers
+  uint32_t* releases = reinterpret_cast<uint32_t*>(smem + C::kOffBar + 2 * C::kStages * 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, kCW);
+      releases[i] = 0u;
     }
     fence_barrier_init();
   }
   __syncthreads();
-  if (warp == kCW) {
+  if constexpr (C::kSelfFed) {
+    if (threadIdx.x == 0) {  // the first stages; the rest are refilled by the consumer warps
+      TileIter f;
+      f.init(p, sc, tb, te);
+      for (int s0 = 0; s0 < C::kStages && f.t < te; ++s0, f.next(p, sc))
+        issue_tile<C>(p, &tmap_k, &tmap_v, smem, descs, full0, s0, f.desc(p, sc));
+    }
+  } else if (warp == kCW) {
     if (lane == 0) producer<C>(p, &tmap_k, &tmap_v, smem, descs, full0, empty0, sc, tb, te);
     return;
   }
@@ -1307,6 +1334,19 @@ __global__ void __launch_bounds__(kThreads, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBl
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty0 + 8 * st);
+    if constexpr (C::kSelfFed) {
+      // the last warp to release this stage refills it with the tile kStages ahead (the wait on
+      // the completed release orders every warp's reads of the stage before the copies)
+      if (lane == 0 && atomicAdd(releases + st, 1u) == kCW - 1) {
+        releases[st] = 0u;
+        const int tn = ti.t + C::kStages;
+        if (tn < te && mbar_wait(empty0 + 8 * st, phase, p.status)) {
+          TileIter f;
+          f.init(p, sc, tn, te);
+          issue_tile<C>(p, &tmap_k, &tmap_v, smem, descs, full0, st, f.desc(p, sc));
+        }
+      }
+    }
     if (++st == C::kStages) {
       st = 0;
       phase ^= 1;
@@ -1544,13 +1584,14 @@ bool make_map(CUtensorMap* map, const void* base, int row_bytes_, uint64_t rows,
 struct Variant {
   int k, v, paged, ng, rope;
   void (*kernel)(const DecodeParams, const CUtensorMap, const CUtensorMap);
-  int smem, ts;
+  int smem, ts, threads;
 };
 
 template <int KS, int VS, bool PG, int NG = 4, bool ROPE = false>
 Variant variant() {
   using C = Cfg<KS, VS, PG, NG, ROPE>;
-  return Variant{KS, VS, PG ? 1 : 0, NG, ROPE ? 1 : 0, decode_kernel<KS, VS, PG, NG, ROPE>, C::kSmemBytes, C::kTS};
+  return Variant{KS, VS, PG ? 1 : 0, NG, ROPE ? 1 : 0, decode_kernel<KS, VS, PG, NG, ROPE>, C::kSmemBytes, C::kTS,
+                 C::kThreadsCta};
 }
 
 constexpr int kNumVariants = 40;
@@ -1647,7 +1688,7 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
   if (occ <= 0) {
     e = cudaFuncSetAttribute(var->kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, var->smem);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var->kernel, kThreads, var->smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, var->kernel, var->threads, var->smem);
     if (e != cudaSuccess) return e;
     if (occ < 1) occ = 1;
     if (dev < kMaxDevices) occ_cache[vi][dev].store(occ, std::memory_order_relaxed);
@@ -1671,7 +1712,7 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
     e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, p);
     if (e != cudaSuccess) return e;
   }
-  e = launch_pdl(var->kernel, dim3(ncta), dim3(kThreads), (size_t)var->smem, st, p, tk, tv);
+  e = launch_pdl(var->kernel, dim3(ncta), dim3(var->threads), (size_t)var->smem, st, p, tk, tv);
   if (e != cudaSuccess) {
     if (dev < kMaxDevices) occ_cache[vi][dev].store(0, std::memory_order_relaxed);  // set up again next call
     return e;
