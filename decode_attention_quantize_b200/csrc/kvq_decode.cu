@@ -97,9 +97,8 @@ struct Cfg {
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
-  // heads staged per pass of the per-pair warp merge: all eight for INT4 KIVI (whose register
-  // allocation suffers from the two-pass form), else four (half the staging, room for a stage)
-  static constexpr int kMergeHeads = (kKivi && kKFmt == FMT_U4) ? 8 : 4;
+  // heads staged per pass of the per-pair warp merge: four (half the staging, room for a stage)
+  static constexpr int kMergeHeads = 4;
   // 128-token stages: three when three still fit next to a second CTA on the SM
   // RoPE: the inverse frequencies (64 fp64), each warp's (base angle, frequency) pairs (64 float2)
   // and the kv head's per-channel key scales (128 fp32)
@@ -250,8 +249,9 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 // on the stage's full barrier, then 2-D TMA boxes of codes and 1-D bulk copies of metadata (or
 // the bf16 residual rows).
 template <class C>
-__device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, uint8_t* stages,
-                           TileDesc* descs, uint32_t full0, int cur, TileDesc d) {
+__device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
+                           const CUtensorMap* tks, const CUtensorMap* tkz, uint8_t* stages, TileDesc* descs,
+                           uint32_t full0, int cur, TileDesc d) {
   const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
   const uint32_t bar = full0 + 8 * cur;
   const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
@@ -274,12 +274,13 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
     if constexpr (C::kKivi) {
       const size_t g0 = (pair_row * (p.cap / 32) + d.t0 / 32) * kHeadDim;
       // element offsets in bytes: fp32 or fp16 metadata
-      const uint8_t* ks8 = reinterpret_cast<const uint8_t*>(p.k_scale);
-      const uint8_t* kz8 = reinterpret_cast<const uint8_t*>(p.k_zero);
       const uint8_t* vs8 = reinterpret_cast<const uint8_t*>(p.v_scale);
       const uint8_t* vz8 = reinterpret_cast<const uint8_t*>(p.v_zero);
-      bulk_g2s(sb + C::kOffKM, ks8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
-      bulk_g2s(sb + C::kOffKM + C::kKMeta / 2, kz8 + g0 * C::kMetaElem, C::kKMeta / 2, bar);
+      // key scales and minima as 128-byte rows through TMA with the 128-byte swizzle, so the query
+      // build's reads (four lanes a 128-byte row apart) fall in distinct banks
+      const int krow = (int)(g0 * C::kMetaElem / 128);
+      tma_2d(sb + C::kOffKM, tks, 0, krow, bar);
+      tma_2d(sb + C::kOffKM + C::kKMeta / 2, tkz, 0, krow, bar);
       bulk_g2s(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
       bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
     } else {
@@ -338,8 +339,8 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
 // have released it.
 template <class C>
 __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                         uint8_t* stages, TileDesc* descs, uint32_t full0, uint32_t empty0,
-                         const Sched& s, int tb, int te) {
+                         const CUtensorMap* tks, const CUtensorMap* tkz, uint8_t* stages, TileDesc* descs,
+                         uint32_t full0, uint32_t empty0, const Sched& s, int tb, int te) {
   TileIter ti;
   ti.init(p, s, tb, te);
   for (int it = 0, st = 0, phase = 0; ti.t < te; ti.next(p, s), ++it) {
@@ -350,7 +351,7 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       st = 0;
       phase ^= 1;
     }
-    issue_tile<C>(p, tk, tv, stages, descs, full0, cur, d);
+    issue_tile<C>(p, tk, tv, tks, tkz, stages, descs, full0, cur, d);
   }
 }
 
@@ -493,6 +494,7 @@ struct Consumer {
   bool qsplit;
   float kmul;        // score multiplier (log2 domain)
   float bias[2];     // KIVI group bias (raw units), heads 2c, 2c+1
+  float qabs;        // KIVI: the largest |q| of the pair's staged queries (all heads)
   int qmode;         // 0: fragments for codes built, 1: for bf16 residual rows
   uint32_t zpk[8][2], zpv[8][2];  // uint8 asymmetric: f16x2 (1024 + zero point)
 };
@@ -527,27 +529,54 @@ __device__ __forceinline__ float4 meta4(const void* base, int i) {
   }
 }
 
+// Elements 4i .. 4i + 3 (fp32, or fp16 when kHalf) of KIVI key group `grp` in a stage region the
+// producer filled by TMA as 128-byte rows with the 128-byte swizzle (16-byte chunk index XOR row).
+template <bool kHalf>
+__device__ __forceinline__ float4 kmeta4_swz(const void* region, int grp, int i) {
+  constexpr int es = kHalf ? 2 : 4;
+  const int b = grp * kHeadDim * es + i * 4 * es;  // byte offset before the swizzle
+  const int row = b >> 7, within = b & 127;
+  const uint8_t* a = static_cast<const uint8_t*>(region) + swz<128>(row, within >> 4) + (within & 15);
+  if constexpr (kHalf) {
+    const uint2 u = *reinterpret_cast<const uint2*>(a);
+    const float2 x = f16x2_to_float2(u.x), y = f16x2_to_float2(u.y);
+    return make_float4(x.x, x.y, y.x, y.y);
+  } else {
+    return *reinterpret_cast<const float4*>(a);
+  }
+}
+
 // Build Q' fragments (head g, this thread's 32 channels 32c..32c+31) from q_s, optionally
 // multiplied by a per-channel fold; with `zmin` also returns sum_d q_d * zmin_d over those
-// channels (the KIVI key-minimum term). fold and zmin hold fp32, or fp16 when kHalf. Returns the
-// power-of-two shift applied to Q'.
-template <int FMT, bool kHalf = false>
+// channels (the KIVI key-minimum term). fold and zmin hold fp32, or fp16 when kHalf. The
+// power-of-two shift applied to Q' (returned) comes from the largest |q'| of the warp, or is
+// given (kGivenShift: from a bound on |q'|, which skips that pass).
+// kSwz: fold and zmin are swizzled KIVI key-metadata regions (kmeta4_swz) of group `grp`.
+template <int FMT, bool kHalf = false, bool kGivenShift = false, bool kSwz = false>
 __device__ __forceinline__ int build_q(const float* q_s, const void* fold, const void* zmin, int g, int c,
-                                       uint32_t (&qh)[8][2], uint32_t (&ql)[8][2], float* bias = nullptr) {
+                                       uint32_t (&qh)[8][2], uint32_t (&ql)[8][2], float* bias = nullptr,
+                                       int given_shift = 0, int grp = 0) {
   const float4* qrow = reinterpret_cast<const float4*>(q_s + q_off(g, 32 * c));
-  // pass 1: the largest |q'| of the warp sets the range shift
-  float mx = 0.0f;
+  auto meta = [&](const void* base, int i) -> float4 {
+    if constexpr (kSwz) return kmeta4_swz<kHalf>(base, grp, 8 * c + i);
+    return meta4<kHalf>(base, 8 * c + i);
+  };
+  int eq = given_shift;
+  if constexpr (!kGivenShift) {
+    // pass 1: the largest |q'| of the warp sets the range shift
+    float mx = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4 q4 = qrow[i];
-    if (fold) {
-      const float4 f4 = meta4<kHalf>(fold, 8 * c + i);
-      q4.x *= f4.x; q4.y *= f4.y; q4.z *= f4.z; q4.w *= f4.w;
+    for (int i = 0; i < 8; ++i) {
+      float4 q4 = qrow[i];
+      if (fold) {
+        const float4 f4 = meta(fold, i);
+        q4.x *= f4.x; q4.y *= f4.y; q4.z *= f4.z; q4.w *= f4.w;
+      }
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w))));
     }
-    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w))));
+    mx = warp_max(mx);
+    eq = range_shift(mx);
   }
-  mx = warp_max(mx);
-  const int eq = range_shift(mx);
   const float sh = pow2i(eq);
   // pass 2: scaled products by local channel, then the fragment split
   float pl[32];
@@ -557,11 +586,11 @@ __device__ __forceinline__ int build_q(const float* q_s, const void* fold, const
     const float4 q4 = qrow[i];
     float4 m4 = make_float4(sh, sh, sh, sh);
     if (fold) {
-      const float4 f4 = meta4<kHalf>(fold, 8 * c + i);
+      const float4 f4 = meta(fold, i);
       m4 = make_float4(f4.x * sh, f4.y * sh, f4.z * sh, f4.w * sh);
     }
     if (zmin) {
-      const float4 z4 = meta4<kHalf>(zmin, 8 * c + i);
+      const float4 z4 = meta(zmin, i);
       bs = fmaf(q4.x, z4.x, fmaf(q4.y, z4.y, fmaf(q4.z, z4.z, fmaf(q4.w, z4.w, bs))));
     }
     pl[4 * i] = q4.x * m4.x;
@@ -701,10 +730,17 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
   if constexpr (C::kRope) rope_warp_angles(rope_theta_s(q_s), rope_angles(q_s) + w * 64, d.t0 + tok_base, 4 * g + c);
   if constexpr (C::kKivi) {
     if (!residual) {
-      const uint8_t* ksm = base + C::kOffKM + w * kHeadDim * C::kMetaElem;
-      const uint8_t* kzm = base + C::kOffKM + C::kKMeta / 2 + w * kHeadDim * C::kMetaElem;
+      // the tile's key scales and minima: swizzled 128-byte rows, group w is this warp's
+      const uint8_t* ksm = base + C::kOffKM;
+      const uint8_t* kzm = base + C::kOffKM + C::kKMeta / 2;
+      // range shift of the group's Q' = q * s from the bound max|q| * max s (one 4-scale load a
+      // lane instead of a pass over the 32 products): Q' stays below 2^15, and its smaller
+      // values keep their ~22 bits in the hi + lo split while within 2^20 of the bound
+      const float4 s4 = kmeta4_swz<C::kHalfMeta>(ksm, w, 4 * g + c);
+      const float sgrp = warp_max(fmaxf(fmaxf(s4.x, s4.y), fmaxf(s4.z, s4.w)));
       float bs;
-      const int eq = build_q<C::kKFmt, C::kHalfMeta>(q_s, ksm, kzm, g, c, S.qh, S.ql, &bs);
+      const int eq = build_q<C::kKFmt, C::kHalfMeta, true, true>(q_s, ksm, kzm, g, c, S.qh, S.ql, &bs,
+                                                                  range_shift(S.qabs * sgrp), w);
       bs += __shfl_xor_sync(0xffffffffu, bs, 1);
       bs += __shfl_xor_sync(0xffffffffu, bs, 2);
       S.bias[0] = __shfl_sync(0xffffffffu, bs, 4 * (2 * c));
@@ -1058,31 +1094,28 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         }
       }
     } else {
-      // one B operand per 32-channel group; KIVI's zero-point term on CUDA cores
-      uint32_t bh[4][2], bl[4][2];
-      float4 s4[4];  // value scales of this thread's four tokens, groups 0..3
+      // one B operand per 32-channel group, built just before that group's MMAs; KIVI's
+      // zero-point term on CUDA cores
+      // value scales of this thread's four tokens, groups 0..3 (fp16 metadata stays packed as
+      // halves until its group is used, which halves the registers it holds)
+      float4 s4[4];
+      uint2 s4h[4];
       float rv[4];   // residual: the power of two each of the four tokens' value rows is scaled by
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         s4[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        s4h[k] = make_uint2(0u, 0u);
         rv[k] = 1.0f;
-        if (!residual && ok[k]) s4[k] = vscale4<C>(base, tk[k]);
+        if constexpr (C::kHalfMeta) {
+          if (!residual && ok[k]) s4h[k] = lds<uint2>(base + C::kOffVM + tk[k] * 8);
+        } else {
+          if (!residual && ok[k]) s4[k] = vscale4<C>(base, tk[k]);
+        }
         if (C::kKivi && residual) {
           const int x = __shfl_sync(0xffffffffu, res_vx, tk[k] & 31);
           rv[k] = pow2i(x);
           s4[k] = make_float4(pow2i(-x), 0.f, 0.f, 0.f);
         }
-      }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float pv[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float sj = j == 0 ? s4[k].x : j == 1 ? s4[k].y : j == 2 ? s4[k].z : s4[k].w;
-          pv[k] = residual ? pt[sb][k] * s4[k].x * pscale : pt[sb][k] * sj * pscale;
-        }
-        split_f16x2(pv[0], pv[1], bh[j][0], bl[j][0]);
-        split_f16x2(pv[2], pv[3], bh[j][1], bl[j][1]);
       }
       if (C::kKivi && !residual) {
 #pragma unroll
@@ -1114,6 +1147,23 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
+        uint32_t bh[2], bl[2];  // P' of group j: tokens (2c, 2c + 1) and (2c + 8, 2c + 9), hi + lo
+        {
+          float pv[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float sj;
+            if constexpr (C::kHalfMeta) {
+              const float2 h2 = f16x2_to_float2((j >> 1) ? s4h[k].y : s4h[k].x);
+              sj = (j & 1) ? h2.y : h2.x;
+            } else {
+              sj = j == 0 ? s4[k].x : j == 1 ? s4[k].y : j == 2 ? s4[k].z : s4[k].w;
+            }
+            pv[k] = residual ? pt[sb][k] * s4[k].x * pscale : pt[sb][k] * sj * pscale;
+          }
+          split_f16x2(pv[0], pv[1], bh[0], bl[0]);
+          split_f16x2(pv[2], pv[3], bh[1], bl[1]);
+        }
         uint32_t pr[2][4];  // [token pair][channel e]: f16x2 (token even, token odd)
         if (residual) {
 #pragma unroll
@@ -1155,10 +1205,8 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           const int mt = 2 * j + half;
-          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bh[j][0],
-                    bh[j][1]);
-          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bl[j][0],
-                    bl[j][1]);
+          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bh[0], bh[1]);
+          mma_16816(S.o[mt], pr[0][2 * half], pr[0][2 * half + 1], pr[1][2 * half], pr[1][2 * half + 1], bl[0], bl[1]);
         }
       }
     }
@@ -1169,7 +1217,8 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
 template <int KS, int VS, bool PAGED, int NG, bool ROPE>
 __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg<KS, VS, PAGED, NG, ROPE>::kMinBlocks)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_v) {
+                  const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_ks,
+                  const __grid_constant__ CUtensorMap tmap_kz) {
   using C = Cfg<KS, VS, PAGED, NG, ROPE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
@@ -1199,10 +1248,10 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
       TileIter f;
       f.init(p, sc, tb, te);
       for (int s0 = 0; s0 < C::kStages && f.t < te; ++s0, f.next(p, sc))
-        issue_tile<C>(p, &tmap_k, &tmap_v, smem, descs, full0, s0, f.desc(p, sc));
+        issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, s0, f.desc(p, sc));
     }
   } else if (warp == kCW) {
-    if (lane == 0) producer<C>(p, &tmap_k, &tmap_v, smem, descs, full0, empty0, sc, tb, te);
+    if (lane == 0) producer<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, empty0, sc, tb, te);
     return;
   }
 
@@ -1276,6 +1325,16 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
 #pragma unroll
       for (int j = 0; j < 4; ++j) S.zacc[j] = 0.0f;
       S.qmode = -1;
+      if constexpr (C::kKivi) {  // first factor of the key groups' shift bound: max |q| of the pair
+        const float4* qrow = reinterpret_cast<const float4*>(q_s + q_off(g, 32 * c));
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float4 q4 = qrow[i];
+          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(q4.x), fabsf(q4.y)), fmaxf(fabsf(q4.z), fabsf(q4.w))));
+        }
+        S.qabs = warp_max(mx);
+      }
       if constexpr (!C::kKivi) {
         const float* fold = nullptr;
         if constexpr (C::kKFold == FOLD_CHANNEL) fold = p.k_scale + (size_t)d.hk * kHeadDim;
@@ -1343,7 +1402,7 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
         if (tn < te && mbar_wait(empty0 + 8 * st, phase, p.status)) {
           TileIter f;
           f.init(p, sc, tn, te);
-          issue_tile<C>(p, &tmap_k, &tmap_v, smem, descs, full0, st, f.desc(p, sc));
+          issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, st, f.desc(p, sc));
         }
       }
     }
@@ -1583,7 +1642,7 @@ bool make_map(CUtensorMap* map, const void* base, int row_bytes_, uint64_t rows,
 
 struct Variant {
   int k, v, paged, ng, rope;
-  void (*kernel)(const DecodeParams, const CUtensorMap, const CUtensorMap);
+  void (*kernel)(const DecodeParams, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap);
   int smem, ts, threads;
 };
 
@@ -1706,13 +1765,23 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
   const int box = p.paged ? p.page_size : var->ts;
   if (!make_map(&tk, p.k_codes, kr, rows, box) || !make_map(&tv, p.v_codes, vr, rows, box))
     return cudaErrorInvalidValue;
+  // KIVI key scales and minima seen as 128-byte rows (4 rows per 32-token group of fp32, 2 of fp16);
+  // a tile's 4 groups are one box
+  CUtensorMap tks = tk, tkz = tk;
+  if (is_kivi(p.k_scheme)) {
+    const int es = kivi_f16(p.k_scheme) ? 2 : 4;
+    const uint64_t mrows = (uint64_t)p.B * p.Hkv * (uint64_t)(p.cap / 32) * es;  // 128 channels * es / 128
+    const int mbox = (var->ts / 32) * es;
+    if (!make_map(&tks, p.k_scale, 128, mrows, mbox) || !make_map(&tkz, p.k_zero, 128, mrows, mbox))
+      return cudaErrorInvalidValue;
+  }
   // Programmatic dependent launches: each kernel may be scheduled while its predecessor
   // drains and waits in griddepcontrol.wait, hiding the launch gaps between the three.
   if (p.paged) {
     e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, p);
     if (e != cudaSuccess) return e;
   }
-  e = launch_pdl(var->kernel, dim3(ncta), dim3(var->threads), (size_t)var->smem, st, p, tk, tv);
+  e = launch_pdl(var->kernel, dim3(ncta), dim3(var->threads), (size_t)var->smem, st, p, tk, tv, tks, tkz);
   if (e != cudaSuccess) {
     if (dev < kMaxDevices) occ_cache[vi][dev].store(0, std::memory_order_relaxed);  // set up again next call
     return e;
