@@ -97,23 +97,26 @@ struct Cfg {
   static constexpr int kQuantBytes = kOffVM + kVMeta;
   static constexpr int kResBytes = kKivi ? 2 * kRT * kHeadDim * 2 : 0;
   static constexpr int kStageBytes = rup(cmax(kQuantBytes, kResBytes), 1024);
-  // heads staged per pass of the per-pair warp merge: four (half the staging, room for a stage)
-  static constexpr int kMergeHeads = 4;
-  // 128-token stages: three when three still fit next to a second CTA on the SM
   // RoPE: the inverse frequencies (64 fp64), each warp's (base angle, frequency) pairs (64 float2)
   // and the kv head's per-channel key scales (128 fp32)
   static constexpr int kRopeBytes = ROPE ? 64 * 8 + kCW * 64 * 8 + kHeadDim * 4 : 0;
-  static constexpr int kFixedBytes = 2048 + kCW * kMergeHeads * kHeadDim * 4 + kCW * 8 * 4 * 2 +
-                                     kCW * kMergeHeads * 4 * 4 + 8 * 144 * 4 + kRopeBytes + 1024;
-  // Dense KIVI: no producer warp. The consumer warps refill the stages themselves (the last warp
-  // to release a stage issues its next tile), so three CTAs of four warps fit on an SM at the
-  // same 168 registers a thread; the others keep a producer warp and two CTAs per SM.
+  // Shared memory of a CTA with `stages` tile stages and `mh` heads staged per pass of the
+  // per-pair warp merge (the layout below, plus 1 KB of alignment slack).
+  static constexpr int smem_for(int stages, int mh) {
+    return stages * kStageBytes + stages * 64 + 2 * stages * 8 + 64 + kCW * mh * kHeadDim * 4 + kCW * 8 * 4 * 2 +
+           kCW * mh * 4 * 4 + 8 * 144 * 4 + kRopeBytes + 1024;
+  }
+  static constexpr int kSmPerSm = 228 * 1024;  // shared memory of an SM (1 KB of it reserved per CTA)
+  static constexpr bool fits(int ctas, int stages, int mh) { return ctas * (smem_for(stages, mh) + 1024) <= kSmPerSm; }
+  // Dense KIVI: no producer warp. The consumer warps refill the stages themselves (the last
+  // warp to release a stage issues its next tile), so three CTAs of four warps fit on an SM at
+  // the same 168 registers a thread. The other kernels keep a producer warp and two CTAs per SM
+  // (three self-fed CTAs of two stages were slower for FP8 and INT4 per group).
   static constexpr bool kSelfFed = kKivi && !PAGED;
   static constexpr int kThreadsCta = kSelfFed ? kCW * 32 : (kCW + 1) * 32;
   static constexpr int kMinBlocks = kSelfFed ? 3 : 2;  // resident CTAs per SM the registers are sized for
-  static constexpr int kStages =
-      kSelfFed ? ((3 * (3 * kStageBytes + kFixedBytes + 1024) <= 227 * 1024) ? 3 : 2)
-               : ((3 * kStageBytes + kFixedBytes <= 112 * 1024) ? 3 : 2);
+  static constexpr int kStages = kSelfFed ? (fits(3, 3, 4) ? 3 : 2) : (fits(2, 3, 4) ? 3 : 2);
+  static constexpr int kMergeHeads = (kSelfFed && !fits(3, kStages, 4)) ? 2 : 4;
   static constexpr int kOffDesc = kStages * kStageBytes;
   static constexpr int kOffBar = kOffDesc + kStages * 64;
   static constexpr int kOffRedO = kOffBar + 2 * kStages * 8 + 64;
@@ -124,7 +127,8 @@ struct Cfg {
   static constexpr int kQStride = 144;          // q row stride (floats): see q_off
   static constexpr int kOffRope = kOffQ + 8 * kQStride * 4;  // 8-byte aligned
   static constexpr int kSmemBytes = kOffRope + kRopeBytes + 1024;  // + alignment slack
-  static_assert(kMinBlocks * (kSmemBytes + 1024) <= 227 * 1024, "the resident CTAs must fit in shared memory");
+  static_assert(kSmemBytes <= smem_for(kStages, kMergeHeads), "layout within its accounting");
+  static_assert(kMinBlocks * (kSmemBytes + 1024) <= kSmPerSm, "the resident CTAs must fit in shared memory");
 };
 
 struct TileDesc {
@@ -456,6 +460,19 @@ __device__ __forceinline__ int residual_row_shift(const uint8_t* row0, int n, in
 template <class T>
 __device__ __forceinline__ T lds(const uint8_t* p) {
   return *reinterpret_cast<const T*>(p);
+}
+
+// A shared-memory load the compiler keeps where it is written (loop-invariant values it would
+// otherwise hoist into registers for the whole loop).
+__device__ __forceinline__ float2 lds_here_f2(const void* p) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_addr(p)));
+  return v;
+}
+__device__ __forceinline__ float lds_here_f(const void* p) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_addr(p)));
+  return v;
 }
 
 // Four 8x8 matrices of 16-bit elements, transposed: lane 8m + r supplies the shared address of
@@ -867,36 +884,34 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
         cvt8x4<C::kKFmt>(wb0, S.zpk[4 + q][0], S.zpk[4 + q][1], h[1][0], h[1][1]);
         cvt8x4<C::kKFmt>(wa1, S.zpk[q][0], S.zpk[q][1], h[2][0], h[2][1]);
         cvt8x4<C::kKFmt>(wb1, S.zpk[4 + q][0], S.zpk[4 + q][1], h[3][0], h[3][1]);
-        uint32_t ahi[2][2][2], alo[2][2][2];  // [row][pair of the k-step slot h][...]: f16x2 (i, i + 64)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 16 * c + 4 * q + e;
-          const float2 bt = rw[i];
-          const float2 fa0 = f16x2_to_float2(h[0][e >> 1]), fb0 = f16x2_to_float2(h[1][e >> 1]);
-          const float2 fa1 = f16x2_to_float2(h[2][e >> 1]), fb1 = f16x2_to_float2(h[3][e >> 1]);
-          // key pair (x, y) = (channel i, channel i + 64) of rows g and g + 8
-          float x0 = (e & 1) ? fa0.y : fa0.x, y0 = (e & 1) ? fb0.y : fb0.x;
-          float x1 = (e & 1) ? fa1.y : fa1.x, y1 = (e & 1) ? fb1.y : fb1.x;
-          if constexpr (C::kKFold == FOLD_CHANNEL) {
-            const float sx = kch[i], sy = kch[i + 64];
-            x0 *= sx; x1 *= sx; y0 *= sy; y1 *= sy;
+        for (int kk = 0; kk < 2; ++kk) {  // k-step 2q + kk: pairs e = 2kk (slot 0) and 2kk + 1 (slot 1)
+          uint32_t ahi[2][2], alo[2][2];  // [row g / g + 8][slot]: f16x2 (channel i, channel i + 64)
+          const float2 fa0 = f16x2_to_float2(h[0][kk]), fb0 = f16x2_to_float2(h[1][kk]);
+          const float2 fa1 = f16x2_to_float2(h[2][kk]), fb1 = f16x2_to_float2(h[3][kk]);
+#pragma unroll
+          for (int hs = 0; hs < 2; ++hs) {
+            const int i = 16 * c + 4 * q + 2 * kk + hs;
+            const float2 bt = lds_here_f2(rw + i);
+            // key pair (x, y) = (channel i, channel i + 64) of rows g and g + 8
+            float x0 = hs ? fa0.y : fa0.x, y0 = hs ? fb0.y : fb0.x;
+            float x1 = hs ? fa1.y : fa1.x, y1 = hs ? fb1.y : fb1.x;
+            if constexpr (C::kKFold == FOLD_CHANNEL) {
+              const float sx = lds_here_f(kch + i), sy = lds_here_f(kch + i + 64);
+              x0 *= sx; x1 *= sx; y0 *= sy; y1 *= sy;
+            }
+            float sn0, cs0, sn1, cs1;
+            __sincosf(fmaf(j0, bt.y, bt.x), &sn0, &cs0);
+            __sincosf(fmaf(j1, bt.y, bt.x), &sn1, &cs1);
+            // (x, y) -> (x cos - y sin, y cos + x sin)
+            split_f16x2(fmaf(x0, cs0, -y0 * sn0), fmaf(y0, cs0, x0 * sn0), ahi[0][hs], alo[0][hs]);
+            split_f16x2(fmaf(x1, cs1, -y1 * sn1), fmaf(y1, cs1, x1 * sn1), ahi[1][hs], alo[1][hs]);
           }
-          float sn0, cs0, sn1, cs1;
-          __sincosf(fmaf(j0, bt.y, bt.x), &sn0, &cs0);
-          __sincosf(fmaf(j1, bt.y, bt.x), &sn1, &cs1);
-          // (x, y) -> (x cos - y sin, y cos + x sin)
-          const int ks_h = e & 1, kk = e >> 1;  // slot pair h and k-step 2q + kk of this pair
-          split_f16x2(fmaf(x0, cs0, -y0 * sn0), fmaf(y0, cs0, x0 * sn0), ahi[0][kk][ks_h], alo[0][kk][ks_h]);
-          split_f16x2(fmaf(x1, cs1, -y1 * sn1), fmaf(y1, cs1, x1 * sn1), ahi[1][kk][ks_h], alo[1][kk][ks_h]);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
           const int ks = 2 * q + kk;
           float(&acc_k)[4] = kk ? a1 : a0;
-          mma_16816(acc_k, ahi[0][kk][0], ahi[1][kk][0], ahi[0][kk][1], ahi[1][kk][1], S.qh[ks][0], S.qh[ks][1]);
-          mma_16816(acc_k, alo[0][kk][0], alo[1][kk][0], alo[0][kk][1], alo[1][kk][1], S.qh[ks][0], S.qh[ks][1]);
-          if (split)
-            mma_16816(acc_k, ahi[0][kk][0], ahi[1][kk][0], ahi[0][kk][1], ahi[1][kk][1], S.ql[ks][0], S.ql[ks][1]);
+          mma_16816(acc_k, ahi[0][0], ahi[1][0], ahi[0][1], ahi[1][1], S.qh[ks][0], S.qh[ks][1]);
+          mma_16816(acc_k, alo[0][0], alo[1][0], alo[0][1], alo[1][1], S.qh[ks][0], S.qh[ks][1]);
+          if (split) mma_16816(acc_k, ahi[0][0], ahi[1][0], ahi[0][1], ahi[1][1], S.ql[ks][0], S.ql[ks][1]);
         }
       }
     } else {
@@ -1518,6 +1533,13 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
     const int c0 = off / W, c1 = (off + n - 1) / W;
     for (int base = c0; base <= c1; base += 32) {
       const int cnt = min(32, c1 - base + 1);
+      const float4* po = reinterpret_cast<const float4*>(p.part_o) + ((size_t)(pair + base) * 8 + j) * (kHeadDim / 4) + lane;
+      // the first partials' rows are loaded together with the (m, l) pairs: one memory round trip
+      constexpr int kEarly = 4;
+      float4 early[kEarly];
+#pragma unroll
+      for (int i = 0; i < kEarly; ++i)
+        if (i < cnt) early[i] = po[(size_t)i * 8 * (kHeadDim / 4)];
       float mi = kNegInf, li = 0.0f;
       if (lane < cnt) {
         const size_t sl = (size_t)(pair + base + lane) * 8 + j;
@@ -1532,8 +1554,17 @@ __global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
       for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
       L = fmaf(L, f, lw);
       acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
-      const float4* po = reinterpret_cast<const float4*>(p.part_o) + ((size_t)(pair + base) * 8 + j) * (kHeadDim / 4) + lane;
-      for (int i = 0; i < cnt; ++i) {
+#pragma unroll
+      for (int i = 0; i < kEarly; ++i) {
+        const float a = __shfl_sync(0xffffffffu, ai, i);
+        if (i < cnt) {
+          acc.x = fmaf(a, early[i].x, acc.x);
+          acc.y = fmaf(a, early[i].y, acc.y);
+          acc.z = fmaf(a, early[i].z, acc.z);
+          acc.w = fmaf(a, early[i].w, acc.w);
+        }
+      }
+      for (int i = kEarly; i < cnt; ++i) {
         const float a = __shfl_sync(0xffffffffu, ai, i);
         const float4 o4 = po[(size_t)i * 8 * (kHeadDim / 4)];
         acc.x = fmaf(a, o4.x, acc.x);
