@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <utility>
@@ -230,11 +231,29 @@ struct TileIter {
 };
 
 // ------------------------------------------------------------------ TMA
-__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+// The cache is streamed once per decode: its tiles are copied with an L2 evict-first policy,
+// so they do not push out what is read again (the split partials, the queries).
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar,
+                                       uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s_ef(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                            uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
           dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
       : "memory");
 }
 
@@ -258,13 +277,14 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
                            uint32_t full0, int cur, TileDesc d) {
   const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
   const uint32_t bar = full0 + 8 * cur;
+  const uint64_t pol = l2_evict_first();
   const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
   if (d.kind == 1) {  // KIVI residual: bf16 rows, whole 32-token slab (inside rcap)
     const size_t r0 = (pair_row * p.rcap + d.t0) * kHeadDim;
     descs[cur] = d;
     mbar_arrive_expect_tx(bar, 2 * kRT * kHeadDim * 2);
-    bulk_g2s(sb, p.k_res + r0, kRT * kHeadDim * 2, bar);
-    bulk_g2s(sb + kRT * kHeadDim * 2, p.v_res + r0, kRT * kHeadDim * 2, bar);
+    bulk_g2s_ef(sb, p.k_res + r0, kRT * kHeadDim * 2, bar, pol);
+    bulk_g2s_ef(sb + kRT * kHeadDim * 2, p.v_res + r0, kRT * kHeadDim * 2, bar, pol);
     return;
   }
   if constexpr (!C::kPaged) {
@@ -273,8 +293,8 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
     const uint32_t bytes = C::kTS * (C::kKRow + C::kVRow) + C::kKMeta + C::kVMeta;
     descs[cur] = d;
     mbar_arrive_expect_tx(bar, bytes);
-    tma_2d(sb + C::kOffK, tk, 0, (int)row0, bar);
-    tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar);
+    tma_2d(sb + C::kOffK, tk, 0, (int)row0, bar, pol);
+    tma_2d(sb + C::kOffV, tv, 0, (int)row0, bar, pol);
     if constexpr (C::kKivi) {
       const size_t g0 = (pair_row * (p.cap / 32) + d.t0 / 32) * kHeadDim;
       // element offsets in bytes: fp32 or fp16 metadata
@@ -283,15 +303,15 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
       // key scales and minima as 128-byte rows through TMA with the 128-byte swizzle, so the query
       // build's reads (four lanes a 128-byte row apart) fall in distinct banks
       const int krow = (int)(g0 * C::kMetaElem / 128);
-      tma_2d(sb + C::kOffKM, tks, 0, krow, bar);
-      tma_2d(sb + C::kOffKM + C::kKMeta / 2, tkz, 0, krow, bar);
-      bulk_g2s(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
-      bulk_g2s(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar);
+      tma_2d(sb + C::kOffKM, tks, 0, krow, bar, pol);
+      tma_2d(sb + C::kOffKM + C::kKMeta / 2, tkz, 0, krow, bar, pol);
+      bulk_g2s_ef(sb + C::kOffVM, vs8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar, pol);
+      bulk_g2s_ef(sb + C::kOffVM + C::kVMeta / 2, vz8 + row0 * 4 * C::kMetaElem, C::kVMeta / 2, bar, pol);
     } else {
-      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar);
-      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar);
-      if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s(sb + C::kOffKM, p.k_scale + row0 * C::kNG, C::kKMeta, bar);
-      if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s(sb + C::kOffVM, p.v_scale + row0 * C::kNG, C::kVMeta, bar);
+      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s_ef(sb + C::kOffKM, p.k_scale + row0, C::kKMeta, bar, pol);
+      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s_ef(sb + C::kOffVM, p.v_scale + row0, C::kVMeta, bar, pol);
+      if constexpr (C::kKFold == FOLD_GROUP) bulk_g2s_ef(sb + C::kOffKM, p.k_scale + row0 * C::kNG, C::kKMeta, bar, pol);
+      if constexpr (C::kVFold == FOLD_GROUP) bulk_g2s_ef(sb + C::kOffVM, p.v_scale + row0 * C::kNG, C::kVMeta, bar, pol);
     }
   } else {
     // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
@@ -327,14 +347,14 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
     for (int i = 0; i < C::kTS / 16; ++i) {
       if (i >= npg || !((valid >> i) & 1u)) continue;
       const size_t prow = ((size_t)page[i] * p.Hkv + d.hk) * ps;
-      tma_2d(sb + C::kOffK + i * ps * C::kKRow, tk, 0, (int)prow, bar);
-      tma_2d(sb + C::kOffV + i * ps * C::kVRow, tv, 0, (int)prow, bar);
-      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar);
-      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar);
+      tma_2d(sb + C::kOffK + i * ps * C::kKRow, tk, 0, (int)prow, bar, pol);
+      tma_2d(sb + C::kOffV + i * ps * C::kVRow, tv, 0, (int)prow, bar, pol);
+      if constexpr (C::kKFold == FOLD_TOKEN) bulk_g2s_ef(sb + C::kOffKM + i * ps * 4, p.k_scale + prow, ps * 4, bar, pol);
+      if constexpr (C::kVFold == FOLD_TOKEN) bulk_g2s_ef(sb + C::kOffVM + i * ps * 4, p.v_scale + prow, ps * 4, bar, pol);
       if constexpr (C::kKFold == FOLD_GROUP)
-        bulk_g2s(sb + C::kOffKM + i * ps * C::kNG * 4, p.k_scale + prow * C::kNG, ps * C::kNG * 4, bar);
+        bulk_g2s_ef(sb + C::kOffKM + i * ps * C::kNG * 4, p.k_scale + prow * C::kNG, ps * C::kNG * 4, bar, pol);
       if constexpr (C::kVFold == FOLD_GROUP)
-        bulk_g2s(sb + C::kOffVM + i * ps * C::kNG * 4, p.v_scale + prow * C::kNG, ps * C::kNG * 4, bar);
+        bulk_g2s_ef(sb + C::kOffVM + i * ps * C::kNG * 4, p.v_scale + prow * C::kNG, ps * C::kNG * 4, bar, pol);
     }
   }
 }
@@ -1504,90 +1524,99 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
 }
 
 // ------------------------------------------------------------------ merge
-// One warp per (pair, query head): lanes read the partials' (m, l) in parallel and combine
+// One warp per query head (b, hq): lanes read the partials' (m, l) in parallel and combine
 // them with shuffles; each lane then accumulates a float4 of channels over the partials.
-// Grid (pairs, 2), four warps per block (heads 4 * blockIdx.y + warp).
-__global__ void __launch_bounds__(128) merge_kernel(const DecodeParams p) {
+// The grid is small (two CTAs of four warps an SM at most, each warp looping over query
+// heads): launched as the decode grid's programmatic dependent, its CTAs take the room the
+// decode CTAs leave on each SM (one next to two 8-bit decode CTAs, the rest as decode CTAs
+// retire) and wait in griddepcontrol.wait, so they start the moment the decode grid completes.
+constexpr int kMergeThreads = 128;
+
+__global__ void __launch_bounds__(kMergeThreads, 6) merge_kernel(const DecodeParams p) {
   grid_dependency_wait();  // the partials of the decode kernel
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pair = blockIdx.x, j = blockIdx.y * 4 + warp;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * (kMergeThreads / 32);
   const int per_seq = p.Hkv * p.HG;
-  const int b = pair / per_seq, hh = pair % per_seq, hk = hh / p.HG, hg = hh % p.HG;
-  const int hl = hg * 8 + j;
-  if (hl >= p.G) return;  // whole warp
-  const int hq = hk * p.G + hl;
-  int off, n, N;
-  if (p.paged) {
-    N = p.plan[p.B];
-    n = (p.plan[b + 1] - p.plan[b]) / per_seq;
-    off = p.plan[b] + hh * n;
-  } else {
-    n = p.nq + p.nr;
-    N = p.n_pairs * n;
-    off = pair * n;
-  }
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float M = kNegInf, L = 0.0f;
-  if (n > 0) {
-    const int W = (N + p.ncta - 1) / p.ncta;
-    const int c0 = off / W, c1 = (off + n - 1) / W;
-    for (int base = c0; base <= c1; base += 32) {
-      const int cnt = min(32, c1 - base + 1);
-      const float4* po = reinterpret_cast<const float4*>(p.part_o) + ((size_t)(pair + base) * 8 + j) * (kHeadDim / 4) + lane;
-      // the first partials' rows are loaded together with the (m, l) pairs: one memory round trip
-      constexpr int kEarly = 4;
-      float4 early[kEarly];
-#pragma unroll
-      for (int i = 0; i < kEarly; ++i)
-        if (i < cnt) early[i] = po[(size_t)i * 8 * (kHeadDim / 4)];
-      float mi = kNegInf, li = 0.0f;
-      if (lane < cnt) {
-        const size_t sl = (size_t)(pair + base + lane) * 8 + j;
-        mi = p.part_ml[sl * 2];
-        li = p.part_ml[sl * 2 + 1];
-      }
-      const float mc = warp_max(fmaxf(M, mi));
-      const float f = (M == kNegInf || mc == kNegInf) ? 0.0f : exp2f(M - mc);
-      const float ai = (mi == kNegInf || mc == kNegInf) ? 0.0f : exp2f(mi - mc);
-      float lw = ai * li;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-      L = fmaf(L, f, lw);
-      acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
-#pragma unroll
-      for (int i = 0; i < kEarly; ++i) {
-        const float a = __shfl_sync(0xffffffffu, ai, i);
-        if (i < cnt) {
-          acc.x = fmaf(a, early[i].x, acc.x);
-          acc.y = fmaf(a, early[i].y, acc.y);
-          acc.z = fmaf(a, early[i].z, acc.z);
-          acc.w = fmaf(a, early[i].w, acc.w);
-        }
-      }
-      for (int i = kEarly; i < cnt; ++i) {
-        const float a = __shfl_sync(0xffffffffu, ai, i);
-        const float4 o4 = po[(size_t)i * 8 * (kHeadDim / 4)];
-        acc.x = fmaf(a, o4.x, acc.x);
-        acc.y = fmaf(a, o4.y, acc.y);
-        acc.z = fmaf(a, o4.z, acc.z);
-        acc.w = fmaf(a, o4.w, acc.w);
-      }
-      M = mc;
+  for (int u = blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5); u < p.B * p.Hq; u += nwarps) {
+    const int b = u / p.Hq, hq = u - b * p.Hq;
+    const int hk = hq / p.G, hl = hq - hk * p.G;
+    const int hg = hl >> 3, j = hl & 7;
+    const int hh = hk * p.HG + hg;
+    const int pair = b * per_seq + hh;
+    int off, n, N;
+    if (p.paged) {
+      N = p.plan[p.B];
+      n = (p.plan[b + 1] - p.plan[b]) / per_seq;
+      off = p.plan[b] + hh * n;
+    } else {
+      n = p.nq + p.nr;
+      N = p.n_pairs * n;
+      off = pair * n;
     }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float M = kNegInf, L = 0.0f;
+    if (n > 0) {
+      const int W = (N + p.ncta - 1) / p.ncta;
+      const int c0 = off / W, c1 = (off + n - 1) / W;
+      for (int base = c0; base <= c1; base += 32) {
+        const int cnt = min(32, c1 - base + 1);
+        const float4* po =
+            reinterpret_cast<const float4*>(p.part_o) + ((size_t)(pair + base) * 8 + j) * (kHeadDim / 4) + lane;
+        // the first partials' rows are loaded together with the (m, l) pairs: one memory round trip
+        constexpr int kEarly = 2;
+        float4 early[kEarly];
+#pragma unroll
+        for (int i = 0; i < kEarly; ++i)
+          if (i < cnt) early[i] = po[(size_t)i * 8 * (kHeadDim / 4)];
+        float mi = kNegInf, li = 0.0f;
+        if (lane < cnt) {
+          const size_t sl = (size_t)(pair + base + lane) * 8 + j;
+          mi = p.part_ml[sl * 2];
+          li = p.part_ml[sl * 2 + 1];
+        }
+        const float mc = warp_max(fmaxf(M, mi));
+        const float f = (M == kNegInf || mc == kNegInf) ? 0.0f : exp2f(M - mc);
+        const float ai = (mi == kNegInf || mc == kNegInf) ? 0.0f : exp2f(mi - mc);
+        float lw = ai * li;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+        L = fmaf(L, f, lw);
+        acc.x *= f; acc.y *= f; acc.z *= f; acc.w *= f;
+#pragma unroll
+        for (int i = 0; i < kEarly; ++i) {
+          const float a = __shfl_sync(0xffffffffu, ai, i);
+          if (i < cnt) {
+            acc.x = fmaf(a, early[i].x, acc.x);
+            acc.y = fmaf(a, early[i].y, acc.y);
+            acc.z = fmaf(a, early[i].z, acc.z);
+            acc.w = fmaf(a, early[i].w, acc.w);
+          }
+        }
+        for (int i = kEarly; i < cnt; ++i) {
+          const float a = __shfl_sync(0xffffffffu, ai, i);
+          const float4 o4 = po[(size_t)i * 8 * (kHeadDim / 4)];
+          acc.x = fmaf(a, o4.x, acc.x);
+          acc.y = fmaf(a, o4.y, acc.y);
+          acc.z = fmaf(a, o4.z, acc.z);
+          acc.w = fmaf(a, o4.w, acc.w);
+        }
+        M = mc;
+      }
+    }
+    float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lse = kNegInf;
+    if (M != kNegInf && L > 0.0f) {
+      ov = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+      lse = (M + log2f(L)) * 0.69314718055994531f;
+    }
+    if (p.rotate) {  // sum p (H v) = H (sum p v): rotate the output back
+      float r[4] = {ov.x, ov.y, ov.z, ov.w};
+      fwht_row32(r, lane);
+      ov = make_float4(r[0], r[1], r[2], r[3]);
+    }
+    reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + hq) * kHeadDim)[lane] = ov;
+    if (lane == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
   }
-  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lse = kNegInf;
-  if (M != kNegInf && L > 0.0f) {
-    ov = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-    lse = (M + log2f(L)) * 0.69314718055994531f;
-  }
-  if (p.rotate) {  // sum p (H v) = H (sum p v): rotate the output back
-    float r[4] = {ov.x, ov.y, ov.z, ov.w};
-    fwht_row32(r, lane);
-    ov = make_float4(r[0], r[1], r[2], r[3]);
-  }
-  reinterpret_cast<float4*>(p.out + ((size_t)b * p.Hq + hq) * kHeadDim)[lane] = ov;
-  if (lane == 0 && p.lse) p.lse[(size_t)b * p.Hq + hq] = lse;
 }
 
 // ------------------------------------------------------------------ paged plan
@@ -1817,7 +1846,11 @@ cudaError_t launch_decode(DecodeParams p, cudaStream_t st) {
     if (dev < kMaxDevices) occ_cache[vi][dev].store(0, std::memory_order_relaxed);  // set up again next call
     return e;
   }
-  e = launch_pdl(merge_kernel, dim3(p.n_pairs, 2), dim3(128), 0, st, p);
+  // merge: two CTAs an SM at most, fewer when there are fewer query heads than warps
+  const long long heads = (long long)p.B * p.Hq;
+  const int mgrid =
+      (int)std::min<long long>(2LL * sm_count(), (heads + kMergeThreads / 32 - 1) / (kMergeThreads / 32));
+  e = launch_pdl(merge_kernel, dim3(mgrid > 0 ? mgrid : 1), dim3(kMergeThreads), 0, st, p);
   if (e != cudaSuccess) return e;
   count_launches(p.paged ? 3 : 2);
   return cudaGetLastError();
