@@ -114,6 +114,10 @@ struct Cfg {
   // the same 168 registers a thread. The other kernels keep a producer warp and two CTAs per SM
   // (three self-fed CTAs of two stages were slower for FP8 and INT4 per group).
   static constexpr bool kSelfFed = kKivi && !PAGED;
+  // 8-bit keys: a pair's query loads are issued before the wait for its first tile (and the
+  // queries are prefetched toward L2 when that tile is issued); measured slower for KIVI and
+  // INT4 per group, whose pair start is cheaper than the registers the overlap costs them
+  static constexpr bool kEarlyPairStart = !kKivi && kKFold != FOLD_GROUP;
   static constexpr int kThreadsCta = kSelfFed ? kCW * 32 : (kCW + 1) * 32;
   static constexpr int kMinBlocks = kSelfFed ? 3 : 2;  // resident CTAs per SM the registers are sized for
   static constexpr int kStages = kSelfFed ? (fits(3, 3, 4) ? 3 : 2) : (fits(2, 3, 4) ? 3 : 2);
@@ -248,6 +252,10 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int
       : "memory");
 }
 
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s_ef(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
                                             uint64_t pol) {
   asm volatile(
@@ -278,6 +286,12 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
   const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
   const uint32_t bar = full0 + 8 * cur;
   const uint64_t pol = l2_evict_first();
+  if (C::kEarlyPairStart && d.first) {  // the pair's queries toward L2, a few tiles before they are loaded
+    const int h0 = d.hg * 8, nh = min(8, p.G - h0);
+    const size_t es = p.q_bf16 ? 2 : 4;
+    const uint8_t* qrow = static_cast<const uint8_t*>(p.q) + ((size_t)d.b * p.Hq + (size_t)d.hk * p.G + h0) * kHeadDim * es;
+    if ((reinterpret_cast<uintptr_t>(qrow) & 15) == 0) bulk_prefetch_l2(qrow, (uint32_t)(nh * kHeadDim * es));
+  }
   const size_t pair_row = (size_t)d.b * p.Hkv + d.hk;
   if (d.kind == 1) {  // KIVI residual: bf16 rows, whole 32-token slab (inside rcap)
     const size_t r0 = (pair_row * p.rcap + d.t0) * kHeadDim;
@@ -1314,9 +1328,9 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
   ti.init(p, sc, tb, te);
   for (int st = 0, phase = 0; ti.t < te; ti.next(p, sc)) {
     const TileDesc d = ti.desc(p, sc);
-    if (!dead && !mbar_wait(full0 + 8 * st, phase, p.status)) dead = true;
-    const uint8_t* base = smem + st * C::kStageBytes;
-    const uint32_t valid = C::kPaged ? descs[st].valid : 0xFFFFFFFFu;
+    if constexpr (!C::kEarlyPairStart) {
+      if (!dead && !mbar_wait(full0 + 8 * st, phase, p.status)) dead = true;
+    }
 
     // ------------------------------------------------ pair start
     if (d.first) {
@@ -1411,6 +1425,11 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
     }
 
     // ------------------------------------------------ tile work
+    if constexpr (C::kEarlyPairStart) {  // the pair start above overlapped the tile's arrival
+      if (!dead && !mbar_wait(full0 + 8 * st, phase, p.status)) dead = true;
+    }
+    const uint8_t* base = smem + st * C::kStageBytes;
+    const uint32_t valid = C::kPaged ? descs[st].valid : 0xFFFFFFFFu;
     const bool residual = C::kKivi && d.kind == 1;
     const int tok_base = residual ? 0 : w * C::kTPW;
     const bool busy = !dead && (residual ? (w == 0) : true) && (d.n - tok_base > 0);
@@ -1473,10 +1492,13 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
           S.zacc[j] += __shfl_xor_sync(0xffffffffu, S.zacc[j], 2);
         }
       }
-      // O is staged and merged kMergeHeads heads at a time (lanes hold heads 2c, 2c + 1)
+      // O is staged and merged kMergeHeads heads at a time (lanes hold heads 2c, 2c + 1); the
+      // group's padding heads (G < 8) are neither merged nor written
       constexpr int kMH = C::kMergeHeads;
+      const int nh = min(8, p.G - d.hg * 8);
 #pragma unroll
       for (int half = 0; half < 8 / kMH; ++half) {
+        if (kMH * half >= nh) break;  // uniform over the CTA
         if ((2 * c) / kMH == half) {
 #pragma unroll
           for (int mt = 0; mt < 8; ++mt)
@@ -1496,7 +1518,7 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
         }
         named_sync(1, kCW * 32);
 #pragma unroll 1
-        for (int j = kMH * half; j < kMH * half + kMH; ++j) {
+        for (int j = kMH * half; j < kMH * half + kMH && j < nh; ++j) {
           float M = kNegInf;
 #pragma unroll
           for (int ww = 0; ww < kCW; ++ww) M = fmaxf(M, red_m[ww * 8 + j]);
