@@ -1597,8 +1597,8 @@ __global__ void __launch_bounds__(kMergeThreads, 6) merge_kernel(const DecodePar
           li = p.part_ml[sl * 2 + 1];
         }
         const float mc = warp_max(fmaxf(M, mi));
-        const float f = (M == kNegInf || mc == kNegInf) ? 0.0f : exp2f(M - mc);
-        const float ai = (mi == kNegInf || mc == kNegInf) ? 0.0f : exp2f(mi - mc);
+        const float f = (M == kNegInf || mc == kNegInf) ? 0.0f : fast_exp2(M - mc);
+        const float ai = (mi == kNegInf || mc == kNegInf) ? 0.0f : fast_exp2(mi - mc);
         float lw = ai * li;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
@@ -1628,8 +1628,13 @@ __global__ void __launch_bounds__(kMergeThreads, 6) merge_kernel(const DecodePar
     float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
     float lse = kNegInf;
     if (M != kNegInf && L > 0.0f) {
-      ov = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
-      lse = (M + log2f(L)) * 0.69314718055994531f;
+      // one reciprocal and the hardware log2: the merge is on the call's critical path, and
+      // both stay far inside the attention tolerance
+      const float inv = __frcp_rn(L);
+      ov = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      float lg;
+      asm("lg2.approx.f32 %0, %1;" : "=f"(lg) : "f"(L));
+      lse = (M + lg) * 0.69314718055994531f;
     }
     if (p.rotate) {  // sum p (H v) = H (sum p v): rotate the output back
       float r[4] = {ov.x, ov.y, ov.z, ov.w};
