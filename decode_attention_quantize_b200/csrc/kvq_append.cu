@@ -398,16 +398,21 @@ __device__ __forceinline__ uint32_t int4_codes(const float (&x)[8], float s) {
   if (quot_range(s)) {
     const float y = __frcp_rn(s);
     const f32x2 y2 = pk2(y, y), ns2 = pk2(-s, -s), m2 = pk2(kRoundMagic, kRoundMagic);
+    uint32_t t[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const f32x2 x2 = pk2(x[2 * k], x[2 * k + 1]);
       const f32x2 q = mul2(x2, y2);
-      const f32x2 t = add2(fma2(fma2(q, ns2, x2), y2, q), m2);  // RN(q - e y) + magic
+      const f32x2 r = add2(fma2(fma2(q, ns2, x2), y2, q), m2);  // RN(q - e y) + magic
       float t0, t1;
-      upk2(t, t0, t1);
-      w |= ((__float_as_uint(t0) & 0xFu) << (8 * k)) | ((__float_as_uint(t1) & 0xFu) << (8 * k + 4));
+      upk2(r, t0, t1);
+      t[2 * k] = __float_as_uint(t0);
+      t[2 * k + 1] = __float_as_uint(t1);
     }
-    return w;
+    // byte k = (nibble of channel 2k, nibble of channel 2k + 1): the low bytes of the even and
+    // of the odd channels gathered by byte permutes, then one shift and one masked merge
+    const uint32_t ev = pack_low_bytes(t[0], t[2], t[4], t[6]), od = pack_low_bytes(t[1], t[3], t[5], t[7]);
+    return (ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u);
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -689,16 +694,62 @@ __global__ void __launch_bounds__(256) requant_kernel(AppendParams p, RescaleWs 
     if (sn[k] == so[k] && zn[k] == zo[k]) keep |= 1u << k;
     if (quot_range(sn[k]) && quot_range(so[k])) fast |= 1u << k;
   }
+  // FP8 per-tensor with both scales in the quotient's range: two codes per packed operation
+  constexpr bool kFp8 = SCHEME == KVQ_FP8_E4M3_PER_TENSOR || SCHEME == KVQ_FP8_E5M2_PER_TENSOR;
+  const bool packed = kFp8 && keep == 0u && fast == 0xFFFFu;
+  // (the residual is formed as q s - x and subtracted, as in quot, so a zero keeps its sign)
+  const f32x2 so2 = pk2(so[0], so[0]), nso2 = pk2(-so[0], -so[0]), sn2 = pk2(sn[0], sn[0]);
+  const f32x2 y2 = pk2(yn[0], yn[0]), ny2 = pk2(-yn[0], -yn[0]);
   const int span = p.paged ? p.max_pages * p.page_size : p.pos0;
   const long long rows = (long long)p.B * span;
+  const bool rows32 = rows < (1LL << 31);  // row index and its (sequence, position) in 32 bits
   for (long long r = (long long)blockIdx.x * 32 + (threadIdx.x >> 3); r < rows; r += (long long)gridDim.x * 32) {
-    const int b = (int)(r / span), pos = (int)(r % span);
+    int b, pos;
+    if (rows32) {
+      b = (int)((unsigned)r / (unsigned)span);
+      pos = (int)r - b * span;
+    } else {
+      b = (int)(r / span);
+      pos = (int)(r % span);
+    }
     if (p.paged && pos >= p.seq_lens[b]) continue;
     size_t row;
     if (!cache_row(p, b, h, pos, row)) continue;
     uint4* ptr = reinterpret_cast<uint4*>(codes + row * kHeadDim + lane8 * 16);
     const uint4 in = *ptr;
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    if constexpr (kFp8) {
+      if (packed) {  // per code the same operations as below: x = v * s_old, z = x / s_new, RN code
+        uint32_t o2[4];
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          uint32_t half_codes[2];
+#pragma unroll
+          for (int hp = 0; hp < 2; ++hp) {
+            uint32_t h2;  // the two codes' values as f16x2 (exact), lower code in the low half
+            if constexpr (SCHEME == KVQ_FP8_E4M3_PER_TENSOR) {
+              asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(w[wi] >> (16 * hp))));
+            } else {
+              h2 = prmt(w[wi], 0u, hp ? 0x3424u : 0x1404u);
+            }
+            float v0, v1;
+            asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n cvt.f32.f16 %0, l;\n cvt.f32.f16 %1, h;\n}\n"
+                : "=f"(v0), "=f"(v1)
+                : "r"(h2));
+            const f32x2 v2 = pk2(v0, v1);
+            const f32x2 x2 = mul2(v2, so2), nx2 = mul2(v2, nso2);  // x and -x, both exact negations
+            const f32x2 q2 = mul2(x2, y2);
+            const f32x2 z2 = fma2(fma2(q2, sn2, nx2), ny2, q2);  // q - RN(q s - x) y
+            float z0, z1;
+            upk2(z2, z0, z1);
+            half_codes[hp] = SCHEME == KVQ_FP8_E4M3_PER_TENSOR ? e4m3x2_rn(z0, z1) : e5m2x2_rn(z0, z1);
+          }
+          o2[wi] = half_codes[0] | (half_codes[1] << 16);
+        }
+        *ptr = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        continue;
+      }
+    }
     uint32_t o[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
