@@ -224,11 +224,13 @@ __device__ __forceinline__ void fwht_row16(float (&x)[8], unsigned mask, int lan
       }
 #pragma unroll
   for (int m = 1; m < 16; m <<= 1) {
-    const bool upper = (lane16 & m) != 0;
+    // upper lane: partner - own; lower lane: own + partner; one fma with the sign (exact:
+    // fma(-1, x, y) rounds y - x and fma(1, x, y) rounds x + y)
+    const float sg = (lane16 & m) ? -1.0f : 1.0f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float y = __shfl_xor_sync(mask, x[k], m);
-      x[k] = upper ? y - x[k] : x[k] + y;
+      x[k] = __fmaf_rn(sg, x[k], y);
     }
   }
 #pragma unroll
