@@ -406,15 +406,18 @@ class GpuWorkload:
                       for b in range(W.B)])
         return self._dev(k, True), self._dev(v, True)
 
-    # one step (eager): append + decode
+    # one step (eager): append + decode, through the library's one-call step (the decode of a
+    # dense 8-bit / INT4 cache then reads the cached tiles while the append runs)
     def step(self, stream=None, k_new=None, v_new=None, q=None):
         d = self.cache.desc
+        q = self.q if q is None else q
         if self.append_token:
             if not self.w.paged:
                 d.num_quantized, d.num_residual = self.saved
-            self.cache.append(self.k_new if k_new is None else k_new, self.v_new if v_new is None else v_new,
-                              stream=stream)
-        self.cache.decode(self.q if q is None else q, self.scale, out=self.out, workspace=self.ws, stream=stream)
+            self.cache.append_decode(self.k_new if k_new is None else k_new, self.v_new if v_new is None else v_new,
+                                     q, self.scale, out=self.out, workspace=self.ws, stream=stream)
+        else:
+            self.cache.decode(q, self.scale, out=self.out, workspace=self.ws, stream=stream)
 
     def decode_lens(self, appended):
         """(per-sequence quantized tokens, residual tokens) seen by a decode. Dense: every step

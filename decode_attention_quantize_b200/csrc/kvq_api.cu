@@ -321,8 +321,14 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* d) {
          round_up((2 * (size_t)d->batch + 2) * sizeof(int32_t));
 }
 
-kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t q_dtype, float softmax_scale,
-                                float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// The decode call; early_from >= 0 when the previous launch on the stream is this library's
+// plain append writing positions from early_from on (see DecodeParams::early_from); with
+// check_only, the argument checks alone.
+kvq_status decode_impl(const kvq_cache_desc* d, const void* q, int32_t q_dtype, float softmax_scale, float* out,
+                       float* lse, void* workspace, size_t workspace_bytes, void* stream, int early_from,
+                       bool check_only) {
   kvq_status st = kvq_validate(d);
   if (st != KVQ_OK) return st;
   if (!q || !out || !aligned16(out) || (q_dtype != KVQ_F32 && q_dtype != KVQ_BF16)) return KVQ_ERR_INVALID_ARG;
@@ -332,6 +338,7 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   const bool paged = d->layout == KVQ_PAGED;
   const bool rope = d->rope_theta > 0.0f;
   if (!decode_supported(d->k_scheme, d->v_scheme, paged, d->group_size, rope)) return KVQ_ERR_UNSUPPORTED;
+  if (check_only) return KVQ_OK;
   const int G = d->num_q_heads / d->num_kv_heads;
   DecodeParams p;
   std::memset(&p, 0, sizeof(p));
@@ -379,7 +386,47 @@ kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t 
   p.part_ml = reinterpret_cast<float*>(ws);
   ws += round_up(slots * 8 * 2 * sizeof(float));
   p.plan = reinterpret_cast<int32_t*>(ws);
+  p.early_from = early_from;
   return from_cuda(launch_decode(p, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+kvq_status kvq_decode_attention(const kvq_cache_desc* d, const void* q, int32_t q_dtype, float softmax_scale,
+                                float* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(d, q, q_dtype, softmax_scale, out, lse, workspace, workspace_bytes, stream, -1, false);
+}
+
+kvq_status kvq_append_decode(kvq_cache_desc* d, const void* k_new, const void* v_new, int32_t in_dtype,
+                             int32_t n_new, const void* q, int32_t q_dtype, float softmax_scale, float* out,
+                             float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  // every check of both calls before anything is launched
+  kvq_status st = decode_impl(d, q, q_dtype, softmax_scale, out, lse, workspace, workspace_bytes, stream, -1, true);
+  if (st != KVQ_OK) return st;
+  if (in_dtype != KVQ_F32 && in_dtype != KVQ_BF16) return KVQ_ERR_INVALID_ARG;
+  if (n_new < 0) return KVQ_ERR_INVALID_ARG;
+  const bool kivi = is_kivi(d->k_scheme);
+  if (n_new > 0) {
+    if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return KVQ_ERR_INVALID_ARG;
+    if (!append_pair_supported(d->k_scheme, d->v_scheme) || (kivi && in_dtype != KVQ_BF16)) return KVQ_ERR_UNSUPPORTED;
+    if (d->layout == KVQ_PAGED) {
+      if (n_new > seq_capacity(d)) return KVQ_ERR_CAPACITY;
+    } else if (kivi) {
+      const int total = d->num_residual + n_new;
+      const int flushed = total - ((total - 1) % d->residual_cap + 1);
+      if ((int64_t)d->num_quantized + flushed > d->capacity) return KVQ_ERR_CAPACITY;
+    } else if ((int64_t)d->num_quantized + n_new > d->capacity) {
+      return KVQ_ERR_CAPACITY;
+    }
+  }
+  // the decode overlaps the append when the append is one launch of the 8-bit / INT4 rows kernel
+  // on a dense cache (it then writes the new positions and nothing else the decode reads)
+  const bool overlap = n_new > 0 && d->layout == KVQ_DENSE && !kivi;
+  const int pos0 = d->num_quantized;
+  st = kvq_quantize_append(d, k_new, v_new, in_dtype, n_new, nullptr, 0u, nullptr, 0, stream);
+  if (st != KVQ_OK) return st;
+  return decode_impl(d, q, q_dtype, softmax_scale, out, lse, workspace, workspace_bytes, stream,
+                     overlap ? pos0 : -1, false);
 }
 
 kvq_status kvq_check_bounded_wait(uint32_t* dev_status, void* stream) {

@@ -118,6 +118,9 @@ struct Cfg {
   // queries are prefetched toward L2 when that tile is issued); measured slower for KIVI and
   // INT4 per group, whose pair start is cheaper than the registers the overlap costs them
   static constexpr bool kEarlyPairStart = !kKivi && kKFold != FOLD_GROUP;
+  // may start while the one-token append of the same step runs (dense, producer warp, codes and
+  // their per-token / per-group scales all reach the consumers through the stages)
+  static constexpr bool kOverlapAppend = !PAGED && !kSelfFed;
   static constexpr int kThreadsCta = kSelfFed ? kCW * 32 : (kCW + 1) * 32;
   static constexpr int kMinBlocks = kSelfFed ? 3 : 2;  // resident CTAs per SM the registers are sized for
   static constexpr int kStages = kSelfFed ? (fits(3, 3, 4) ? 3 : 2) : (fits(2, 3, 4) ? 3 : 2);
@@ -381,9 +384,14 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
                          uint32_t full0, uint32_t empty0, const Sched& s, int tb, int te) {
   TileIter ti;
   ti.init(p, s, tb, te);
+  bool waited = !C::kOverlapAppend || p.early_from < 0;
   for (int it = 0, st = 0, phase = 0; ti.t < te; ti.next(p, s), ++it) {
     if (it >= C::kStages && !mbar_wait(empty0 + 8 * st, phase ^ 1, p.status)) return;
     const TileDesc d = ti.desc(p, s);
+    if (!waited && d.t0 + p.ts > p.early_from) {  // this tile holds positions the append writes
+      grid_dependency_wait();
+      waited = true;
+    }
     const int cur = st;
     if (++st == C::kStages) {
       st = 0;
@@ -1271,7 +1279,9 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
   using C = Cfg<KS, VS, PAGED, NG, ROPE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-  grid_dependency_wait();    // the cache, the queries and the plan come from earlier kernels
+  // the cache, the queries and the plan come from earlier kernels (after an overlapped append,
+  // only the tiles it writes: the producer waits before the first of them)
+  if (!C::kOverlapAppend || p.early_from < 0) grid_dependency_wait();
   grid_launch_dependents();  // the merge may be scheduled now; it waits for this grid to finish
   const Sched sc = make_sched(p);
   const int tb = blockIdx.x * sc.W;

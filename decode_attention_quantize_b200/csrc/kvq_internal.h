@@ -87,6 +87,10 @@ struct DecodeParams {
   int rotate;                   // rotate each query, and each output back
   int group;                    // INT4 per-group: channels per group (selects the kernel)
   float rope_theta;             // > 0: keys cached before RoPE, rotated at their positions here
+  // >= 0: the kernel runs as the programmatic dependent of an append that writes token
+  // positions from here on (and nothing else the decode reads): tiles before it are read
+  // before the wait for that append, the others after it. < 0: wait at the start.
+  int early_from;
 };
 
 constexpr int kMaxCtas = 1024;

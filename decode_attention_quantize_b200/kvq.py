@@ -42,7 +42,7 @@ EXPORTS = [
     "kvq_abi_version", "kvq_status_string", "kvq_validate", "kvq_cache_bytes",
     "kvq_append_workspace_bytes", "kvq_quantize_append", "kvq_dequantize",
     "kvq_decode_workspace_bytes", "kvq_decode_attention", "kvq_get_device_status", "kvq_launch_count",
-    "kvq_decode_attention_noalloc", "kvq_check_bounded_wait",
+    "kvq_decode_attention_noalloc", "kvq_check_bounded_wait", "kvq_append_decode",
 ]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -93,12 +93,13 @@ def _load():
     L.kvq_decode_attention.argtypes = [P, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.kvq_get_device_status.argtypes = [P, vp, i32, vp]
     L.kvq_launch_count.restype = ctypes.c_uint64
+    L.kvq_append_decode.argtypes = [P, vp, vp, i32, i32, vp, i32, ctypes.c_float, vp, vp, vp, sz, vp]
     L.kvq_decode_attention_noalloc.argtypes = [P, vp, i32, ctypes.c_float, vp, vp, vp]
     L.kvq_decode_attention_noalloc.restype = ctypes.c_int
     L.kvq_check_bounded_wait.argtypes = [vp, vp]
     L.kvq_check_bounded_wait.restype = ctypes.c_int
     for name in ("kvq_validate", "kvq_cache_bytes", "kvq_quantize_append", "kvq_dequantize",
-                 "kvq_decode_attention", "kvq_get_device_status"):
+                 "kvq_decode_attention", "kvq_get_device_status", "kvq_append_decode"):
         getattr(L, name).restype = ctypes.c_int
     return L
 
@@ -231,6 +232,29 @@ def kvq_decode_attention(desc: KvqDesc, q, softmax_scale: float, out=None, lse=N
                                     _ptr(out), _ptr(lse), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
            "kvq_decode_attention")
+    return out, lse
+
+
+def kvq_append_decode(desc: KvqDesc, k_new, v_new, q, softmax_scale: float, out=None, lse=None, workspace=None,
+                      stream=None):
+    """One decode step: a plain append of k_new / v_new [B, Hkv, n, D], then decode attention of
+    q [B, Hq, D] over the updated cache; returns (out, lse)."""
+    _need(k_new is not None and v_new is not None and k_new.dim() == 4, "k_new, v_new: [B, Hkv, n, D] tensors")
+    n = int(k_new.shape[2])
+    _check_shape(k_new, (desc.batch, desc.num_kv_heads, n, desc.head_dim), "k_new")
+    _check_shape(v_new, (desc.batch, desc.num_kv_heads, n, desc.head_dim), "v_new")
+    _need(k_new.dtype == v_new.dtype, f"k_new and v_new dtypes differ ({k_new.dtype}, {v_new.dtype})")
+    _need(q is not None and q.dim() == 3, "q: [B, Hq, D] tensor")
+    if out is None:
+        out = torch.empty(tuple(q.shape), dtype=torch.float32, device=q.device)
+    _check_decode_args(desc, q, out, lse)
+    if workspace is None:
+        workspace = decode_workspace(desc, q.device)
+    _check_device([("k_new", k_new), ("v_new", v_new), ("workspace", workspace)], q.device)
+    _check(lib.kvq_append_decode(ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), n, _ptr(q),
+                                 _dtype_code(q), float(softmax_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "kvq_append_decode")
     return out, lse
 
 
@@ -399,6 +423,20 @@ class QuantizedKVCache:
             workspace = self._decode_ws
         return kvq_decode_attention(self.desc, q, softmax_scale, out=out, lse=lse, workspace=workspace,
                                     stream=stream)
+
+    def append_decode(self, k, v, q, softmax_scale=None, out=None, lse=None, workspace=None, stream=None):
+        """One decode step: append k, v with the cache's scales as they are, then decode q. The
+        decode of a dense 8-bit or INT4 cache starts reading the cached tiles while the append
+        runs. Not with a rescaling schedule (use append, then decode)."""
+        _need(self.schedule is None, "append_decode: the cache has a rescaling schedule")
+        if softmax_scale is None:
+            softmax_scale = 1.0 / math.sqrt(self.spec.D)
+        if workspace is None:
+            if self._decode_ws is None:
+                self._decode_ws = decode_workspace(self.desc, self.device)
+            workspace = self._decode_ws
+        return kvq_append_decode(self.desc, k, v, q, softmax_scale, out=out, lse=lse, workspace=workspace,
+                                 stream=stream)
 
     def status(self, clear=False):
         return kvq_get_device_status(self.desc, clear=clear)

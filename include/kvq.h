@@ -245,6 +245,25 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_cache_desc* desc, const void* 
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * One decode step in one call: kvq_quantize_append(desc, k_new, v_new, in_dtype, n_new,
+ * NULL, 0, ...) (a plain append: the cache's scales as they are), then
+ * kvq_decode_attention(desc, q, ...) over the updated cache, on `stream`, with the same
+ * arguments, layouts, results and errors as those two calls. Every check of both runs before
+ * anything is launched. "KV Cache Quantization" (infra.bea.ai), §4 FP8 KV cache: the cache is
+ * appended to and read back at every decode step; this call overlaps the two.
+ *   workspace  decode workspace (kvq_decode_workspace_bytes; a plain append needs none)
+ * On a dense cache with 8-bit or INT4-per-group schemes (not KIVI) the decode kernel is
+ * launched as the programmatic dependent of the append and reads the cached tiles that hold
+ * no new position while the append runs; it waits for the append before the tiles that do.
+ * Otherwise the two run one after the other. Not for a cache whose scales must grow with the
+ * block (KVQ_APPEND_RESCALE) or be calibrated from it: call the two entry points.
+ */
+KVQ_API kvq_status kvq_append_decode(kvq_cache_desc* desc, const void* k_new, const void* v_new, int32_t in_dtype,
+                                     int32_t n_new, const void* q, int32_t q_dtype, float softmax_scale,
+                                     float* out, float* lse, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/*
  * Test support; the pages have no counterpart. Launches one warp that waits on a
  * shared-memory barrier nothing ever arrives at, through the same bounded wait every kernel
  * of the library uses for its copy barriers. After about one second the wait gives up, sets

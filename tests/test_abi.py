@@ -263,3 +263,32 @@ def test_prerope_validation():
     need = L.kvq_decode_workspace_bytes(ctypes.byref(d))
     assert L.kvq_decode_attention(ctypes.byref(d), buf, 1, ctypes.c_float(0.088), buf, None, buf, need,
                                   None) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_append_decode_checks_both_calls_before_launch():
+    # every check of the append and of the decode runs before anything is launched: a failing
+    # decode argument leaves the descriptor's length unchanged (no append happened)
+    from decode_attention_quantize_b200 import kvq
+    L = kvq.lib
+    buf = 0x20000
+    d = _desc(num_quantized=100)
+    need = L.kvq_decode_workspace_bytes(ctypes.byref(d))
+
+    def call(n_new=1, q_dtype=1, scale=0.088, out=buf, ws_bytes=None, in_dtype=kvq.KVQ_BF16, k=buf):
+        return L.kvq_append_decode(ctypes.byref(d), k, buf, in_dtype, n_new, buf, q_dtype, ctypes.c_float(scale),
+                                   out, None, buf, need if ws_bytes is None else ws_bytes, None)
+
+    assert call(ws_bytes=need - 1) == kvq.KVQ_ERR_WORKSPACE
+    assert call(q_dtype=7) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(scale=-1.0) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(out=buf + 4) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(n_new=-1) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(in_dtype=5) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(k=buf + 2) == kvq.KVQ_ERR_INVALID_ARG  # misaligned new keys
+    assert call(n_new=157) == kvq.KVQ_ERR_CAPACITY      # 100 + 157 > 256
+    assert d.num_quantized == 100
+    # KIVI appends take bf16 only
+    d3 = _desc(k_scheme=5, v_scheme=5, k_zero=buf, v_zero=buf, k_res=buf, v_res=buf)
+    need3 = L.kvq_decode_workspace_bytes(ctypes.byref(d3))
+    assert L.kvq_append_decode(ctypes.byref(d3), buf, buf, kvq.KVQ_F32, 1, buf, 1, ctypes.c_float(0.088), buf,
+                               None, buf, need3, None) == kvq.KVQ_ERR_UNSUPPORTED
