@@ -285,7 +285,7 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 template <class C>
 __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
                            const CUtensorMap* tks, const CUtensorMap* tkz, uint8_t* stages, TileDesc* descs,
-                           uint32_t full0, int cur, TileDesc d) {
+                           uint32_t full0, int cur, TileDesc d, const int (&pages)[C::kTS / 16]) {
   const uint32_t sb = smem_addr(stages + cur * C::kStageBytes);
   const uint32_t bar = full0 + 8 * cur;
   const uint64_t pol = l2_evict_first();
@@ -334,15 +334,13 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
     // paged: page i of the tile -> rows (page * Hkv + hk) * page_size of the pool
     const int ps = p.page_size;
     const int npg = (d.n + ps - 1) / ps;
-    const int pi0 = d.t0 / ps;
     int page[C::kTS / 16];
     uint32_t valid = 0, nvalid = 0;
 #pragma unroll
     for (int i = 0; i < C::kTS / 16; ++i) {
       page[i] = -1;
       if (i < npg) {
-        const int pi = pi0 + i;
-        const int id = pi < p.max_pages ? p.page_table[(size_t)d.b * p.max_pages + pi] : -1;
+        const int id = pages[i];  // read from the page table one tile ahead (load_tile_pages)
         page[i] = id;
         if (id >= 0 && id < p.num_pages) {
           valid |= 1u << i;
@@ -376,6 +374,20 @@ __device__ void issue_tile(const DecodeParams& p, const CUtensorMap* tk, const C
   }
 }
 
+// Paged: the page ids of tile d's pages (ids outside the table read as -1; validated when
+// the tile is issued). Called one tile ahead, so the loads overlap the wait for a free stage.
+template <class C>
+__device__ __forceinline__ void load_tile_pages(const DecodeParams& p, const TileDesc& d, int (&pages)[C::kTS / 16]) {
+  const int ps = p.page_size;
+  const int npg = (d.n + ps - 1) / ps;
+  const int pi0 = d.t0 / ps;
+#pragma unroll
+  for (int i = 0; i < C::kTS / 16; ++i) {
+    const int pi = pi0 + i;
+    pages[i] = (i < npg && pi < p.max_pages) ? p.page_table[(size_t)d.b * p.max_pages + pi] : -1;
+  }
+}
+
 // The producer warp's loop (one elected lane): each stage is refilled once the consumer warps
 // have released it.
 template <class C>
@@ -385,9 +397,14 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
   TileIter ti;
   ti.init(p, s, tb, te);
   bool waited = !C::kOverlapAppend || p.early_from < 0;
-  for (int it = 0, st = 0, phase = 0; ti.t < te; ti.next(p, s), ++it) {
+  int pages[C::kTS / 16];
+  TileDesc d;
+  if (ti.t < te) {
+    d = ti.desc(p, s);
+    if constexpr (C::kPaged) load_tile_pages<C>(p, d, pages);
+  }
+  for (int it = 0, st = 0, phase = 0; ti.t < te; ++it) {
     if (it >= C::kStages && !mbar_wait(empty0 + 8 * st, phase ^ 1, p.status)) return;
-    const TileDesc d = ti.desc(p, s);
     if (!waited && d.t0 + p.ts > p.early_from) {  // this tile holds positions the append writes
       grid_dependency_wait();
       waited = true;
@@ -397,7 +414,12 @@ __device__ void producer(const DecodeParams& p, const CUtensorMap* tk, const CUt
       st = 0;
       phase ^= 1;
     }
-    issue_tile<C>(p, tk, tv, tks, tkz, stages, descs, full0, cur, d);
+    issue_tile<C>(p, tk, tv, tks, tkz, stages, descs, full0, cur, d, pages);
+    ti.next(p, s);
+    if (ti.t < te) {  // the next tile's descriptor and (paged) page ids, ahead of its stage
+      d = ti.desc(p, s);
+      if constexpr (C::kPaged) load_tile_pages<C>(p, d, pages);
+    }
   }
 }
 
@@ -1302,12 +1324,13 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
     fence_barrier_init();
   }
   __syncthreads();
+  const int no_pages[C::kTS / 16] = {};  // dense tiles: no page ids
   if constexpr (C::kSelfFed) {
     if (threadIdx.x == 0) {  // the first stages; the rest are refilled by the consumer warps
       TileIter f;
       f.init(p, sc, tb, te);
       for (int s0 = 0; s0 < C::kStages && f.t < te; ++s0, f.next(p, sc))
-        issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, s0, f.desc(p, sc));
+        issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, s0, f.desc(p, sc), no_pages);
     }
   } else if (warp == kCW) {
     if (lane == 0) producer<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, empty0, sc, tb, te);
@@ -1466,7 +1489,7 @@ __global__ void __launch_bounds__(Cfg<KS, VS, PAGED, NG, ROPE>::kThreadsCta, Cfg
         if (tn < te && mbar_wait(empty0 + 8 * st, phase, p.status)) {
           TileIter f;
           f.init(p, sc, tn, te);
-          issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, st, f.desc(p, sc));
+          issue_tile<C>(p, &tmap_k, &tmap_v, &tmap_ks, &tmap_kz, smem, descs, full0, st, f.desc(p, sc), no_pages);
         }
       }
     }
