@@ -1224,6 +1224,12 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
           }
         }
       }
+      // p * 2^evn once per token (a power of two: exact, so p * 2^evn * s rounds as p * s * 2^evn);
+      // KIVI INT4 keeps the per-group form, whose fewer live registers its allocation prefers
+      constexpr bool kHoist = C::kVFmt != FMT_U4;
+      float pp2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pp2[k] = kHoist ? pt[sb][k] * pscale : pt[sb][k];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         uint32_t bh[2], bl[2];  // P' of group j: tokens (2c, 2c + 1) and (2c + 8, 2c + 9), hi + lo
@@ -1238,7 +1244,10 @@ __device__ __forceinline__ void warp_tile(Consumer<C>& S, const DecodeParams& p,
             } else {
               sj = j == 0 ? s4[k].x : j == 1 ? s4[k].y : j == 2 ? s4[k].z : s4[k].w;
             }
-            pv[k] = residual ? pt[sb][k] * s4[k].x * pscale : pt[sb][k] * sj * pscale;
+            if constexpr (kHoist)
+              pv[k] = residual ? pp2[k] * s4[k].x : pp2[k] * sj;
+            else
+              pv[k] = residual ? pp2[k] * s4[k].x * pscale : pp2[k] * sj * pscale;
           }
           split_f16x2(pv[0], pv[1], bh[0], bl[0]);
           split_f16x2(pv[2], pv[3], bh[1], bl[1]);
