@@ -72,6 +72,12 @@ def test_fused_step_variants():
     fused_steps(S.INT8_SYM_PER_TENSOR, S.UINT8_ASYM_PER_CHANNEL, 64, [1, 1], B=3, Hq=24, Hkv=3)  # G = 8
 
 
+def test_fused_step_without_new_tokens():
+    # n_new = 0: nothing is appended, so the decode is not a dependent of an append and waits at
+    # its start as the plain decode does
+    fused_steps(S.FP8_E4M3_PER_TENSOR, S.FP8_E4M3_PER_TENSOR, 200, [1, 0, 1])
+
+
 def test_fused_step_kivi_runs_in_sequence():
     # KIVI (the flush may rewrite a whole group) takes the two calls one after the other
     fused_steps(S.KIVI_INT4, S.KIVI_INT4, 250, [3, 4, 1])
