@@ -225,6 +225,19 @@ def test_binding_checks_shapes_before_any_device_call():
         paged.append(good_kv, good_kv, new_lens=torch.zeros(3, dtype=torch.int32))
     with pytest.raises(ValueError, match="new_lens: int32"):
         paged.append(good_kv, good_kv, new_lens=torch.zeros(2, dtype=torch.int64))
+    # the one-call step checks the new rows and the query before anything is launched
+    for k, v in bad:
+        with pytest.raises(ValueError):
+            cache.append_decode(k, v, q)
+    with pytest.raises(ValueError, match="q: shape"):
+        cache.append_decode(good_kv, good_kv, torch.zeros(2, 4, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="out: shape"):
+        cache.append_decode(good_kv, good_kv, q, out=torch.zeros(2, 8, 127))
+    scheduled = kvq.QuantizedKVCache(kvq.CacheSpec(2, 8, 2, kvq.FP8_E4M3_PER_TENSOR, kvq.FP8_E4M3_PER_TENSOR,
+                                                   capacity=256), device="cpu", rescale_every=1024)
+    with pytest.raises(ValueError, match="rescaling schedule"):
+        scheduled.append_decode(good_kv, good_kv, q)
+    assert cache.num_quantized == 0  # nothing was appended
 
 
 def test_fp16_kivi_metadata_halves_the_metadata_bytes():
