@@ -1,6 +1,7 @@
 // Split-KV decode attention over the quantized cache (sm_100a).
 //
-// One CTA = 4 consumer warps + 1 producer warp. The grid is a persistent-style set of
+// One CTA = 4 consumer warps + 1 producer warp (dense KIVI: the consumer warps refill the
+// stages themselves, see Cfg::kSelfFed). The grid is a persistent-style set of
 // CTAs; the flattened list of (batch, kv_head, head-group) token tiles is cut into equal
 // contiguous ranges, one per CTA, so every SM streams the same number of bytes however
 // the sequence lengths vary. Tiles of codes reach shared memory by 2-D TMA with hardware
